@@ -1,0 +1,176 @@
+"""NumPy front end of the CPU oracle (``dashkv_oracle.c``).
+
+Test infrastructure only: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` use this module; the product library never
+imports it.  Every function takes and returns NumPy arrays; floating-point
+inputs are widened to float64 before they reach the C code, so bf16 values
+arrive exactly.
+
+The steps follow the pages' method (see the C file's header for the exact
+definitions and the passages they come from): sign-random-projection key
+codes, a full-precision query scored against those codes, exact top-k with
+sinks and a recent window, then exact softmax attention over the selected
+tokens only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dashkv_oracle.c")
+_LIB = os.path.join(_HERE, "libdashkv_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle in place (gcc, OpenMP) and return the .so path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P, I, I64, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
+        L.dko_splitmix64_nth.argtypes = [U64, U64]
+        L.dko_splitmix64_nth.restype = U64
+        L.dko_hyperplanes.argtypes = [U64, I, I, P]
+        L.dko_encode.argtypes = [I, I, I, I, I64, P, I, I, P, P, P, P]
+        L.dko_append.argtypes = [I, I, I, I, I64, P, I, I, P, P, P, P, P, P, P]
+        L.dko_scores.argtypes = [I, I, I, I, I, I64, P, I, I, P, P, P, P, P]
+        L.dko_scores.restype = ctypes.c_double
+        L.dko_select.argtypes = [I, I, I64, P, P, I, I, I, P, P, I]
+        L.dko_select.restype = I
+        L.dko_attend.argtypes = [I, I, I, I, I64, P, I, I, P, P, P, P, P, I, P, P]
+        L.dko_set_threads.argtypes = [I]
+        L.dko_get_threads.restype = I
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def set_threads(n: int) -> None:
+    lib().dko_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().dko_get_threads())
+
+
+def splitmix64_nth(seed: int, n: int) -> int:
+    return int(lib().dko_splitmix64_nth(seed & (2**64 - 1), n))
+
+
+def hyperplanes(seed: int, bits: int, d: int) -> np.ndarray:
+    """R[j][i] in {+1, -1}, shape [bits, d], int8."""
+    R = np.empty((bits, d), dtype=np.int8)
+    lib().dko_hyperplanes(seed & (2**64 - 1), bits, d, _p(R))
+    return R
+
+
+class Layout:
+    """Dense ([B,Hkv,n_cap,d]) or paged ([P,page,Hkv,d] + page table) KV layout."""
+
+    def __init__(self, B, Hkv, d, bits, n_cap=0, page_table=None, page=0):
+        self.B, self.Hkv, self.d, self.bits = int(B), int(Hkv), int(d), int(bits)
+        self.n_cap = int(n_cap)
+        self.page = int(page)
+        self.page_table = None if page_table is None else _i32(page_table)
+        self.max_pages = 0 if page_table is None else int(self.page_table.shape[1])
+        self.w64 = max(1, self.bits // 64)
+
+    def args(self):
+        return (self.B, self.Hkv, self.d, self.bits, self.n_cap,
+                _p(self.page_table), self.max_pages, self.page)
+
+
+def encode(layout: Layout, K, seq_lens, R, codes: np.ndarray | None = None) -> np.ndarray:
+    """Codes for tokens [0, seq_lens[b]) in the layout's code shape (uint64)."""
+    K = _f64(K)
+    seq = _i32(seq_lens)
+    R = np.ascontiguousarray(R, dtype=np.int8)
+    if codes is None:
+        if layout.page:
+            P = K.shape[0]
+            codes = np.zeros((P, layout.Hkv, layout.page, layout.w64), dtype=np.uint64)
+        else:
+            codes = np.zeros((layout.B, layout.Hkv, layout.n_cap, layout.w64), dtype=np.uint64)
+    lib().dko_encode(*layout.args(), _p(K), _p(seq), _p(R), _p(codes))
+    return codes
+
+
+def append(layout: Layout, K: np.ndarray, V: np.ndarray, codes: np.ndarray, seq_lens: np.ndarray,
+           k_new, v_new, R) -> None:
+    """In-place append of one token per (b, kv head); K, V float64, seq_lens int32."""
+    assert K.dtype == np.float64 and V.dtype == np.float64 and seq_lens.dtype == np.int32
+    lib().dko_append(*layout.args(), _p(K), _p(V), _p(codes), _p(seq_lens),
+                     _p(_f64(k_new)), _p(_f64(v_new)), _p(np.ascontiguousarray(R, dtype=np.int8)))
+
+
+def scores(layout: Layout, Hq, q, codes, seq_lens, R):
+    """(scores [B,Hkv,n_cap] float64 (NaN beyond seq_len), bound on |s|)."""
+    n_cap = layout.n_cap if not layout.page else layout.max_pages * layout.page
+    out = np.full((layout.B, layout.Hkv, n_cap), np.nan)
+    # the C side uses n_cap as the scores row length (and, dense, as the KV row count)
+    B, Hkv, d, bits, _, pt, mp, page = layout.args()
+    bound = lib().dko_scores(B, int(Hq), Hkv, d, bits, n_cap, pt, mp, page,
+                             _p(_f64(q)), _p(np.ascontiguousarray(codes, dtype=np.uint64)),
+                             _p(_i32(seq_lens)), _p(np.ascontiguousarray(R, dtype=np.int8)), _p(out))
+    return out, float(bound)
+
+
+def select(scores_arr, seq_lens, topk, sink, window, cap=None):
+    """(sel_idx [B,Hkv,cap] int32 ascending, -1 padded; sel_cnt [B,Hkv] int32)."""
+    s = _f64(scores_arr)
+    B, Hkv, n_cap = s.shape
+    cap = int(cap if cap is not None else topk + sink + window)
+    idx = np.empty((B, Hkv, cap), dtype=np.int32)
+    cnt = np.empty((B, Hkv), dtype=np.int32)
+    rc = lib().dko_select(B, Hkv, n_cap, _p(_i32(seq_lens)), _p(s), int(topk), int(sink),
+                          int(window), _p(idx), _p(cnt), cap)
+    if rc != 0:
+        raise ValueError("selection larger than cap")
+    return idx, cnt
+
+
+def attend(layout: Layout, Hq, q, K, V, sel_idx, sel_cnt):
+    """(out [B,Hq,d] float64, lse [B,Hq] float64)."""
+    sel_idx = _i32(sel_idx)
+    cap = sel_idx.shape[-1]
+    out = np.empty((layout.B, int(Hq), layout.d))
+    lse = np.empty((layout.B, int(Hq)))
+    B, Hkv, d, _, n_cap, pt, mp, page = layout.args()
+    lib().dko_attend(B, int(Hq), Hkv, d, n_cap, pt, mp, page, _p(_f64(q)), _p(_f64(K)), _p(_f64(V)),
+                     _p(sel_idx), _p(_i32(sel_cnt)), cap, _p(out), _p(lse))
+    return out, lse
+
+
+def decode_step(layout: Layout, Hq, q, K, V, codes, seq_lens, R, topk, sink, window):
+    """Score -> select -> attend for one decode query batch (no append)."""
+    sc, bound = scores(layout, Hq, q, codes, seq_lens, R)
+    idx, cnt = select(sc, seq_lens, topk, sink, window)
+    out, lse = attend(layout, Hq, q, K, V, idx, cnt)
+    return dict(scores=sc, bound=bound, sel_idx=idx, sel_cnt=cnt, out=out, lse=lse)
