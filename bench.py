@@ -1,0 +1,363 @@
+"""Decode-step benchmark: append -> hash-score + top-k select -> sparse attention.
+
+One step = one decode query per sequence of the batch: append the new key /
+value (with its code), score every cached key from its code, select top-k +
+sinks + window, attend over the selection.  Default workload: B=4 sequences of
+128K cached tokens, Hq=32, Hkv=8, d=128, 128-bit codes, k=2048, S=4, W=512
+(synthetic 1/64-grid Gaussian K/V/Q with planted needles).
+
+L2 is flushed (a 2 x L2 buffer is written) before every timed step; each step
+is timed with CUDA events on the launching stream.  Multi-GPU: one replica per
+rank (weak scaling, no data-path collective); NCCL only for the barrier and
+the max-over-ranks of the timings.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dashkv|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hash_indexed_top_b200 import workloads as W  # noqa: E402
+
+METRIC = "sparse-decode queries/s at 128K ctx; achieved HBM GB/s vs ~8 TB/s peak"
+SPEC_HBM_GBS = 8000.0
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
+    return dict(hbm_gbs=6650.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while timing."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if (args.impl == "dashkv" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available() and args.impl == "dashkv":
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
+    """Time the CPU oracle's decode step (score + select + attend) on one
+    sequence of the workload (all its KV / query heads), after one untimed
+    oracle encode of that sequence's cache."""
+    from oracle import oracle as O
+    one = cfg.scaled(B=1, steps=n_steps)
+    w = W.make_workload(one, device="cpu", steps=n_steps)
+    R = O.hyperplanes(W.HYPERPLANE_SEED, cfg.bits, cfg.d)
+    L = O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=w.n_cap)
+    K = w.K.double().numpy()
+    V = w.V.double().numpy()
+    seq = w.seq_lens.numpy().astype(np.int32).copy()
+    codes = O.encode(L, K, seq, R)
+    times = []
+    for s in range(n_steps):
+        O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
+        t0 = time.perf_counter()
+        O.decode_step(L, cfg.Hq, w.q[s].double().numpy(), K, V, codes, seq, R, cfg.topk, cfg.sink, cfg.window)
+        times.append(time.perf_counter() - t0)
+    return dict(times=times, cores=O.get_threads(),
+                sample=f"sequence {seq_index} of {cfg.B} (N={cfg.N}, all {cfg.Hkv} KV / {cfg.Hq} query heads), "
+                       f"{n_steps} decode steps, oracle encode untimed")
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    warm = max(0, args.warmup)
+    r = oracle_sample(cfg, warm + args.steps)
+    t = r["times"][warm:]
+    value = len(t) / sum(t)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(t) / len(t),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+                   "bits": cfg.bits, "topk": cfg.topk, "sink": cfg.sink, "window": cfg.window,
+                   "per_step_sample": "one sequence's decode query"},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_dashkv(args, cfg, world, rank, local):
+    from hash_indexed_top_b200 import build
+    from hash_indexed_top_b200 import dashkv as dk
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: the dashkv arm needs a CUDA device")
+    build.build()
+    dev = torch.device("cuda", local)
+    total = args.warmup + args.steps + args.e2e_steps
+    w = W.make_workload(cfg, device=dev, steps=total)
+    eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
+                    cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED)
+    codes = dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged)
+    cache = dk.KVCache(w.K, w.V, codes, w.page_table)
+    seq = w.seq_lens.clone()
+    ws = eng.workspace(cache.capacity, dev)
+    buf = eng.alloc_step(dev)
+    flush = W.flush_buffer(dev)
+    stream = torch.cuda.current_stream(dev)
+    eng.encode_keys(cache, seq)
+    torch.cuda.synchronize(dev)
+    assert eng.get_error() == 0
+
+    def step(s):
+        eng.append_keys(cache, w.k_new[s], w.v_new[s], seq)
+        eng.select(cache, w.q[s], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+        eng.sparse_decode(cache, w.q[s], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+
+    for s in range(args.warmup):
+        flush.fill_(s)
+        step(s)
+    torch.cuda.synchronize(dev)
+
+    # ---- device-timed steps (+ per-kernel trace events)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(K)]
+    n_before = seq.clone()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        wall0 = time.perf_counter()
+        for i in range(K):
+            flush.fill_(i)
+            e = ev[i]
+            e[0].record(stream)
+            eng.set_trace(e[2:4])
+            eng.append_keys(cache, w.k_new[args.warmup + i], w.v_new[args.warmup + i], seq)
+            eng.set_trace(e[4:8])
+            eng.select(cache, w.q[args.warmup + i], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            eng.set_trace(e[8:10])
+            eng.sparse_decode(cache, w.q[args.warmup + i], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+            eng.set_trace(None)
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    barrier(world)
+    assert eng.get_error() == 0
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    kern = {
+        "append_keys": [e[2].elapsed_time(e[3]) for e in ev],
+        "score_hist": [e[4].elapsed_time(e[5]) for e in ev],
+        "collect_select": [e[6].elapsed_time(e[7]) for e in ev],
+        "sparse_decode": [e[8].elapsed_time(e[9]) for e in ev],
+    }
+    sum_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = sum_ms / K
+    value = world * cfg.B * K / (sum_ms / 1e3)
+
+    # ---- algorithmic bytes (codes of every cached key + selected K/V rows + q in / out)
+    lens_mid = n_before.double() + 1 + (K - 1) / 2.0  # mean cache length over the timed steps
+    code_bytes = float(lens_mid.sum()) * cfg.Hkv * cfg.bits / 8
+    sel_rows = float(buf["sel_cnt"].sum())
+    kv_bytes = sel_rows * 2 * cfg.d * 2
+    qo_bytes = cfg.B * cfg.Hq * cfg.d * (2 + 4)
+    step_bytes = code_bytes + kv_bytes + qo_bytes
+    peaks = measured_peaks()
+    kms = {k: statistics.mean(v) for k, v in kern.items()}
+    score_gbs = code_bytes / (kms["score_hist"] * 1e-3) / 1e9
+    decode_gbs = kv_bytes / (kms["sparse_decode"] * 1e-3) / 1e9
+    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    E = args.e2e_steps
+    e2e = None
+    if E > 0:
+        hq = w.q.cpu().pin_memory()
+        hk = w.k_new.cpu().pin_memory()
+        hv = w.v_new.cpu().pin_memory()
+        h_out = torch.empty_like(buf["out"], device="cpu").pin_memory()
+        h_lse = torch.empty_like(buf["lse"], device="cpu").pin_memory()
+        dq = torch.empty_like(w.q[0])
+        dkn = torch.empty_like(w.k_new[0])
+        dvn = torch.empty_like(w.v_new[0])
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(E)]
+        barrier(world)
+        for i in range(E):
+            s = args.warmup + K + i
+            flush.fill_(i)
+            eev[i][0].record(stream)
+            dq.copy_(hq[s], non_blocking=True)
+            dkn.copy_(hk[s], non_blocking=True)
+            dvn.copy_(hv[s], non_blocking=True)
+            eng.append_keys(cache, dkn, dvn, seq)
+            eng.select(cache, dq, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            eng.sparse_decode(cache, dq, buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+            h_out.copy_(buf["out"], non_blocking=True)
+            h_lse.copy_(buf["lse"], non_blocking=True)
+            eev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        assert eng.get_error() == 0
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), world)
+        h2d = dq.numel() * dq.element_size() + dkn.numel() * dkn.element_size() * 2
+        d2h = h_out.numel() * 4 + h_lse.numel() * 4
+        e2e = {"value": world * cfg.B * E / (e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": E}
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_steps > 0:
+        r = oracle_sample(cfg, args.cpu_steps)
+        cpu = {"value": len(r["times"]) / sum(r["times"]), "unit": "queries/s", "cores": r["cores"],
+               "kind": "oracle", "sample": r["sample"]}
+
+    clk = clocks.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+                       "bits": cfg.bits, "topk": cfg.topk, "sink": cfg.sink, "window": cfg.window,
+                       "layout": "paged" if w.paged else "dense", "l2": "flushed before every step (2 x L2 write)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "score_hist", "achieved": score_gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": score_gbs / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"], "frac_of_8tbs": score_gbs / SPEC_HBM_GBS,
+                         "algorithmic_bytes_per_launch": code_bytes, "traffic": None},
+            "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_gbs,
+                              "frac": step_gbs / peaks["hbm_gbs"], "frac_of_8tbs": step_gbs / SPEC_HBM_GBS,
+                              "code_bytes": code_bytes, "selected_kv_bytes": kv_bytes, "q_out_bytes": qo_bytes},
+            "kernels_ms": kms,
+            "kernel_gbs": {"score_hist": score_gbs, "sparse_decode": decode_gbs},
+            "codes_scanned_per_s": float(lens_mid.sum()) * cfg.Hkv / (ms_per_step * 1e-3),
+            "selected_kv_bytes_per_s": kv_bytes / (ms_per_step * 1e-3),
+            "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 4 * K, "clocks": clk,
+            "wall_s_timed_region": wall,
+        }
+        print(json.dumps(line), flush=True)
+    eng.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["dashkv", "reference"], default="dashkv")
+    ap.add_argument("--config", default="c128k", choices=sorted(W.CONFIGS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-steps", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = W.CONFIGS[args.config]
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, world, rank)
+        else:
+            run_dashkv(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

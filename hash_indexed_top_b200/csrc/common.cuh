@@ -1,0 +1,93 @@
+// common.cuh -- layout addressing, hyperplane bits and the device error word
+// shared by the kernels of libdashkv (one translation unit: dashkv.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dkv {
+
+constexpr int kMaxBits = 128;
+constexpr int kMaxDim = 128;
+constexpr int kSmCountFallback = 148;
+
+// Device error word (one per device that loads the library).  Bits:
+enum : unsigned { kErrCapacity = 1u, kErrPage = 2u };
+__device__ unsigned g_error_word;
+
+__device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }
+
+// Hyperplanes as sign bits: bit (i % 32) of word [j * (d / 32) + i / 32] is set
+// when R[j][i] = -1.  2 KB at bits = d = 128, passed by value as a kernel
+// parameter (constant bank), so no device allocation is needed.
+struct RBits {
+    uint32_t w[kMaxBits * kMaxDim / 32];
+};
+
+// Cache addressing.  page_size == 0 selects the dense layout.
+struct KV {
+    __nv_bfloat16 *k;
+    __nv_bfloat16 *v;
+    uint64_t *codes;
+    int64_t n_cap;             // dense rows per (b, h)
+    const int32_t *page_table; // [B][max_pages]
+    int32_t max_pages;
+    int32_t num_pages;
+    int32_t page_size;         // 0 = dense
+    int32_t Hkv;
+    int32_t d;
+    int32_t W;                 // 64-bit code words per key
+
+    __host__ __device__ int64_t capacity() const {
+        return page_size ? (int64_t)max_pages * page_size : n_cap;
+    }
+    // Physical page of token t of sequence b, or -1 (error word set) when the
+    // page table entry is out of range.
+    __device__ __forceinline__ int64_t page_of(int b, int64_t t) const {
+        int32_t p = __ldg(page_table + (int64_t)b * max_pages + t / page_size);
+        if (p < 0 || p >= num_pages) {
+            raise_error(kErrPage);
+            return -1;
+        }
+        return p;
+    }
+    // Element offset of row (b, h, t) in k / v, or -1.
+    __device__ __forceinline__ int64_t row(int b, int h, int64_t t) const {
+        if (!page_size) return (((int64_t)b * Hkv + h) * n_cap + t) * d;
+        int64_t p = page_of(b, t);
+        if (p < 0) return -1;
+        return ((p * page_size + t % page_size) * Hkv + h) * (int64_t)d;
+    }
+    // Word offset of the code of (b, h, t), or -1.
+    __device__ __forceinline__ int64_t code(int b, int h, int64_t t) const {
+        if (!page_size) return (((int64_t)b * Hkv + h) * n_cap + t) * W;
+        int64_t p = page_of(b, t);
+        if (p < 0) return -1;
+        return ((p * Hkv + h) * page_size + t % page_size) * (int64_t)W;
+    }
+};
+
+// Sequence length clamped to the capacity (error word set when it exceeds it).
+__device__ __forceinline__ int64_t clamp_len(const KV &kv, const int32_t *seq_lens, int b) {
+    int64_t n = __ldg(seq_lens + b);
+    int64_t cap = kv.capacity();
+    if (n > cap) {
+        raise_error(kErrCapacity);
+        n = cap;
+    }
+    return n < 0 ? 0 : n;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+// Order-preserving map from fp32 to uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace dkv

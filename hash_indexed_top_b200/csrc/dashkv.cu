@@ -1,0 +1,424 @@
+// dashkv.cu -- the C ABI declared in include/dashkv.h: host-side validation,
+// context, workspace carving and kernel launches.  Every stage of the decode
+// step runs in the kernels of encode.cuh, select.cuh and decode.cuh; this file
+// only checks arguments and enqueues them.  The library allocates no device
+// memory: the caller passes every buffer, including the workspace.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "../../include/dashkv.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "encode.cuh"
+#include "select.cuh"
+
+using namespace dkv;
+
+struct dashkv_ctx {
+    dashkv_config cfg;
+    RBits R;
+    int device;
+    int sm_count;
+    void **trace;   // optional cudaEvent_t pairs around each kernel of a call
+    int n_trace;
+};
+
+namespace {
+// Records the tracing events around the kernels of one call.
+struct Tracer {
+    const dashkv_ctx *ctx;
+    cudaStream_t st;
+    int k = 0;
+    Tracer(const dashkv_ctx *c, cudaStream_t s) : ctx(c), st(s) {}
+    void before() {
+        if (ctx->trace && 2 * k + 1 < ctx->n_trace) cudaEventRecord((cudaEvent_t)ctx->trace[2 * k], st);
+    }
+    void after() {
+        if (ctx->trace && 2 * k + 1 < ctx->n_trace) cudaEventRecord((cudaEvent_t)ctx->trace[2 * k + 1], st);
+        ++k;
+    }
+};
+}  // namespace
+
+namespace {
+
+// splitmix64: output number n (n >= 1) of the stream that starts at `seed`.
+uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
+    uint64_t z = seed + n * 0x9E3779B97F4A7C15ULL;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+// R[j][i] = -1 iff the top bit of output j*d+i+1 is set; packed as sign bits.
+void build_rbits(uint64_t seed, int bits, int d, RBits *R) {
+    memset(R, 0, sizeof(*R));
+    for (int j = 0; j < bits; ++j)
+        for (int i = 0; i < d; ++i)
+            if (splitmix64_at(seed, (uint64_t)j * d + i + 1) >> 63) R->w[j * (d / 32) + i / 32] |= 1u << (i % 32);
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+dashkv_status check_config(const dashkv_config *c) {
+    if (!c) return DASHKV_ERR_INVALID_ARG;
+    if (c->batch <= 0 || c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->topk <= 0 || c->sink < 0 ||
+        c->window < 0 || c->page_size < 0 || c->reserved != 0)
+        return DASHKV_ERR_INVALID_ARG;
+    if (c->num_q_heads % c->num_kv_heads) return DASHKV_ERR_INVALID_ARG;
+    const int G = c->num_q_heads / c->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return DASHKV_ERR_UNSUPPORTED;
+    if (c->head_dim != 64 && c->head_dim != 128) return DASHKV_ERR_UNSUPPORTED;
+    if (c->bits != 32 && c->bits != 64 && c->bits != 128) return DASHKV_ERR_UNSUPPORTED;
+    if (c->page_size && (c->page_size % 32 || c->page_size > 1024)) return DASHKV_ERR_UNSUPPORTED;
+    if (c->num_kv_heads > 32) return DASHKV_ERR_UNSUPPORTED;
+    if ((int64_t)c->topk + c->sink + c->window > 0x7fffffff / 2) return DASHKV_ERR_INVALID_ARG;
+    return DASHKV_OK;
+}
+
+dashkv_status check_view(const dashkv_ctx *ctx, const dashkv_kv_view *kv, bool need_kv, bool need_codes) {
+    if (!kv) return DASHKV_ERR_INVALID_ARG;
+    const dashkv_config &c = ctx->cfg;
+    if (need_kv && (!kv->k || !kv->v || !aligned(kv->k, 16) || !aligned(kv->v, 16))) return DASHKV_ERR_INVALID_ARG;
+    if (need_codes && (!kv->codes || !aligned(kv->codes, c.bits == 128 ? 16 : 8))) return DASHKV_ERR_INVALID_ARG;
+    if (c.page_size) {
+        if (!kv->page_table || kv->max_pages <= 0 || kv->num_pages <= 0) return DASHKV_ERR_INVALID_ARG;
+    } else {
+        if (kv->page_table || kv->n_cap <= 0) return DASHKV_ERR_INVALID_ARG;
+    }
+    const int64_t cap = c.page_size ? (int64_t)kv->max_pages * c.page_size : kv->n_cap;
+    if (cap > 0x7fffffffLL) return DASHKV_ERR_INVALID_ARG;  // token ids are int32
+    return DASHKV_OK;
+}
+
+KV make_kv(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
+    KV o;
+    o.k = static_cast<__nv_bfloat16 *>(kv->k);
+    o.v = static_cast<__nv_bfloat16 *>(kv->v);
+    o.codes = kv->codes;
+    o.n_cap = kv->n_cap;
+    o.page_table = kv->page_table;
+    o.max_pages = kv->max_pages;
+    o.num_pages = kv->num_pages;
+    o.page_size = ctx->cfg.page_size;
+    o.Hkv = ctx->cfg.num_kv_heads;
+    o.d = ctx->cfg.head_dim;
+    o.W = ctx->cfg.bits >= 64 ? ctx->cfg.bits / 64 : 1;
+    return o;
+}
+
+int64_t view_capacity(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
+    return ctx->cfg.page_size ? (int64_t)kv->max_pages * ctx->cfg.page_size : kv->n_cap;
+}
+
+// ---- workspace: [scores | cand | hist | state | arrive(3 x BH) | seg_cnt | partials]
+struct WsLayout {
+    size_t scores, cand, hist, state, arrive, seg_cnt, part, total;
+};
+
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
+    const size_t BH = (size_t)c.batch * c.num_kv_heads;
+    const size_t G = (size_t)(c.num_q_heads / c.num_kv_heads);
+    WsLayout L;
+    size_t o = 0;
+    L.scores = o;  o = align_up(o + BH * (size_t)max_tokens * 4);
+    L.cand = o;    o = align_up(o + BH * (size_t)max_tokens * 4);
+    L.hist = o;    o = align_up(o + BH * kBins * 4);
+    L.state = o;   o = align_up(o + BH * sizeof(SelState));
+    L.arrive = o;  o = align_up(o + 3 * BH * 4);
+    L.seg_cnt = o; o = align_up(o + BH * kMaxSelCtas * 4);
+    L.part = o;    o = align_up(o + BH * kMaxSplits * G * (c.head_dim + 2) * 4);
+    L.total = o;
+    return L;
+}
+
+dashkv_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? DASHKV_OK : DASHKV_ERR_CUDA;
+}
+
+int sel_ctas(const dashkv_ctx *ctx, int64_t cap) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    int n = (2 * ctx->sm_count) / BH;
+    if (n < 1) n = 1;
+    const int64_t by_tokens = ceil_div(cap, 1024);
+    if (n > by_tokens) n = (int)by_tokens;
+    if (n > kMaxSelCtas) n = kMaxSelCtas;
+    return n < 1 ? 1 : n;
+}
+
+int attn_splits(const dashkv_ctx *ctx) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int64_t cap_sel = (int64_t)ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
+    int64_t n = ceil_div(4 * ctx->sm_count, BH);
+    const int64_t by_rows = ceil_div(cap_sel, 128);
+    if (n > by_rows) n = by_rows;
+    if (n > kMaxSplits) n = kMaxSplits;
+    return n < 1 ? 1 : (int)n;
+}
+
+// ---- template dispatch
+template <int BITS, int D>
+void set_attrs_bd() {
+    cudaFuncSetAttribute(encode_keys_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)EncodeShape<BITS, D>::SMEM);
+    cudaFuncSetAttribute(score_hist_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+}
+
+void set_attrs() {
+    set_attrs_bd<32, 64>();  set_attrs_bd<32, 128>();
+    set_attrs_bd<64, 64>();  set_attrs_bd<64, 128>();
+    set_attrs_bd<128, 64>(); set_attrs_bd<128, 128>();
+}
+
+template <int BITS, int D>
+void launch_encode_bd(const dashkv_ctx *ctx, const KV &kv, const int32_t *seq_lens, cudaStream_t st) {
+    using S = EncodeShape<BITS, D>;
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int64_t tiles = ceil_div(kv.capacity(), S::KT);
+    int64_t gx = ceil_div(8 * ctx->sm_count, BH);
+    if (gx > tiles) gx = tiles;
+    if (gx < 1) gx = 1;
+    encode_keys_kernel<BITS, D><<<dim3((unsigned)gx, BH), S::THREADS, S::SMEM, st>>>(kv, seq_lens, ctx->R, tiles);
+}
+
+template <int D>
+void launch_encode_d(const dashkv_ctx *ctx, const KV &kv, const int32_t *s, cudaStream_t st) {
+    switch (ctx->cfg.bits) {
+        case 32: launch_encode_bd<32, D>(ctx, kv, s, st); break;
+        case 64: launch_encode_bd<64, D>(ctx, kv, s, st); break;
+        default: launch_encode_bd<128, D>(ctx, kv, s, st); break;
+    }
+}
+
+template <int BITS, int D>
+void launch_append_bd(const dashkv_ctx *ctx, const KV &kv, const void *kn, const void *vn, int32_t *seq,
+                      cudaStream_t st) {
+    append_keys_kernel<BITS, D><<<ctx->cfg.batch, 32 * ctx->cfg.num_kv_heads, 0, st>>>(
+        kv, static_cast<const __nv_bfloat16 *>(kn), static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R);
+}
+
+template <int D>
+void launch_append_d(const dashkv_ctx *ctx, const KV &kv, const void *kn, const void *vn, int32_t *seq,
+                     cudaStream_t st) {
+    switch (ctx->cfg.bits) {
+        case 32: launch_append_bd<32, D>(ctx, kv, kn, vn, seq, st); break;
+        case 64: launch_append_bd<64, D>(ctx, kv, kn, vn, seq, st); break;
+        default: launch_append_bd<128, D>(ctx, kv, kn, vn, seq, st); break;
+    }
+}
+
+template <int BITS, int D>
+void launch_score_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                     int nctas, cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
+    score_hist_kernel<BITS, D><<<dim3(nctas, BH), kSelThreads, ScoreShape<BITS>::SMEM, st>>>(
+        kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, ctx->cfg.topk, nctas);
+}
+
+template <int D>
+void launch_score_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                    int nctas, cudaStream_t st) {
+    switch (ctx->cfg.bits) {
+        case 32: launch_score_bd<32, D>(ctx, kv, q, seq, ws, nctas, st); break;
+        case 64: launch_score_bd<64, D>(ctx, kv, q, seq, ws, nctas, st); break;
+        default: launch_score_bd<128, D>(ctx, kv, q, seq, ws, nctas, st); break;
+    }
+}
+
+template <int D, int G>
+void launch_decode_dg(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *si, const int32_t *sc,
+                      float *out, float *lse, const AttnWS &ws, cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int splits = attn_splits(ctx);
+    const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
+    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    sparse_decode_kernel<D, G><<<dim3(splits, BH), kAttnThreads, 0, st>>>(
+        kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws, splits,
+        scale_log2);
+}
+
+template <int D>
+void launch_decode_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *si, const int32_t *sc,
+                     float *out, float *lse, const AttnWS &ws, cudaStream_t st) {
+    switch (ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads) {
+        case 1: launch_decode_dg<D, 1>(ctx, kv, q, si, sc, out, lse, ws, st); break;
+        case 2: launch_decode_dg<D, 2>(ctx, kv, q, si, sc, out, lse, ws, st); break;
+        case 4: launch_decode_dg<D, 4>(ctx, kv, q, si, sc, out, lse, ws, st); break;
+        default: launch_decode_dg<D, 8>(ctx, kv, q, si, sc, out, lse, ws, st); break;
+    }
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+const char *dashkv_status_str(dashkv_status s) {
+    switch (s) {
+        case DASHKV_OK: return "ok";
+        case DASHKV_ERR_INVALID_ARG: return "invalid argument";
+        case DASHKV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case DASHKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case DASHKV_ERR_CAPACITY: return "sequence length beyond cache capacity";
+        case DASHKV_ERR_CUDA: return "CUDA error";
+        case DASHKV_ERR_DEVICE: return "page id out of range";
+        case DASHKV_ERR_NO_DEVICE: return "no CUDA device";
+    }
+    return "unknown status";
+}
+
+dashkv_status dashkv_hyperplanes(uint64_t seed, int32_t bits, int32_t d, int8_t *host_out) {
+    if (!host_out || bits <= 0 || d <= 0 || bits > kMaxBits || d > kMaxDim || d % 32) return DASHKV_ERR_INVALID_ARG;
+    RBits R;
+    build_rbits(seed, bits, d, &R);
+    for (int j = 0; j < bits; ++j)
+        for (int i = 0; i < d; ++i) host_out[j * d + i] = ((R.w[j * (d / 32) + i / 32] >> (i % 32)) & 1u) ? -1 : 1;
+    return DASHKV_OK;
+}
+
+dashkv_status dashkv_create(const dashkv_config *cfg, dashkv_ctx **out) {
+    if (!out) return DASHKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    dashkv_status st = check_config(cfg);
+    if (st != DASHKV_OK) return st;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return DASHKV_ERR_NO_DEVICE;
+    }
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = kSmCountFallback;
+    dashkv_ctx *c = static_cast<dashkv_ctx *>(calloc(1, sizeof(dashkv_ctx)));
+    if (!c) return DASHKV_ERR_INVALID_ARG;
+    c->cfg = *cfg;
+    c->device = dev;
+    c->sm_count = sms;
+    build_rbits(cfg->seed, cfg->bits, cfg->head_dim, &c->R);
+    set_attrs();
+    if (cudaGetLastError() != cudaSuccess) {
+        free(c);
+        return DASHKV_ERR_CUDA;
+    }
+    *out = c;
+    return DASHKV_OK;
+}
+
+void dashkv_destroy(dashkv_ctx *ctx) { free(ctx); }
+
+size_t dashkv_workspace_size(const dashkv_ctx *ctx, int64_t max_tokens) {
+    if (!ctx || max_tokens < 0) return 0;
+    return ws_layout(ctx->cfg, max_tokens).total;
+}
+
+dashkv_status dashkv_encode_keys(dashkv_ctx *ctx, const dashkv_kv_view *kv, const int32_t *seq_lens, void *stream) {
+    if (!ctx || !seq_lens) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, true);
+    if (s != DASHKV_OK) return s;
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_encode_d<64>(ctx, k, seq_lens, st);
+    else launch_encode_d<128>(ctx, k, seq_lens, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_append_keys(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *k_new, const void *v_new,
+                                 int32_t *seq_lens, void *stream) {
+    if (!ctx || !seq_lens || !k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))
+        return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, true);
+    if (s != DASHKV_OK) return s;
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_append_d<64>(ctx, k, k_new, v_new, seq_lens, st);
+    else launch_append_d<128>(ctx, k, k_new, v_new, seq_lens, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q, const int32_t *seq_lens,
+                            int32_t *sel_idx, int32_t *sel_cnt, float *scores, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    if (!ctx || !q || !seq_lens || !sel_idx || !sel_cnt || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, false, true);
+    if (s != DASHKV_OK) return s;
+    const int64_t cap = view_capacity(ctx, kv);
+    const WsLayout L = ws_layout(ctx->cfg, cap);
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
+    char *w = static_cast<char *>(workspace);
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    SelWS ws;
+    ws.scores = scores ? scores : reinterpret_cast<float *>(w + L.scores);
+    ws.ld = cap;
+    ws.cand = reinterpret_cast<int32_t *>(w + L.cand);
+    ws.hist = reinterpret_cast<uint32_t *>(w + L.hist);
+    ws.state = reinterpret_cast<SelState *>(w + L.state);
+    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive);
+    ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int nctas = sel_ctas(ctx, cap);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_score_d<64>(ctx, k, q, seq_lens, ws, nctas, st);
+    else launch_score_d<128>(ctx, k, q, seq_lens, ws, nctas, st);
+    tr.after();
+    const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
+    tr.before();
+    collect_kernel<<<dim3(nctas, BH), kSelThreads, 0, st>>>(seq_lens, ws, nctas, ctx->cfg.sink, ctx->cfg.window,
+                                                            cap_sel, sel_idx, sel_cnt);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
+                                   const int32_t *sel_idx, const int32_t *sel_cnt, float *out, float *lse,
+                                   void *workspace, size_t workspace_bytes, void *stream) {
+    if (!ctx || !q || !sel_idx || !sel_cnt || !out || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, false);
+    if (s != DASHKV_OK) return s;
+    const WsLayout L = ws_layout(ctx->cfg, view_capacity(ctx, kv));
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
+    char *w = static_cast<char *>(workspace);
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    AttnWS ws;
+    ws.part = reinterpret_cast<float *>(w + L.part);
+    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive) + 2 * BH;
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, st);
+    else launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_set_trace(dashkv_ctx *ctx, void **events, int32_t n_events) {
+    if (!ctx || n_events < 0 || (events && n_events < 2)) return DASHKV_ERR_INVALID_ARG;
+    ctx->trace = events;
+    ctx->n_trace = events ? n_events : 0;
+    return DASHKV_OK;
+}
+
+dashkv_status dashkv_get_error(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DASHKV_ERR_CUDA;
+    unsigned w = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (w && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (w & kErrPage) return DASHKV_ERR_DEVICE;
+    if (w & kErrCapacity) return DASHKV_ERR_CAPACITY;
+    return DASHKV_OK;
+}
+
+}  // extern "C"

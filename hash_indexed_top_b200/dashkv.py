@@ -1,0 +1,230 @@
+"""Python binding of ``libdashkv.so`` (C ABI in ``include/dashkv.h``).
+
+Argument marshalling only: every stage of the decode step runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams; tensors
+are passed to the C calls as raw pointers.  There is no CPU fallback -- if the
+shared library is missing or no CUDA device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdashkv.so")
+
+STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace missing or too small",
+    4: "sequence length beyond cache capacity", 5: "CUDA error", 6: "page id out of range", 7: "no CUDA device",
+}
+
+SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_encode_keys",
+           "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
+           "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_status_str")
+
+
+class DashKVError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call}: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("bits", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("sink", ctypes.c_int32), ("window", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+
+
+class KVView(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("n_cap", ctypes.c_int64), ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdashkv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with hash_indexed_top_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t
+        L.dashkv_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(P)]
+        L.dashkv_create.restype = ctypes.c_int
+        L.dashkv_destroy.argtypes = [P]
+        L.dashkv_destroy.restype = None
+        L.dashkv_workspace_size.argtypes = [P, ctypes.c_int64]
+        L.dashkv_workspace_size.restype = SZ
+        L.dashkv_encode_keys.argtypes = [P, ctypes.POINTER(KVView), P, P]
+        L.dashkv_append_keys.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P]
+        L.dashkv_select.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
+        L.dashkv_sparse_decode.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
+        L.dashkv_get_error.argtypes = [P]
+        L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
+        L.dashkv_set_trace.argtypes = [P, P, I32]
+        L.dashkv_status_str.argtypes = [ctypes.c_int]
+        L.dashkv_status_str.restype = ctypes.c_char_p
+        for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode",
+                  "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(call: str, status: int) -> None:
+    if status != 0:
+        raise DashKVError(call, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def hyperplanes(seed: int, bits: int, d: int) -> torch.Tensor:
+    """The +-1 hyperplanes [bits, d] (int8, host) a context with this seed uses."""
+    out = torch.empty((bits, d), dtype=torch.int8)
+    _check("dashkv_hyperplanes", lib().dashkv_hyperplanes(seed & (2**64 - 1), bits, d, _ptr(out)))
+    return out
+
+
+@dataclasses.dataclass
+class KVCache:
+    """Device tensors of one cache.  Dense: k, v [B,Hkv,n_cap,d] bf16, codes
+    [B,Hkv,n_cap,W] int64.  Paged: k, v [P,page,Hkv,d], codes [P,Hkv,page,W],
+    page_table [B,max_pages] int32."""
+    k: torch.Tensor
+    v: torch.Tensor
+    codes: torch.Tensor
+    page_table: Optional[torch.Tensor] = None
+
+    @property
+    def paged(self) -> bool:
+        return self.page_table is not None
+
+    @property
+    def page_size(self) -> int:
+        return int(self.k.shape[1]) if self.paged else 0
+
+    @property
+    def capacity(self) -> int:
+        return int(self.page_table.shape[1]) * self.page_size if self.paged else int(self.k.shape[2])
+
+    def view(self) -> KVView:
+        if self.paged:
+            return KVView(self.k.data_ptr(), self.v.data_ptr(), self.codes.data_ptr(), 0,
+                          self.page_table.data_ptr(), int(self.page_table.shape[1]), int(self.k.shape[0]))
+        return KVView(self.k.data_ptr(), self.v.data_ptr(), self.codes.data_ptr(), int(self.k.shape[2]),
+                      None, 0, 0)
+
+    @staticmethod
+    def empty_codes_like(k: torch.Tensor, bits: int, paged: bool) -> torch.Tensor:
+        W = max(1, bits // 64)
+        if paged:
+            P, ps, Hkv, _ = k.shape
+            return torch.zeros((P, Hkv, ps, W), dtype=torch.int64, device=k.device)
+        B, Hkv, n_cap, _ = k.shape
+        return torch.zeros((B, Hkv, n_cap, W), dtype=torch.int64, device=k.device)
+
+
+class DashKV:
+    """One problem configuration (shapes, bits, k, S, W, layout, seed)."""
+
+    def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, bits: int, topk: int,
+                 sink: int, window: int, page_size: int = 0, seed: int = 0x5EEDDA5B):
+        if not torch.cuda.is_available():
+            raise RuntimeError("hash_indexed_top_b200 needs a CUDA device (B200, sm_100a)")
+        self.cfg = Config(batch, num_q_heads, num_kv_heads, head_dim, bits, topk, sink, window, page_size, 0,
+                          seed & (2**64 - 1))
+        self.sel_cap = topk + sink + window
+        h = ctypes.c_void_p()
+        _check("dashkv_create", lib().dashkv_create(ctypes.byref(self.cfg), ctypes.byref(h)))
+        self._ctx = h
+        self._ws = None
+
+    def close(self) -> None:
+        if self._ctx:
+            lib().dashkv_destroy(self._ctx)
+            self._ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---- workspace
+    def workspace_size(self, max_tokens: int) -> int:
+        return int(lib().dashkv_workspace_size(self._ctx, int(max_tokens)))
+
+    def workspace(self, max_tokens: int, device=None) -> torch.Tensor:
+        """A zero-filled workspace (kept and reused while it is large enough)."""
+        need = self.workspace_size(max_tokens)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(need, dtype=torch.uint8, device=device or torch.cuda.current_device())
+        return self._ws
+
+    # ---- the four calls
+    def encode_keys(self, cache: KVCache, seq_lens: torch.Tensor, stream=None) -> None:
+        v = cache.view()
+        _check("dashkv_encode_keys", lib().dashkv_encode_keys(self._ctx, ctypes.byref(v), _ptr(seq_lens),
+                                                              _stream(stream)))
+
+    def append_keys(self, cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor, seq_lens: torch.Tensor,
+                    stream=None) -> None:
+        v = cache.view()
+        _check("dashkv_append_keys", lib().dashkv_append_keys(self._ctx, ctypes.byref(v), _ptr(k_new),
+                                                              _ptr(v_new), _ptr(seq_lens), _stream(stream)))
+
+    def select(self, cache: KVCache, q: torch.Tensor, seq_lens: torch.Tensor, sel_idx: torch.Tensor,
+               sel_cnt: torch.Tensor, scores: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+        ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
+        v = cache.view()
+        _check("dashkv_select", lib().dashkv_select(self._ctx, ctypes.byref(v), _ptr(q), _ptr(seq_lens),
+                                                    _ptr(sel_idx), _ptr(sel_cnt), _ptr(scores), _ptr(ws),
+                                                    ws.numel(), _stream(stream)))
+
+    def sparse_decode(self, cache: KVCache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
+                      out: torch.Tensor, lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+        ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
+        v = cache.view()
+        _check("dashkv_sparse_decode", lib().dashkv_sparse_decode(self._ctx, ctypes.byref(v), _ptr(q),
+                                                                  _ptr(sel_idx), _ptr(sel_cnt), _ptr(out),
+                                                                  _ptr(lse), _ptr(ws), ws.numel(),
+                                                                  _stream(stream)))
+
+    def set_trace(self, events: Optional[list] = None) -> None:
+        """Record torch.cuda.Event pairs around each kernel of the following calls (None: off)."""
+        if events is None:
+            self._trace = None
+            _check("dashkv_set_trace", lib().dashkv_set_trace(self._ctx, None, 0))
+            return
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        self._trace = arr  # keep alive while tracing
+        _check("dashkv_set_trace", lib().dashkv_set_trace(self._ctx, arr, len(events)))
+
+    def get_error(self, stream=None) -> int:
+        """Synchronise the stream; return (and clear) the device error status."""
+        return int(lib().dashkv_get_error(_stream(stream)))
+
+    # ---- convenience: output buffers for one step
+    def alloc_step(self, device) -> dict:
+        B, Hq, Hkv, d = self.cfg.batch, self.cfg.num_q_heads, self.cfg.num_kv_heads, self.cfg.head_dim
+        return dict(sel_idx=torch.empty((B, Hkv, self.sel_cap), dtype=torch.int32, device=device),
+                    sel_cnt=torch.empty((B, Hkv), dtype=torch.int32, device=device),
+                    out=torch.empty((B, Hq, d), dtype=torch.float32, device=device),
+                    lse=torch.empty((B, Hq), dtype=torch.float32, device=device))

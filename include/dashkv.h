@@ -1,0 +1,183 @@
+/*
+ * dashkv.h -- C ABI of the decode-step hash-score -> top-k -> exact sparse
+ * attention library for NVIDIA B200 (sm_100a).
+ *
+ * One decode step over a long KV cache runs in four stages:
+ *
+ *   1. hash_encode  every cached key k (head dim d) becomes `bits` sign bits
+ *                   against seeded Rademacher (+1/-1) hyperplanes R:
+ *                   bit_j = [ sum_i R[j][i] k[i] >= 0 ]  (a tie at 0 gives 1).
+ *                   DASH-KV page, section "从平方到线性：复杂度降低的数学原理"
+ *                   (locality-sensitive hashing of the keys) and section
+ *                   "技术架构：动态混合精度机制" (a light key-side encoder).
+ *   2. asym_score   the query stays in full precision; it is projected onto
+ *                   the same hyperplanes and scored against the packed key
+ *                   codes, s_t = sum_j qp_j (2 bit_tj - 1); with grouped
+ *                   query attention the scores of the query heads that share
+ *                   a KV head are summed.  DASH-KV page, section
+ *                   "DASH-KV的核心创新：非对称深度哈希" (asymmetric encoding);
+ *                   Spherical KV page, section 2.1 ADA (logits straight from
+ *                   compact codes, no dense key is rebuilt).
+ *   3. select       the top-k scores per (sequence, KV head), ties to the
+ *                   lower index, united with the first S (sink) and last W
+ *                   (window) tokens.  DeepSeek DSA->CSA/HCA page, section
+ *                   "从 DSA 说起" (indexer then top-k) and the SWA paragraph
+ *                   of its CSA section; DySCO page, Q3 (attention sinks).
+ *   4. attention    softmax(q K^T / sqrt(d)) V over the selected tokens only,
+ *                   fp32 accumulation, one output per query head.
+ *                   DeepSeek DSA->CSA/HCA page, section "从 DSA 说起"
+ *                   (real attention on the top-k only).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers marked "device" are CUDA device pointers; the caller owns and
+ *    allocates every buffer.  The library allocates no device memory.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and never synchronises the host, except
+ *    dashkv_get_error().
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns a status and launches nothing.  Problems only the
+ *    device can see (a page id outside [0, num_pages), a sequence length
+ *    beyond the cache capacity) set a per-device error word that
+ *    dashkv_get_error() reads and clears; the affected tokens are skipped.
+ *  - Layouts (B sequences, Hkv KV heads, Hq = G * Hkv query heads,
+ *    W = max(1, bits / 64) 64-bit code words per key):
+ *      keys / values, dense : bf16 [B][Hkv][n_cap][d]
+ *      keys / values, paged : bf16 [num_pages][page_size][Hkv][d]
+ *      codes, dense         : u64  [B][Hkv][n_cap][W]
+ *      codes, paged         : u64  [num_pages][Hkv][page_size][W]
+ *      token t of sequence b lives in physical page
+ *      page_table[b * max_pages + t / page_size], slot t % page_size.
+ *      Hyperplane j's bit sits in code word j / 64 at bit position j % 64;
+ *      a 32-bit code occupies the low half of its word (high half zero).
+ *      queries q : bf16 [B][Hq][d]; query head h reads KV head h / G.
+ *  - seq_lens (device int32 [B]) holds each sequence's cached length; the
+ *    current decode step's own key is expected to be appended first, so the
+ *    recent window includes it.
+ */
+#ifndef DASHKV_H
+#define DASHKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dashkv_status {
+    DASHKV_OK = 0,
+    DASHKV_ERR_INVALID_ARG = 1,  /* null pointer, bad shape or size                  */
+    DASHKV_ERR_UNSUPPORTED = 2,  /* d, bits, G or page_size outside the supported set */
+    DASHKV_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required       */
+    DASHKV_ERR_CAPACITY = 4,     /* device error word: a sequence outgrew its cache   */
+    DASHKV_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, sync, copy)   */
+    DASHKV_ERR_DEVICE = 6,       /* device error word: bad page id in page_table      */
+    DASHKV_ERR_NO_DEVICE = 7     /* no usable CUDA device                             */
+} dashkv_status;
+
+/* Problem description.  Supported: head_dim in {64, 128}; bits in
+ * {32, 64, 128}; num_q_heads = G * num_kv_heads with G in {1, 2, 4, 8};
+ * topk >= 1; sink, window >= 0; page_size 0 (dense) or a multiple of 32 up
+ * to 1024. */
+typedef struct dashkv_config {
+    int32_t batch;          /* B  */
+    int32_t num_q_heads;    /* Hq */
+    int32_t num_kv_heads;   /* Hkv */
+    int32_t head_dim;       /* d  */
+    int32_t bits;           /* hash bits per key (b) */
+    int32_t topk;           /* k  */
+    int32_t sink;           /* S: first tokens always kept */
+    int32_t window;         /* W: last tokens always kept  */
+    int32_t page_size;      /* 0 = dense layout            */
+    int32_t reserved;       /* must be 0 */
+    uint64_t seed;          /* hyperplane seed             */
+} dashkv_config;
+
+/* The KV cache the calls read (and dashkv_append_keys writes). */
+typedef struct dashkv_kv_view {
+    void *k;                      /* device bf16 keys   (layout above)               */
+    void *v;                      /* device bf16 values (layout above)               */
+    uint64_t *codes;              /* device key codes   (layout above)               */
+    int64_t n_cap;                /* dense: token capacity per (b, kv head)          */
+    const int32_t *page_table;    /* device [B][max_pages]; NULL = dense layout      */
+    int32_t max_pages;            /* paged: row length of page_table                 */
+    int32_t num_pages;            /* paged: physical pages held by k, v and codes    */
+} dashkv_kv_view;
+
+typedef struct dashkv_ctx dashkv_ctx;
+
+/* Validate `cfg` and build a context holding it and the hyperplanes R
+ * (host memory only; R[j][i] is -1 when the top bit of splitmix64 output
+ * number j*d+i+1 from `seed` is set, else +1).  *out receives the context;
+ * release it with dashkv_destroy().  Binds to the CUDA device current at
+ * this call (queried for its SM count). */
+dashkv_status dashkv_create(const dashkv_config *cfg, dashkv_ctx **out);
+void dashkv_destroy(dashkv_ctx *ctx);
+
+/* Bytes of device workspace dashkv_select / dashkv_sparse_decode need for
+ * caches of at most `max_tokens` tokens per sequence (dense: n_cap; paged:
+ * max_pages * page_size).  The workspace must be zero-filled once before its
+ * first use; every call that returns DASHKV_OK leaves it ready for the next
+ * one.  Select and decode may share one workspace; calls that use the same
+ * workspace must not overlap on the GPU. */
+size_t dashkv_workspace_size(const dashkv_ctx *ctx, int64_t max_tokens);
+
+/* Stage 1 for a whole cache: write the codes of tokens [0, seq_lens[b]) of
+ * every (b, kv head) into kv->codes.  Reads kv->k.  seq_lens: device int32 [B]. */
+dashkv_status dashkv_encode_keys(dashkv_ctx *ctx, const dashkv_kv_view *kv,
+                                 const int32_t *seq_lens, void *stream);
+
+/* One decode step's cache append: k_new / v_new (device bf16 [B][Hkv][d])
+ * are written at position seq_lens[b] of every (b, kv head), their codes
+ * into kv->codes, then seq_lens[b] is incremented on the device. */
+dashkv_status dashkv_append_keys(dashkv_ctx *ctx, const dashkv_kv_view *kv,
+                                 const void *k_new, const void *v_new,
+                                 int32_t *seq_lens, void *stream);
+
+/* Stages 2 and 3.  q: device bf16 [B][Hq][d].  Writes, per (b, kv head),
+ * the ascending, duplicate-free selected token ids into
+ * sel_idx (device int32 [B][Hkv][topk + sink + window], unused tail = -1)
+ * and their number into sel_cnt (device int32 [B][Hkv]).
+ * scores (optional, may be NULL): device fp32 [B][Hkv][max_tokens]
+ * receives s_t for t < seq_lens[b] (other entries untouched).
+ * Reads kv->codes (and kv->page_table), never kv->k / kv->v. */
+dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
+                            const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
+                            float *scores, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* Stage 4.  Exact softmax attention of every query head over the rows its
+ * KV head selected: out (device fp32 [B][Hq][d]); lse (optional, device
+ * fp32 [B][Hq]) receives log sum_t exp(q.K_t / sqrt(d)) (-inf when nothing
+ * is selected, out = 0 then).  sel_idx / sel_cnt as dashkv_select writes
+ * them; ids must be < seq_lens[b]. */
+dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
+                                   const int32_t *sel_idx, const int32_t *sel_cnt,
+                                   float *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
+/* Synchronise `stream`, then read and clear the current device's error
+ * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, or
+ * DASHKV_ERR_CUDA when the stream reports an error. */
+dashkv_status dashkv_get_error(void *stream);
+
+/* The hyperplanes a context built with (seed, bits, d) uses, as int8 +1/-1
+ * in host memory [bits][d]. */
+dashkv_status dashkv_hyperplanes(uint64_t seed, int32_t bits, int32_t head_dim, int8_t *host_out);
+
+/* Optional kernel tracing for profiling.  While `events` is non-NULL, every
+ * following call on this context records events[2k] (a cudaEvent_t) on its
+ * stream right before the k-th kernel it launches and events[2k + 1] right
+ * after it (k counts from 0 within each call; kernels beyond n_events / 2 are
+ * not traced).  The array must stay valid until tracing is turned off with
+ * events = NULL.  The caller owns the events. */
+dashkv_status dashkv_set_trace(dashkv_ctx *ctx, void **events, int32_t n_events);
+
+/* Static string naming a status. */
+const char *dashkv_status_str(dashkv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DASHKV_H */

@@ -1,0 +1,128 @@
+"""Test harness: run the same seeded workload through the CUDA library (via
+its C ABI binding) and through the CPU oracle, and compare.
+
+Bars: codes, scores and selected indices bit-identical; attention outputs and
+log-sum-exp within |err| <= 1e-3 + 8e-3 |ref| per element.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from hash_indexed_top_b200 import dashkv as dk
+from hash_indexed_top_b200 import workloads as W
+from oracle import oracle as O
+
+ATOL, RTOL = 1e-3, 8e-3
+
+
+class GpuRun:
+    def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED):
+        self.cfg, self.w = cfg, w
+        dev = w.K.device
+        self.eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
+                             cfg.page_size if w.paged else 0, seed)
+        codes = dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged)
+        self.cache = dk.KVCache(w.K, w.V, codes, w.page_table)
+        self.seq = w.seq_lens.clone()
+        self.buf = self.eng.alloc_step(dev)
+        self.scores = torch.full((cfg.B, cfg.Hkv, self.cache.capacity), float("nan"), device=dev)
+
+    def encode(self):
+        self.eng.encode_keys(self.cache, self.seq)
+
+    def append(self, s: int):
+        self.eng.append_keys(self.cache, self.w.k_new[s], self.w.v_new[s], self.seq)
+
+    def select_decode(self, q: torch.Tensor):
+        b = self.buf
+        self.eng.select(self.cache, q, self.seq, b["sel_idx"], b["sel_cnt"], self.scores)
+        self.eng.sparse_decode(self.cache, q, b["sel_idx"], b["sel_cnt"], b["out"], b["lse"])
+
+    def error(self) -> int:
+        return self.eng.get_error()
+
+    def close(self):
+        self.eng.close()
+
+
+class OracleRun:
+    """Oracle state over the full cache (small workloads)."""
+
+    def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED):
+        self.cfg = cfg
+        self.R = O.hyperplanes(seed, cfg.bits, cfg.d)
+        if w.paged:
+            self.L = O.Layout(cfg.B, cfg.Hkv, cfg.d, cfg.bits, page_table=w.page_table.cpu().numpy(),
+                              page=cfg.page_size)
+        else:
+            self.L = O.Layout(cfg.B, cfg.Hkv, cfg.d, cfg.bits, n_cap=w.n_cap)
+        self.K = w.K.cpu().double().numpy().copy()
+        self.V = w.V.cpu().double().numpy().copy()
+        self.seq = w.seq_lens.cpu().numpy().astype(np.int32).copy()
+        self.codes = O.encode(self.L, self.K, self.seq, self.R)
+        self.w = w
+
+    def append(self, s: int):
+        O.append(self.L, self.K, self.V, self.codes, self.seq, self.w.k_new[s].cpu().double().numpy(),
+                 self.w.v_new[s].cpu().double().numpy(), self.R)
+
+    def step(self, q: torch.Tensor) -> dict:
+        return O.decode_step(self.L, self.cfg.Hq, q.cpu().double().numpy(), self.K, self.V, self.codes,
+                             self.seq, self.R, self.cfg.topk, self.cfg.sink, self.cfg.window)
+
+
+def within_tol(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    both_inf = np.isneginf(got) & np.isneginf(ref)
+    err = np.abs(got - ref)
+    return both_inf | (err <= ATOL + RTOL * np.abs(ref))
+
+
+def compare_step(g: GpuRun, o: OracleRun, r: dict, what: str = "") -> dict:
+    """Assert parity of one step; returns a few diagnostics."""
+    gc = g.cache.codes.cpu().numpy().view(np.uint64)
+    assert np.array_equal(gc, o.codes), f"{what}: codes differ at {np.argwhere(gc != o.codes)[:5].tolist()}"
+    assert np.array_equal(g.seq.cpu().numpy(), o.seq), f"{what}: seq_lens differ"
+    gs = g.scores.cpu().numpy()
+    os_ = r["scores"].astype(np.float32)
+    for b in range(o.cfg.B):
+        n = int(o.seq[b])
+        a, e = gs[b, :, :n], os_[b, :, :n]
+        assert np.array_equal(a.view(np.uint32), e.view(np.uint32)), \
+            f"{what}: scores differ (b={b}) at {np.argwhere(a != e)[:5].tolist()}"
+    gi = g.buf["sel_idx"].cpu().numpy()
+    gn = g.buf["sel_cnt"].cpu().numpy()
+    assert np.array_equal(gn, r["sel_cnt"]), f"{what}: sel_cnt {gn.ravel()[:8]} vs {r['sel_cnt'].ravel()[:8]}"
+    assert np.array_equal(gi, r["sel_idx"]), f"{what}: sel_idx differ"
+    out = g.buf["out"].cpu().double().numpy()
+    lse = g.buf["lse"].cpu().double().numpy()
+    ok = within_tol(out, r["out"])
+    assert ok.all(), f"{what}: out max err {np.nanmax(np.abs(out - r['out'])):.3e}"
+    okl = within_tol(lse, r["lse"])
+    assert okl.all(), f"{what}: lse max err {np.nanmax(np.abs(lse - r['lse'])):.3e}"
+    fin = np.isfinite(r["out"])
+    return dict(max_err=float(np.abs(out - r["out"])[fin].max()) if fin.any() else 0.0)
+
+
+def run_parity(cfg: W.Config, steps: int, device="cuda", w: W.Workload | None = None, mutate=None) -> list:
+    """Encode, then `steps` x (append, select, decode) on GPU and oracle, comparing every step."""
+    if w is None:
+        w = W.make_workload(cfg, device="cpu", steps=steps)
+    if mutate is not None:
+        w = mutate(w)
+    g = GpuRun(cfg, w.to(device))
+    o = OracleRun(cfg, w)
+    g.encode()
+    diags = []
+    try:
+        for s in range(steps):
+            g.append(s)
+            o.append(s)
+            q = w.q[s]
+            g.select_decode(q.to(device))
+            r = o.step(q)
+            assert g.error() == 0
+            diags.append(compare_step(g, o, r, f"{cfg.name} step {s}"))
+    finally:
+        g.close()
+    return diags

@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point its header declares, validates configurations before it
+touches a device, and its hyperplane generator agrees with the oracle's
+independently written one."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+from hash_indexed_top_b200 import build as B
+from hash_indexed_top_b200 import dashkv as dk
+from oracle import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "dashkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dashkv_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_calls():
+    fns = header_functions()
+    for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode"):
+        assert f in fns
+
+
+def test_library_exports_every_declared_symbol():
+    fns = header_functions()
+    assert set(fns) == set(dk.SYMBOLS)
+    L = dk.lib()
+    for f in fns:
+        assert getattr(L, f) is not None
+    out = subprocess.run(["nm", "-D", "--defined-only", dk.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(dashkv_\w+)", out))
+    assert set(fns) <= exported
+
+
+def test_status_strings():
+    L = dk.lib()
+    for code, text in dk.STATUS.items():
+        assert L.dashkv_status_str(code).decode() == text
+
+
+@pytest.mark.parametrize("seed,bits,d", [(0x5EEDDA5B, 128, 128), (1, 64, 128), (7, 32, 64), (2**63 + 5, 128, 64)])
+def test_library_hyperplanes_match_oracle(seed, bits, d):
+    a = dk.hyperplanes(seed, bits, d).numpy()
+    b = O.hyperplanes(seed, bits, d)
+    assert np.array_equal(a, b)
+
+
+def _cfg(**kw):
+    base = dict(batch=1, num_q_heads=4, num_kv_heads=1, head_dim=64, bits=32, topk=8, sink=0, window=0,
+                page_size=0, reserved=0, seed=1)
+    base.update(kw)
+    return dk.Config(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=96), 2), (dict(bits=48), 2), (dict(bits=256), 2), (dict(num_q_heads=12, num_kv_heads=1), 2),
+    (dict(num_q_heads=6, num_kv_heads=4), 1), (dict(topk=0), 1), (dict(sink=-1), 1), (dict(page_size=48), 2),
+    (dict(batch=0), 1), (dict(reserved=3), 1), (dict(num_q_heads=64, num_kv_heads=64), 2),
+])
+def test_create_rejects_bad_configs(kw, status):
+    h = ctypes.c_void_p()
+    cfg = _cfg(**kw)
+    assert dk.lib().dashkv_create(ctypes.byref(cfg), ctypes.byref(h)) == status
+    assert not h.value
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="host without a GPU only")
+def test_create_without_device_reports_no_device():
+    h = ctypes.c_void_p()
+    cfg = _cfg()
+    assert dk.lib().dashkv_create(ctypes.byref(cfg), ctypes.byref(h)) == 7
+    with pytest.raises(RuntimeError):
+        dk.DashKV(1, 4, 1, 64, 32, 8, 0, 0)
