@@ -64,7 +64,7 @@ class ClockSampler:
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -192,7 +192,10 @@ def run_dashkv(args, cfg, world, rank, local):
     build.build()
     dev = torch.device("cuda", local)
     total = args.warmup + args.steps + args.e2e_steps
-    w = W.make_workload(cfg, device=dev, steps=total)
+    # capacity also covers the extra replays of the timed graphs that keep the
+    # clock sampler busy (each replay appends one token per sequence)
+    w = W.make_workload(cfg, device=dev, steps=total + args.trace_steps,
+                        extra_cap=args.steps * args.clock_reps)
     eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
                     cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED)
     codes = dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged)
@@ -206,47 +209,77 @@ def run_dashkv(args, cfg, world, rank, local):
     torch.cuda.synchronize(dev)
     assert eng.get_error() == 0
 
-    def step(s):
-        eng.append_keys(cache, w.k_new[s], w.v_new[s], seq)
-        eng.select(cache, w.q[s], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
-        eng.sparse_decode(cache, w.q[s], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+    # One CUDA graph per step (append -> select -> decode on that step's inputs);
+    # capture runs nothing.  The timed graphs carry no trace events (an event
+    # between two kernels would stop the next one from launching early); a
+    # second set with trace events around every kernel gives the per-kernel
+    # durations, replayed right after the timed steps.
+    K = args.steps
+    T = min(K, args.trace_steps)
+    n_graph = args.warmup + K + T
+
+    def capture(s, e=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if e is not None:
+                eng.set_trace(e[2:4])
+            eng.append_keys(cache, w.k_new[s], w.v_new[s], seq)
+            if e is not None:
+                eng.set_trace(e[4:8])
+            eng.select(cache, w.q[s], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            if e is not None:
+                eng.set_trace(e[8:10])
+            eng.sparse_decode(cache, w.q[s], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+            if e is not None:
+                eng.set_trace(None)
+        return g
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(n_graph)]
+    for e in ev:  # materialise the CUDA events (torch creates them on first record)
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize(dev)
+    graphs = [capture(s) for s in range(args.warmup + K)]
+    traced = [capture(args.warmup + K + i, ev[args.warmup + K + i]) for i in range(T)]
 
     for s in range(args.warmup):
         flush.fill_(s)
-        step(s)
+        graphs[s].replay()
     torch.cuda.synchronize(dev)
+    assert eng.get_error() == 0
 
-    # ---- device-timed steps (+ per-kernel trace events)
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(K)]
+    # ---- device-timed steps
     n_before = seq.clone()
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
         wall0 = time.perf_counter()
-        for i in range(K):
-            flush.fill_(i)
-            e = ev[i]
-            e[0].record(stream)
-            eng.set_trace(e[2:4])
-            eng.append_keys(cache, w.k_new[args.warmup + i], w.v_new[args.warmup + i], seq)
-            eng.set_trace(e[4:8])
-            eng.select(cache, w.q[args.warmup + i], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
-            eng.set_trace(e[8:10])
-            eng.sparse_decode(cache, w.q[args.warmup + i], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
-            eng.set_trace(None)
-            e[1].record(stream)
-        torch.cuda.synchronize(dev)
-        wall = time.perf_counter() - wall0
+        for rep in range(args.clock_reps):
+            for i in range(K):
+                s = args.warmup + i
+                flush.fill_(i)
+                ev[s][0].record(stream)
+                graphs[s].replay()
+                ev[s][1].record(stream)
+            torch.cuda.synchronize(dev)
+            if rep == 0:
+                step_ms = [ev[args.warmup + i][0].elapsed_time(ev[args.warmup + i][1]) for i in range(K)]
+                wall = time.perf_counter() - wall0
+                # traced replays: per-kernel durations on the same workload
+                for i in range(T):
+                    flush.fill_(i)
+                    traced[i].replay()
+                torch.cuda.synchronize(dev)
+                tb = args.warmup + K
+                kern = {
+                    "append_keys": [ev[tb + i][2].elapsed_time(ev[tb + i][3]) for i in range(T)],
+                    "score_hist": [ev[tb + i][4].elapsed_time(ev[tb + i][5]) for i in range(T)],
+                    "collect_select": [ev[tb + i][6].elapsed_time(ev[tb + i][7]) for i in range(T)],
+                    "sparse_decode": [ev[tb + i][8].elapsed_time(ev[tb + i][9]) for i in range(T)],
+                }
     barrier(world)
     assert eng.get_error() == 0
-    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    kern = {
-        "append_keys": [e[2].elapsed_time(e[3]) for e in ev],
-        "score_hist": [e[4].elapsed_time(e[5]) for e in ev],
-        "collect_select": [e[6].elapsed_time(e[7]) for e in ev],
-        "sparse_decode": [e[8].elapsed_time(e[9]) for e in ev],
-    }
+    del graphs, traced
     sum_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = sum_ms / K
     value = world * cfg.B * K / (sum_ms / 1e3)
@@ -279,7 +312,7 @@ def run_dashkv(args, cfg, world, rank, local):
         eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(E)]
         barrier(world)
         for i in range(E):
-            s = args.warmup + K + i
+            s = args.warmup + K + T + i
             flush.fill_(i)
             eev[i][0].record(stream)
             dq.copy_(hq[s], non_blocking=True)
@@ -328,6 +361,7 @@ def run_dashkv(args, cfg, world, rank, local):
             "codes_scanned_per_s": float(lens_mid.sum()) * cfg.Hkv / (ms_per_step * 1e-3),
             "selected_kv_bytes_per_s": kv_bytes / (ms_per_step * 1e-3),
             "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 4 * K, "clocks": clk,
+            "timing": "one CUDA graph per step (append, select, decode; programmatic dependent launches); events around each replay; kernels_ms from separately traced replays",
             "wall_s_timed_region": wall,
         }
         print(json.dumps(line), flush=True)
@@ -343,6 +377,10 @@ def main():
     ap.add_argument("--config", default="c128k", choices=sorted(W.CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-steps", type=int, default=2)
+    ap.add_argument("--trace-steps", type=int, default=10,
+                    help="extra traced steps for the per-kernel durations")
+    ap.add_argument("--clock-reps", type=int, default=20,
+                    help="replays of the timed steps while clocks are sampled (only the first is reported)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

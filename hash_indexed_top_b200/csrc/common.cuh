@@ -79,6 +79,13 @@ __device__ __forceinline__ int64_t clamp_len(const KV &kv, const int32_t *seq_le
     return n < 0 ? 0 : n;
 }
 
+// Programmatic dependent launch.  wait(): block until the preceding kernel of
+// the stream has completed and its writes are visible (a no-op when this kernel
+// was launched without the programmatic-serialization attribute).  trigger():
+// allow the following kernel to be scheduled early (it still waits in wait()).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 

@@ -7,6 +7,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <type_traits>
+
 #include "../../include/dashkv.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -31,11 +33,15 @@ struct Tracer {
     cudaStream_t st;
     int k = 0;
     Tracer(const dashkv_ctx *c, cudaStream_t s) : ctx(c), st(s) {}
+    // External records: under stream capture they become event-record nodes of
+    // the graph (timeable on every replay) rather than capture dependencies.
     void before() {
-        if (ctx->trace && 2 * k + 1 < ctx->n_trace) cudaEventRecord((cudaEvent_t)ctx->trace[2 * k], st);
+        if (ctx->trace && 2 * k + 1 < ctx->n_trace)
+            cudaEventRecordWithFlags((cudaEvent_t)ctx->trace[2 * k], st, cudaEventRecordExternal);
     }
     void after() {
-        if (ctx->trace && 2 * k + 1 < ctx->n_trace) cudaEventRecord((cudaEvent_t)ctx->trace[2 * k + 1], st);
+        if (ctx->trace && 2 * k + 1 < ctx->n_trace)
+            cudaEventRecordWithFlags((cudaEvent_t)ctx->trace[2 * k + 1], st, cudaEventRecordExternal);
         ++k;
     }
 };
@@ -119,13 +125,17 @@ struct WsLayout {
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Internal score / candidate rows are padded to a multiple of 64 tokens.
+int64_t row_ld(int64_t max_tokens) { return (max_tokens + 63) / 64 * 64; }
+
 WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
     const size_t BH = (size_t)c.batch * c.num_kv_heads;
     const size_t G = (size_t)(c.num_q_heads / c.num_kv_heads);
+    const size_t ld = (size_t)row_ld(max_tokens);
     WsLayout L;
     size_t o = 0;
-    L.scores = o;  o = align_up(o + BH * (size_t)max_tokens * 4);
-    L.cand = o;    o = align_up(o + BH * (size_t)max_tokens * 4);
+    L.scores = o;  o = align_up(o + BH * ld * 4);
+    L.cand = o;    o = align_up(o + BH * ld * 4);
     L.hist = o;    o = align_up(o + BH * kBins * 4);
     L.state = o;   o = align_up(o + BH * sizeof(SelState));
     L.arrive = o;  o = align_up(o + 3 * BH * 4);
@@ -135,13 +145,31 @@ WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
     return L;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while its predecessor drains; it synchronises itself with griddep_wait().
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 dashkv_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? DASHKV_OK : DASHKV_ERR_CUDA;
 }
 
-int sel_ctas(const dashkv_ctx *ctx, int64_t cap) {
+// CTAs per (b, kv head) for a kernel with `per_sm` resident CTAs per SM.
+int sel_ctas(const dashkv_ctx *ctx, int64_t cap, int per_sm) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
-    int n = (2 * ctx->sm_count) / BH;
+    int n = (per_sm * ctx->sm_count) / BH;
     if (n < 1) n = 1;
     const int64_t by_tokens = ceil_div(cap, 1024);
     if (n > by_tokens) n = (int)by_tokens;
@@ -152,8 +180,8 @@ int sel_ctas(const dashkv_ctx *ctx, int64_t cap) {
 int attn_splits(const dashkv_ctx *ctx) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int64_t cap_sel = (int64_t)ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
-    int64_t n = ceil_div(4 * ctx->sm_count, BH);
-    const int64_t by_rows = ceil_div(cap_sel, 128);
+    int64_t n = (2 * ctx->sm_count) / BH;  // one wave of two CTAs per SM
+    const int64_t by_rows = ceil_div(cap_sel, 64);
     if (n > by_rows) n = by_rows;
     if (n > kMaxSplits) n = kMaxSplits;
     return n < 1 ? 1 : (int)n;
@@ -168,7 +196,16 @@ void set_attrs_bd() {
                          (int)ScoreShape<BITS>::SMEM);
 }
 
+template <int D, int G>
+void set_attr_decode() {
+    cudaFuncSetAttribute(sparse_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)DecodeShape<D, G>::SMEM);
+}
+
 void set_attrs() {
+    set_attr_decode<64, 1>();  set_attr_decode<64, 2>();  set_attr_decode<64, 4>();  set_attr_decode<64, 8>();
+    set_attr_decode<128, 1>(); set_attr_decode<128, 2>(); set_attr_decode<128, 4>(); set_attr_decode<128, 8>();
+    cudaFuncSetAttribute(collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(CollectSmem));
     set_attrs_bd<32, 64>();  set_attrs_bd<32, 128>();
     set_attrs_bd<64, 64>();  set_attrs_bd<64, 128>();
     set_attrs_bd<128, 64>(); set_attrs_bd<128, 128>();
@@ -197,8 +234,10 @@ void launch_encode_d(const dashkv_ctx *ctx, const KV &kv, const int32_t *s, cuda
 template <int BITS, int D>
 void launch_append_bd(const dashkv_ctx *ctx, const KV &kv, const void *kn, const void *vn, int32_t *seq,
                       cudaStream_t st) {
-    append_keys_kernel<BITS, D><<<ctx->cfg.batch, 32 * ctx->cfg.num_kv_heads, 0, st>>>(
-        kv, static_cast<const __nv_bfloat16 *>(kn), static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R);
+    int threads = ctx->cfg.num_kv_heads * BITS;
+    if (threads > kAppendThreads) threads = kAppendThreads;
+    launch_pdl(append_keys_kernel<BITS, D>, dim3(ctx->cfg.batch), dim3(threads), 0, st, kv,
+               static_cast<const __nv_bfloat16 *>(kn), static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R);
 }
 
 template <int D>
@@ -216,8 +255,8 @@ void launch_score_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
                      int nctas, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
-    score_hist_kernel<BITS, D><<<dim3(nctas, BH), kSelThreads, ScoreShape<BITS>::SMEM, st>>>(
-        kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, ctx->cfg.topk, nctas);
+    launch_pdl(score_hist_kernel<BITS, D>, dim3(nctas, BH), dim3(kScoreThreads), ScoreShape<BITS>::SMEM, st, kv,
+               static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, ctx->cfg.topk, nctas);
 }
 
 template <int D>
@@ -237,9 +276,9 @@ void launch_decode_dg(const dashkv_ctx *ctx, const KV &kv, const void *q, const 
     const int splits = attn_splits(ctx);
     const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    sparse_decode_kernel<D, G><<<dim3(splits, BH), kAttnThreads, 0, st>>>(
-        kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws, splits,
-        scale_log2);
+    launch_pdl(sparse_decode_kernel<D, G>, dim3(splits, BH), dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st, kv,
+               static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws, splits,
+               scale_log2);
 }
 
 template <int D>
@@ -357,8 +396,10 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     char *w = static_cast<char *>(workspace);
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     SelWS ws;
-    ws.scores = scores ? scores : reinterpret_cast<float *>(w + L.scores);
-    ws.ld = cap;
+    ws.scores = reinterpret_cast<float *>(w + L.scores);
+    ws.ld = row_ld(cap);
+    ws.scores_out = scores;
+    ws.ld_out = cap;
     ws.cand = reinterpret_cast<int32_t *>(w + L.cand);
     ws.hist = reinterpret_cast<uint32_t *>(w + L.hist);
     ws.state = reinterpret_cast<SelState *>(w + L.state);
@@ -366,16 +407,17 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
     const KV k = make_kv(ctx, kv);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int nctas = sel_ctas(ctx, cap);
+    const int nscore = sel_ctas(ctx, cap, 1);    // score kernel: one 1024-thread CTA per SM
+    const int ncollect = sel_ctas(ctx, cap, 2);  // collect kernel: two 512-thread CTAs per SM
     Tracer tr(ctx, st);
     tr.before();
-    if (ctx->cfg.head_dim == 64) launch_score_d<64>(ctx, k, q, seq_lens, ws, nctas, st);
-    else launch_score_d<128>(ctx, k, q, seq_lens, ws, nctas, st);
+    if (ctx->cfg.head_dim == 64) launch_score_d<64>(ctx, k, q, seq_lens, ws, nscore, st);
+    else launch_score_d<128>(ctx, k, q, seq_lens, ws, nscore, st);
     tr.after();
     const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     tr.before();
-    collect_kernel<<<dim3(nctas, BH), kSelThreads, 0, st>>>(seq_lens, ws, nctas, ctx->cfg.sink, ctx->cfg.window,
-                                                            cap_sel, sel_idx, sel_cnt);
+    launch_pdl(collect_kernel, dim3(ncollect, BH), dim3(kSelThreads), sizeof(CollectSmem), st, ws, ncollect,
+               ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
     tr.after();
     return launch_status();
 }

@@ -4,18 +4,21 @@
 // the tokens that matter are attended in full precision).
 //
 // Gathered split-K flash-decode: grid = (splits, B * Hkv).  Each CTA takes a
-// contiguous slice of one (b, kv head)'s selected ids, gathers each K/V row
-// once (16-byte loads, LPR = d/8 lanes per row) and serves all G query heads of
-// the group from it, keeping a running (max, sum, acc) per head in fp32 with
-// base-2 exponentials.  The per-CTA partials go to the workspace; the last CTA
-// of the (b, h) (atomic arrival counter, no waiting) merges them with a
+// contiguous slice of one (b, kv head)'s selected ids.  A lane group of LPR
+// lanes owns one row at a time (DPL = d / LPR dims per lane), gathers its K and
+// V slices with 16-byte loads once, and serves all G query heads of the group
+// from them.  Rows are processed in tiles of RT per lane group: the logits of
+// the tile are formed first, then one running-max update and one rescale of
+// the accumulators per tile (fp32, base-2 exponentials).  Each CTA merges its
+// lane groups' states in shared memory and writes one partial; the last CTA of
+// the (b, h) (atomic arrival counter, no waiting) merges the partials with a
 // log-sum-exp reduction and writes out / lse.
 #pragma once
 #include "common.cuh"
 
 namespace dkv {
 
-constexpr int kAttnThreads = 128;
+constexpr int kAttnThreads = 256;
 constexpr int kMaxSplits = 256;
 
 struct AttnWS {
@@ -24,123 +27,256 @@ struct AttnWS {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(kAttnThreads)
+struct DecodeShape {
+    static constexpr int DPL = G >= 4 ? 32 / G : 16;   // dims per lane
+    static constexpr int LPR = D / DPL;                // lanes per row
+    static constexpr int RPW = 32 / LPR;               // rows per warp step
+    static constexpr int NWARP = kAttnThreads / 32;
+    static constexpr int NST = NWARP * RPW;            // lane groups (running states) per CTA
+    static constexpr int RT0 = RPW >= 8 ? 1 : 8 / RPW;
+    static constexpr int RT = RT0 * G > 32 ? 32 / G : RT0;  // rows per lane group per tile (<= 32 logits)
+    static constexpr int TROWS = RPW * RT;             // rows per warp tile
+    static constexpr int STAGES = TROWS <= 4 ? 3 : 2;  // cp.async pipeline depth per warp
+    static constexpr int CPR = D / 8;                  // 16-byte chunks per K (or V) row
+    // per warp: STAGES buffers x TROWS rows x (K, V) x D bf16
+    static constexpr size_t STAGE_BYTES = (size_t)NWARP * STAGES * TROWS * 2 * D * 2;
+    static constexpr size_t SMEM = STAGE_BYTES + (size_t)NST * G * (D + 2) * 4 + 16;
+};
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// 2^x on the SFU (approximate, flushes denormal results to zero: weights below
+// 2^-126 of the running maximum vanish, far inside the fp32 accumulation error).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kAttnThreads, 2)
 sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                      const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt, int cap_sel,
                      float *__restrict__ out, float *__restrict__ lse, AttnWS ws, int splits, float scale_log2) {
-    constexpr int LPR = D / 8;        // lanes per row (8 bf16 = 16 B each)
-    constexpr int RPW = 32 / LPR;     // rows per warp step
-    constexpr int NWARP = kAttnThreads / 32;
-    constexpr int NST = NWARP * RPW;  // independent running states per CTA
-    constexpr int U = 4;              // rows in flight per lane group
-    __shared__ float s_m[NST][G], s_l[NST][G];
-    __shared__ float s_acc[NST][G][D];
+    using S = DecodeShape<D, G>;
+    constexpr int DPL = S::DPL, LPR = S::LPR, RPW = S::RPW, NST = S::NST, RT = S::RT;
+    constexpr int TROWS = S::TROWS, CPR = S::CPR, NWARP = S::NWARP, STAGES = S::STAGES;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(smem_raw);               // [NWARP][STAGES][TROWS][2][D]
+    float *s_acc = reinterpret_cast<float *>(smem_raw + S::STAGE_BYTES);              // [NST][G][D]
+    float *s_m = s_acc + NST * G * D;                                                  // [NST][G]
+    float *s_l = s_m + NST * G;                                                        // [NST][G]
     __shared__ int s_last;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = lane / LPR, li = lane % LPR;
     const int bh = blockIdx.y, b = bh / kv.Hkv, h = bh % kv.Hkv;
     const int split = blockIdx.x;
-    int cnt = sel_cnt[bh];
-    if (cnt > cap_sel) cnt = cap_sel;
-    if (cnt < 0) cnt = 0;
     const int64_t cap_tokens = kv.capacity();
-    const int per = (cnt + splits - 1) / splits;
-    const int r0 = split * per;
-    const int r1 = r0 + per < cnt ? r0 + per : cnt;
 
-    float qf[G][8];
+    // this lane's slice of every query head of the group
+    float qf[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(q + ((int64_t)b * Hq + h * G + g) * D) + li);
-        qf[g][0] = bf16_lo(raw.x); qf[g][1] = bf16_hi(raw.x);
-        qf[g][2] = bf16_lo(raw.y); qf[g][3] = bf16_hi(raw.y);
-        qf[g][4] = bf16_lo(raw.z); qf[g][5] = bf16_hi(raw.z);
-        qf[g][6] = bf16_lo(raw.w); qf[g][7] = bf16_hi(raw.w);
+        const __nv_bfloat16 *qr = q + ((int64_t)b * Hq + h * G + g) * D + li * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; e += 2) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(qr + e);
+            qf[g][e] = bf16_lo(w);
+            qf[g][e + 1] = bf16_hi(w);
+        }
     }
-    float m[G], l[G], acc[G][8];
+    float m[G], l[G], acc[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
         l[g] = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = 0.0f;
+        for (int e = 0; e < DPL; ++e) acc[g][e] = 0.0f;
     }
 
+    // q is an input of the step; the selection comes from the preceding kernel
+    griddep_wait();
+    griddep_trigger();
+    int cnt = sel_cnt[bh];
+    if (cnt > cap_sel) cnt = cap_sel;
+    if (cnt < 0) cnt = 0;
+    const int per = (cnt + splits - 1) / splits;
+    const int r0 = split * per;
+    const int r1 = r0 + per < cnt ? r0 + per : cnt;
+
     const int32_t *ids = sel_idx + (int64_t)bh * cap_sel;
-    const int stride = NST;
-    // warp-uniform loop (the dot-product reduction shuffles across the whole warp)
-    for (int rw = r0 + warp * RPW; rw < r1; rw += stride * U) {
-        uint4 kr[U], vr[U];
-        bool ok[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int r = rw + sub + u * stride;
-            ok[u] = false;
-            kr[u] = make_uint4(0, 0, 0, 0);
-            vr[u] = make_uint4(0, 0, 0, 0);
-            if (r < r1) {
-                const int t = __ldg(ids + r);
-                int64_t off = -1;
-                if (t >= 0 && t < cap_tokens) off = kv.row(b, h, t);
-                else raise_error(kErrCapacity);
-                if (off >= 0) {
-                    ok[u] = true;
-                    kr[u] = __ldg(reinterpret_cast<const uint4 *>(kv.k + off) + li);
-                    vr[u] = __ldg(reinterpret_cast<const uint4 *>(kv.v + off) + li);
-                }
-            }
+    __nv_bfloat16 *wstage = stage + (size_t)warp * STAGES * TROWS * 2 * D;
+    // Token of row `base + lane` of a tile (lanes < TROWS), -1 when the row is
+    // outside the slice or its id lies outside the cache.
+    auto tile_token = [&](int base) -> int {
+        const int r = base + lane;
+        if (lane >= TROWS || r >= r1) return -1;
+        const int t = __ldg(ids + r);
+        if (t < 0 || t >= cap_tokens) {
+            raise_error(kErrCapacity);
+            return -1;
         }
+        if (kv.page_size && kv.page_of(b, t) < 0) return -1;
+        return t;
+    };
+    // Gather a tile's K and V rows into buffer `buf` (zero-filled when invalid);
+    // tok: this lane's tile_token() of the tile.
+    auto prefetch = [&](int tok, int buf) {
+        __nv_bfloat16 *dst0 = wstage + (size_t)buf * TROWS * 2 * D;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            // lanes of a row group share ok[u] (same row); groups differ only at the tail
-            float kf[8] = {bf16_lo(kr[u].x), bf16_hi(kr[u].x), bf16_lo(kr[u].y), bf16_hi(kr[u].y),
-                           bf16_lo(kr[u].z), bf16_hi(kr[u].z), bf16_lo(kr[u].w), bf16_hi(kr[u].w)};
-            float vf[8] = {bf16_lo(vr[u].x), bf16_hi(vr[u].x), bf16_lo(vr[u].y), bf16_hi(vr[u].y),
-                           bf16_lo(vr[u].z), bf16_hi(vr[u].z), bf16_lo(vr[u].w), bf16_hi(vr[u].w)};
+        for (int x = lane; x < TROWS * 2 * CPR; x += 32) {
+            const int j = x / (2 * CPR), c = x % (2 * CPR);
+            const int t = __shfl_sync(0xffffffffu, tok, j);
+            const bool isv = c >= CPR;
+            const int cc = isv ? c - CPR : c;
+            const int64_t off = t >= 0 ? kv.row(b, h, t) : 0;
+            const __nv_bfloat16 *src = (isv ? kv.v : kv.k) + off + cc * 8;
+            cp_async16(dst0 + ((size_t)j * 2 + (isv ? 1 : 0)) * D + cc * 8, src, t >= 0 ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+
+    constexpr int WSTEP = NWARP * TROWS;  // rows per CTA tile round
+    int base = r0 + warp * TROWS;
+    int tok[STAGES];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float dot = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) dot = fmaf(qf[g][e], kf[e], dot);
-#pragma unroll
-                for (int o = LPR / 2; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                if (ok[u]) {
-                    const float x = dot * scale_log2;
-                    const float mn = fmaxf(m[g], x);
-                    const float c = exp2f(m[g] - mn);
-                    const float p = exp2f(x - mn);
-                    l[g] = fmaf(l[g], c, p);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(acc[g][e], c, p * vf[e]);
-                    m[g] = mn;
-                }
-            }
+    for (int s = 0; s < STAGES - 1; ++s) {
+        tok[s] = -1;
+        if (base + s * WSTEP < r1) {
+            tok[s] = tile_token(base + s * WSTEP);
+            prefetch(tok[s], s);
+        } else {
+            cp_async_commit();
         }
     }
+    for (int k = 0; base < r1; base += WSTEP, ++k) {
+        const int buf = k % STAGES;
+        const int ahead = base + (STAGES - 1) * WSTEP;
+        const int abuf = (k + STAGES - 1) % STAGES;
+        if (ahead < r1) {
+            tok[abuf] = tile_token(ahead);
+            prefetch(tok[abuf], abuf);
+        } else {
+            cp_async_commit();
+        }
+        cp_async_wait<STAGES - 1>();
+        __syncwarp();
+        const __nv_bfloat16 *tile = wstage + (size_t)buf * TROWS * 2 * D;
+
+        float x[RT][G];  // logits, then softmax weights
+        bool ok[RT];
+#pragma unroll
+        for (int j = 0; j < RT; ++j) {
+            const int jr = j * RPW + sub;  // row within the tile
+            ok[j] = __shfl_sync(0xffffffffu, tok[buf], jr) >= 0;
+            const __nv_bfloat16 *kr = tile + (size_t)jr * 2 * D + li * DPL;
+            float kf[DPL];
+            if constexpr (DPL >= 8) {
+#pragma unroll
+                for (int e = 0; e < DPL; e += 8) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(kr + e);
+                    kf[e + 0] = bf16_lo(w.x); kf[e + 1] = bf16_hi(w.x); kf[e + 2] = bf16_lo(w.y); kf[e + 3] = bf16_hi(w.y);
+                    kf[e + 4] = bf16_lo(w.z); kf[e + 5] = bf16_hi(w.z); kf[e + 6] = bf16_lo(w.w); kf[e + 7] = bf16_hi(w.w);
+                }
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2 *>(kr);
+                kf[0] = bf16_lo(w.x); kf[1] = bf16_hi(w.x); kf[2] = bf16_lo(w.y); kf[3] = bf16_hi(w.y);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float d0 = 0.0f, d1 = 0.0f;
+#pragma unroll
+                for (int e = 0; e < DPL; e += 2) {
+                    d0 = fmaf(qf[g][e], kf[e], d0);
+                    d1 = fmaf(qf[g][e + 1], kf[e + 1], d1);
+                }
+                x[j][g] = d0 + d1;
+            }
+        }
+#pragma unroll
+        for (int o = LPR / 2; o; o >>= 1)
+#pragma unroll
+            for (int j = 0; j < RT; ++j)
+#pragma unroll
+                for (int g = 0; g < G; ++g) x[j][g] += __shfl_xor_sync(0xffffffffu, x[j][g], o);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < RT; ++j) {
+                x[j][g] = ok[j] ? x[j][g] * scale_log2 : -INFINITY;
+                tmax = fmaxf(tmax, x[j][g]);
+            }
+            if (tmax == -INFINITY) {  // no valid row in this lane group's tile
+#pragma unroll
+                for (int j = 0; j < RT; ++j) x[j][g] = 0.0f;
+                continue;
+            }
+            const float mn = fmaxf(m[g], tmax);
+            const float c = fast_exp2(m[g] - mn);
+            m[g] = mn;
+            float psum = 0.0f;
+#pragma unroll
+            for (int j = 0; j < RT; ++j) { x[j][g] = fast_exp2(x[j][g] - mn); psum += x[j][g]; }
+            l[g] = fmaf(l[g], c, psum);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[g][e] *= c;
+        }
+        // P.V for the tile
+#pragma unroll
+        for (int j = 0; j < RT; ++j) {
+            const int jr = j * RPW + sub;
+            const __nv_bfloat16 *vrow = tile + ((size_t)jr * 2 + 1) * D + li * DPL;
+            float vf[DPL];
+            if constexpr (DPL >= 8) {
+#pragma unroll
+                for (int e = 0; e < DPL; e += 8) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(vrow + e);
+                    vf[e + 0] = bf16_lo(w.x); vf[e + 1] = bf16_hi(w.x); vf[e + 2] = bf16_lo(w.y); vf[e + 3] = bf16_hi(w.y);
+                    vf[e + 4] = bf16_lo(w.z); vf[e + 5] = bf16_hi(w.z); vf[e + 6] = bf16_lo(w.w); vf[e + 7] = bf16_hi(w.w);
+                }
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2 *>(vrow);
+                vf[0] = bf16_lo(w.x); vf[1] = bf16_hi(w.x); vf[2] = bf16_lo(w.y); vf[3] = bf16_hi(w.y);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) acc[g][e] = fmaf(x[j][g], vf[e], acc[g][e]);
+        }
+        __syncwarp();  // the buffer is refilled by a later prefetch
+    }
+    cp_async_wait<0>();
 
     // merge the NST running states of this CTA
     const int st = warp * RPW + sub;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        if (li == 0) { s_m[st][g] = m[g]; s_l[st][g] = l[g]; }
+        if (li == 0) { s_m[st * G + g] = m[g]; s_l[st * G + g] = l[g]; }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s_acc[st][g][8 * li + e] = acc[g][e];
+        for (int e = 0; e < DPL; ++e) s_acc[(st * G + g) * D + li * DPL + e] = acc[g][e];
     }
     __syncthreads();
     float *part = ws.part + ((int64_t)bh * kMaxSplits + split) * G * (D + 2);
     for (int x = tid; x < G * D; x += kAttnThreads) {
         const int g = x / D, i = x % D;
         float M = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < NST; ++s) M = fmaxf(M, s_m[s][g]);
+#pragma unroll 8
+        for (int s = 0; s < NST; ++s) M = fmaxf(M, s_m[s * G + g]);
         float L = 0.0f, Acc = 0.0f;
         if (M != -INFINITY) {
-#pragma unroll
+#pragma unroll 8
             for (int s = 0; s < NST; ++s) {
-                const float c = exp2f(s_m[s][g] - M);
-                L = fmaf(s_l[s][g], c, L);
-                Acc = fmaf(s_acc[s][g][i], c, Acc);
+                const float c = fast_exp2(s_m[s * G + g] - M);
+                L = fmaf(s_l[s * G + g], c, L);
+                Acc = fmaf(s_acc[(s * G + g) * D + i], c, Acc);
             }
         }
         part[g * (D + 2) + i] = Acc;
@@ -154,16 +290,16 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const float *base = ws.part + (int64_t)bh * kMaxSplits * G * (D + 2);
+    const float *pbase = ws.part + (int64_t)bh * kMaxSplits * G * (D + 2);
     for (int x = tid; x < G * D; x += kAttnThreads) {
         const int g = x / D, i = x % D;
         float M = -INFINITY;
-        for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(base + (s * G + g) * (D + 2) + D));
+        for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(pbase + (s * G + g) * (D + 2) + D));
         float L = 0.0f, Acc = 0.0f;
         if (M != -INFINITY) {
             for (int s = 0; s < splits; ++s) {
-                const float *ps = base + (s * G + g) * (D + 2);
-                const float c = exp2f(__ldcg(ps + D) - M);
+                const float *ps = pbase + (s * G + g) * (D + 2);
+                const float c = fast_exp2(__ldcg(ps + D) - M);
                 L = fmaf(__ldcg(ps + D + 1), c, L);
                 Acc = fmaf(__ldcg(ps + i), c, Acc);
             }

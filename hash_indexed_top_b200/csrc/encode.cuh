@@ -103,72 +103,83 @@ encode_keys_kernel(KV kv, const int32_t *__restrict__ seq_lens, const RBits R, i
 }
 
 // ---------------------------------------------------------------------------
-// Decode-step append.  One CTA per sequence, one warp per kv head: copy the new
-// K/V rows into slot seq_lens[b], encode the key (lane owns hyperplanes
-// lane + 32 m; the sign bits are gathered with warp ballots), then bump
-// seq_lens[b].
-template <int BITS, int D>
-__global__ void append_keys_kernel(KV kv, const __nv_bfloat16 *__restrict__ k_new,
-                                   const __nv_bfloat16 *__restrict__ v_new, int32_t *seq_lens,
-                                   const RBits R) {
-    __shared__ uint32_t Rb[BITS * D / 32];
-    __shared__ float kf[32][D];
-    __shared__ int s_ok;
-    const int b = blockIdx.x;
-    const int h = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int e = threadIdx.x; e < BITS * D / 32; e += blockDim.x) Rb[e] = R.w[e];
+// Decode-step append.  One CTA per sequence: copy the new K/V rows of every kv
+// head into slot seq_lens[b], encode each new key (one thread per
+// (head, hyperplane); the sign bits of a warp are gathered with one ballot),
+// then bump seq_lens[b] once every head is done.
+constexpr int kAppendThreads = 1024;
 
+template <int BITS, int D>
+__global__ void __launch_bounds__(kAppendThreads)
+append_keys_kernel(KV kv, const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *__restrict__ v_new,
+                   int32_t *seq_lens, const RBits R) {
+    constexpr int WPR = D / 32;                 // R words per hyperplane
+    __shared__ uint32_t Rb[BITS * WPR];         // [j][word]
+    __shared__ float kf[32][D];
+    __shared__ uint32_t code32[32][BITS / 32];
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int Hkv = kv.Hkv;
+    for (int e = tid; e < BITS * WPR; e += blockDim.x) Rb[e] = R.w[e];
+
+    griddep_wait();
+    griddep_trigger();  // the scorer may start building its LUT meanwhile
+    // every thread checks the slot itself (no extra barrier); thread 0 reports
     const int64_t pos = seq_lens[b];
-    if (threadIdx.x == 0) {
-        int ok = pos >= 0 && pos < kv.capacity();
-        if (!ok) raise_error(kErrCapacity);
-        if (ok && kv.page_size) ok = kv.page_of(b, pos) >= 0;
-        s_ok = ok;
+    bool ok = pos >= 0 && pos < kv.capacity();
+    if (ok && kv.page_size) {
+        const int32_t p = __ldg(kv.page_table + (int64_t)b * kv.max_pages + pos / kv.page_size);
+        ok = p >= 0 && p < kv.num_pages;
+        if (!ok && tid == 0) raise_error(kErrPage);
+    } else if (!ok && tid == 0) {
+        raise_error(kErrCapacity);
     }
-    __syncthreads();
-    const bool ok = s_ok != 0;
-    if (ok && h < kv.Hkv) {
-        const int64_t r = kv.row(b, h, pos);
-        const uint4 *ksrc = reinterpret_cast<const uint4 *>(k_new + ((int64_t)b * kv.Hkv + h) * D);
-        const uint4 *vsrc = reinterpret_cast<const uint4 *>(v_new + ((int64_t)b * kv.Hkv + h) * D);
-        constexpr int CPR = D / 8;
-        for (int c = lane; c < 2 * CPR; c += 32) {
-            if (c < CPR) {
-                uint4 x = __ldg(ksrc + c);
-                reinterpret_cast<uint4 *>(kv.k + r)[c] = x;
-                kf[h][8 * c + 0] = bf16_lo(x.x); kf[h][8 * c + 1] = bf16_hi(x.x);
-                kf[h][8 * c + 2] = bf16_lo(x.y); kf[h][8 * c + 3] = bf16_hi(x.y);
-                kf[h][8 * c + 4] = bf16_lo(x.z); kf[h][8 * c + 5] = bf16_hi(x.z);
-                kf[h][8 * c + 6] = bf16_lo(x.w); kf[h][8 * c + 7] = bf16_hi(x.w);
-            } else {
-                reinterpret_cast<uint4 *>(kv.v + r)[c - CPR] = __ldg(vsrc + (c - CPR));
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    if (ok) {
+        for (int c = tid; c < 2 * Hkv * CPR; c += blockDim.x) {
+            const int isv = c >= Hkv * CPR;
+            const int cc = isv ? c - Hkv * CPR : c;
+            const int h = cc / CPR, part = cc % CPR;
+            const int64_t r = kv.row(b, h, pos);
+            const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + ((int64_t)b * Hkv + h) * D);
+            const uint4 x = __ldg(src + part);
+            reinterpret_cast<uint4 *>((isv ? kv.v : kv.k) + r)[part] = x;
+            if (!isv) {
+                float *dst = &kf[h][8 * part];
+                dst[0] = bf16_lo(x.x); dst[1] = bf16_hi(x.x); dst[2] = bf16_lo(x.y); dst[3] = bf16_hi(x.y);
+                dst[4] = bf16_lo(x.z); dst[5] = bf16_hi(x.z); dst[6] = bf16_lo(x.w); dst[7] = bf16_hi(x.w);
             }
         }
-        __syncwarp();
-        uint32_t words[BITS / 32];
+    }
+    __syncthreads();
+    if (ok) {
+        // thread -> (head, hyperplane): a warp covers 32 consecutive hyperplanes of one head
+        for (int x = tid; x < Hkv * BITS; x += blockDim.x) {
+            const int h = x / BITS, j = x % BITS;
+            uint32_t rw[WPR];
 #pragma unroll
-        for (int m = 0; m < BITS / 32; ++m) {
-            const int j = lane + 32 * m;
+            for (int w = 0; w < WPR; ++w) rw[w] = Rb[j * WPR + w];
             float acc = 0.0f;
+#pragma unroll
             for (int i = 0; i < D; ++i) {
-                float rf = ((Rb[j * (D / 32) + i / 32] >> (i % 32)) & 1u) ? -1.0f : 1.0f;
+                const float rf = ((rw[i / 32] >> (i % 32)) & 1u) ? -1.0f : 1.0f;
                 acc = fmaf(rf, kf[h][i], acc);
             }
-            words[m] = __ballot_sync(0xffffffffu, acc >= 0.0f);
-        }
-        if (lane == 0) {
-            int64_t c = kv.code(b, h, pos);
-            if (BITS == 32) {
-                kv.codes[c] = (uint64_t)words[0];
-            } else {
-#pragma unroll
-                for (int w = 0; w < BITS / 64; ++w)
-                    kv.codes[c + w] = (uint64_t)words[2 * w] | ((uint64_t)words[2 * w + 1] << 32);
-            }
+            const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
+            if (lane == 0) code32[h][j / 32] = word;
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0 && ok) seq_lens[b] = (int32_t)(pos + 1);
+    if (ok) {
+        constexpr int W = BITS >= 64 ? BITS / 64 : 1;
+        for (int x = tid; x < Hkv * W; x += blockDim.x) {
+            const int h = x / W, w = x % W;
+            const int64_t c = kv.code(b, h, pos);
+            kv.codes[c + w] = BITS == 32 ? (uint64_t)code32[h][0]
+                                         : ((uint64_t)code32[h][2 * w] | ((uint64_t)code32[h][(2 * w + 1) % (BITS / 32)] << 32));
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && ok) seq_lens[b] = (int32_t)(pos + 1);
 }
 
 }  // namespace dkv

@@ -37,7 +37,9 @@ namespace dkv {
 constexpr int kBins = 4096;
 constexpr int kSelThreads = 512;
 constexpr int kMaxSelCtas = 512;
-constexpr int kCandSmem = 2048;  // in-bin candidates resolved in shared memory
+constexpr int kCandSmem = 2048;   // in-bin candidates ranked in shared memory
+constexpr int kListSmem = 8192;   // candidate list held in shared memory by the resolver
+constexpr int kCollectTile = kSelThreads * 16;
 
 enum : int { kStateNormal = 0, kStateAll = 1, kStateEmpty = 2 };
 
@@ -46,15 +48,16 @@ struct SelState {
     int32_t above1;   // tokens in bins > T1
     int32_t cnt_T1;   // tokens in bin T1
     int32_t flags;
-    float A;          // score bound used for binning
-    float inv_w;      // bins per unit score
+    float inv2A;      // 1 / (2 A): scores map to [0, 1] over [-A, A]
+    float pad;
     int32_t kk;       // min(topk, N)
     int32_t n;        // N (clamped)
 };
 
 struct SelWS {
-    float *scores;       // [BH][ld]
-    int64_t ld;          // row length (cache capacity in tokens)
+    float *scores;       // [BH][ld] internal score rows (ld multiple of 64)
+    float *scores_out;   // optional user copy [BH][ld_out]
+    int64_t ld, ld_out;
     int32_t *cand;       // [BH][ld]
     uint32_t *hist;      // [BH][kBins]        zero between calls
     SelState *state;     // [BH]
@@ -62,9 +65,10 @@ struct SelWS {
     int32_t *seg_cnt;    // [BH][kMaxSelCtas]
 };
 
-__device__ __forceinline__ int score_bin(float s, float A, float inv_w) {
-    int bin = (int)((s + A) * inv_w);
-    return bin < 0 ? 0 : (bin > kBins - 1 ? kBins - 1 : bin);
+// Monotone map of a score to one of kBins bins (x in [0, 1] over [-A, A]).
+__device__ __forceinline__ int score_bin(float s, float inv2A) {
+    const float x = __saturatef(fmaf(s, inv2A, 0.5f));
+    return (int)(x * (float)(kBins - 1));
 }
 
 // Token range [t0, t1) of CTA `c` of `nctas` over a length-n sequence; ranges
@@ -76,8 +80,9 @@ __device__ __forceinline__ void cta_range(int64_t n, int c, int nctas, int64_t &
     if (t0 > n) t0 = n;
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim = kSelThreads).
+// Block-wide exclusive scan of one int per thread (blockDim = NT).
 // Returns the exclusive prefix; *total gets the block sum.  All threads must call.
+template <int NT = kSelThreads>
 __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
@@ -89,81 +94,118 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
     if (lane == 31) s_warp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = lane < kSelThreads / 32 ? s_warp[lane] : 0;
+        int w = lane < NT / 32 ? s_warp[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int y = __shfl_up_sync(0xffffffffu, w, o);
             if (lane >= o) w += y;
         }
-        if (lane < kSelThreads / 32) s_warp[lane] = w;  // inclusive warp prefix
+        if (lane < NT / 32) s_warp[lane] = w;  // inclusive warp prefix
     }
     __syncthreads();
     int before = warp ? s_warp[warp - 1] : 0;
-    *total = s_warp[kSelThreads / 32 - 1];
+    *total = s_warp[NT / 32 - 1];
     __syncthreads();  // s_warp may be reused right after
     return before + x - v;
 }
 
 // ---------------------------------------------------------------------------
 // Score + histogram.
+//
+// One CTA of 1024 threads per SM.  The byte-LUT (256 rows x 256 B; row v holds
+// LUT_c[v] for the T tables, replicated 32/T times) sits at a shared address
+// whose low 16 bits are zero, so one byte-permute of (code word, per-lane
+// offset) yields the complete shared address of a lookup:
+//   addr = lut_base | byte << 8 | 4 * (copy * T + table).
+// Lane l reads its token's bytes rotated by rho = l % T, so at each step the
+// 32 lanes touch 32 distinct banks.
+constexpr int kScoreThreads = 1024;
+
 template <int BITS>
 struct ScoreShape {
     static constexpr int T = BITS / 8;         // byte tables
     static constexpr int COPIES = 32 / T;      // interleaved copies: lanes hit distinct banks
     static constexpr int NW = BITS / 32;       // 32-bit code words per token
-    static constexpr size_t LUT_BYTES = 256 * 256;  // 256 byte values x 256-byte rows
-    static constexpr size_t SMEM = LUT_BYTES + kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;
+    static constexpr uint32_t LUT_BYTES = 256 * 256;
+    static constexpr uint32_t LOW_BYTES = kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;  // hist + scratch
+    // dynamic smem: low region, then the LUT at the next 64 KB boundary
+    static constexpr size_t SMEM = 2 * 65536 + LOW_BYTES;
+    using Vec = typename std::conditional<BITS == 128, uint4, uint2>::type;  // one token's code
 };
 
 // Rotate the token's code bytes by rho (byte r of the result = byte (r + rho)
-// mod 4*NW of the input), so every lane reads its tables in a staggered order.
+// mod 4*NW of the input).
+// Branch-free: word rotation by rho / 4 as two select stages, then a funnel
+// shift by 8 (rho % 4) bits across neighbouring words.
 template <int NW>
-__device__ __forceinline__ void rotate_bytes(uint32_t (&w)[NW], int rho) {
-    if (NW == 4) {
-        if (rho & 8) { uint32_t a = w[0], c = w[1]; w[0] = w[2]; w[1] = w[3]; w[2] = a; w[3] = c; }
-        if (rho & 4) { uint32_t a = w[0]; w[0] = w[1]; w[1] = w[2]; w[2] = w[3]; w[3] = a; }
-    } else if (NW == 2) {
-        if (rho & 4) { uint32_t a = w[0]; w[0] = w[1]; w[1] = a; }
-    }
-    const int sh = 8 * (rho & 3);
-    uint32_t o[NW];
+__device__ __forceinline__ void rotate_bytes(uint32_t (&w)[NW], bool by8, bool by4, uint32_t sh) {
+    uint32_t a[NW], c[NW];
 #pragma unroll
-    for (int k = 0; k < NW; ++k) o[k] = __funnelshift_r(w[k], w[(k + 1) % NW], sh);
+    for (int k = 0; k < NW; ++k) a[k] = (NW == 4 && by8) ? w[(k + 2) % NW] : w[k];
 #pragma unroll
-    for (int k = 0; k < NW; ++k) w[k] = o[k];
+    for (int k = 0; k < NW; ++k) c[k] = (NW >= 2 && by4) ? a[(k + 1) % NW] : a[k];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) w[k] = __funnelshift_r(c[k], c[(k + 1) % NW], sh);
 }
 
 template <int BITS>
-__device__ __forceinline__ void load_code(const uint64_t *p, uint32_t (&w)[BITS / 32]) {
-    if (BITS == 128) {
-        uint4 x = __ldcs(reinterpret_cast<const uint4 *>(p));
-        w[0] = x.x; w[1] = x.y; w[2 % (BITS / 32)] = x.z; w[3 % (BITS / 32)] = x.w;
+__device__ __forceinline__ void unpack_code(const typename ScoreShape<BITS>::Vec &x, uint32_t (&w)[BITS / 32]) {
+    if constexpr (BITS == 128) {
+        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+    } else if constexpr (BITS == 64) {
+        w[0] = x.x; w[1] = x.y;
     } else {
-        uint2 x = __ldcs(reinterpret_cast<const uint2 *>(p));
         w[0] = x.x;
-        if (BITS == 64) w[1 % (BITS / 32)] = x.y;
     }
 }
 
+// Shared-memory load from a 32-bit shared address.  Not volatile: its address
+// always depends on code words loaded after the barrier that publishes the LUT,
+// so it cannot be scheduled before that barrier.
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// Score of one (rotated) code: sum over its T bytes of the lane's table entries.
+template <int BITS>
+__device__ __forceinline__ float lut_score(const uint32_t (&w)[BITS / 32], const uint32_t (&off)[BITS / 8]) {
+    constexpr int T = BITS / 8;
+    float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+    for (int r = 0; r < T; r += 2) {
+        s0 += lds_f32(__byte_perm(w[r >> 2], off[r], 0x7604u | ((uint32_t)(r & 3) << 4)));
+        s1 += lds_f32(__byte_perm(w[(r + 1) >> 2], off[r + 1], 0x7604u | ((uint32_t)((r + 1) & 3) << 4)));
+    }
+    return (s0 + s1) + 0.0f;  // + 0 turns a -0 into +0
+}
+
 template <int BITS, int D>
-__global__ void __launch_bounds__(kSelThreads, 2)
+__global__ void __launch_bounds__(kScoreThreads, 1)
 score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                   const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int nctas) {
     using S = ScoreShape<BITS>;
+    using Vec = typename S::Vec;
     constexpr int T = S::T, NW = S::NW;
+    constexpr int NWARPS = kScoreThreads / 32;
     extern __shared__ __align__(1024) unsigned char smem[];
-    unsigned char *lut = smem;                                            // [256][256 B]
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + S::LUT_BYTES);   // [kBins]
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);                  // [kBins]
     float *qsum = reinterpret_cast<float *>(hist + kBins);                // [D]
     float *Qp = qsum + kMaxDim;                                           // [BITS]
     float *red = Qp + kMaxBits;                                           // [64]
+    const uint32_t smem_s = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t lut_s = (smem_s + S::LOW_BYTES + 65535u) & ~65535u;     // 64 KB aligned
+    unsigned char *lut = smem + (lut_s - smem_s);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.y, b = bh / kv.Hkv, h = bh % kv.Hkv;
-    const int64_t n = clamp_len(kv, seq_lens, b);
-
-    for (int i = tid; i < kBins; i += kSelThreads) hist[i] = 0;
-    for (int i = tid; i < D; i += kSelThreads) {
+    if (lut_s + 65536u > smem_s + (uint32_t)S::SMEM) {  // cannot happen with a small static region
+        if (tid == 0) raise_error(kErrCapacity);
+        return;
+    }
+    for (int i = tid; i < kBins; i += kScoreThreads) hist[i] = 0;
+    for (int i = tid; i < D; i += kScoreThreads) {
         const __nv_bfloat16 *qh = q + ((int64_t)b * Hq + (int64_t)h * G) * D + i;
         float s = 0.0f;
         for (int g = 0; g < G; ++g) s += __bfloat162float(qh[(int64_t)g * D]);
@@ -188,70 +230,75 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         for (int j = lane; j < BITS; j += 32) a += fabsf(Qp[j]);
 #pragma unroll
         for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) {
-            red[0] = a;
-            red[1] = a > 0.0f ? (float)kBins / (2.0f * a) : 0.0f;
-        }
+        if (lane == 0) red[0] = a > 0.0f ? 0.5f / a : 0.0f;
     }
-    // LUT_c[v] for the T byte tables, replicated COPIES times per 256-byte row:
-    // word (v * 64 + copy * T + c).
+    // LUT rows: word (v * 64 + copy * T + c) holds LUT_c[v]; lane l fills word l
+    // of each row it owns (copy = l / T, c = l % T), so stores never conflict.
     {
-        const int v = tid & 255;
-        for (int c = tid >> 8; c < T; c += kSelThreads / 256) {
+        const int c = lane % T;
+        float qv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) qv[u] = Qp[8 * c + u];
+        for (int v = warp; v < 256; v += NWARPS) {
             float val = 0.0f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) val += ((v >> u) & 1) ? Qp[8 * c + u] : -Qp[8 * c + u];
-            float *row = reinterpret_cast<float *>(lut + v * 256);
-#pragma unroll
-            for (int cp = 0; cp < S::COPIES; ++cp) row[cp * T + c] = val;
+            for (int u = 0; u < 8; ++u) val += ((v >> u) & 1) ? qv[u] : -qv[u];
+            reinterpret_cast<float *>(lut + v * 256)[lane] = val;
         }
     }
     __syncthreads();
-    const float A = red[0], inv_w = red[1];
+    const float inv2A = red[0];
+    // everything above depends on q only; codes and lengths come from the append
+    griddep_wait();
+    const int64_t n = clamp_len(kv, seq_lens, b);
 
     int64_t t0, t1;
     cta_range(n, blockIdx.x, nctas, t0, t1);
     const int rho = lane % T, copy = lane / T;
+    const bool rot8 = (rho & 8) != 0, rot4 = (rho & 4) != 0;
+    const uint32_t rot_sh = 8u * (uint32_t)(rho & 3);
     uint32_t off[T];
 #pragma unroll
-    for (int r = 0; r < T; ++r) off[r] = 4u * (uint32_t)(copy * T + (rho + r) % T);
+    for (int r = 0; r < T; ++r) off[r] = lut_s | 4u * (uint32_t)(copy * T + (rho + r) % T);
 
     float *srow = ws.scores + (int64_t)bh * ws.ld;
-    constexpr int U = 4;
-    constexpr int NWARPS = kSelThreads / 32;
-    for (int64_t g0 = t0 + warp * 32; g0 < t1; g0 += (int64_t)NWARPS * 32 * U) {
-        uint32_t w[U][NW];
+    float *urow = ws.scores_out ? ws.scores_out + (int64_t)bh * ws.ld_out : nullptr;
+    const int nloc = (int)(t1 - t0);  // tokens of this CTA (< 2^31)
+    // lane's code pointer for local token index i (dense layout; paged via page table)
+    const Vec *dense = reinterpret_cast<const Vec *>(kv.codes) + ((int64_t)bh * kv.n_cap + t0);
+    auto fetch = [&](int i) -> Vec {  // i: local index of this lane's token (i < nloc)
+        if (!kv.page_size) return __ldcs(dense + i);
+        const int64_t c = kv.code(b, h, t0 + i);
+        return c >= 0 ? __ldcs(reinterpret_cast<const Vec *>(kv.codes + c)) : Vec{};
+    };
+
+    constexpr int STEP = NWARPS * 32;
+    int i = warp * 32 + lane;
+    Vec nxt0 = i < nloc ? fetch(i) : Vec{};
+    Vec nxt1 = i + STEP < nloc ? fetch(i + STEP) : Vec{};
+    for (int g = warp * 32; g < nloc; g += 2 * STEP, i += 2 * STEP) {
+        const Vec cur0 = nxt0, cur1 = nxt1;
+        if (i + 2 * STEP < nloc) nxt0 = fetch(i + 2 * STEP);
+        if (i + 3 * STEP < nloc) nxt1 = fetch(i + 3 * STEP);
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t t = g0 + (int64_t)u * NWARPS * 32 + lane;
-#pragma unroll
-            for (int k = 0; k < NW; ++k) w[u][k] = 0;
-            if (t < t1) {
-                int64_t c = kv.code(b, h, t);
-                if (c >= 0) load_code<BITS>(kv.codes + c, w[u]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t t = g0 + (int64_t)u * NWARPS * 32 + lane;
-            rotate_bytes<NW>(w[u], rho);
-            float s = 0.0f;
-#pragma unroll
-            for (int r = 0; r < T; ++r) {
-                uint32_t addr = __byte_perm(w[u][r >> 2], off[r], 0x7604u | ((uint32_t)(r & 3) << 4));
-                s += *reinterpret_cast<const float *>(lut + addr);
-            }
-            s += 0.0f;
-            if (t < t1) {
-                srow[t] = s;
-                atomicAdd(&hist[score_bin(s, A, inv_w)], 1u);
+        for (int u = 0; u < 2; ++u) {
+            const int iu = i + u * STEP;
+            uint32_t w[NW];
+            unpack_code<BITS>(u ? cur1 : cur0, w);
+            rotate_bytes<NW>(w, rot8, rot4, rot_sh);
+            const float s = lut_score<BITS>(w, off);
+            if (iu < nloc) {
+                srow[t0 + iu] = s;
+                if (urow) urow[t0 + iu] = s;
+                atomicAdd(&hist[score_bin(s, inv2A)], 1u);
             }
         }
     }
+    griddep_trigger();
     __syncthreads();
     uint32_t *ghist = ws.hist + (int64_t)bh * kBins;
-    for (int i = tid; i < kBins; i += kSelThreads)
-        if (hist[i]) atomicAdd(ghist + i, hist[i]);
+    for (int k = tid; k < kBins; k += kScoreThreads)
+        if (hist[k]) atomicAdd(ghist + k, hist[k]);
 
     // ---- last CTA of this (b, h): locate the threshold bin
     __shared__ int s_last;
@@ -262,22 +309,22 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int i = tid; i < kBins; i += kSelThreads) {
-        hist[i] = __ldcg(ghist + i);
-        ghist[i] = 0;
+    for (int k = tid; k < kBins; k += kScoreThreads) {
+        hist[k] = __ldcg(ghist + k);
+        ghist[k] = 0;
     }
     __syncthreads();
     const int64_t kk = topk < n ? topk : n;
-    constexpr int PER = kBins / kSelThreads;  // bins per thread, thread 0 owns the top
+    constexpr int PER = kBins / kScoreThreads;  // bins per thread, thread 0 owns the top
     int local = 0;
     const int top = kBins - 1 - tid * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) local += hist[top - e];
     int total;
-    const int before = block_excl_scan(local, s_warp, &total);
+    const int before = block_excl_scan<kScoreThreads>(local, s_warp, &total);
     if (tid == 0) {
         SelState st;
-        st.A = A; st.inv_w = inv_w; st.kk = (int32_t)kk; st.n = (int32_t)n;
+        st.inv2A = inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
         st.T1 = kBins; st.above1 = 0; st.cnt_T1 = 0;
         st.flags = n == 0 ? kStateEmpty : (kk >= n ? kStateAll : kStateNormal);
         ws.state[bh] = st;
@@ -300,200 +347,266 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
 }
 
 // ---------------------------------------------------------------------------
-// Resolve helpers (run by the last CTA of a (b, h) in collect_kernel).
+// Collect + resolve.
+//
+// The candidate list of a (b, h) is the concatenation, in CTA order, of every
+// CTA's segment (tokens of its range with bin >= T1, ascending), so the list
+// is in ascending token order.  The resolver addresses it through a ListView:
+// either a shared-memory copy (tokens + order keys) or, when the list is too
+// long for that, the segments in global memory.
+struct ListView {
+    const int32_t *s_t;        // shared copy (or null)
+    const uint32_t *s_key;
+    const int32_t *cand;       // global segments
+    const float *srow;
+    const int *s_seg_off;      // exclusive prefix of the segment sizes [nctas + 1]
+    int nctas, n;
 
-// Visit the concatenated segments (ascending token order) in tiles of
-// kSelThreads; f(e_valid, t) is called by every thread for every tile.
-template <class F>
-__device__ __forceinline__ void for_list_tiles(const SelWS &ws, int bh, int nctas, int n,
-                                               const int *s_seg_cnt, F &&f) {
-    const int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
-    for (int c = 0; c < nctas; ++c) {
-        int64_t t0, t1;
-        cta_range(n, c, nctas, t0, t1);
-        const int cnt = s_seg_cnt[c];
-        for (int base = 0; base < cnt; base += kSelThreads) {
-            const int e = base + threadIdx.x;
-            const bool valid = e < cnt;
-            const int t = valid ? __ldcg(cand + t0 + e) : 0;
-            f(valid, t);
+    __device__ __forceinline__ void get(int e, int &t, uint32_t &key) const {
+        if (s_t) {
+            t = s_t[e];
+            key = s_key[e];
+            return;
         }
+        int lo = 0, hi = nctas;  // segment c with s_seg_off[c] <= e < s_seg_off[c + 1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_seg_off[mid] <= e) lo = mid; else hi = mid;
+        }
+        int64_t t0, t1;
+        cta_range(n, lo, nctas, t0, t1);
+        t = __ldcg(cand + t0 + (e - s_seg_off[lo]));
+        key = float_key(__ldcg(srow + t));
     }
+};
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-__device__ __forceinline__ void write_selection(const SelWS &ws, int bh, int nctas, const SelState &st,
-                                                int S, int W, int cap_sel, int32_t *sel_idx,
-                                                int32_t *sel_cnt, const int *s_seg_cnt, uint32_t Tkey,
-                                                int IT, int *s_warp) {
-    const int n = st.n;
-    int32_t *out = sel_idx + (int64_t)bh * cap_sel;
-    const float *srow = ws.scores + (int64_t)bh * ws.ld;
-    const int s_end = S < n ? S : n;                  // sinks [0, s_end)
-    const int w_beg = n - W > s_end ? n - W : s_end;  // window [w_beg, n)
-    int pos;
-    if (st.flags == kStateAll) {
-        for (int t = threadIdx.x; t < n; t += kSelThreads) out[t] = t;
-        pos = n;
-    } else if (st.flags == kStateEmpty) {
-        pos = 0;
-    } else {
-        for (int t = threadIdx.x; t < s_end; t += kSelThreads) out[t] = t;
-        pos = s_end;
-        for_list_tiles(ws, bh, nctas, n, s_seg_cnt, [&](bool valid, int t) {
-            bool keep = false;
-            if (valid && t >= s_end && t < w_beg) {
-                const float s = __ldcg(srow + t);
-                const int bin = score_bin(s, st.A, st.inv_w);
-                const uint32_t key = float_key(s);
-                keep = bin > st.T1 || (bin == st.T1 && (key > Tkey || (key == Tkey && t <= IT)));
-            }
-            int tot;
-            const int p = block_excl_scan(keep ? 1 : 0, s_warp, &tot);
-            if (keep && pos + p < cap_sel) out[pos + p] = t;
-            pos += tot;
-        });
-        for (int t = w_beg + threadIdx.x; t < n; t += kSelThreads)
-            if (pos + (t - w_beg) < cap_sel) out[pos + (t - w_beg)] = t;
-        pos += n - w_beg;
-        if (pos > cap_sel) pos = cap_sel;  // unreachable when the threshold is consistent
+// For every list element in order, f(e, t, key) -> bool; returns, per thread,
+// the exclusive rank of its first kept element and the block total.  Each thread
+// owns a contiguous run of elements so one block scan orders everything.
+template <class Pred, class Emit>
+__device__ __forceinline__ int ordered_pass(const ListView &L, int M, int *s_warp, Pred &&pred, Emit &&emit) {
+    const int per = (M + kSelThreads - 1) / kSelThreads;
+    const int e0 = threadIdx.x * per;
+    const int e1 = min(M, e0 + per);
+    int cnt = 0;
+    for (int e = e0; e < e1; ++e) {
+        int t; uint32_t key;
+        L.get(e, t, key);
+        cnt += pred(t, key) ? 1 : 0;
     }
-    for (int r = pos + threadIdx.x; r < cap_sel; r += kSelThreads) out[r] = -1;
-    if (threadIdx.x == 0) sel_cnt[bh] = pos;
+    int total;
+    int r = block_excl_scan(cnt, s_warp, &total);
+    if (cnt)
+        for (int e = e0; e < e1; ++e) {
+            int t; uint32_t key;
+            L.get(e, t, key);
+            if (pred(t, key)) emit(r++, t);
+        }
+    return total;
 }
 
-// ---------------------------------------------------------------------------
+struct CollectSmem {
+    int32_t list_t[kListSmem];
+    uint32_t list_key[kListSmem];
+    uint32_t ck[kCandSmem];
+    int32_t ci[kCandSmem];
+    uint32_t h[2048];
+    int seg_off[kMaxSelCtas + 1];
+    int warp[32];
+    int misc[8];
+    int last;
+};
+
 __global__ void __launch_bounds__(kSelThreads)
-collect_kernel(const int32_t *__restrict__ seq_lens_unused, SelWS ws, int nctas, int S, int W, int cap_sel,
-               int32_t *sel_idx, int32_t *sel_cnt) {
-    __shared__ int s_warp[32];
-    __shared__ int s_last;
-    __shared__ int s_seg_cnt[kMaxSelCtas];
-    __shared__ uint32_t s_ck[kCandSmem];
-    __shared__ int s_ci[kCandSmem];
-    __shared__ uint32_t s_h[2048];
-    __shared__ int s_misc[8];
-    (void)seq_lens_unused;
-
+collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    CollectSmem &sm = *reinterpret_cast<CollectSmem *>(smem_raw);
     const int tid = threadIdx.x;
     const int bh = blockIdx.y;
+    griddep_wait();
     const SelState st = ws.state[bh];
     const int n = st.n;
     int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
     const float *srow = ws.scores + (int64_t)bh * ws.ld;
 
+    // ---- this CTA's segment: tokens of [t0, t1) with bin >= T1, ascending
     int count = 0;
     if (st.flags == kStateNormal) {
         int64_t t0, t1;
         cta_range(n, blockIdx.x, nctas, t0, t1);
-        for (int64_t base = t0; base < t1; base += kSelThreads) {
-            const int64_t t = base + tid;
-            bool f = false;
-            if (t < t1) f = score_bin(__ldcg(srow + t), st.A, st.inv_w) >= st.T1;
+        for (int64_t base = t0; base < t1; base += kCollectTile) {
+            const int64_t tb = base + (int64_t)tid * 16;
+            uint32_t flags = 0;
+            if (tb + 16 <= t1) {
+                const float4 *p = reinterpret_cast<const float4 *>(srow + tb);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 x = __ldcg(p + v);
+                    flags |= (uint32_t)(score_bin(x.x, st.inv2A) >= st.T1) << (4 * v + 0);
+                    flags |= (uint32_t)(score_bin(x.y, st.inv2A) >= st.T1) << (4 * v + 1);
+                    flags |= (uint32_t)(score_bin(x.z, st.inv2A) >= st.T1) << (4 * v + 2);
+                    flags |= (uint32_t)(score_bin(x.w, st.inv2A) >= st.T1) << (4 * v + 3);
+                }
+            } else {
+                for (int j = 0; j < 16; ++j)
+                    if (tb + j < t1) flags |= (uint32_t)(score_bin(__ldcg(srow + tb + j), st.inv2A) >= st.T1) << j;
+            }
             int tot;
-            const int p = block_excl_scan(f ? 1 : 0, s_warp, &tot);
-            if (f) cand[t0 + count + p] = (int32_t)t;
+            int r = block_excl_scan(__popc(flags), sm.warp, &tot);
+            while (flags) {
+                const int j = __ffs(flags) - 1;
+                flags &= flags - 1;
+                cand[t0 + count + r++] = (int32_t)(tb + j);
+            }
             count += tot;
         }
     }
+    griddep_trigger();
     if (tid == 0) ws.seg_cnt[(int64_t)bh * kMaxSelCtas + blockIdx.x] = count;
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(ws.arrive + gridDim.y + bh, 1u) == (unsigned)(nctas - 1);
+    if (tid == 0) sm.last = atomicAdd(ws.arrive + gridDim.y + bh, 1u) == (unsigned)(nctas - 1);
     __syncthreads();
-    if (!s_last) return;
+    if (!sm.last) return;
     __threadfence();
 
-    // ---- resolve the exact threshold (Tkey, IT) inside bin T1
-    for (int c = tid; c < nctas; c += kSelThreads) s_seg_cnt[c] = __ldcg(ws.seg_cnt + (int64_t)bh * kMaxSelCtas + c);
+    // ---- the last CTA of (b, h): list offsets, exact threshold, final selection
+    {
+        const int c = tid;
+        const int v = c < nctas ? __ldcg(ws.seg_cnt + (int64_t)bh * kMaxSelCtas + c) : 0;
+        int tot;
+        const int ex = block_excl_scan(v, sm.warp, &tot);
+        if (c < nctas) sm.seg_off[c] = ex;
+        if (c == 0) sm.seg_off[nctas] = tot;
+    }
     __syncthreads();
+    const int M = sm.seg_off[nctas];
+    ListView L{nullptr, nullptr, cand, srow, sm.seg_off, nctas, n};
+    if (st.flags == kStateNormal && M <= kListSmem) {
+        // one parallel round over the whole list (each element finds its segment)
+        for (int e = tid; e < M; e += kSelThreads) {
+            int t; uint32_t key;
+            L.get(e, t, key);
+            sm.list_t[e] = t;
+            sm.list_key[e] = key;
+        }
+        __syncthreads();
+        L.s_t = sm.list_t;
+        L.s_key = sm.list_key;
+    }
+
+    const float inv2A = st.inv2A;
+    const int T1 = st.T1;
     uint32_t Tkey = 0;
     int IT = 0x7fffffff;
     if (st.flags == kStateNormal) {
         const int need1 = st.kk - st.above1;  // 1 <= need1 <= cnt_T1
+        auto in_bin = [&](uint32_t key) { return score_bin(key_to_float(key), inv2A) == T1; };
         if (need1 < st.cnt_T1 && st.cnt_T1 <= kCandSmem) {
-            if (tid == 0) s_misc[0] = 0;
+            // rank the in-bin candidates by (score desc, token asc)
+            if (tid == 0) sm.misc[0] = 0;
             __syncthreads();
-            for_list_tiles(ws, bh, nctas, n, s_seg_cnt, [&](bool valid, int t) {
-                if (valid) {
-                    const float s = __ldcg(srow + t);
-                    if (score_bin(s, st.A, st.inv_w) == st.T1) {
-                        const int slot = atomicAdd(&s_misc[0], 1);
-                        s_ck[slot] = float_key(s);
-                        s_ci[slot] = t;
-                    }
+            for (int e = tid; e < M; e += kSelThreads) {
+                int t; uint32_t key;
+                L.get(e, t, key);
+                if (in_bin(key)) {
+                    const int slot = atomicAdd(&sm.misc[0], 1);
+                    sm.ck[slot] = key;
+                    sm.ci[slot] = t;
                 }
-            });
-            __syncthreads();
-            const int c1 = s_misc[0];
-            for (int e = tid; e < c1; e += kSelThreads) {
-                const uint32_t ke = s_ck[e];
-                const int ie = s_ci[e];
-                int rank = 0;
-                for (int f = 0; f < c1; ++f) {
-                    const uint32_t kf = s_ck[f];
-                    rank += (kf > ke) || (kf == ke && s_ci[f] < ie);
-                }
-                if (rank == need1 - 1) { s_misc[1] = (int)ke; s_misc[2] = ie; }
             }
             __syncthreads();
-            Tkey = (uint32_t)s_misc[1];
-            IT = s_misc[2];
+            const int c1 = sm.misc[0];
+            for (int e = tid; e < c1; e += kSelThreads) {
+                const uint32_t ke = sm.ck[e];
+                const int ie = sm.ci[e];
+                int rank = 0;
+                for (int f = 0; f < c1; ++f) {
+                    const uint32_t kf = sm.ck[f];
+                    rank += (kf > ke) || (kf == ke && sm.ci[f] < ie);
+                }
+                if (rank == need1 - 1) { sm.misc[1] = (int)ke; sm.misc[2] = ie; }
+            }
+            __syncthreads();
+            Tkey = (uint32_t)sm.misc[1];
+            IT = sm.misc[2];
         } else if (need1 < st.cnt_T1) {
-            // Large tie-heavy bin: radix-select the key over the in-bin tokens
-            // (11/11/10 bits), then the need-th tied token in index order.
+            // Large, tie-heavy bin: radix-select the order key over the in-bin
+            // tokens (11/11/10 bits), then the need-th tied token in list order.
             uint32_t prefix = 0, mask = 0;
             int need = need1;
-            const int shifts[3] = {21, 10, 0};
-            const int widths[3] = {11, 11, 10};
+#pragma unroll 1
             for (int p = 0; p < 3; ++p) {
-                const int sh = shifts[p], nb = 1 << widths[p];
-                for (int i = tid; i < 2048; i += kSelThreads) s_h[i] = 0;
+                const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0);
+                const int nb = p == 2 ? 1024 : 2048;
+                for (int i = tid; i < 2048; i += kSelThreads) sm.h[i] = 0;
                 __syncthreads();
-                for_list_tiles(ws, bh, nctas, n, s_seg_cnt, [&](bool valid, int t) {
-                    if (valid) {
-                        const float s = __ldcg(srow + t);
-                        const uint32_t key = float_key(s);
-                        if (score_bin(s, st.A, st.inv_w) == st.T1 && (key & mask) == prefix)
-                            atomicAdd(&s_h[(key >> sh) & (nb - 1)], 1u);
-                    }
-                });
+                for (int e = tid; e < M; e += kSelThreads) {
+                    int t; uint32_t key;
+                    L.get(e, t, key);
+                    if (in_bin(key) && (key & mask) == prefix) atomicAdd(&sm.h[(key >> sh) & (nb - 1)], 1u);
+                }
                 __syncthreads();
                 if (tid == 0) {
                     int run = 0, dd = nb - 1;
-                    for (; dd >= 0; --dd) {
-                        if (run + (int)s_h[dd] >= need) break;
-                        run += s_h[dd];
+                    for (; dd > 0; --dd) {
+                        if (run + (int)sm.h[dd] >= need) break;
+                        run += sm.h[dd];
                     }
-                    s_misc[3] = dd;
-                    s_misc[4] = need - run;
+                    sm.misc[3] = dd;
+                    sm.misc[4] = need - run;
                 }
                 __syncthreads();
-                prefix |= (uint32_t)s_misc[3] << sh;
+                prefix |= (uint32_t)sm.misc[3] << sh;
                 mask |= (uint32_t)(nb - 1) << sh;
-                need = s_misc[4];
+                need = sm.misc[4];
                 __syncthreads();
             }
             Tkey = prefix;
-            // the need-th token (index order) among bin == T1 and key == Tkey
-            int run = 0;
-            if (tid == 0) s_misc[5] = 0x7fffffff;
+            if (tid == 0) sm.misc[5] = 0x7fffffff;
             __syncthreads();
-            for_list_tiles(ws, bh, nctas, n, s_seg_cnt, [&](bool valid, int t) {
-                bool m = false;
-                if (valid) {
-                    const float s = __ldcg(srow + t);
-                    m = score_bin(s, st.A, st.inv_w) == st.T1 && float_key(s) == Tkey;
-                }
-                int tot;
-                const int p = block_excl_scan(m ? 1 : 0, s_warp, &tot);
-                if (m && run + p + 1 == need) s_misc[5] = t;
-                run += tot;
-            });
+            const int want = need;
+            ordered_pass(L, M, sm.warp,
+                         [&](int t, uint32_t key) { return in_bin(key) && key == Tkey; },
+                         [&](int rank, int t) { if (rank + 1 == want) sm.misc[5] = t; });
             __syncthreads();
-            IT = s_misc[5];
+            IT = sm.misc[5];
         }
     }
-    write_selection(ws, bh, nctas, st, S, W, cap_sel, sel_idx, sel_cnt, s_seg_cnt, Tkey, IT, s_warp);
+
+    // ---- emit: sinks, kept list tokens in the middle range, window
+    int32_t *out = sel_idx + (int64_t)bh * cap_sel;
+    const int s_end = S < n ? S : n;                  // sinks [0, s_end)
+    const int w_beg = n - W > s_end ? n - W : s_end;  // window [w_beg, n)
+    int pos;
+    if (st.flags == kStateAll) {
+        for (int t = tid; t < n; t += kSelThreads) out[t] = t;
+        pos = n;
+    } else if (st.flags == kStateEmpty) {
+        pos = 0;
+    } else {
+        for (int t = tid; t < s_end; t += kSelThreads) out[t] = t;
+        pos = s_end;
+        const int kept = ordered_pass(
+            L, M, sm.warp,
+            [&](int t, uint32_t key) {
+                if (t < s_end || t >= w_beg) return false;
+                const int bin = score_bin(key_to_float(key), inv2A);
+                return bin > T1 || (bin == T1 && (key > Tkey || (key == Tkey && t <= IT)));
+            },
+            [&](int rank, int t) { if (pos + rank < cap_sel) out[pos + rank] = t; });
+        pos += kept;
+        for (int t = w_beg + tid; t < n; t += kSelThreads)
+            if (pos + (t - w_beg) < cap_sel) out[pos + (t - w_beg)] = t;
+        pos += n - w_beg;
+        if (pos > cap_sel) pos = cap_sel;  // unreachable when the threshold is consistent
+    }
+    for (int r = pos + tid; r < cap_sel; r += kSelThreads) out[r] = -1;
+    if (tid == 0) sel_cnt[bh] = pos;
     if (tid == 0) ws.arrive[gridDim.y + bh] = 0;
 }
 

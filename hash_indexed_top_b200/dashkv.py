@@ -213,7 +213,10 @@ class DashKV:
             self._trace = None
             _check("dashkv_set_trace", lib().dashkv_set_trace(self._ctx, None, 0))
             return
-        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        handles = [e.cuda_event for e in events]
+        if not all(handles):
+            raise ValueError("set_trace: record each event once first (torch creates CUDA events lazily)")
+        arr = (ctypes.c_void_p * len(events))(*handles)
         self._trace = arr  # keep alive while tracing
         _check("dashkv_set_trace", lib().dashkv_set_trace(self._ctx, arr, len(events)))
 

@@ -74,7 +74,8 @@ class OracleRun:
 
 def within_tol(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
     both_inf = np.isneginf(got) & np.isneginf(ref)
-    err = np.abs(got - ref)
+    with np.errstate(invalid="ignore"):
+        err = np.abs(got - ref)
     return both_inf | (err <= ATOL + RTOL * np.abs(ref))
 
 
