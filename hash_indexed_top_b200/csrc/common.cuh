@@ -13,7 +13,7 @@ constexpr int kMaxDim = 128;
 constexpr int kSmCountFallback = 148;
 
 // Device error word (one per device that loads the library).  Bits:
-enum : unsigned { kErrCapacity = 1u, kErrPage = 2u };
+enum : unsigned { kErrCapacity = 1u, kErrPage = 2u, kErrTimeout = 4u };
 __device__ unsigned g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }

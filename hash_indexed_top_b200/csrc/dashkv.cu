@@ -22,6 +22,9 @@ struct dashkv_ctx {
     RBits R;
     int device;
     int sm_count;
+    int coop;        // cooperative launches supported
+    int fused_pdl;   // combine cooperative with programmatic serialization
+    int force_two_kernel;
     void **trace;   // optional cudaEvent_t pairs around each kernel of a call
     int n_trace;
 };
@@ -70,7 +73,7 @@ bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 dashkv_status check_config(const dashkv_config *c) {
     if (!c) return DASHKV_ERR_INVALID_ARG;
     if (c->batch <= 0 || c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->topk <= 0 || c->sink < 0 ||
-        c->window < 0 || c->page_size < 0 || c->reserved != 0)
+        c->window < 0 || c->page_size < 0 || (c->flags & ~DASHKV_FLAG_TWO_KERNEL_SELECT))
         return DASHKV_ERR_INVALID_ARG;
     if (c->num_q_heads % c->num_kv_heads) return DASHKV_ERR_INVALID_ARG;
     const int G = c->num_q_heads / c->num_kv_heads;
@@ -120,7 +123,7 @@ int64_t view_capacity(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
 
 // ---- workspace: [scores | cand | hist | state | arrive(3 x BH) | seg_cnt | partials]
 struct WsLayout {
-    size_t scores, cand, hist, state, arrive, seg_cnt, part, total;
+    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, bar, inbin_n, inbin, def_mid, total;
 };
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -136,11 +139,16 @@ WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
     size_t o = 0;
     L.scores = o;  o = align_up(o + BH * ld * 4);
     L.cand = o;    o = align_up(o + BH * ld * 4);
+    L.ckey = o;    o = align_up(o + BH * ld * 4);
     L.hist = o;    o = align_up(o + BH * kBins * 4);
     L.state = o;   o = align_up(o + BH * sizeof(SelState));
     L.arrive = o;  o = align_up(o + 3 * BH * 4);
     L.seg_cnt = o; o = align_up(o + BH * kMaxSelCtas * 4);
     L.part = o;    o = align_up(o + BH * kMaxSplits * G * (c.head_dim + 2) * 4);
+    L.bar = o;     o = align_up(o + BH * 2 * 4);
+    L.inbin_n = o; o = align_up(o + BH * 4);
+    L.inbin = o;   o = align_up(o + BH * kInbinMax * 16);
+    L.def_mid = o; o = align_up(o + BH * kMaxSelCtas * 4);
     L.total = o;
     return L;
 }
@@ -188,11 +196,32 @@ int attn_splits(const dashkv_ctx *ctx) {
 }
 
 // ---- template dispatch
+// The scorer places its LUT at the first 64 KB boundary above its low region;
+// that needs the static shared memory (plus the 1 KB the system reserves) to
+// leave room for the low region below 64 KB.
+template <int BITS, int D>
+bool score_layout_ok() {
+    cudaFuncAttributes a[4];
+    cudaFuncGetAttributes(&a[0], score_hist_kernel<BITS, D, false>);
+    cudaFuncGetAttributes(&a[1], score_hist_kernel<BITS, D, true>);
+    cudaFuncGetAttributes(&a[2], select_fused_kernel<BITS, D, false>);
+    cudaFuncGetAttributes(&a[3], select_fused_kernel<BITS, D, true>);
+    for (auto &x : a)
+        if (x.sharedSizeBytes + 1024 + ScoreShape<BITS>::LOW_BYTES > 65536) return false;
+    return true;
+}
+
 template <int BITS, int D>
 void set_attrs_bd() {
     cudaFuncSetAttribute(encode_keys_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)EncodeShape<BITS, D>::SMEM);
-    cudaFuncSetAttribute(score_hist_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(score_hist_kernel<BITS, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(score_hist_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)ScoreShape<BITS>::SMEM);
 }
 
@@ -255,8 +284,51 @@ void launch_score_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
                      int nctas, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
-    launch_pdl(score_hist_kernel<BITS, D>, dim3(nctas, BH), dim3(kScoreThreads), ScoreShape<BITS>::SMEM, st, kv,
+    auto kern = kv.page_size ? score_hist_kernel<BITS, D, true> : score_hist_kernel<BITS, D, false>;
+    launch_pdl(kern, dim3(nctas, BH), dim3(kScoreThreads), ScoreShape<BITS>::SMEM, st, kv,
                static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, ctx->cfg.topk, nctas);
+}
+
+// The fused selection needs every CTA resident at once: one per SM.
+bool use_fused(const dashkv_ctx *ctx, int64_t cap) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    return ctx->coop && !ctx->force_two_kernel && sel_ctas(ctx, cap, 1) * BH <= ctx->sm_count;
+}
+
+// Fused selection: cooperative launch (all CTAs resident together; the kernel
+// synchronises the CTAs of each (b, h) with bounded waits) that may also start
+// early behind the preceding kernel.
+template <int BITS, int D>
+void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                     int nctas, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
+    const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
+    auto kern = kv.page_size ? select_fused_kernel<BITS, D, true> : select_fused_kernel<BITS, D, false>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nctas, BH);
+    cfg.blockDim = dim3(kScoreThreads);
+    cfg.dynamicSmemBytes = ScoreShape<BITS>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ctx->fused_pdl ? 2 : 1;
+    cudaLaunchKernelEx(&cfg, kern, kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R,
+                       ws, ctx->cfg.topk, nctas, ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
+}
+
+template <int D>
+void launch_fused_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                    int nctas, int32_t *si, int32_t *sc, cudaStream_t st) {
+    switch (ctx->cfg.bits) {
+        case 32: launch_fused_bd<32, D>(ctx, kv, q, seq, ws, nctas, si, sc, st); break;
+        case 64: launch_fused_bd<64, D>(ctx, kv, q, seq, ws, nctas, si, sc, st); break;
+        default: launch_fused_bd<128, D>(ctx, kv, q, seq, ws, nctas, si, sc, st); break;
+    }
 }
 
 template <int D>
@@ -307,6 +379,7 @@ const char *dashkv_status_str(dashkv_status s) {
         case DASHKV_ERR_CUDA: return "CUDA error";
         case DASHKV_ERR_DEVICE: return "page id out of range";
         case DASHKV_ERR_NO_DEVICE: return "no CUDA device";
+        case DASHKV_ERR_TIMEOUT: return "in-kernel wait timed out";
     }
     return "unknown status";
 }
@@ -337,8 +410,21 @@ dashkv_status dashkv_create(const dashkv_config *cfg, dashkv_ctx **out) {
     c->cfg = *cfg;
     c->device = dev;
     c->sm_count = sms;
+    int coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) coop = 0;
+    c->coop = coop;
+    c->fused_pdl = 1;
+    c->force_two_kernel = (cfg->flags & DASHKV_FLAG_TWO_KERNEL_SELECT) != 0;
     build_rbits(cfg->seed, cfg->bits, cfg->head_dim, &c->R);
     set_attrs();
+    const bool layout_ok =
+        cfg->head_dim == 64
+            ? (cfg->bits == 32 ? score_layout_ok<32, 64>() : cfg->bits == 64 ? score_layout_ok<64, 64>() : score_layout_ok<128, 64>())
+            : (cfg->bits == 32 ? score_layout_ok<32, 128>() : cfg->bits == 64 ? score_layout_ok<64, 128>() : score_layout_ok<128, 128>());
+    if (!layout_ok) {
+        free(c);
+        return DASHKV_ERR_UNSUPPORTED;
+    }
     if (cudaGetLastError() != cudaSuccess) {
         free(c);
         return DASHKV_ERR_CUDA;
@@ -401,15 +487,35 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     ws.scores_out = scores;
     ws.ld_out = cap;
     ws.cand = reinterpret_cast<int32_t *>(w + L.cand);
+    ws.ckey = reinterpret_cast<uint32_t *>(w + L.ckey);
     ws.hist = reinterpret_cast<uint32_t *>(w + L.hist);
     ws.state = reinterpret_cast<SelState *>(w + L.state);
     ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive);
     ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
+    ws.bar = reinterpret_cast<uint32_t *>(w + L.bar);
+    ws.inbin_n = reinterpret_cast<uint32_t *>(w + L.inbin_n);
+    ws.inbin = reinterpret_cast<uint4 *>(w + L.inbin);
+    ws.def_mid = reinterpret_cast<int32_t *>(w + L.def_mid);
     const KV k = make_kv(ctx, kv);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int nscore = sel_ctas(ctx, cap, 1);    // score kernel: one 1024-thread CTA per SM
     const int ncollect = sel_ctas(ctx, cap, 2);  // collect kernel: two 512-thread CTAs per SM
     Tracer tr(ctx, st);
+    auto copy_scores = [&]() {
+        if (!scores) return;
+        const int gx = (int)((cap + 255) / 256 < 64 ? (cap + 255) / 256 : 64);
+        launch_pdl(copy_scores_kernel, dim3(gx > 0 ? gx : 1, BH), dim3(256), 0, st,
+                   (const float *)ws.scores, ws.ld, scores, ws.ld_out, seq_lens, ctx->cfg.num_kv_heads, cap);
+    };
+    if (use_fused(ctx, cap)) {
+        // every CTA of the grid fits at once (one per SM): fused selection
+        tr.before();
+        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nscore, sel_idx, sel_cnt, st);
+        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nscore, sel_idx, sel_cnt, st);
+        tr.after();
+        copy_scores();
+        return launch_status();
+    }
     tr.before();
     if (ctx->cfg.head_dim == 64) launch_score_d<64>(ctx, k, q, seq_lens, ws, nscore, st);
     else launch_score_d<128>(ctx, k, q, seq_lens, ws, nscore, st);
@@ -419,6 +525,7 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     launch_pdl(collect_kernel, dim3(ncollect, BH), dim3(kSelThreads), sizeof(CollectSmem), st, ws, ncollect,
                ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
     tr.after();
+    copy_scores();
     return launch_status();
 }
 
@@ -445,6 +552,11 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
     return launch_status();
 }
 
+int32_t dashkv_select_kernels(const dashkv_ctx *ctx, int64_t max_tokens) {
+    if (!ctx) return 0;
+    return use_fused(ctx, max_tokens) ? 1 : 2;
+}
+
 dashkv_status dashkv_set_trace(dashkv_ctx *ctx, void **events, int32_t n_events) {
     if (!ctx || n_events < 0 || (events && n_events < 2)) return DASHKV_ERR_INVALID_ARG;
     ctx->trace = events;
@@ -458,6 +570,7 @@ dashkv_status dashkv_get_error(void *stream) {
     unsigned w = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return DASHKV_ERR_CUDA;
     if (w && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (w & kErrTimeout) return DASHKV_ERR_TIMEOUT;
     if (w & kErrPage) return DASHKV_ERR_DEVICE;
     if (w & kErrCapacity) return DASHKV_ERR_CAPACITY;
     return DASHKV_OK;

@@ -63,6 +63,12 @@ struct SelWS {
     SelState *state;     // [BH]
     uint32_t *arrive;    // [2][BH]            zero between calls
     int32_t *seg_cnt;    // [BH][kMaxSelCtas]
+    uint32_t *ckey;      // [BH][ld] order keys of the segment entries (fused selection)
+    // fused selection only
+    uint32_t *bar;       // [BH][2] barrier (arrivals, generation); arrivals zero between calls
+    uint32_t *inbin_n;   // [BH]   in-bin list length (cleared at barrier 1)
+    uint4 *inbin;        // [BH][kInbinMax] (order key, token, cta, 0)
+    int32_t *def_mid;    // [BH][kMaxSelCtas]
 };
 
 // Monotone map of a score to one of kBins bins (x in [0, 1] over [-A, A]).
@@ -120,6 +126,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
 // Lane l reads its token's bytes rotated by rho = l % T, so at each step the
 // 32 lanes touch 32 distinct banks.
 constexpr int kScoreThreads = 1024;
+constexpr int kScoreThreadsConst = kScoreThreads;
 
 template <int BITS>
 struct ScoreShape {
@@ -128,9 +135,12 @@ struct ScoreShape {
     static constexpr int NW = BITS / 32;       // 32-bit code words per token
     static constexpr uint32_t LUT_BYTES = 256 * 256;
     static constexpr uint32_t LOW_BYTES = kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;  // hist + scratch
-    // dynamic smem: low region, then the LUT at the next 64 KB boundary
-    static constexpr size_t SMEM = 2 * 65536 + LOW_BYTES;
     using Vec = typename std::conditional<BITS == 128, uint4, uint2>::type;  // one token's code
+    // per-thread cp.async ring of upcoming codes (one token per thread per stage)
+    static constexpr int STAGES = 5;
+    static constexpr uint32_t RING_BYTES = STAGES * kScoreThreadsConst * sizeof(Vec);
+    // dynamic smem: low region, the LUT at the next 64 KB boundary, then the ring
+    static constexpr size_t SMEM = 2 * 65536 + RING_BYTES;
 };
 
 // Rotate the token's code bytes by rho (byte r of the result = byte (r + rho)
@@ -181,15 +191,26 @@ __device__ __forceinline__ float lut_score(const uint32_t (&w)[BITS / 32], const
     return (s0 + s1) + 0.0f;  // + 0 turns a -0 into +0
 }
 
-template <int BITS, int D>
-__global__ void __launch_bounds__(kScoreThreads, 1)
-score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
-                  const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int nctas) {
+
+// ---------------------------------------------------------------------------
+// Score phase shared by the fused and the two-kernel selection: LUT prologue
+// (depends on q only, so it runs before waiting on the preceding kernel), then
+// stream this CTA's codes, write the fp32 scores and build the CTA histogram
+// in shared memory.  Ends with the histogram complete (after a barrier).
+struct ScoreOut {
+    int64_t n, t0, t1;
+    float inv2A;
+    unsigned char *lut;  // 64 KB LUT region, free for reuse once scoring is done
+};
+
+template <int BITS, int D, bool PAGED>
+__device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
+                                                const int32_t *__restrict__ seq_lens, const RBits &R,
+                                                const SelWS &ws, int nctas, unsigned char *smem) {
     using S = ScoreShape<BITS>;
     using Vec = typename S::Vec;
     constexpr int T = S::T, NW = S::NW;
     constexpr int NWARPS = kScoreThreads / 32;
-    extern __shared__ __align__(1024) unsigned char smem[];
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem);                  // [kBins]
     float *qsum = reinterpret_cast<float *>(hist + kBins);                // [D]
     float *Qp = qsum + kMaxDim;                                           // [BITS]
@@ -200,10 +221,7 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.y, b = bh / kv.Hkv, h = bh % kv.Hkv;
-    if (lut_s + 65536u > smem_s + (uint32_t)S::SMEM) {  // cannot happen with a small static region
-        if (tid == 0) raise_error(kErrCapacity);
-        return;
-    }
+
     for (int i = tid; i < kBins; i += kScoreThreads) hist[i] = 0;
     for (int i = tid; i < D; i += kScoreThreads) {
         const __nv_bfloat16 *qh = q + ((int64_t)b * Hq + (int64_t)h * G) * D + i;
@@ -247,13 +265,16 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         }
     }
     __syncthreads();
-    const float inv2A = red[0];
+    ScoreOut o;
+    o.inv2A = red[0];
+    o.lut = lut;
     // everything above depends on q only; codes and lengths come from the append
     griddep_wait();
-    const int64_t n = clamp_len(kv, seq_lens, b);
+    o.n = clamp_len(kv, seq_lens, b);
+    cta_range(o.n, blockIdx.x, nctas, o.t0, o.t1);
+    const int64_t t0 = o.t0, t1 = o.t1;
+    const float inv2A = o.inv2A;
 
-    int64_t t0, t1;
-    cta_range(n, blockIdx.x, nctas, t0, t1);
     const int rho = lane % T, copy = lane / T;
     const bool rot8 = (rho & 8) != 0, rot4 = (rho & 4) != 0;
     const uint32_t rot_sh = 8u * (uint32_t)(rho & 3);
@@ -261,48 +282,119 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
 #pragma unroll
     for (int r = 0; r < T; ++r) off[r] = lut_s | 4u * (uint32_t)(copy * T + (rho + r) % T);
 
-    float *srow = ws.scores + (int64_t)bh * ws.ld;
-    float *urow = ws.scores_out ? ws.scores_out + (int64_t)bh * ws.ld_out : nullptr;
     const int nloc = (int)(t1 - t0);  // tokens of this CTA (< 2^31)
-    // lane's code pointer for local token index i (dense layout; paged via page table)
-    const Vec *dense = reinterpret_cast<const Vec *>(kv.codes) + ((int64_t)bh * kv.n_cap + t0);
-    auto fetch = [&](int i) -> Vec {  // i: local index of this lane's token (i < nloc)
-        if (!kv.page_size) return __ldcs(dense + i);
-        const int64_t c = kv.code(b, h, t0 + i);
-        return c >= 0 ? __ldcs(reinterpret_cast<const Vec *>(kv.codes + c)) : Vec{};
-    };
 
-    constexpr int STEP = NWARPS * 32;
-    int i = warp * 32 + lane;
-    Vec nxt0 = i < nloc ? fetch(i) : Vec{};
-    Vec nxt1 = i + STEP < nloc ? fetch(i + STEP) : Vec{};
-    for (int g = warp * 32; g < nloc; g += 2 * STEP, i += 2 * STEP) {
-        const Vec cur0 = nxt0, cur1 = nxt1;
-        if (i + 2 * STEP < nloc) nxt0 = fetch(i + 2 * STEP);
-        if (i + 3 * STEP < nloc) nxt1 = fetch(i + 3 * STEP);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int iu = i + u * STEP;
-            uint32_t w[NW];
-            unpack_code<BITS>(u ? cur1 : cur0, w);
-            rotate_bytes<NW>(w, rot8, rot4, rot_sh);
-            const float s = lut_score<BITS>(w, off);
-            if (iu < nloc) {
-                srow[t0 + iu] = s;
-                if (urow) urow[t0 + iu] = s;
-                atomicAdd(&hist[score_bin(s, inv2A)], 1u);
+    // Each thread streams tokens tid, tid + NT, ... through its own slots of a
+    // STAGES-deep cp.async ring: it only ever reads codes it copied itself, so
+    // the ring needs no barriers, and STAGES - 1 codes per thread stay in flight.
+    constexpr int NT = kScoreThreads;
+    constexpr int STAGES = S::STAGES;
+    constexpr int VB = (int)sizeof(Vec);
+    const uint32_t ring_s = lut_s + 65536u + (uint32_t)tid * VB;  // this thread's slot of stage 0
+    const unsigned char *ring = lut + 65536 + tid * VB;
+    const Vec *dense = reinterpret_cast<const Vec *>(kv.codes) + ((int64_t)bh * kv.n_cap + t0);
+    float *srow = ws.scores + (int64_t)bh * ws.ld + t0;
+    auto issue = [&](int k) {  // copy the code of token k * NT + tid into stage k % STAGES
+        const int i = k * NT + tid;
+        const void *src = dense;
+        int bytes = 0;
+        if (i < nloc) {
+            if (!PAGED) {
+                src = dense + i;
+                bytes = VB;
+            } else {
+                const int64_t c = kv.code(b, h, t0 + i);
+                if (c >= 0) { src = kv.codes + c; bytes = VB; }
             }
         }
+        const uint32_t dst = ring_s + (uint32_t)((k % STAGES) * NT * VB);
+        if (VB == 16)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+        else
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const int nk = (nloc + NT - 1) / NT;  // stages this CTA streams
+#pragma unroll
+    for (int k = 0; k < STAGES - 1; ++k) issue(k);
+    for (int k = 0; k < nk; ++k) {
+        issue(k + STAGES - 1);
+        asm volatile("cp.async.wait_group %0;" ::"n"(STAGES - 1) : "memory");
+        const int i = k * NT + tid;
+        if (i < nloc) {
+            const Vec code = *reinterpret_cast<const Vec *>(ring + (k % STAGES) * NT * VB);
+            uint32_t w[NW];
+            unpack_code<BITS>(code, w);
+            rotate_bytes<NW>(w, rot8, rot4, rot_sh);
+            const float s = lut_score<BITS>(w, off);
+            srow[i] = s;
+            atomicAdd(&hist[score_bin(s, inv2A)], 1u);
+        }
     }
-    griddep_trigger();
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
+    return o;
+}
+
+// Optional user copy of the scores: entries [0, seq_lens[b]) of every row.
+__global__ void copy_scores_kernel(const float *__restrict__ src, int64_t ld, float *__restrict__ dst, int64_t ld_out,
+                                   const int32_t *__restrict__ seq_lens, int Hkv, int64_t cap) {
+    griddep_wait();
+    const int bh = blockIdx.y;
+    int64_t n = seq_lens[bh / Hkv];
+    if (n > cap) n = cap;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x)
+        dst[(int64_t)bh * ld_out + t] = src[(int64_t)bh * ld + t];
+}
+
+// Threshold bin from a complete histogram in shared memory: the bin T1 that
+// holds the kk-th largest score, the count above it and in it.  All threads
+// call; the results land in out[0..2] (shared).  Requires 0 < kk < total.
+template <int NT>
+__device__ __forceinline__ void threshold_bin(const uint32_t *hist, int64_t kk, int *s_warp, int *out) {
+    constexpr int PER = kBins / NT;  // bins per thread, thread 0 owns the top
+    const int tid = threadIdx.x;
+    int local = 0;
+    const int top = kBins - 1 - tid * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) local += hist[top - e];
+    int total;
+    const int before = block_excl_scan<NT>(local, s_warp, &total);
+    if (before < kk && before + local >= kk) {
+        int run = before;
+        for (int e = 0; e < PER; ++e) {
+            const int bin = top - e;
+            if (run + (int)hist[bin] >= kk) {
+                out[0] = bin;
+                out[1] = run;
+                out[2] = (int)hist[bin];
+                break;
+            }
+            run += hist[bin];
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Two-kernel selection, first kernel: score + histogram; the last CTA of a
+// (b, h) (arrival counter, no waiting) locates the threshold bin.
+template <int BITS, int D, bool PAGED>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
+                  const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int nctas) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ int s_last;
+    __shared__ int s_warp[32];
+    __shared__ int s_thr[4];
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.y;
+    const ScoreOut so = score_phase<BITS, D, PAGED>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
+    griddep_trigger();
     uint32_t *ghist = ws.hist + (int64_t)bh * kBins;
     for (int k = tid; k < kBins; k += kScoreThreads)
         if (hist[k]) atomicAdd(ghist + k, hist[k]);
-
-    // ---- last CTA of this (b, h): locate the threshold bin
-    __shared__ int s_last;
-    __shared__ int s_warp[32];
     __threadfence();
     __syncthreads();
     if (tid == 0) s_last = atomicAdd(ws.arrive + bh, 1u) == (unsigned)(nctas - 1);
@@ -313,47 +405,29 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         hist[k] = __ldcg(ghist + k);
         ghist[k] = 0;
     }
+    if (tid == 0) { s_thr[0] = kBins; s_thr[1] = 0; s_thr[2] = 0; }
     __syncthreads();
+    const int64_t n = so.n;
     const int64_t kk = topk < n ? topk : n;
-    constexpr int PER = kBins / kScoreThreads;  // bins per thread, thread 0 owns the top
-    int local = 0;
-    const int top = kBins - 1 - tid * PER;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) local += hist[top - e];
-    int total;
-    const int before = block_excl_scan<kScoreThreads>(local, s_warp, &total);
+    if (n > 0 && kk < n) threshold_bin<kScoreThreads>(hist, kk, s_warp, s_thr);
     if (tid == 0) {
         SelState st;
-        st.inv2A = inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
-        st.T1 = kBins; st.above1 = 0; st.cnt_T1 = 0;
+        st.inv2A = so.inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
+        st.T1 = s_thr[0]; st.above1 = s_thr[1]; st.cnt_T1 = s_thr[2];
         st.flags = n == 0 ? kStateEmpty : (kk >= n ? kStateAll : kStateNormal);
         ws.state[bh] = st;
+        ws.arrive[bh] = 0;
     }
-    __syncthreads();
-    if (n > 0 && kk < n && before < kk && before + local >= kk) {
-        int run = before;
-        for (int e = 0; e < PER; ++e) {
-            const int bin = top - e;
-            if (run + (int)hist[bin] >= kk) {
-                ws.state[bh].T1 = bin;
-                ws.state[bh].above1 = run;
-                ws.state[bh].cnt_T1 = (int)hist[bin];
-                break;
-            }
-            run += hist[bin];
-        }
-    }
-    if (tid == 0) ws.arrive[bh] = 0;
 }
 
 // ---------------------------------------------------------------------------
-// Collect + resolve.
+// Resolve + emit (one CTA of NT threads per (b, h)).
 //
 // The candidate list of a (b, h) is the concatenation, in CTA order, of every
-// CTA's segment (tokens of its range with bin >= T1, ascending), so the list
-// is in ascending token order.  The resolver addresses it through a ListView:
-// either a shared-memory copy (tokens + order keys) or, when the list is too
-// long for that, the segments in global memory.
+// scoring CTA's segment (tokens of its range with bin >= T1, ascending), so the
+// list is in ascending token order.  The resolver addresses it through a
+// ListView: either a shared-memory copy (tokens + order keys) or, when the
+// list is too long for that, the segments in global memory.
 struct ListView {
     const int32_t *s_t;        // shared copy (or null)
     const uint32_t *s_key;
@@ -384,12 +458,12 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// For every list element in order, f(e, t, key) -> bool; returns, per thread,
-// the exclusive rank of its first kept element and the block total.  Each thread
-// owns a contiguous run of elements so one block scan orders everything.
-template <class Pred, class Emit>
+// For every list element in order, pred(t, key) -> keep; emit(rank, t) for the
+// kept ones in list order.  Each thread owns a contiguous run of elements so one
+// block scan orders everything.  Returns the number kept.
+template <int NT, class Pred, class Emit>
 __device__ __forceinline__ int ordered_pass(const ListView &L, int M, int *s_warp, Pred &&pred, Emit &&emit) {
-    const int per = (M + kSelThreads - 1) / kSelThreads;
+    const int per = (M + NT - 1) / NT;
     const int e0 = threadIdx.x * per;
     const int e1 = min(M, e0 + per);
     int cnt = 0;
@@ -399,7 +473,7 @@ __device__ __forceinline__ int ordered_pass(const ListView &L, int M, int *s_war
         cnt += pred(t, key) ? 1 : 0;
     }
     int total;
-    int r = block_excl_scan(cnt, s_warp, &total);
+    int r = block_excl_scan<NT>(cnt, s_warp, &total);
     if (cnt)
         for (int e = e0; e < e1; ++e) {
             int t; uint32_t key;
@@ -409,9 +483,10 @@ __device__ __forceinline__ int ordered_pass(const ListView &L, int M, int *s_war
     return total;
 }
 
-struct CollectSmem {
-    int32_t list_t[kListSmem];
-    uint32_t list_key[kListSmem];
+template <int LIST_CAP>
+struct ResolveSmem {
+    int32_t list_t[LIST_CAP];
+    uint32_t list_key[LIST_CAP];
     uint32_t ck[kCandSmem];
     int32_t ci[kCandSmem];
     uint32_t h[2048];
@@ -421,74 +496,28 @@ struct CollectSmem {
     int last;
 };
 
-__global__ void __launch_bounds__(kSelThreads)
-collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    CollectSmem &sm = *reinterpret_cast<CollectSmem *>(smem_raw);
+// Exact threshold (Tkey, IT) inside bin T1, then the final ascending selection.
+// seg_cnt: the per-CTA segment sizes of this (b, h) in global memory.
+template <int NT, int LIST_CAP>
+__device__ void resolve_emit(const SelWS &ws, int bh, int nctas, const SelState &st, int S, int W, int cap_sel,
+                             int32_t *sel_idx, int32_t *sel_cnt, ResolveSmem<LIST_CAP> &sm) {
     const int tid = threadIdx.x;
-    const int bh = blockIdx.y;
-    griddep_wait();
-    const SelState st = ws.state[bh];
     const int n = st.n;
-    int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
+    const int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
     const float *srow = ws.scores + (int64_t)bh * ws.ld;
-
-    // ---- this CTA's segment: tokens of [t0, t1) with bin >= T1, ascending
-    int count = 0;
-    if (st.flags == kStateNormal) {
-        int64_t t0, t1;
-        cta_range(n, blockIdx.x, nctas, t0, t1);
-        for (int64_t base = t0; base < t1; base += kCollectTile) {
-            const int64_t tb = base + (int64_t)tid * 16;
-            uint32_t flags = 0;
-            if (tb + 16 <= t1) {
-                const float4 *p = reinterpret_cast<const float4 *>(srow + tb);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float4 x = __ldcg(p + v);
-                    flags |= (uint32_t)(score_bin(x.x, st.inv2A) >= st.T1) << (4 * v + 0);
-                    flags |= (uint32_t)(score_bin(x.y, st.inv2A) >= st.T1) << (4 * v + 1);
-                    flags |= (uint32_t)(score_bin(x.z, st.inv2A) >= st.T1) << (4 * v + 2);
-                    flags |= (uint32_t)(score_bin(x.w, st.inv2A) >= st.T1) << (4 * v + 3);
-                }
-            } else {
-                for (int j = 0; j < 16; ++j)
-                    if (tb + j < t1) flags |= (uint32_t)(score_bin(__ldcg(srow + tb + j), st.inv2A) >= st.T1) << j;
-            }
-            int tot;
-            int r = block_excl_scan(__popc(flags), sm.warp, &tot);
-            while (flags) {
-                const int j = __ffs(flags) - 1;
-                flags &= flags - 1;
-                cand[t0 + count + r++] = (int32_t)(tb + j);
-            }
-            count += tot;
-        }
-    }
-    griddep_trigger();
-    if (tid == 0) ws.seg_cnt[(int64_t)bh * kMaxSelCtas + blockIdx.x] = count;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sm.last = atomicAdd(ws.arrive + gridDim.y + bh, 1u) == (unsigned)(nctas - 1);
-    __syncthreads();
-    if (!sm.last) return;
-    __threadfence();
-
-    // ---- the last CTA of (b, h): list offsets, exact threshold, final selection
     {
         const int c = tid;
         const int v = c < nctas ? __ldcg(ws.seg_cnt + (int64_t)bh * kMaxSelCtas + c) : 0;
         int tot;
-        const int ex = block_excl_scan(v, sm.warp, &tot);
+        const int ex = block_excl_scan<NT>(v, sm.warp, &tot);
         if (c < nctas) sm.seg_off[c] = ex;
         if (c == 0) sm.seg_off[nctas] = tot;
     }
     __syncthreads();
     const int M = sm.seg_off[nctas];
     ListView L{nullptr, nullptr, cand, srow, sm.seg_off, nctas, n};
-    if (st.flags == kStateNormal && M <= kListSmem) {
-        // one parallel round over the whole list (each element finds its segment)
-        for (int e = tid; e < M; e += kSelThreads) {
+    if (st.flags == kStateNormal && M <= LIST_CAP) {
+        for (int e = tid; e < M; e += NT) {  // one parallel round over the whole list
             int t; uint32_t key;
             L.get(e, t, key);
             sm.list_t[e] = t;
@@ -510,7 +539,7 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
             // rank the in-bin candidates by (score desc, token asc)
             if (tid == 0) sm.misc[0] = 0;
             __syncthreads();
-            for (int e = tid; e < M; e += kSelThreads) {
+            for (int e = tid; e < M; e += NT) {
                 int t; uint32_t key;
                 L.get(e, t, key);
                 if (in_bin(key)) {
@@ -521,7 +550,7 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
             }
             __syncthreads();
             const int c1 = sm.misc[0];
-            for (int e = tid; e < c1; e += kSelThreads) {
+            for (int e = tid; e < c1; e += NT) {
                 const uint32_t ke = sm.ck[e];
                 const int ie = sm.ci[e];
                 int rank = 0;
@@ -543,9 +572,9 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
             for (int p = 0; p < 3; ++p) {
                 const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0);
                 const int nb = p == 2 ? 1024 : 2048;
-                for (int i = tid; i < 2048; i += kSelThreads) sm.h[i] = 0;
+                for (int i = tid; i < 2048; i += NT) sm.h[i] = 0;
                 __syncthreads();
-                for (int e = tid; e < M; e += kSelThreads) {
+                for (int e = tid; e < M; e += NT) {
                     int t; uint32_t key;
                     L.get(e, t, key);
                     if (in_bin(key) && (key & mask) == prefix) atomicAdd(&sm.h[(key >> sh) & (nb - 1)], 1u);
@@ -570,9 +599,9 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
             if (tid == 0) sm.misc[5] = 0x7fffffff;
             __syncthreads();
             const int want = need;
-            ordered_pass(L, M, sm.warp,
-                         [&](int t, uint32_t key) { return in_bin(key) && key == Tkey; },
-                         [&](int rank, int t) { if (rank + 1 == want) sm.misc[5] = t; });
+            ordered_pass<NT>(L, M, sm.warp,
+                             [&](int t, uint32_t key) { return in_bin(key) && key == Tkey; },
+                             [&](int rank, int t) { if (rank + 1 == want) sm.misc[5] = t; });
             __syncthreads();
             IT = sm.misc[5];
         }
@@ -584,14 +613,14 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
     const int w_beg = n - W > s_end ? n - W : s_end;  // window [w_beg, n)
     int pos;
     if (st.flags == kStateAll) {
-        for (int t = tid; t < n; t += kSelThreads) out[t] = t;
+        for (int t = tid; t < n; t += NT) out[t] = t;
         pos = n;
     } else if (st.flags == kStateEmpty) {
         pos = 0;
     } else {
-        for (int t = tid; t < s_end; t += kSelThreads) out[t] = t;
+        for (int t = tid; t < s_end; t += NT) out[t] = t;
         pos = s_end;
-        const int kept = ordered_pass(
+        const int kept = ordered_pass<NT>(
             L, M, sm.warp,
             [&](int t, uint32_t key) {
                 if (t < s_end || t >= w_beg) return false;
@@ -600,14 +629,318 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
             },
             [&](int rank, int t) { if (pos + rank < cap_sel) out[pos + rank] = t; });
         pos += kept;
-        for (int t = w_beg + tid; t < n; t += kSelThreads)
+        for (int t = w_beg + tid; t < n; t += NT)
             if (pos + (t - w_beg) < cap_sel) out[pos + (t - w_beg)] = t;
         pos += n - w_beg;
         if (pos > cap_sel) pos = cap_sel;  // unreachable when the threshold is consistent
     }
-    for (int r = pos + tid; r < cap_sel; r += kSelThreads) out[r] = -1;
+    for (int r = pos + tid; r < cap_sel; r += NT) out[r] = -1;
     if (tid == 0) sel_cnt[bh] = pos;
+}
+
+// ---------------------------------------------------------------------------
+// Two-kernel selection, second kernel: ordered compaction of each CTA's tokens
+// with bin >= T1 into its segment; the last CTA of a (b, h) resolves and emits.
+using CollectSmem = ResolveSmem<kListSmem>;
+
+__global__ void __launch_bounds__(kSelThreads)
+collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    CollectSmem &sm = *reinterpret_cast<CollectSmem *>(smem_raw);
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.y;
+    griddep_wait();
+    const SelState st = ws.state[bh];
+    const int n = st.n;
+    int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
+    const float *srow = ws.scores + (int64_t)bh * ws.ld;
+
+    int count = 0;
+    if (st.flags == kStateNormal) {
+        int64_t t0, t1;
+        cta_range(n, blockIdx.x, nctas, t0, t1);
+        for (int64_t base = t0; base < t1; base += kCollectTile) {
+            const int64_t tb = base + (int64_t)tid * 16;
+            uint32_t flags = 0;
+            if (tb + 16 <= t1) {
+                const float4 *p = reinterpret_cast<const float4 *>(srow + tb);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 x = __ldcg(p + v);
+                    flags |= (uint32_t)(score_bin(x.x, st.inv2A) >= st.T1) << (4 * v + 0);
+                    flags |= (uint32_t)(score_bin(x.y, st.inv2A) >= st.T1) << (4 * v + 1);
+                    flags |= (uint32_t)(score_bin(x.z, st.inv2A) >= st.T1) << (4 * v + 2);
+                    flags |= (uint32_t)(score_bin(x.w, st.inv2A) >= st.T1) << (4 * v + 3);
+                }
+            } else {
+                for (int j = 0; j < 16; ++j)
+                    if (tb + j < t1) flags |= (uint32_t)(score_bin(__ldcg(srow + tb + j), st.inv2A) >= st.T1) << j;
+            }
+            int tot;
+            int r = block_excl_scan<kSelThreads>(__popc(flags), sm.warp, &tot);
+            while (flags) {
+                const int j = __ffs(flags) - 1;
+                flags &= flags - 1;
+                cand[t0 + count + r++] = (int32_t)(tb + j);
+            }
+            count += tot;
+        }
+    }
+    griddep_trigger();
+    if (tid == 0) ws.seg_cnt[(int64_t)bh * kMaxSelCtas + blockIdx.x] = count;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sm.last = atomicAdd(ws.arrive + gridDim.y + bh, 1u) == (unsigned)(nctas - 1);
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
+    resolve_emit<kSelThreads, kListSmem>(ws, bh, nctas, st, S, W, cap_sel, sel_idx, sel_cnt, sm);
     if (tid == 0) ws.arrive[gridDim.y + bh] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Fused selection: one kernel, all CTAs of a (b, h) co-resident (cooperative
+// launch, at most one CTA per SM), two barriers per (b, h).
+//   stream + histogram -> barrier 1 -> every CTA finds T1 from the summed
+//   histogram, compacts its own tokens with bin >= T1 into its segment, counts
+//   the definite ones (bin > T1) in the middle range and appends its few in-bin
+//   tokens to a shared list -> barrier 2 -> every CTA ranks the in-bin list
+//   (score desc, token asc), derives every CTA's count of selected middle
+//   tokens, hence its own output offset, and writes its tokens in order; CTA 0
+//   writes the sinks, the window, the padding and the count.
+// A bin with more than kInbinMax tokens (heavy ties) takes the exact resolver
+// of the two-kernel path, run by CTA 0 after barrier 2.
+constexpr int kInbinMax = 1024;
+constexpr unsigned kSpinLimit = 1u << 24;  // ~1.7 s of 100 ns naps: then report a timeout
+
+// Barrier among the `nparts` CTAs of one (b, h): bar[0] counts arrivals, bar[1]
+// is the generation the last arrival advances.  Bounded wait: a CTA that gives
+// up records kErrTimeout and carries on.  reset: a word the last arrival
+// clears before releasing the others.
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void bh_barrier(uint32_t *bar, unsigned nparts, uint32_t *reset) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t g = ld_acquire(bar + 1);
+        __threadfence();
+        if (atomicAdd(bar, 1u) == nparts - 1) {
+            bar[0] = 0;
+            if (reset) *reset = 0;
+            __threadfence();
+            atomicAdd(bar + 1, 1u);
+        } else {
+            unsigned spins = 0;
+            while (ld_acquire(bar + 1) == g) {
+                if (++spins > kSpinLimit) {
+                    raise_error(kErrTimeout);
+                    break;
+                }
+                __nanosleep(100);
+            }
+            __threadfence();
+        }
+    }
+    __syncthreads();
+}
+
+template <int BITS, int D, bool PAGED>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
+                    const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int nctas, int S,
+                    int W, int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
+    constexpr int NT = kScoreThreads;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ int s_warp[32];
+    __shared__ int s_thr[4];
+    __shared__ int s_misc[4];
+    __shared__ int s_mid[kMaxSelCtas];
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.y, cta = blockIdx.x;
+    const ScoreOut so = score_phase<BITS, D, PAGED>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *ghist = ws.hist + (int64_t)bh * kBins;
+    for (int k = tid; k < kBins; k += NT)
+        if (hist[k]) atomicAdd(ghist + k, hist[k]);
+    griddep_trigger();
+    bh_barrier(ws.bar + 2 * bh, nctas, ws.inbin_n + bh);  // (1): histogram complete
+
+    const int64_t n = so.n, t0 = so.t0, t1 = so.t1;
+    const int64_t kk = topk < n ? topk : n;
+    const bool normal = n > 0 && kk < n;
+    if (tid == 0) { s_thr[0] = kBins; s_thr[1] = 0; s_thr[2] = 0; }
+    if (normal) {
+        for (int k = tid; k < kBins; k += NT) hist[k] = __ldcg(ghist + k);
+        __syncthreads();
+        threshold_bin<NT>(hist, kk, s_warp, s_thr);
+    }
+    __syncthreads();
+    const int T1 = s_thr[0], above1 = s_thr[1], cnt_T1 = s_thr[2];
+    const bool fallback = normal && cnt_T1 > kInbinMax;
+    const int s_end = (int)(S < n ? S : n);
+    const int w_beg = (int)(n - W > s_end ? n - W : s_end);
+    const float inv2A = so.inv2A;
+    int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
+    const float *srow = ws.scores + (int64_t)bh * ws.ld;
+
+    // ---- own range: segment of tokens with bin >= T1 (ascending), definite
+    // middle count, in-bin tokens appended to the shared list
+    uint32_t *ckey = ws.ckey + (int64_t)bh * ws.ld;
+    int seg = 0, defmid = 0;
+    if (normal) {
+        for (int64_t base = t0; base < t1; base += (int64_t)NT * 32) {
+            const int64_t tb = base + (int64_t)tid * 32;
+            float x[32];
+            if (tb + 32 <= t1) {
+                const float4 *p = reinterpret_cast<const float4 *>(srow + tb);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 f = __ldcg(p + v);
+                    x[4 * v] = f.x; x[4 * v + 1] = f.y; x[4 * v + 2] = f.z; x[4 * v + 3] = f.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = tb + e < t1 ? __ldcg(srow + tb + e) : -INFINITY;
+            }
+            uint32_t flags = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int bin = tb + e < t1 ? score_bin(x[e], inv2A) : -1;
+                if (bin >= T1) flags |= 1u << e;
+                if (bin > T1) defmid += (tb + e >= s_end && tb + e < w_beg);
+            }
+            int tot;
+            int r = block_excl_scan<NT>(__popc(flags), s_warp, &tot);
+            uint32_t f = flags;
+            while (f) {
+                const int j = __ffs(f) - 1;
+                f &= f - 1;
+                const int64_t t = tb + j;
+                const float sj = srow[t];  // L1 hit: this thread just read it
+                const uint32_t key = float_key(sj);
+                cand[t0 + seg + r] = (int32_t)t;
+                ckey[t0 + seg + r] = key;
+                ++r;
+                if (!fallback && score_bin(sj, inv2A) == T1) {
+                    const unsigned slot = atomicAdd(ws.inbin_n + bh, 1u);
+                    if (slot < (unsigned)kInbinMax)
+                        ws.inbin[(int64_t)bh * kInbinMax + slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, 0u);
+                }
+            }
+            seg += tot;
+        }
+        int tot;
+        block_excl_scan<NT>(defmid, s_warp, &tot);
+        defmid = tot;
+    }
+    if (tid == 0) {
+        ws.seg_cnt[(int64_t)bh * kMaxSelCtas + cta] = seg;
+        ws.def_mid[(int64_t)bh * kMaxSelCtas + cta] = defmid;
+    }
+    bh_barrier(ws.bar + 2 * bh, nctas, nullptr);  // (2): segments, counts, in-bin list complete
+
+    int32_t *out = sel_idx + (int64_t)bh * cap_sel;
+    if (!normal || fallback) {
+        if (cta != 0) return;
+        for (int k = tid; k < kBins; k += NT) ghist[k] = 0;
+        SelState st;
+        st.T1 = T1; st.above1 = above1; st.cnt_T1 = cnt_T1;
+        st.flags = n == 0 ? kStateEmpty : (normal ? kStateNormal : kStateAll);
+        st.inv2A = inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
+        resolve_emit<NT, 4096>(ws, bh, nctas, st, S, W, cap_sel, sel_idx, sel_cnt,
+                               *reinterpret_cast<ResolveSmem<4096> *>(so.lut));
+        return;
+    }
+
+    // ---- fast path: rank the in-bin list (every CTA, redundantly; it is short)
+    uint4 *s_inb = reinterpret_cast<uint4 *>(so.lut);  // reuses the LUT region
+    const int c1 = cnt_T1;                            // == number of list entries
+    for (int e = tid; e < c1; e += NT) s_inb[e] = __ldcg(ws.inbin + (int64_t)bh * kInbinMax + e);
+    for (int c = tid; c < nctas; c += NT) s_mid[c] = __ldcg(ws.def_mid + (int64_t)bh * kMaxSelCtas + c);
+    if (tid == 0) { s_misc[0] = 0; s_misc[1] = 0x7fffffff; }
+    __syncthreads();
+    const int need1 = (int)kk - above1;  // 1 <= need1 <= c1
+    if (need1 < c1) {
+        for (int e = tid; e < c1; e += NT) {
+            const uint32_t ke = s_inb[e].x, ie = s_inb[e].y;
+            int rank = 0;
+            for (int f = 0; f < c1; ++f) {
+                const uint32_t kf = s_inb[f].x;
+                rank += (kf > ke) || (kf == ke && s_inb[f].y < ie);
+            }
+            if (rank == need1 - 1) { s_misc[0] = (int)ke; s_misc[1] = (int)ie; }
+        }
+        __syncthreads();
+    }
+    const uint32_t Tkey = (uint32_t)s_misc[0];
+    const int IT = s_misc[1];
+    auto keep_inbin = [&](uint32_t key, int t) { return key > Tkey || (key == Tkey && t <= IT); };
+    // selected in-bin tokens in the middle range, credited to their CTA
+    for (int e = tid; e < c1; e += NT) {
+        const int t = (int)s_inb[e].y;
+        if (t >= s_end && t < w_beg && keep_inbin(s_inb[e].x, t)) atomicAdd(&s_mid[s_inb[e].z], 1);
+    }
+    __syncthreads();
+    int total_mid;
+    const int before = block_excl_scan<NT>(tid < nctas ? s_mid[tid] : 0, s_warp, &total_mid);
+    if (tid == cta) s_misc[2] = before;
+    __syncthreads();
+    const int obase = s_end + s_misc[2];
+
+    // own segment: keep bin > T1, or in-bin under the (Tkey, IT) rule; middle only
+    {
+        const int per = (seg + NT - 1) / NT;
+        const int e0 = tid * per, e1 = min(seg, e0 + per);
+        constexpr int MAXPER = 8;  // elements held in registers per thread (else re-read)
+        int tt[MAXPER];
+        uint32_t kk2[MAXPER];
+        auto keep = [&](int t, uint32_t key) {
+            if (t < s_end || t >= w_beg) return false;
+            return score_bin(key_to_float(key), inv2A) > T1 || keep_inbin(key, t);
+        };
+#pragma unroll
+        for (int j = 0; j < MAXPER; ++j) {
+            const int e = e0 + j;
+            tt[j] = e < e1 ? __ldcg(cand + t0 + e) : -1;
+            kk2[j] = e < e1 ? __ldcg(ckey + t0 + e) : 0u;
+        }
+        int cnt = 0;
+#pragma unroll
+        for (int j = 0; j < MAXPER; ++j) cnt += (e0 + j < e1) && keep(tt[j], kk2[j]);
+        for (int e = e0 + MAXPER; e < e1; ++e) cnt += keep(__ldcg(cand + t0 + e), __ldcg(ckey + t0 + e));
+        int tot;
+        int r = block_excl_scan<NT>(cnt, s_warp, &tot);
+        if (cnt) {
+#pragma unroll
+            for (int j = 0; j < MAXPER; ++j)
+                if (e0 + j < e1 && keep(tt[j], kk2[j])) {
+                    if (obase + r < cap_sel) out[obase + r] = tt[j];
+                    ++r;
+                }
+            for (int e = e0 + MAXPER; e < e1; ++e) {
+                const int t = __ldcg(cand + t0 + e);
+                if (keep(t, __ldcg(ckey + t0 + e))) {
+                    if (obase + r < cap_sel) out[obase + r] = t;
+                    ++r;
+                }
+            }
+        }
+    }
+    if (cta == 0) {
+        for (int t = tid; t < s_end; t += NT) out[t] = t;
+        const int wpos = s_end + total_mid;
+        for (int t = w_beg + tid; t < n; t += NT)
+            if (wpos + (t - w_beg) < cap_sel) out[wpos + (t - w_beg)] = t;
+        int total = wpos + (int)(n - w_beg);
+        if (total > cap_sel) total = cap_sel;
+        for (int r = total + tid; r < cap_sel; r += NT) out[r] = -1;
+        if (tid == 0) sel_cnt[bh] = total;
+        for (int k = tid; k < kBins; k += NT) ghist[k] = 0;
+    }
 }
 
 }  // namespace dkv

@@ -20,11 +20,14 @@ LIB_PATH = os.path.join(_HERE, "libdashkv.so")
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace missing or too small",
     4: "sequence length beyond cache capacity", 5: "CUDA error", 6: "page id out of range", 7: "no CUDA device",
+    8: "in-kernel wait timed out",
 }
+
+FLAG_TWO_KERNEL_SELECT = 1
 
 SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_encode_keys",
            "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
-           "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_status_str")
+           "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str")
 
 
 class DashKVError(RuntimeError):
@@ -37,7 +40,7 @@ class Config(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("bits", ctypes.c_int32), ("topk", ctypes.c_int32),
                 ("sink", ctypes.c_int32), ("window", ctypes.c_int32), ("page_size", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+                ("flags", ctypes.c_int32), ("seed", ctypes.c_uint64)]
 
 
 class KVView(ctypes.Structure):
@@ -70,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.dashkv_get_error.argtypes = [P]
         L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
         L.dashkv_set_trace.argtypes = [P, P, I32]
+        L.dashkv_select_kernels.argtypes = [P, ctypes.c_int64]
+        L.dashkv_select_kernels.restype = I32
         L.dashkv_status_str.argtypes = [ctypes.c_int]
         L.dashkv_status_str.restype = ctypes.c_char_p
         for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode",
@@ -143,10 +148,12 @@ class DashKV:
     """One problem configuration (shapes, bits, k, S, W, layout, seed)."""
 
     def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, bits: int, topk: int,
-                 sink: int, window: int, page_size: int = 0, seed: int = 0x5EEDDA5B):
+                 sink: int, window: int, page_size: int = 0, seed: int = 0x5EEDDA5B,
+                 two_kernel_select: bool = False):
         if not torch.cuda.is_available():
             raise RuntimeError("hash_indexed_top_b200 needs a CUDA device (B200, sm_100a)")
-        self.cfg = Config(batch, num_q_heads, num_kv_heads, head_dim, bits, topk, sink, window, page_size, 0,
+        flags = FLAG_TWO_KERNEL_SELECT if two_kernel_select else 0
+        self.cfg = Config(batch, num_q_heads, num_kv_heads, head_dim, bits, topk, sink, window, page_size, flags,
                           seed & (2**64 - 1))
         self.sel_cap = topk + sink + window
         h = ctypes.c_void_p()
@@ -206,6 +213,10 @@ class DashKV:
                                                                   _ptr(sel_idx), _ptr(sel_cnt), _ptr(out),
                                                                   _ptr(lse), _ptr(ws), ws.numel(),
                                                                   _stream(stream)))
+
+    def select_kernels(self, max_tokens: int) -> int:
+        """1 when dashkv_select runs the fused kernel for this cache size, 2 for score + collect."""
+        return int(lib().dashkv_select_kernels(self._ctx, int(max_tokens)))
 
     def set_trace(self, events: Optional[list] = None) -> None:
         """Record torch.cuda.Event pairs around each kernel of the following calls (None: off)."""

@@ -188,6 +188,18 @@ def make_workload(cfg: Config, device="cpu", steps: Optional[int] = None, extra_
                     needle_pos=pos.to(dev))
 
 
-def flush_buffer(device, l2_bytes: int = 126 * 1024 * 1024) -> torch.Tensor:
-    """A buffer of twice the L2 size; writing it evicts everything cached."""
-    return torch.empty(int(2 * l2_bytes) // 4, dtype=torch.int32, device=device)
+class L2Flush:
+    """Cold-cache state between timed steps: write a buffer of twice the L2
+    size (evicting everything cached), then read a second, clean buffer of the
+    same size so that L2 holds only clean lines and no write-back of the flush
+    data lands inside the next timed step."""
+
+    def __init__(self, device, l2_bytes: int = 126 * 1024 * 1024):
+        n = int(2 * l2_bytes) // 4
+        self.dirty = torch.empty(n, dtype=torch.int32, device=device)
+        self.clean = torch.zeros(n, dtype=torch.int32, device=device)
+        self.sink = torch.empty((), dtype=torch.int64, device=device)
+
+    def __call__(self, i: int = 0) -> None:
+        self.dirty.fill_(i)
+        torch.sum(self.clean, out=self.sink)

@@ -73,8 +73,15 @@ typedef enum dashkv_status {
     DASHKV_ERR_CAPACITY = 4,     /* device error word: a sequence outgrew its cache   */
     DASHKV_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, sync, copy)   */
     DASHKV_ERR_DEVICE = 6,       /* device error word: bad page id in page_table      */
-    DASHKV_ERR_NO_DEVICE = 7     /* no usable CUDA device                             */
+    DASHKV_ERR_NO_DEVICE = 7,    /* no usable CUDA device                             */
+    DASHKV_ERR_TIMEOUT = 8       /* device error word: a bounded in-kernel wait gave up */
 } dashkv_status;
+
+/* Selection path.  By default dashkv_select runs one cooperative kernel
+ * whose CTAs (one per SM, so at most the SM count of them) synchronise per
+ * (sequence, kv head); when B * Hkv exceeds the SM count, or with this flag,
+ * it runs two ordinary kernels instead.  Both give identical results. */
+#define DASHKV_FLAG_TWO_KERNEL_SELECT 1
 
 /* Problem description.  Supported: head_dim in {64, 128}; bits in
  * {32, 64, 128}; num_q_heads = G * num_kv_heads with G in {1, 2, 4, 8};
@@ -90,7 +97,7 @@ typedef struct dashkv_config {
     int32_t sink;           /* S: first tokens always kept */
     int32_t window;         /* W: last tokens always kept  */
     int32_t page_size;      /* 0 = dense layout            */
-    int32_t reserved;       /* must be 0 */
+    int32_t flags;          /* DASHKV_FLAG_* bits; 0 = defaults */
     uint64_t seed;          /* hyperplane seed             */
 } dashkv_config;
 
@@ -158,13 +165,20 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    size_t workspace_bytes, void *stream);
 
 /* Synchronise `stream`, then read and clear the current device's error
- * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, or
- * DASHKV_ERR_CUDA when the stream reports an error. */
+ * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, DASHKV_ERR_TIMEOUT
+ * (the selection's CTAs could not all be resident together, e.g. because other
+ * work held the SMs; its output is then invalid), or DASHKV_ERR_CUDA when the
+ * stream reports an error. */
 dashkv_status dashkv_get_error(void *stream);
 
 /* The hyperplanes a context built with (seed, bits, d) uses, as int8 +1/-1
  * in host memory [bits][d]. */
 dashkv_status dashkv_hyperplanes(uint64_t seed, int32_t bits, int32_t head_dim, int8_t *host_out);
+
+/* Number of kernels dashkv_select launches for caches of `max_tokens` tokens
+ * per sequence: 1 (fused, cooperative) or 2 (score, then collect); 0 when ctx
+ * is NULL.  For profiling tools that trace individual kernels. */
+int32_t dashkv_select_kernels(const dashkv_ctx *ctx, int64_t max_tokens);
 
 /* Optional kernel tracing for profiling.  While `events` is non-NULL, every
  * following call on this context records events[2k] (a cudaEvent_t) on its

@@ -17,11 +17,11 @@ ATOL, RTOL = 1e-3, 8e-3
 
 
 class GpuRun:
-    def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED):
+    def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED, two_kernel: bool = False):
         self.cfg, self.w = cfg, w
         dev = w.K.device
         self.eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
-                             cfg.page_size if w.paged else 0, seed)
+                             cfg.page_size if w.paged else 0, seed, two_kernel_select=two_kernel)
         codes = dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged)
         self.cache = dk.KVCache(w.K, w.V, codes, w.page_table)
         self.seq = w.seq_lens.clone()
@@ -105,13 +105,14 @@ def compare_step(g: GpuRun, o: OracleRun, r: dict, what: str = "") -> dict:
     return dict(max_err=float(np.abs(out - r["out"])[fin].max()) if fin.any() else 0.0)
 
 
-def run_parity(cfg: W.Config, steps: int, device="cuda", w: W.Workload | None = None, mutate=None) -> list:
+def run_parity(cfg: W.Config, steps: int, device="cuda", w: W.Workload | None = None, mutate=None,
+               two_kernel: bool = False) -> list:
     """Encode, then `steps` x (append, select, decode) on GPU and oracle, comparing every step."""
     if w is None:
         w = W.make_workload(cfg, device="cpu", steps=steps)
     if mutate is not None:
         w = mutate(w)
-    g = GpuRun(cfg, w.to(device))
+    g = GpuRun(cfg, w.to(device), two_kernel=two_kernel)
     o = OracleRun(cfg, w)
     g.encode()
     diags = []

@@ -36,26 +36,33 @@ def built():
     build.build()
 
 
+PATHS = {"fused": False, "two_kernel": True}
+
+
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(CASES))
-def test_parity(name):
+def test_parity(name, path):
     cfg, steps = CASES[name]
-    diags = run_parity(cfg, steps)
+    diags = run_parity(cfg, steps, two_kernel=PATHS[path])
     assert len(diags) == steps
 
 
-def test_topk_covers_everything_is_dense_attention():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_topk_covers_everything_is_dense_attention(path):
     cfg = W.Config("allk", B=2, Hq=8, Hkv=2, d=128, N=700, n_min=300, bits=64, topk=5000, sink=4, window=16,
                    steps=1, needles=2, seed=80)
-    run_parity(cfg, 1)
+    run_parity(cfg, 1, two_kernel=PATHS[path])
 
 
-def test_sinks_and_window_overlap_short_sequences():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_sinks_and_window_overlap_short_sequences(path):
     cfg = W.Config("overlap", B=4, Hq=4, Hkv=1, d=64, N=60, n_min=1, bits=32, topk=5, sink=20, window=50,
                    steps=2, needles=0, seed=81)
-    run_parity(cfg, 2)
+    run_parity(cfg, 2, two_kernel=PATHS[path])
 
 
-def test_zero_query_all_scores_tie():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_zero_query_all_scores_tie(path):
     # q = 0 makes every score 0: one histogram bin holds every token, so the
     # exact threshold comes from the radix path and ties go to the lowest ids.
     cfg = W.Config("zeroq", B=1, Hq=4, Hkv=1, d=128, N=9000, bits=128, topk=700, sink=3, window=5,
@@ -64,10 +71,11 @@ def test_zero_query_all_scores_tie():
     def mutate(w):
         w.q.zero_()
         return w
-    run_parity(cfg, 1, mutate=mutate)
+    run_parity(cfg, 1, mutate=mutate, two_kernel=PATHS[path])
 
 
-def test_repeated_keys_heavy_ties():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_repeated_keys_heavy_ties(path):
     # only 3 distinct keys: huge tie groups at the threshold, in small-bin and radix regimes
     cfg = W.Config("ties", B=2, Hq=8, Hkv=2, d=128, N=5000, bits=64, topk=1500, sink=0, window=0,
                    steps=1, needles=0, seed=83)
@@ -77,16 +85,17 @@ def test_repeated_keys_heavy_ties():
         idx = torch.arange(w.K.shape[2]) % 3
         w.K[:] = pat[:, :, idx]
         return w
-    run_parity(cfg, 1, mutate=mutate)
+    run_parity(cfg, 1, mutate=mutate, two_kernel=PATHS[path])
 
 
-def test_empty_sequence_selects_nothing():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_empty_sequence_selects_nothing(path):
     cfg = W.Config("empty", B=3, Hq=4, Hkv=2, d=64, N=200, bits=64, topk=10, sink=2, window=2,
                    steps=0, needles=0, seed=84)
     w = W.make_workload(cfg, steps=0)
     w.seq_lens[1] = 0
     from pipeline import GpuRun, OracleRun, compare_step
-    g = GpuRun(cfg, w.to("cuda"))
+    g = GpuRun(cfg, w.to("cuda"), two_kernel=PATHS[path])
     o = OracleRun(cfg, w)
     g.encode()
     q = torch.zeros((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16)
@@ -100,11 +109,12 @@ def test_empty_sequence_selects_nothing():
     g.close()
 
 
-def test_repeat_calls_are_deterministic_and_leave_workspace_clean():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_repeat_calls_are_deterministic_and_leave_workspace_clean(path):
     cfg, _ = CASES["c128k_small"]
     w = W.make_workload(cfg, steps=1).to("cuda")
     from pipeline import GpuRun
-    g = GpuRun(cfg, w)
+    g = GpuRun(cfg, w, two_kernel=PATHS[path])
     g.encode()
     g.append(0)
     outs = []

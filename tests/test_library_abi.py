@@ -61,7 +61,7 @@ def test_library_hyperplanes_match_oracle(seed, bits, d):
 
 def _cfg(**kw):
     base = dict(batch=1, num_q_heads=4, num_kv_heads=1, head_dim=64, bits=32, topk=8, sink=0, window=0,
-                page_size=0, reserved=0, seed=1)
+                page_size=0, flags=0, seed=1)
     base.update(kw)
     return dk.Config(**base)
 
@@ -69,7 +69,7 @@ def _cfg(**kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(head_dim=96), 2), (dict(bits=48), 2), (dict(bits=256), 2), (dict(num_q_heads=12, num_kv_heads=1), 2),
     (dict(num_q_heads=6, num_kv_heads=4), 1), (dict(topk=0), 1), (dict(sink=-1), 1), (dict(page_size=48), 2),
-    (dict(batch=0), 1), (dict(reserved=3), 1), (dict(num_q_heads=64, num_kv_heads=64), 2),
+    (dict(batch=0), 1), (dict(flags=6), 1), (dict(num_q_heads=64, num_kv_heads=64), 2),
 ])
 def test_create_rejects_bad_configs(kw, status):
     h = ctypes.c_void_p()
