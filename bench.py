@@ -382,7 +382,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-steps", type=int, default=2)
     ap.add_argument("--two-kernel-select", action="store_true",
-                    help="use the non-cooperative two-kernel selection path")
+                    help="use the two-kernel selection path")
     ap.add_argument("--trace-steps", type=int, default=10,
                     help="extra traced steps for the per-kernel durations")
     ap.add_argument("--clock-reps", type=int, default=20,

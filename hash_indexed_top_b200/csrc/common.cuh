@@ -11,9 +11,12 @@ namespace dkv {
 constexpr int kMaxBits = 128;
 constexpr int kMaxDim = 128;
 constexpr int kSmCountFallback = 148;
+// One 128-byte line per (b, h) for every workspace word that CTAs update
+// atomically, so that different (b, h) never serialise on one L2 line.
+constexpr int kSyncStride = 32;
 
 // Device error word (one per device that loads the library).  Bits:
-enum : unsigned { kErrCapacity = 1u, kErrPage = 2u, kErrTimeout = 4u };
+enum : unsigned { kErrCapacity = 1u, kErrPage = 2u };
 __device__ unsigned g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }
@@ -93,6 +96,42 @@ __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x 
 __device__ __forceinline__ uint32_t float_key(float f) {
     uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Rotate the token's code bytes by rho (byte r of the result = byte (r + rho)
+// mod 4*NW of the input).
+// Branch-free: word rotation by rho / 4 as two select stages, then a funnel
+// shift by 8 (rho % 4) bits across neighbouring words.
+template <int NW>
+__device__ __forceinline__ void rotate_bytes(uint32_t (&w)[NW], bool by8, bool by4, uint32_t sh) {
+    uint32_t a[NW], c[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) a[k] = (NW == 4 && by8) ? w[(k + 2) % NW] : w[k];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) c[k] = (NW >= 2 && by4) ? a[(k + 1) % NW] : a[k];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) w[k] = __funnelshift_r(c[k], c[(k + 1) % NW], sh);
+}
+
+// Code storage.  Token t's code (b bits = T = b/8 bytes, LSB-first, hyperplane j
+// in byte j/8 bit j%8) is stored with its bytes rotated by t mod T: stored byte
+// p holds code byte (p + t mod T) mod T.  The scorer's lane that handles token t
+// reads its bytes in exactly that order, so the swizzle replaces a per-token
+// register rotation.  w: the code as BITS/32 little-endian 32-bit words.
+template <int BITS>
+__device__ __forceinline__ void store_code_rotated(uint64_t *dst, const uint32_t (&w)[BITS / 32], int64_t t) {
+    constexpr int NW = BITS / 32;
+    const int rho = (int)(t % (BITS / 8));
+    uint32_t r[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) r[k] = w[k];
+    rotate_bytes<NW>(r, (rho & 8) != 0, (rho & 4) != 0, 8u * (uint32_t)(rho & 3));
+    if constexpr (NW == 1) {
+        dst[0] = (uint64_t)r[0];
+    } else {
+#pragma unroll
+        for (int k = 0; k < NW / 2; ++k) dst[k] = (uint64_t)r[2 * k] | ((uint64_t)r[2 * k + 1] << 32);
+    }
 }
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

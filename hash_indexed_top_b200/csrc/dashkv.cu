@@ -22,8 +22,7 @@ struct dashkv_ctx {
     RBits R;
     int device;
     int sm_count;
-    int coop;        // cooperative launches supported
-    int fused_pdl;   // combine cooperative with programmatic serialization
+    int cluster_max;  // CTAs per (b, h) cluster of the fused selection; 0: no cluster launch
     int force_two_kernel;
     void **trace;   // optional cudaEvent_t pairs around each kernel of a call
     int n_trace;
@@ -121,9 +120,9 @@ int64_t view_capacity(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
     return ctx->cfg.page_size ? (int64_t)kv->max_pages * ctx->cfg.page_size : kv->n_cap;
 }
 
-// ---- workspace: [scores | cand | hist | state | arrive(3 x BH) | seg_cnt | partials]
+// ---- workspace: [scores | cand | ckey | hist | state | arrive(3 x BH lines) | seg_cnt | partials]
 struct WsLayout {
-    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, bar, inbin_n, inbin, def_mid, total;
+    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, total;
 };
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -142,13 +141,9 @@ WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
     L.ckey = o;    o = align_up(o + BH * ld * 4);
     L.hist = o;    o = align_up(o + BH * kBins * 4);
     L.state = o;   o = align_up(o + BH * sizeof(SelState));
-    L.arrive = o;  o = align_up(o + 3 * BH * 4);
+    L.arrive = o;  o = align_up(o + 3 * BH * kSyncStride * 4);
     L.seg_cnt = o; o = align_up(o + BH * kMaxSelCtas * 4);
     L.part = o;    o = align_up(o + BH * kMaxSplits * G * (c.head_dim + 2) * 4);
-    L.bar = o;     o = align_up(o + BH * 2 * 4);
-    L.inbin_n = o; o = align_up(o + BH * 4);
-    L.inbin = o;   o = align_up(o + BH * kInbinMax * 16);
-    L.def_mid = o; o = align_up(o + BH * kMaxSelCtas * 4);
     L.total = o;
     return L;
 }
@@ -289,15 +284,55 @@ void launch_score_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
                static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, ctx->cfg.topk, nctas);
 }
 
-// The fused selection needs every CTA resident at once: one per SM.
-bool use_fused(const dashkv_ctx *ctx, int64_t cap) {
-    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
-    return ctx->coop && !ctx->force_two_kernel && sel_ctas(ctx, cap, 1) * BH <= ctx->sm_count;
+// Fused selection whenever cluster launches are available (and not disabled).
+bool use_fused(const dashkv_ctx *ctx) { return !ctx->force_two_kernel && ctx->cluster_max > 0; }
+
+// CTAs per cluster for one call: at most the context's choice, and no more
+// than one per 1024 tokens of capacity.
+int fused_cluster(const dashkv_ctx *ctx, int64_t cap) {
+    const int64_t by_tokens = ceil_div(cap, 1024);
+    const int c = ctx->cluster_max < by_tokens ? ctx->cluster_max : (int)by_tokens;
+    return c < 1 ? 1 : c;
 }
 
-// Fused selection: cooperative launch (all CTAs resident together; the kernel
-// synchronises the CTAs of each (b, h) with bounded waits) that may also start
-// early behind the preceding kernel.
+// Largest cluster size C <= kMaxCluster for which all B * Hkv clusters of the
+// fused selection are resident at once (one wave, one CTA per SM); 1 when
+// even single CTAs need several waves; 0 without cluster launch support.
+template <int BITS, int D>
+int pick_cluster(const dashkv_ctx *ctx) {
+    int ok = 0;
+    if (cudaDeviceGetAttribute(&ok, cudaDevAttrClusterLaunch, ctx->device) != cudaSuccess || !ok) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    int c = ctx->sm_count / BH;
+    if (c > kMaxCluster) c = kMaxCluster;
+    for (; c > 1; --c) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(c, BH);
+        cfg.blockDim = dim3(kScoreThreads);
+        cfg.dynamicSmemBytes = ScoreShape<BITS>::SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, select_fused_kernel<BITS, D, false>, &cfg) == cudaSuccess &&
+            nclusters >= BH)
+            break;
+        cudaGetLastError();
+    }
+    return c < 1 ? 1 : c;
+}
+
+// Fused selection: a grid of (C, B * Hkv) CTAs in clusters of C (one cluster
+// per (b, h)) that may also start early behind the preceding kernel.
 template <int BITS, int D>
 void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
                      int nctas, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
@@ -311,14 +346,16 @@ void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
     cfg.dynamicSmemBytes = ScoreShape<BITS>::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nctas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = ctx->fused_pdl ? 2 : 1;
+    cfg.numAttrs = 2;
     cudaLaunchKernelEx(&cfg, kern, kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R,
-                       ws, ctx->cfg.topk, nctas, ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
+                       ws, ctx->cfg.topk, ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
 }
 
 template <int D>
@@ -379,7 +416,6 @@ const char *dashkv_status_str(dashkv_status s) {
         case DASHKV_ERR_CUDA: return "CUDA error";
         case DASHKV_ERR_DEVICE: return "page id out of range";
         case DASHKV_ERR_NO_DEVICE: return "no CUDA device";
-        case DASHKV_ERR_TIMEOUT: return "in-kernel wait timed out";
     }
     return "unknown status";
 }
@@ -410,13 +446,13 @@ dashkv_status dashkv_create(const dashkv_config *cfg, dashkv_ctx **out) {
     c->cfg = *cfg;
     c->device = dev;
     c->sm_count = sms;
-    int coop = 0;
-    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) coop = 0;
-    c->coop = coop;
-    c->fused_pdl = 1;
     c->force_two_kernel = (cfg->flags & DASHKV_FLAG_TWO_KERNEL_SELECT) != 0;
     build_rbits(cfg->seed, cfg->bits, cfg->head_dim, &c->R);
     set_attrs();
+    c->cluster_max =
+        cfg->head_dim == 64
+            ? (cfg->bits == 32 ? pick_cluster<32, 64>(c) : cfg->bits == 64 ? pick_cluster<64, 64>(c) : pick_cluster<128, 64>(c))
+            : (cfg->bits == 32 ? pick_cluster<32, 128>(c) : cfg->bits == 64 ? pick_cluster<64, 128>(c) : pick_cluster<128, 128>(c));
     const bool layout_ok =
         cfg->head_dim == 64
             ? (cfg->bits == 32 ? score_layout_ok<32, 64>() : cfg->bits == 64 ? score_layout_ok<64, 64>() : score_layout_ok<128, 64>())
@@ -492,10 +528,6 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     ws.state = reinterpret_cast<SelState *>(w + L.state);
     ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive);
     ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
-    ws.bar = reinterpret_cast<uint32_t *>(w + L.bar);
-    ws.inbin_n = reinterpret_cast<uint32_t *>(w + L.inbin_n);
-    ws.inbin = reinterpret_cast<uint4 *>(w + L.inbin);
-    ws.def_mid = reinterpret_cast<int32_t *>(w + L.def_mid);
     const KV k = make_kv(ctx, kv);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int nscore = sel_ctas(ctx, cap, 1);    // score kernel: one 1024-thread CTA per SM
@@ -507,11 +539,11 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
         launch_pdl(copy_scores_kernel, dim3(gx > 0 ? gx : 1, BH), dim3(256), 0, st,
                    (const float *)ws.scores, ws.ld, scores, ws.ld_out, seq_lens, ctx->cfg.num_kv_heads, cap);
     };
-    if (use_fused(ctx, cap)) {
-        // every CTA of the grid fits at once (one per SM): fused selection
+    if (use_fused(ctx)) {
+        const int nc = fused_cluster(ctx, cap);
         tr.before();
-        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nscore, sel_idx, sel_cnt, st);
-        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nscore, sel_idx, sel_cnt, st);
+        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nc, sel_idx, sel_cnt, st);
+        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nc, sel_idx, sel_cnt, st);
         tr.after();
         copy_scores();
         return launch_status();
@@ -541,7 +573,7 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     AttnWS ws;
     ws.part = reinterpret_cast<float *>(w + L.part);
-    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive) + 2 * BH;
+    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive) + 2 * BH * kSyncStride;
     const KV k = make_kv(ctx, kv);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Tracer tr(ctx, st);
@@ -554,7 +586,8 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
 
 int32_t dashkv_select_kernels(const dashkv_ctx *ctx, int64_t max_tokens) {
     if (!ctx) return 0;
-    return use_fused(ctx, max_tokens) ? 1 : 2;
+    (void)max_tokens;
+    return use_fused(ctx) ? 1 : 2;
 }
 
 dashkv_status dashkv_set_trace(dashkv_ctx *ctx, void **events, int32_t n_events) {
@@ -570,7 +603,6 @@ dashkv_status dashkv_get_error(void *stream) {
     unsigned w = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return DASHKV_ERR_CUDA;
     if (w && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return DASHKV_ERR_CUDA;
-    if (w & kErrTimeout) return DASHKV_ERR_TIMEOUT;
     if (w & kErrPage) return DASHKV_ERR_DEVICE;
     if (w & kErrCapacity) return DASHKV_ERR_CAPACITY;
     return DASHKV_OK;

@@ -51,6 +51,19 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
+// Packed fp32 fused multiply-add (two lanes of fp32 per instruction on sm_100):
+// (a.x * b.x + c.x, a.y * b.y + c.y), each rounded once like fmaf.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&d);
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t x) { return make_float2(bf16_lo(x), bf16_hi(x)); }
+
 // 2^x on the SFU (approximate, flushes denormal results to zero: weights below
 // 2^-126 of the running maximum vanish, far inside the fp32 accumulation error).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -128,17 +141,24 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     };
     // Gather a tile's K and V rows into buffer `buf` (zero-filled when invalid);
     // tok: this lane's tile_token() of the tile.
+    // Lane l copies row l / LPT of the tile: chunks l % LPT, l % LPT + LPT, ...
+    // of its K and V rows (so each lane computes one row address per tile).
+    constexpr int LPT = 32 / TROWS;               // lanes per tile row
+    constexpr int CPL = 2 * CPR / LPT;            // 16-byte chunks per lane (K then V)
     auto prefetch = [&](int tok, int buf) {
         __nv_bfloat16 *dst0 = wstage + (size_t)buf * TROWS * 2 * D;
+        const int j = lane / LPT, c0 = lane % LPT;
+        const int t = __shfl_sync(0xffffffffu, tok, j);
+        const int64_t off = t >= 0 ? kv.row(b, h, t) : 0;
+        const int nbytes = t >= 0 ? 16 : 0;
+        __nv_bfloat16 *dst = dst0 + (size_t)j * 2 * D;
 #pragma unroll
-        for (int x = lane; x < TROWS * 2 * CPR; x += 32) {
-            const int j = x / (2 * CPR), c = x % (2 * CPR);
-            const int t = __shfl_sync(0xffffffffu, tok, j);
-            const bool isv = c >= CPR;
+        for (int m = 0; m < CPL; ++m) {
+            const int c = c0 + m * LPT;       // chunk of the (K, V) pair of rows
+            const bool isv = c >= CPR;        // compile-time per m when LPT divides CPR
             const int cc = isv ? c - CPR : c;
-            const int64_t off = t >= 0 ? kv.row(b, h, t) : 0;
             const __nv_bfloat16 *src = (isv ? kv.v : kv.k) + off + cc * 8;
-            cp_async16(dst0 + ((size_t)j * 2 + (isv ? 1 : 0)) * D + cc * 8, src, t >= 0 ? 16 : 0);
+            cp_async16(dst + (isv ? D : 0) + cc * 8, src, nbytes);
         }
         cp_async_commit();
     };
@@ -191,13 +211,11 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float d0 = 0.0f, d1 = 0.0f;
+                float2 d2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                for (int e = 0; e < DPL; e += 2) {
-                    d0 = fmaf(qf[g][e], kf[e], d0);
-                    d1 = fmaf(qf[g][e + 1], kf[e + 1], d1);
-                }
-                x[j][g] = d0 + d1;
+                for (int e = 0; e < DPL; e += 2)
+                    d2 = ffma2(make_float2(qf[g][e], qf[g][e + 1]), make_float2(kf[e], kf[e + 1]), d2);
+                x[j][g] = d2.x + d2.y;
             }
         }
 #pragma unroll
@@ -247,9 +265,15 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                 vf[0] = bf16_lo(w.x); vf[1] = bf16_hi(w.x); vf[2] = bf16_lo(w.y); vf[3] = bf16_hi(w.y);
             }
 #pragma unroll
-            for (int g = 0; g < G; ++g)
+            for (int g = 0; g < G; ++g) {
+                const float2 p2 = make_float2(x[j][g], x[j][g]);
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) acc[g][e] = fmaf(x[j][g], vf[e], acc[g][e]);
+                for (int e = 0; e < DPL; e += 2) {
+                    const float2 a2 = ffma2(p2, make_float2(vf[e], vf[e + 1]), make_float2(acc[g][e], acc[g][e + 1]));
+                    acc[g][e] = a2.x;
+                    acc[g][e + 1] = a2.y;
+                }
+            }
         }
         __syncwarp();  // the buffer is refilled by a later prefetch
     }
@@ -286,29 +310,54 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     // the last CTA of this (b, h) merges the splits
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(ws.arrive + bh, 1u) == (unsigned)(splits - 1);
+    if (tid == 0) s_last = atomicAdd(ws.arrive + (int64_t)kSyncStride * bh, 1u) == (unsigned)(splits - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
     const float *pbase = ws.part + (int64_t)bh * kMaxSplits * G * (D + 2);
+    // per-(split, head) scale 2^(m_s - M_g) and the total sum L_g, then the
+    // weighted sum of the accumulators with all split loads in flight
+    float *s_c = s_acc;                  // [splits][G] (the CTA states are no longer needed)
+    float *s_L = s_acc + kMaxSplits * G; // [G]
+    float *s_M = s_L + G;                // [G]
+    for (int x = tid; x < splits * G; x += kAttnThreads) {
+        const int sp = x / G, g = x % G;
+        s_c[x] = __ldcg(pbase + (sp * G + g) * (D + 2) + D);      // m_s
+        s_c[kMaxSplits * G + 2 * G + x] = __ldcg(pbase + (sp * G + g) * (D + 2) + D + 1);  // l_s
+    }
+    __syncthreads();
+    if (tid < G) {
+        const int g = tid;
+        float M = -INFINITY;
+        for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, s_c[sp * G + g]);
+        float L = 0.0f;
+        for (int sp = 0; sp < splits; ++sp) {
+            const float c = M == -INFINITY ? 0.0f : fast_exp2(s_c[sp * G + g] - M);
+            L = fmaf(s_c[kMaxSplits * G + 2 * G + sp * G + g], c, L);
+            s_c[sp * G + g] = c;
+        }
+        s_L[g] = L;
+        s_M[g] = M;
+    }
+    __syncthreads();
     for (int x = tid; x < G * D; x += kAttnThreads) {
         const int g = x / D, i = x % D;
-        float M = -INFINITY;
-        for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(pbase + (s * G + g) * (D + 2) + D));
-        float L = 0.0f, Acc = 0.0f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < splits; ++s) {
-                const float *ps = pbase + (s * G + g) * (D + 2);
-                const float c = fast_exp2(__ldcg(ps + D) - M);
-                L = fmaf(__ldcg(ps + D + 1), c, L);
-                Acc = fmaf(__ldcg(ps + i), c, Acc);
-            }
+        float Acc = 0.0f;
+        int sp = 0;
+        for (; sp + 8 <= splits; sp += 8) {
+            float a[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a[u] = __ldcg(pbase + ((sp + u) * G + g) * (D + 2) + i);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) Acc = fmaf(a[u], s_c[(sp + u) * G + g], Acc);
         }
+        for (; sp < splits; ++sp) Acc = fmaf(__ldcg(pbase + (sp * G + g) * (D + 2) + i), s_c[sp * G + g], Acc);
+        const float L = s_L[g];
         const int64_t oq = (int64_t)b * Hq + h * G + g;
         out[oq * D + i] = L > 0.0f ? Acc / L : 0.0f;
-        if (i == 0 && lse) lse[oq] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        if (i == 0 && lse) lse[oq] = L > 0.0f ? (s_M[g] + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
-    if (tid == 0) ws.arrive[bh] = 0;
+    if (tid == 0) ws.arrive[(int64_t)kSyncStride * bh] = 0;
 }
 
 }  // namespace dkv

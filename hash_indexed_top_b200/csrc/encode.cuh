@@ -25,7 +25,7 @@ struct EncodeShape {
     static constexpr int THREADS = 128;
     static constexpr int KT = THREADS / NG;            // keys per tile
     static constexpr int KS_LD = KT + 1;               // padded row of the transposed tile
-    static constexpr size_t SMEM = sizeof(float) * ((size_t)D * BITS + (size_t)D * KS_LD);
+    static constexpr size_t SMEM = sizeof(float) * ((size_t)D * BITS + (size_t)D * KS_LD) + 8 * KT * NG + 8;
 };
 
 template <int BITS, int D>
@@ -35,6 +35,7 @@ encode_keys_kernel(KV kv, const int32_t *__restrict__ seq_lens, const RBits R, i
     extern __shared__ float4 smem_f4[];
     float *Rf = reinterpret_cast<float *>(smem_f4);  // [D][BITS]
     float *ks = Rf + D * BITS;                       // [D][KS_LD]
+    uint64_t *words = reinterpret_cast<uint64_t *>(ks + D * S::KS_LD);  // [KT][NG] code words of the tile
 
     const int bh = blockIdx.y;
     const int b = bh / kv.Hkv, h = bh % kv.Hkv;
@@ -91,13 +92,18 @@ encode_keys_kernel(KV kv, const int32_t *__restrict__ seq_lens, const RBits R, i
                 acc[4 * q + 3] = fmaf(r.w, kx, acc[4 * q + 3]);
             }
         }
-        const int64_t t = t0 + key;
-        if (t < n) {
-            uint64_t word = 0;
+        uint64_t word = 0;
 #pragma unroll
-            for (int jj = 0; jj < S::JPT; ++jj) word |= (uint64_t)(acc[jj] >= 0.0f) << jj;
+        for (int jj = 0; jj < S::JPT; ++jj) word |= (uint64_t)(acc[jj] >= 0.0f) << jj;
+        words[key * S::NG + grp] = word;
+        __syncthreads();
+        const int64_t t = t0 + key;
+        if (grp == 0 && t < n) {
+            uint32_t w32[BITS / 32];
+#pragma unroll
+            for (int k = 0; k < BITS / 32; ++k) w32[k] = (uint32_t)(words[key * S::NG + k / 2] >> (32 * (k % 2)));
             int64_t c = kv.code(b, h, t);
-            if (c >= 0) kv.codes[c + grp] = word;
+            if (c >= 0) store_code_rotated<BITS>(kv.codes + c, w32, t);
         }
     }
 }
@@ -170,12 +176,11 @@ append_keys_kernel(KV kv, const __nv_bfloat16 *__restrict__ k_new, const __nv_bf
     }
     __syncthreads();
     if (ok) {
-        constexpr int W = BITS >= 64 ? BITS / 64 : 1;
-        for (int x = tid; x < Hkv * W; x += blockDim.x) {
-            const int h = x / W, w = x % W;
-            const int64_t c = kv.code(b, h, pos);
-            kv.codes[c + w] = BITS == 32 ? (uint64_t)code32[h][0]
-                                         : ((uint64_t)code32[h][2 * w] | ((uint64_t)code32[h][(2 * w + 1) % (BITS / 32)] << 32));
+        for (int h = tid; h < Hkv; h += blockDim.x) {
+            uint32_t w32[BITS / 32];
+#pragma unroll
+            for (int k = 0; k < BITS / 32; ++k) w32[k] = code32[h][k];
+            store_code_rotated<BITS>(kv.codes + kv.code(b, h, pos), w32, pos);
         }
     }
     __syncthreads();

@@ -40,6 +40,9 @@ constexpr int kMaxSelCtas = 512;
 constexpr int kCandSmem = 2048;   // in-bin candidates ranked in shared memory
 constexpr int kListSmem = 8192;   // candidate list held in shared memory by the resolver
 constexpr int kCollectTile = kSelThreads * 16;
+// The fused selection records, per 32-token chunk of a CTA's range, the largest
+// bin in the chunk (uint16 in shared memory, for the first kCmaxCap chunks).
+constexpr int kCmaxCap = 16384;
 
 enum : int { kStateNormal = 0, kStateAll = 1, kStateEmpty = 2 };
 
@@ -61,14 +64,9 @@ struct SelWS {
     int32_t *cand;       // [BH][ld]
     uint32_t *hist;      // [BH][kBins]        zero between calls
     SelState *state;     // [BH]
-    uint32_t *arrive;    // [2][BH]            zero between calls
+    uint32_t *arrive;    // [2][BH] x kSyncStride   zero between calls
     int32_t *seg_cnt;    // [BH][kMaxSelCtas]
-    uint32_t *ckey;      // [BH][ld] order keys of the segment entries (fused selection)
-    // fused selection only
-    uint32_t *bar;       // [BH][2] barrier (arrivals, generation); arrivals zero between calls
-    uint32_t *inbin_n;   // [BH]   in-bin list length (cleared at barrier 1)
-    uint4 *inbin;        // [BH][kInbinMax] (order key, token, cta, 0)
-    int32_t *def_mid;    // [BH][kMaxSelCtas]
+    uint32_t *ckey;      // [BH][ld] order keys of spilled candidates (fused selection)
 };
 
 // Monotone map of a score to one of kBins bins (x in [0, 1] over [-A, A]).
@@ -134,7 +132,8 @@ struct ScoreShape {
     static constexpr int COPIES = 32 / T;      // interleaved copies: lanes hit distinct banks
     static constexpr int NW = BITS / 32;       // 32-bit code words per token
     static constexpr uint32_t LUT_BYTES = 256 * 256;
-    static constexpr uint32_t LOW_BYTES = kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;  // hist + scratch
+    static constexpr uint32_t SCRATCH_BYTES = kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;  // hist + scratch
+    static constexpr uint32_t LOW_BYTES = SCRATCH_BYTES + kCmaxCap * 2;               // + chunk maxima
     using Vec = typename std::conditional<BITS == 128, uint4, uint2>::type;  // one token's code
     // per-thread cp.async ring of upcoming codes (one token per thread per stage)
     static constexpr int STAGES = 5;
@@ -142,21 +141,6 @@ struct ScoreShape {
     // dynamic smem: low region, the LUT at the next 64 KB boundary, then the ring
     static constexpr size_t SMEM = 2 * 65536 + RING_BYTES;
 };
-
-// Rotate the token's code bytes by rho (byte r of the result = byte (r + rho)
-// mod 4*NW of the input).
-// Branch-free: word rotation by rho / 4 as two select stages, then a funnel
-// shift by 8 (rho % 4) bits across neighbouring words.
-template <int NW>
-__device__ __forceinline__ void rotate_bytes(uint32_t (&w)[NW], bool by8, bool by4, uint32_t sh) {
-    uint32_t a[NW], c[NW];
-#pragma unroll
-    for (int k = 0; k < NW; ++k) a[k] = (NW == 4 && by8) ? w[(k + 2) % NW] : w[k];
-#pragma unroll
-    for (int k = 0; k < NW; ++k) c[k] = (NW >= 2 && by4) ? a[(k + 1) % NW] : a[k];
-#pragma unroll
-    for (int k = 0; k < NW; ++k) w[k] = __funnelshift_r(c[k], c[(k + 1) % NW], sh);
-}
 
 template <int BITS>
 __device__ __forceinline__ void unpack_code(const typename ScoreShape<BITS>::Vec &x, uint32_t (&w)[BITS / 32]) {
@@ -199,11 +183,13 @@ __device__ __forceinline__ float lut_score(const uint32_t (&w)[BITS / 32], const
 // in shared memory.  Ends with the histogram complete (after a barrier).
 struct ScoreOut {
     int64_t n, t0, t1;
+    int R;               // tokens per warp range (multiple of 32)
     float inv2A;
     unsigned char *lut;  // 64 KB LUT region, free for reuse once scoring is done
+    uint16_t *cmax;      // [kCmaxCap] largest bin per 32-token chunk (CMAX only)
 };
 
-template <int BITS, int D, bool PAGED>
+template <int BITS, int D, bool PAGED, bool CMAX = false>
 __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                                                 const int32_t *__restrict__ seq_lens, const RBits &R,
                                                 const SelWS &ws, int nctas, unsigned char *smem) {
@@ -268,6 +254,7 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     ScoreOut o;
     o.inv2A = red[0];
     o.lut = lut;
+    o.cmax = reinterpret_cast<uint16_t *>(smem + S::SCRATCH_BYTES);
     // everything above depends on q only; codes and lengths come from the append
     griddep_wait();
     o.n = clamp_len(kv, seq_lens, b);
@@ -275,18 +262,26 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     const int64_t t0 = o.t0, t1 = o.t1;
     const float inv2A = o.inv2A;
 
+    // Lane l always handles tokens with t % 32 == l, whose stored bytes are
+    // rotated by rho = l % T (see store_code_rotated): at step r it reads byte r,
+    // which is code byte (r + rho) % T, from table (r + rho) % T in copy l / T.
     const int rho = lane % T, copy = lane / T;
-    const bool rot8 = (rho & 8) != 0, rot4 = (rho & 4) != 0;
-    const uint32_t rot_sh = 8u * (uint32_t)(rho & 3);
     uint32_t off[T];
 #pragma unroll
     for (int r = 0; r < T; ++r) off[r] = lut_s | 4u * (uint32_t)(copy * T + (rho + r) % T);
 
     const int nloc = (int)(t1 - t0);  // tokens of this CTA (< 2^31)
-
-    // Each thread streams tokens tid, tid + NT, ... through its own slots of a
-    // STAGES-deep cp.async ring: it only ever reads codes it copied itself, so
-    // the ring needs no barriers, and STAGES - 1 codes per thread stay in flight.
+    // Warp w streams the contiguous range [w R, (w + 1) R) of the CTA's tokens,
+    // 32 at a time (lane = token), so its scores come out in token order.
+    constexpr int NWARP = kScoreThreads / 32;
+    const int wlen = (int)(ceil_div(ceil_div(nloc, NWARP), 32) * 32);
+    o.R = wlen;
+    const int wb = warp * wlen;                               // warp's first local token
+    const int we = min(nloc, wb + wlen);                      // one past its last
+    const int nk = we > wb ? (we - wb + 31) / 32 : 0;         // 32-token steps of this warp
+    // Each thread streams its tokens through its own slots of a STAGES-deep
+    // cp.async ring: it only ever reads codes it copied itself, so the ring needs
+    // no barriers, and STAGES - 1 codes per thread stay in flight.
     constexpr int NT = kScoreThreads;
     constexpr int STAGES = S::STAGES;
     constexpr int VB = (int)sizeof(Vec);
@@ -294,11 +289,11 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     const unsigned char *ring = lut + 65536 + tid * VB;
     const Vec *dense = reinterpret_cast<const Vec *>(kv.codes) + ((int64_t)bh * kv.n_cap + t0);
     float *srow = ws.scores + (int64_t)bh * ws.ld + t0;
-    auto issue = [&](int k) {  // copy the code of token k * NT + tid into stage k % STAGES
-        const int i = k * NT + tid;
+    auto issue = [&](int k, int slot) {  // copy the code of token wb + 32 k + lane into `slot`
+        const int i = wb + 32 * k + lane;
         const void *src = dense;
         int bytes = 0;
-        if (i < nloc) {
+        if (k < nk && i < we) {
             if (!PAGED) {
                 src = dense + i;
                 bytes = VB;
@@ -307,28 +302,36 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
                 if (c >= 0) { src = kv.codes + c; bytes = VB; }
             }
         }
-        const uint32_t dst = ring_s + (uint32_t)((k % STAGES) * NT * VB);
+        const uint32_t dst = ring_s + (uint32_t)(slot * NT * VB);
         if (VB == 16)
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
         else
             asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    const int nk = (nloc + NT - 1) / NT;  // stages this CTA streams
 #pragma unroll
-    for (int k = 0; k < STAGES - 1; ++k) issue(k);
+    for (int k = 0; k < STAGES - 1; ++k) issue(k, k);
+    int slot = 0, islot = STAGES - 1;
     for (int k = 0; k < nk; ++k) {
-        issue(k + STAGES - 1);
+        issue(k + STAGES - 1, islot);
+        islot = islot == STAGES - 1 ? 0 : islot + 1;
         asm volatile("cp.async.wait_group %0;" ::"n"(STAGES - 1) : "memory");
-        const int i = k * NT + tid;
-        if (i < nloc) {
-            const Vec code = *reinterpret_cast<const Vec *>(ring + (k % STAGES) * NT * VB);
+        const int i = wb + 32 * k + lane;
+        const Vec code = *reinterpret_cast<const Vec *>(ring + slot * NT * VB);
+        slot = slot == STAGES - 1 ? 0 : slot + 1;
+        int bin = 0;
+        if (i < we) {
             uint32_t w[NW];
             unpack_code<BITS>(code, w);
-            rotate_bytes<NW>(w, rot8, rot4, rot_sh);
             const float s = lut_score<BITS>(w, off);
             srow[i] = s;
-            atomicAdd(&hist[score_bin(s, inv2A)], 1u);
+            bin = score_bin(s, inv2A);
+            atomicAdd(&hist[bin], 1u);
+        }
+        if constexpr (CMAX) {
+            const unsigned m = __reduce_max_sync(0xffffffffu, (unsigned)bin);
+            const int c = (wb >> 5) + k;  // chunk of local tokens [32 c, 32 c + 32)
+            if (lane == 0 && c < kCmaxCap) o.cmax[c] = (uint16_t)m;
         }
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -397,7 +400,7 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         if (hist[k]) atomicAdd(ghist + k, hist[k]);
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(ws.arrive + bh, 1u) == (unsigned)(nctas - 1);
+    if (tid == 0) s_last = atomicAdd(ws.arrive + (int64_t)kSyncStride * bh, 1u) == (unsigned)(nctas - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
@@ -416,7 +419,7 @@ score_hist_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         st.T1 = s_thr[0]; st.above1 = s_thr[1]; st.cnt_T1 = s_thr[2];
         st.flags = n == 0 ? kStateEmpty : (kk >= n ? kStateAll : kStateNormal);
         ws.state[bh] = st;
-        ws.arrive[bh] = 0;
+        ws.arrive[(int64_t)kSyncStride * bh] = 0;
     }
 }
 
@@ -690,163 +693,235 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
     if (tid == 0) ws.seg_cnt[(int64_t)bh * kMaxSelCtas + blockIdx.x] = count;
     __threadfence();
     __syncthreads();
-    if (tid == 0) sm.last = atomicAdd(ws.arrive + gridDim.y + bh, 1u) == (unsigned)(nctas - 1);
+    if (tid == 0) sm.last = atomicAdd(ws.arrive + (int64_t)kSyncStride * (gridDim.y + bh), 1u) == (unsigned)(nctas - 1);
     __syncthreads();
     if (!sm.last) return;
     __threadfence();
     resolve_emit<kSelThreads, kListSmem>(ws, bh, nctas, st, S, W, cap_sel, sel_idx, sel_cnt, sm);
-    if (tid == 0) ws.arrive[gridDim.y + bh] = 0;
+    if (tid == 0) ws.arrive[(int64_t)kSyncStride * (gridDim.y + bh)] = 0;
 }
 
 // ---------------------------------------------------------------------------
-// Fused selection: one kernel, all CTAs of a (b, h) co-resident (cooperative
-// launch, at most one CTA per SM), two barriers per (b, h).
-//   stream + histogram -> barrier 1 -> every CTA finds T1 from the summed
-//   histogram, compacts its own tokens with bin >= T1 into its segment, counts
-//   the definite ones (bin > T1) in the middle range and appends its few in-bin
-//   tokens to a shared list -> barrier 2 -> every CTA ranks the in-bin list
-//   (score desc, token asc), derives every CTA's count of selected middle
+// Fused selection: one kernel, one thread-block cluster of C CTAs per (b, h)
+// (C <= kMaxCluster, one 1024-thread CTA per SM).  The CTAs of a cluster are
+// scheduled together and exchange their small per-CTA results through
+// distributed shared memory, with hardware cluster barriers:
+//   stream + histogram (+ per-chunk maximum bins) -> barrier 1 -> every CTA
+//   finds T1 from the cluster's histograms (coarse 64-bin super-bins first,
+//   then the 64 bins of the one that holds the k-th score), keeps its tokens
+//   with bin >= T1 (only chunks whose maximum bin reaches T1 are re-read),
+//   counts the definite ones (bin > T1) of the middle range and lists its
+//   few in-bin ones -> barrier 2 -> every CTA gathers the in-bin lists, ranks
+//   them (score desc, token asc), derives each CTA's count of selected middle
 //   tokens, hence its own output offset, and writes its tokens in order; CTA 0
-//   writes the sinks, the window, the padding and the count.
-// A bin with more than kInbinMax tokens (heavy ties) takes the exact resolver
-// of the two-kernel path, run by CTA 0 after barrier 2.
+//   writes the sinks, the window, the padding and the count -> barrier 3 (no
+//   CTA leaves while another may still read its shared memory).
+// A threshold bin with more than kInbinMax tokens (heavy ties), or a sequence
+// with n <= k, takes the exact resolver of the two-kernel path, run by CTA 0
+// over segments in global memory after barrier 2.
 constexpr int kInbinMax = 1024;
-constexpr unsigned kSpinLimit = 1u << 24;  // ~1.7 s of 100 ns naps: then report a timeout
+constexpr int kMaxCluster = 16;
 
-// Barrier among the `nparts` CTAs of one (b, h): bar[0] counts arrivals, bar[1]
-// is the generation the last arrival advances.  Bounded wait: a CTA that gives
-// up records kErrTimeout and carries on.  reset: a word the last arrival
-// clears before releasing the others.
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+    cluster_arrive();
+    cluster_wait();
+}
+// Address, in the cluster's shared window, of the object at `p` (this CTA's
+// shared memory) in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
     uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
     return v;
 }
 
-__device__ __forceinline__ void bh_barrier(uint32_t *bar, unsigned nparts, uint32_t *reset) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t g = ld_acquire(bar + 1);
-        __threadfence();
-        if (atomicAdd(bar, 1u) == nparts - 1) {
-            bar[0] = 0;
-            if (reset) *reset = 0;
-            __threadfence();
-            atomicAdd(bar + 1, 1u);
-        } else {
-            unsigned spins = 0;
-            while (ld_acquire(bar + 1) == g) {
-                if (++spins > kSpinLimit) {
-                    raise_error(kErrTimeout);
-                    break;
-                }
-                __nanosleep(100);
-            }
-            __threadfence();
+// Threshold of the cluster's summed histogram, computed by one full warp from
+// the CTAs' super-bin counts (coarse[64], super-bin s = bins [64 s, 64 s + 64))
+// and histograms (hist[kBins]), both read in place in every CTA's shared
+// memory.  out = {T1, tokens above T1, tokens in T1} as threshold_bin.
+__device__ __forceinline__ void cluster_threshold(const uint32_t *coarse, const uint32_t *hist, int nranks,
+                                                  int64_t kk, int *out) {
+    const int lane = threadIdx.x & 31;
+    // lane l holds super-bins 63 - 2l (upper) and 62 - 2l (lower): lane 0 the top
+    uint32_t cu = 0, cl = 0;
+    for (int r = 0; r < nranks; ++r) {
+        cu += ld_cluster_u32(cluster_addr(coarse + (63 - 2 * lane), r));
+        cl += ld_cluster_u32(cluster_addr(coarse + (62 - 2 * lane), r));
+    }
+    int64_t incl = (int64_t)cu + cl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int64_t excl = incl - cu - cl;
+    const bool here = excl < kk && kk <= incl;
+    int sb = 0;
+    int64_t above = 0;
+    if (here) {
+        if (excl + cu >= kk) { sb = 63 - 2 * lane; above = excl; }
+        else { sb = 62 - 2 * lane; above = excl + cu; }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+    sb = __shfl_sync(0xffffffffu, sb, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    // the 64 bins of super-bin sb, the same way
+    const int bu = 64 * sb + 63 - 2 * lane, bl = bu - 1;
+    uint32_t fu = 0, fl = 0;
+    for (int r = 0; r < nranks; ++r) {
+        fu += ld_cluster_u32(cluster_addr(hist + bu, r));
+        fl += ld_cluster_u32(cluster_addr(hist + bl, r));
+    }
+    int64_t fincl = (int64_t)fu + fl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, fincl, o);
+        if (lane >= o) fincl += y;
+    }
+    const int64_t fexcl = above + fincl - fu - fl;
+    fincl += above;
+    if (fexcl < kk && kk <= fincl) {
+        if (fexcl + fu >= kk) { out[0] = bu; out[1] = (int)fexcl; out[2] = (int)fu; }
+        else { out[0] = bl; out[1] = (int)(fexcl + fu); out[2] = (int)fl; }
+    }
+}
+
+// Smallest finite float s with score_bin(s, inv2A) >= T, or +inf if there is
+// none, so that for every finite s:  s >= result  <=>  score_bin(s) >= T.
+// score_bin is monotone in s (a correctly rounded fma with a non-negative
+// factor, a clamp, a scale and a truncation), hence monotone along the
+// order-preserving keys.  A full warp first tests the 32 keys around the
+// algebraic estimate; if the boundary is not among them it narrows the whole
+// key range 32-fold per round.  Every lane returns the result.
+__device__ __forceinline__ float bin_floor_value(int T, float inv2A) {
+    const int lane = threadIdx.x & 31;
+    if (T <= 0) return -INFINITY;
+    if (T >= kBins) return INFINITY;
+    auto P = [&](uint32_t key) { return score_bin(key_to_float(key), inv2A) >= T; };
+    if (inv2A > 0.0f) {
+        const float est = ((float)T / (float)(kBins - 1) - 0.5f) / inv2A;
+        const uint32_t k0 = float_key(est) - 16u;
+        const uint32_t b = __ballot_sync(0xffffffffu, P(k0 + (uint32_t)lane));
+        const int f = __ffs(b) - 1;  // a boundary inside the window: false below lane f, true from it
+        if (f > 0 && b == (0xffffffffu << f)) return key_to_float(k0 + (uint32_t)f);
+    }
+    const uint32_t none = 0xff800000u;     // key of +inf: one past the key of FLT_MAX
+    uint64_t lo = 0x00800000u, hi = none;  // key of -FLT_MAX; answer in [lo, hi]
+    while (lo < hi) {
+        const uint64_t n = hi - lo;
+        const uint64_t step = (n + 31) / 32;
+        const uint64_t x = lo + (uint64_t)lane * step;
+        const uint32_t b = __ballot_sync(0xffffffffu, x < hi && P((uint32_t)x));
+        if (b) {
+            const int f = __ffs(b) - 1;    // false at lo + (f - 1) step, true at lo + f step
+            hi = lo + (uint64_t)f * step;
+            if (f) lo += (uint64_t)(f - 1) * step + 1;
+        } else {                           // every tested point is false
+            const uint64_t last = (n - 1) / step < 31 ? (n - 1) / step : 31;
+            lo += last * step + 1;
         }
     }
-    __syncthreads();
+    return key_to_float((uint32_t)lo);     // `none` maps to +inf
 }
 
 template <int BITS, int D, bool PAGED>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
-                    const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int nctas, int S,
-                    int W, int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
+                    const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int S, int W,
+                    int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
     constexpr int NT = kScoreThreads;
+    constexpr int NWARP = NT / 32;
+    constexpr int CW = 64;  // candidates per warp kept in shared memory (more go to the global segment)
+    constexpr int FB = 8;   // hit chunks whose scores one warp loads per round trip
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ int s_warp[32];
     __shared__ int s_thr[4];
     __shared__ int s_misc[4];
-    __shared__ int s_mid[kMaxSelCtas];
-    const int tid = threadIdx.x;
-    const int bh = blockIdx.y, cta = blockIdx.x;
-    const ScoreOut so = score_phase<BITS, D, PAGED>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
-    uint32_t *ghist = ws.hist + (int64_t)bh * kBins;
-    for (int k = tid; k < kBins; k += NT)
-        if (hist[k]) atomicAdd(ghist + k, hist[k]);
+    __shared__ float s_theta[2];
+    __shared__ uint32_t s_coarse[64];      // this CTA's histogram per super-bin (read by the cluster)
+    __shared__ int s_pub[2];               // this CTA's in-bin entries, definite middle tokens (read by the cluster)
+    __shared__ int s_cinb[kMaxCluster + 1], s_mid[kMaxCluster];
+    __shared__ int s_wcnt[NWARP], s_wdef[NWARP], s_wkeep[NWARP];
+    __shared__ int s_ninb;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.y, cta = blockIdx.x;  // cta = rank in the cluster (cluster = the row of CTAs)
+    const int nctas = gridDim.x;
+    const ScoreOut so = score_phase<BITS, D, PAGED, true>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
+    const uint32_t *hist = reinterpret_cast<const uint32_t *>(smem);
     griddep_trigger();
-    bh_barrier(ws.bar + 2 * bh, nctas, ws.inbin_n + bh);  // (1): histogram complete
-
+    {   // super-bin counts: 16 threads per super-bin, 4 bins each
+        uint32_t c = hist[4 * tid] + hist[4 * tid + 1] + hist[4 * tid + 2] + hist[4 * tid + 3];
+#pragma unroll
+        for (int o = 8; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if ((lane & 15) == 0) s_coarse[tid >> 4] = c;
+    }
     const int64_t n = so.n, t0 = so.t0, t1 = so.t1;
     const int64_t kk = topk < n ? topk : n;
     const bool normal = n > 0 && kk < n;
-    if (tid == 0) { s_thr[0] = kBins; s_thr[1] = 0; s_thr[2] = 0; }
-    if (normal) {
-        for (int k = tid; k < kBins; k += NT) hist[k] = __ldcg(ghist + k);
-        __syncthreads();
-        threshold_bin<NT>(hist, kk, s_warp, s_thr);
+    if (tid == 0) { s_thr[0] = kBins; s_thr[1] = 0; s_thr[2] = 0; s_ninb = 0; }
+    cluster_sync();  // (1): every histogram of the cluster is complete
+    const float inv2A = so.inv2A;
+    if (normal && warp == 0) {
+        cluster_threshold(s_coarse, hist, nctas, kk, s_thr);
+        __syncwarp();
+        const int T1w = s_thr[0];
+        const float th = bin_floor_value(T1w, inv2A);
+        const float th2 = bin_floor_value(T1w + 1, inv2A);
+        if (lane == 0) { s_theta[0] = th; s_theta[1] = th2; }
     }
     __syncthreads();
     const int T1 = s_thr[0], above1 = s_thr[1], cnt_T1 = s_thr[2];
     const bool fallback = normal && cnt_T1 > kInbinMax;
     const int s_end = (int)(S < n ? S : n);
     const int w_beg = (int)(n - W > s_end ? n - W : s_end);
-    const float inv2A = so.inv2A;
     int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
-    const float *srow = ws.scores + (int64_t)bh * ws.ld;
-
-    // ---- own range: segment of tokens with bin >= T1 (ascending), definite
-    // middle count, in-bin tokens appended to the shared list
     uint32_t *ckey = ws.ckey + (int64_t)bh * ws.ld;
-    int seg = 0, defmid = 0;
-    if (normal) {
-        for (int64_t base = t0; base < t1; base += (int64_t)NT * 32) {
-            const int64_t tb = base + (int64_t)tid * 32;
-            float x[32];
-            if (tb + 32 <= t1) {
-                const float4 *p = reinterpret_cast<const float4 *>(srow + tb);
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 f = __ldcg(p + v);
-                    x[4 * v] = f.x; x[4 * v + 1] = f.y; x[4 * v + 2] = f.z; x[4 * v + 3] = f.w;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = tb + e < t1 ? __ldcg(srow + tb + e) : -INFINITY;
-            }
-            uint32_t flags = 0;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int bin = tb + e < t1 ? score_bin(x[e], inv2A) : -1;
-                if (bin >= T1) flags |= 1u << e;
-                if (bin > T1) defmid += (tb + e >= s_end && tb + e < w_beg);
-            }
-            int tot;
-            int r = block_excl_scan<NT>(__popc(flags), s_warp, &tot);
-            uint32_t f = flags;
-            while (f) {
-                const int j = __ffs(f) - 1;
-                f &= f - 1;
-                const int64_t t = tb + j;
-                const float sj = srow[t];  // L1 hit: this thread just read it
-                const uint32_t key = float_key(sj);
-                cand[t0 + seg + r] = (int32_t)t;
-                ckey[t0 + seg + r] = key;
-                ++r;
-                if (!fallback && score_bin(sj, inv2A) == T1) {
-                    const unsigned slot = atomicAdd(ws.inbin_n + bh, 1u);
-                    if (slot < (unsigned)kInbinMax)
-                        ws.inbin[(int64_t)bh * kInbinMax + slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, 0u);
-                }
-            }
-            seg += tot;
-        }
-        int tot;
-        block_excl_scan<NT>(defmid, s_warp, &tot);
-        defmid = tot;
-    }
-    if (tid == 0) {
-        ws.seg_cnt[(int64_t)bh * kMaxSelCtas + cta] = seg;
-        ws.def_mid[(int64_t)bh * kMaxSelCtas + cta] = defmid;
-    }
-    bh_barrier(ws.bar + 2 * bh, nctas, nullptr);  // (2): segments, counts, in-bin list complete
-
+    const float *srow = ws.scores + (int64_t)bh * ws.ld;
     int32_t *out = sel_idx + (int64_t)bh * cap_sel;
+
     if (!normal || fallback) {
+        // ---- exact resolver of the two-kernel path (heavy ties, everything or nothing selected):
+        // CTA segments [t0, t0 + seg) of the tokens with bin >= T1, ascending
+        int seg = 0;
+        if (normal) {
+            for (int64_t base = t0; base < t1; base += (int64_t)NT * 32) {
+                const int64_t tb = base + (int64_t)tid * 32;
+                uint32_t flags = 0;
+                for (int e = 0; e < 32; ++e)
+                    if (tb + e < t1 && score_bin(__ldcg(srow + tb + e), inv2A) >= T1) flags |= 1u << e;
+                int tot;
+                int r = block_excl_scan<NT>(__popc(flags), s_warp, &tot);
+                while (flags) {
+                    const int j = __ffs(flags) - 1;
+                    flags &= flags - 1;
+                    cand[t0 + seg + r++] = (int32_t)(tb + j);
+                }
+                seg += tot;
+            }
+        }
+        if (tid == 0) ws.seg_cnt[(int64_t)bh * kMaxSelCtas + cta] = seg;
+        __threadfence();
+        cluster_sync();  // (2): segments complete (nothing reads another CTA's shared memory after this)
         if (cta != 0) return;
-        for (int k = tid; k < kBins; k += NT) ghist[k] = 0;
         SelState st;
         st.T1 = T1; st.above1 = above1; st.cnt_T1 = cnt_T1;
         st.flags = n == 0 ? kStateEmpty : (normal ? kStateNormal : kStateAll);
@@ -856,13 +931,106 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         return;
     }
 
-    // ---- fast path: rank the in-bin list (every CTA, redundantly; it is short)
-    uint4 *s_inb = reinterpret_cast<uint4 *>(so.lut);  // reuses the LUT region
-    const int c1 = cnt_T1;                            // == number of list entries
-    for (int e = tid; e < c1; e += NT) s_inb[e] = __ldcg(ws.inbin + (int64_t)bh * kInbinMax + e);
-    for (int c = tid; c < nctas; c += NT) s_mid[c] = __ldcg(ws.def_mid + (int64_t)bh * kMaxSelCtas + c);
+    // ---- fast path.  Warp w owns the 32-token chunks of its range; only the
+    // chunks whose maximum bin reaches T1 are re-read (lane = token, FB chunks
+    // per round trip).  A token is a candidate iff its score >= theta (exactly
+    // bin >= T1) and in the threshold bin iff also score < theta2.  The warp
+    // keeps its candidates in token order with their order keys -- the first CW
+    // in shared memory, the rest in its slice of the global segment -- lists the
+    // in-bin ones for the cluster and counts the definite middle ones.
+    uint4 *s_loc = reinterpret_cast<uint4 *>(so.lut);                      // this CTA's in-bin tokens
+    uint2 *wcand = reinterpret_cast<uint2 *>(so.lut + 16384) + warp * CW;  // per-warp candidates
+    uint4 *s_inb = reinterpret_cast<uint4 *>(so.lut + 32768);              // the cluster's in-bin tokens
+    const float theta = s_theta[0], theta2 = s_theta[1];
+    const int wb = warp * so.R;
+    const int we = (int)min((int64_t)(wb + so.R), t1 - t0);
+    const int nch = we > wb ? (we - wb + 31) >> 5 : 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    int ncand = 0, ndef = 0;
+    for (int cb = 0; cb < nch; cb += 32) {
+        const int gc = (wb >> 5) + cb + lane;
+        const bool hc = cb + lane < nch && (gc >= kCmaxCap || (int)so.cmax[gc] >= T1);
+        uint32_t hm = __ballot_sync(0xffffffffu, hc);
+        while (hm) {
+            float sv[FB];
+            int ci[FB];
+#pragma unroll
+            for (int f = 0; f < FB; ++f) {
+                ci[f] = -1;
+                sv[f] = 0.0f;
+                if (hm) {
+                    ci[f] = cb + __ffs(hm) - 1;
+                    hm &= hm - 1;
+                    const int i = wb + 32 * ci[f] + lane;
+                    if (i < we) sv[f] = __ldcg(srow + t0 + i);
+                }
+            }
+            // all loads land before any is used: one round trip per FB chunks
+#pragma unroll
+            for (int f = 0; f < FB; ++f) asm volatile("" ::"f"(sv[f]));
+#pragma unroll
+            for (int f = 0; f < FB; ++f) {
+                if (ci[f] < 0) break;
+                const int i = wb + 32 * ci[f] + lane;
+                const bool hit = i < we && sv[f] >= theta;
+                const uint32_t ball = __ballot_sync(0xffffffffu, hit);
+                if (hit) {
+                    const int j = ncand + __popc(ball & lt);
+                    const int t = (int)(t0 + i);
+                    const uint32_t key = float_key(sv[f]);
+                    if (j < CW) wcand[j] = make_uint2((uint32_t)t, key);
+                    else { cand[t0 + wb + j] = t; ckey[t0 + wb + j] = key; }
+                    if (sv[f] < theta2) {
+                        const int slot = atomicAdd(&s_ninb, 1);
+                        if (slot < kInbinMax) s_loc[slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, 0u);
+                    } else if (t >= s_end && t < w_beg) {
+                        ++ndef;
+                    }
+                }
+                ncand += __popc(ball);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
+    if (lane == 0) { s_wcnt[warp] = ncand; s_wdef[warp] = ndef; }
+    __syncthreads();
+    if (warp == 0) {
+        int d = s_wdef[lane];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (lane == 0) { s_pub[0] = min(s_ninb, kInbinMax); s_pub[1] = d; }
+    }
+    cluster_sync();  // (2): every CTA's in-bin list and counts are published
+
+    // ---- gather the cluster's in-bin lists (their sizes sum to cnt_T1)
+    if (warp == 0) {
+        int ni = 0, nd = 0;
+        if (lane < nctas) {
+            ni = (int)ld_cluster_u32(cluster_addr(&s_pub[0], lane));
+            nd = (int)ld_cluster_u32(cluster_addr(&s_pub[1], lane));
+        }
+        int incl = ni;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane < nctas) { s_cinb[lane] = incl - ni; s_mid[lane] = nd; }
+        if (lane == nctas - 1) s_cinb[nctas] = incl;
+    }
+    __syncthreads();
+    const int c1 = min(s_cinb[nctas], kInbinMax);  // == cnt_T1
+    for (int e = tid; e < c1; e += NT) {
+        int r = 0;
+        while (r + 1 < nctas && s_cinb[r + 1] <= e) ++r;
+        s_inb[e] = ld_cluster_v4(cluster_addr(s_loc + (e - s_cinb[r]), r));
+    }
     if (tid == 0) { s_misc[0] = 0; s_misc[1] = 0x7fffffff; }
     __syncthreads();
+    cluster_arrive();  // (3): done with the other CTAs' shared memory
+
+    // ---- rank the in-bin list (every CTA, redundantly; it is short)
     const int need1 = (int)kk - above1;  // 1 <= need1 <= c1
     if (need1 < c1) {
         for (int e = tid; e < c1; e += NT) {
@@ -878,69 +1046,62 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     }
     const uint32_t Tkey = (uint32_t)s_misc[0];
     const int IT = s_misc[1];
-    auto keep_inbin = [&](uint32_t key, int t) { return key > Tkey || (key == Tkey && t <= IT); };
+    auto keep = [&](int t, uint32_t key) {
+        if (t < s_end || t >= w_beg) return false;
+        return key_to_float(key) >= theta2 || key > Tkey || (key == Tkey && t <= IT);
+    };
     // selected in-bin tokens in the middle range, credited to their CTA
     for (int e = tid; e < c1; e += NT) {
         const int t = (int)s_inb[e].y;
-        if (t >= s_end && t < w_beg && keep_inbin(s_inb[e].x, t)) atomicAdd(&s_mid[s_inb[e].z], 1);
+        const uint32_t key = s_inb[e].x;
+        if (t >= s_end && t < w_beg && (key > Tkey || (key == Tkey && t <= IT))) atomicAdd(&s_mid[s_inb[e].z], 1);
     }
     __syncthreads();
-    int total_mid;
-    const int before = block_excl_scan<NT>(tid < nctas ? s_mid[tid] : 0, s_warp, &total_mid);
-    if (tid == cta) s_misc[2] = before;
+    int before = 0, total_mid = 0;
+    for (int r = 0; r < nctas; ++r) {
+        before += r < cta ? s_mid[r] : 0;
+        total_mid += s_mid[r];
+    }
+    // ---- each warp: kept count, prefix over warps, ordered emission
+    auto cand_at = [&](int j, int &t, uint32_t &key) {
+        if (j < CW) { const uint2 c = wcand[j]; t = (int)c.x; key = c.y; }
+        else { t = __ldcg(cand + t0 + wb + j); key = __ldcg(ckey + t0 + wb + j); }
+    };
+    int nkeep = 0;
+    for (int j = lane; j < ncand; j += 32) {
+        int t; uint32_t key;
+        cand_at(j, t, key);
+        nkeep += keep(t, key);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) nkeep += __shfl_xor_sync(0xffffffffu, nkeep, o);
+    if (lane == 0) s_wkeep[warp] = nkeep;
     __syncthreads();
-    const int obase = s_end + s_misc[2];
-
-    // own segment: keep bin > T1, or in-bin under the (Tkey, IT) rule; middle only
-    {
-        const int per = (seg + NT - 1) / NT;
-        const int e0 = tid * per, e1 = min(seg, e0 + per);
-        constexpr int MAXPER = 8;  // elements held in registers per thread (else re-read)
-        int tt[MAXPER];
-        uint32_t kk2[MAXPER];
-        auto keep = [&](int t, uint32_t key) {
-            if (t < s_end || t >= w_beg) return false;
-            return score_bin(key_to_float(key), inv2A) > T1 || keep_inbin(key, t);
-        };
-#pragma unroll
-        for (int j = 0; j < MAXPER; ++j) {
-            const int e = e0 + j;
-            tt[j] = e < e1 ? __ldcg(cand + t0 + e) : -1;
-            kk2[j] = e < e1 ? __ldcg(ckey + t0 + e) : 0u;
+    int wpos = s_end + before;
+    for (int w2 = 0; w2 < warp; ++w2) wpos += s_wkeep[w2];
+    for (int jb = 0; jb < ncand; jb += 32) {
+        const int j = jb + lane;
+        int t = 0; uint32_t key = 0;
+        if (j < ncand) cand_at(j, t, key);
+        const bool k2 = j < ncand && keep(t, key);
+        const uint32_t ball = __ballot_sync(0xffffffffu, k2);
+        if (k2) {
+            const int p = wpos + __popc(ball & lt);
+            if (p < cap_sel) out[p] = t;
         }
-        int cnt = 0;
-#pragma unroll
-        for (int j = 0; j < MAXPER; ++j) cnt += (e0 + j < e1) && keep(tt[j], kk2[j]);
-        for (int e = e0 + MAXPER; e < e1; ++e) cnt += keep(__ldcg(cand + t0 + e), __ldcg(ckey + t0 + e));
-        int tot;
-        int r = block_excl_scan<NT>(cnt, s_warp, &tot);
-        if (cnt) {
-#pragma unroll
-            for (int j = 0; j < MAXPER; ++j)
-                if (e0 + j < e1 && keep(tt[j], kk2[j])) {
-                    if (obase + r < cap_sel) out[obase + r] = tt[j];
-                    ++r;
-                }
-            for (int e = e0 + MAXPER; e < e1; ++e) {
-                const int t = __ldcg(cand + t0 + e);
-                if (keep(t, __ldcg(ckey + t0 + e))) {
-                    if (obase + r < cap_sel) out[obase + r] = t;
-                    ++r;
-                }
-            }
-        }
+        wpos += __popc(ball);
     }
     if (cta == 0) {
         for (int t = tid; t < s_end; t += NT) out[t] = t;
-        const int wpos = s_end + total_mid;
+        const int wpos0 = s_end + total_mid;
         for (int t = w_beg + tid; t < n; t += NT)
-            if (wpos + (t - w_beg) < cap_sel) out[wpos + (t - w_beg)] = t;
-        int total = wpos + (int)(n - w_beg);
+            if (wpos0 + (t - w_beg) < cap_sel) out[wpos0 + (t - w_beg)] = t;
+        int total = wpos0 + (int)(n - w_beg);
         if (total > cap_sel) total = cap_sel;
         for (int r = total + tid; r < cap_sel; r += NT) out[r] = -1;
         if (tid == 0) sel_cnt[bh] = total;
-        for (int k = tid; k < kBins; k += NT) ghist[k] = 0;
     }
+    cluster_wait();  // (3): no CTA leaves while another may still read its shared memory
 }
 
 }  // namespace dkv

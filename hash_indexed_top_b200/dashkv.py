@@ -20,7 +20,6 @@ LIB_PATH = os.path.join(_HERE, "libdashkv.so")
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace missing or too small",
     4: "sequence length beyond cache capacity", 5: "CUDA error", 6: "page id out of range", 7: "no CUDA device",
-    8: "in-kernel wait timed out",
 }
 
 FLAG_TWO_KERNEL_SELECT = 1
@@ -96,6 +95,27 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream: Optional[torch.cuda.Stream]):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def canonical_codes(codes: torch.Tensor, bits: int) -> torch.Tensor:
+    """Undo the storage rotation of key codes (host or device tensor, int64).
+
+    The library stores token t's code with its T = bits/8 bytes rotated by
+    t mod T (stored byte p = code byte (p + t mod T) mod T); the token position
+    is the second-to-last axis in both layouts (dense [B,Hkv,n_cap,W], paged
+    [P,Hkv,page,W], page a multiple of 32).  Returns the codes with hyperplane j
+    at word j/64, bit j%64."""
+    T = bits // 8
+    W = codes.shape[-1]
+    n = codes.shape[-2]
+    b = codes.contiguous().view(torch.uint8).reshape(*codes.shape[:-1], W * 8)
+    rho = torch.arange(n, device=codes.device) % T
+    src = (torch.arange(T, device=codes.device)[None, :] - rho[:, None]) % T  # original c <- stored (c - rho) mod T
+    idx = src.expand(*b.shape[:-1], T)
+    orig = torch.gather(b[..., :T], -1, idx)
+    full = torch.zeros_like(b)
+    full[..., :T] = orig
+    return full.reshape(*codes.shape[:-1], W * 8).view(torch.int64).reshape(codes.shape)
 
 
 def hyperplanes(seed: int, bits: int, d: int) -> torch.Tensor:

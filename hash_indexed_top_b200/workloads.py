@@ -202,4 +202,4 @@ class L2Flush:
 
     def __call__(self, i: int = 0) -> None:
         self.dirty.fill_(i)
-        torch.sum(self.clean, out=self.sink)
+        torch.sum(self.clean, dim=0, out=self.sink)

@@ -48,8 +48,13 @@
  *      codes, paged         : u64  [num_pages][Hkv][page_size][W]
  *      token t of sequence b lives in physical page
  *      page_table[b * max_pages + t / page_size], slot t % page_size.
- *      Hyperplane j's bit sits in code word j / 64 at bit position j % 64;
- *      a 32-bit code occupies the low half of its word (high half zero).
+ *      Code bits: hyperplane j is bit j % 8 of code byte j / 8 (T = bits/8
+ *      bytes, little-endian, i.e. word j / 64 bit j % 64 before the rotation
+ *      below; a 32-bit code occupies the low half of its word, high half 0).
+ *      Storage rotation: token t's T code bytes are stored rotated by t mod T
+ *      (stored byte p holds code byte (p + t mod T) mod T), the order in which
+ *      the scorer's lanes consume them.  (Paged: page_size is a multiple of 32,
+ *      so the slot index gives the same t mod T.)
  *      queries q : bf16 [B][Hq][d]; query head h reads KV head h / G.
  *  - seq_lens (device int32 [B]) holds each sequence's cached length; the
  *    current decode step's own key is expected to be appended first, so the
@@ -73,14 +78,15 @@ typedef enum dashkv_status {
     DASHKV_ERR_CAPACITY = 4,     /* device error word: a sequence outgrew its cache   */
     DASHKV_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, sync, copy)   */
     DASHKV_ERR_DEVICE = 6,       /* device error word: bad page id in page_table      */
-    DASHKV_ERR_NO_DEVICE = 7,    /* no usable CUDA device                             */
-    DASHKV_ERR_TIMEOUT = 8       /* device error word: a bounded in-kernel wait gave up */
+    DASHKV_ERR_NO_DEVICE = 7     /* no usable CUDA device                             */
 } dashkv_status;
 
-/* Selection path.  By default dashkv_select runs one cooperative kernel
- * whose CTAs (one per SM, so at most the SM count of them) synchronise per
- * (sequence, kv head); when B * Hkv exceeds the SM count, or with this flag,
- * it runs two ordinary kernels instead.  Both give identical results. */
+/* Selection path.  By default dashkv_select runs one kernel with one
+ * thread-block cluster per (sequence, kv head): its CTAs (one per SM, up to
+ * 16 per cluster) exchange histograms and boundary tokens through distributed
+ * shared memory and hardware cluster barriers.  Without cluster launch
+ * support, or with this flag, it runs two ordinary kernels instead.  Both give
+ * identical results. */
 #define DASHKV_FLAG_TWO_KERNEL_SELECT 1
 
 /* Problem description.  Supported: head_dim in {64, 128}; bits in
@@ -165,10 +171,8 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    size_t workspace_bytes, void *stream);
 
 /* Synchronise `stream`, then read and clear the current device's error
- * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, DASHKV_ERR_TIMEOUT
- * (the selection's CTAs could not all be resident together, e.g. because other
- * work held the SMs; its output is then invalid), or DASHKV_ERR_CUDA when the
- * stream reports an error. */
+ * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, or DASHKV_ERR_CUDA
+ * when the stream reports an error. */
 dashkv_status dashkv_get_error(void *stream);
 
 /* The hyperplanes a context built with (seed, bits, d) uses, as int8 +1/-1
@@ -176,7 +180,7 @@ dashkv_status dashkv_get_error(void *stream);
 dashkv_status dashkv_hyperplanes(uint64_t seed, int32_t bits, int32_t head_dim, int8_t *host_out);
 
 /* Number of kernels dashkv_select launches for caches of `max_tokens` tokens
- * per sequence: 1 (fused, cooperative) or 2 (score, then collect); 0 when ctx
+ * per sequence: 1 (fused, clustered) or 2 (score, then collect); 0 when ctx
  * is NULL.  For profiling tools that trace individual kernels. */
 int32_t dashkv_select_kernels(const dashkv_ctx *ctx, int64_t max_tokens);
 

@@ -81,7 +81,7 @@ def within_tol(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
 
 def compare_step(g: GpuRun, o: OracleRun, r: dict, what: str = "") -> dict:
     """Assert parity of one step; returns a few diagnostics."""
-    gc = g.cache.codes.cpu().numpy().view(np.uint64)
+    gc = dk.canonical_codes(g.cache.codes, o.cfg.bits).cpu().numpy().view(np.uint64)
     assert np.array_equal(gc, o.codes), f"{what}: codes differ at {np.argwhere(gc != o.codes)[:5].tolist()}"
     assert np.array_equal(g.seq.cpu().numpy(), o.seq), f"{what}: seq_lens differ"
     gs = g.scores.cpu().numpy()

@@ -85,3 +85,19 @@ def test_create_without_device_reports_no_device():
     assert dk.lib().dashkv_create(ctypes.byref(cfg), ctypes.byref(h)) == 7
     with pytest.raises(RuntimeError):
         dk.DashKV(1, 4, 1, 64, 32, 8, 0, 0)
+
+
+@pytest.mark.parametrize("bits", [32, 64, 128])
+def test_canonical_codes_undoes_the_storage_rotation(bits):
+    # stored byte p of token t holds code byte (p + t mod T) mod T
+    T, W = bits // 8, max(1, bits // 64)
+    rng = np.random.default_rng(bits)
+    orig = rng.integers(0, 256, size=(2, 3, 70, W * 8), dtype=np.uint8)
+    orig[..., T:] = 0
+    stored = np.zeros_like(orig)
+    for t in range(70):
+        for p in range(T):
+            stored[:, :, t, p] = orig[:, :, t, (p + t % T) % T]
+    st = torch.from_numpy(stored.copy()).view(torch.int64).reshape(2, 3, 70, W)
+    back = dk.canonical_codes(st, bits).view(torch.uint8).reshape(2, 3, 70, W * 8).numpy()
+    assert np.array_equal(back, orig)
