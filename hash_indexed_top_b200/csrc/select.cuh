@@ -116,20 +116,22 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
 // ---------------------------------------------------------------------------
 // Score + histogram.
 //
-// One CTA of 1024 threads per SM.  The byte-LUT (256 rows x 256 B; row v holds
-// LUT_c[v] for the T tables, replicated 32/T times) sits at a shared address
-// whose low 16 bits are zero, so one byte-permute of (code word, per-lane
-// offset) yields the complete shared address of a lookup:
-//   addr = lut_base | byte << 8 | 4 * (copy * T + table).
-// Lane l reads its token's bytes rotated by rho = l % T, so at each step the
-// 32 lanes touch 32 distinct banks.
+// One CTA of 1024 threads per SM.  The byte-LUT (256 rows x 256 B; word j of
+// row v holds LUT_{j mod T}[v], j = 0..63) sits at a shared address whose low
+// 16 bits are zero.  Lane l handles tokens t = l (mod 32), stored rotated by
+// t mod T (stored byte r = code byte (r + l) mod T), so at step r it needs
+// table (l + r) mod T, i.e. word l + r of the row of its byte.  One
+// byte-permute of (code word, lane base) yields the row address
+//   lut_base | byte << 8 | 4 l
+// and the load adds the immediate 4 r: one permute, one load and one add per
+// byte, with a single per-lane register.  At each step the 32 lanes read
+// words l + r of their rows: 32 distinct banks.
 constexpr int kScoreThreads = 1024;
 constexpr int kScoreThreadsConst = kScoreThreads;
 
 template <int BITS>
 struct ScoreShape {
     static constexpr int T = BITS / 8;         // byte tables
-    static constexpr int COPIES = 32 / T;      // interleaved copies: lanes hit distinct banks
     static constexpr int NW = BITS / 32;       // 32-bit code words per token
     static constexpr uint32_t LUT_BYTES = 256 * 256;
     static constexpr uint32_t SCRATCH_BYTES = kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;  // hist + scratch
@@ -156,22 +158,33 @@ __device__ __forceinline__ void unpack_code(const typename ScoreShape<BITS>::Vec
 // Shared-memory load from a 32-bit shared address.  Not volatile: its address
 // always depends on code words loaded after the barrier that publishes the LUT,
 // so it cannot be scheduled before that barrier.
+template <int IMM>
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
     float v;
-    asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(IMM));
     return v;
 }
 
+// Terms r = 0 .. R - 1 of a score (even r into s0, odd r into s1, ascending).
+template <int BITS, int R>
+struct LutTerms {
+    static __device__ __forceinline__ void add(const uint32_t (&w)[BITS / 32], uint32_t base, float &s0, float &s1) {
+        LutTerms<BITS, R - 1>::add(w, base, s0, s1);
+        constexpr int r = R - 1;
+        const float v = lds_f32<4 * r>(__byte_perm(w[r >> 2], base, 0x7604u | ((uint32_t)(r & 3) << 4)));
+        if (r % 2 == 0) s0 += v; else s1 += v;
+    }
+};
+template <int BITS>
+struct LutTerms<BITS, 0> {
+    static __device__ __forceinline__ void add(const uint32_t (&)[BITS / 32], uint32_t, float &, float &) {}
+};
+
 // Score of one (rotated) code: sum over its T bytes of the lane's table entries.
 template <int BITS>
-__device__ __forceinline__ float lut_score(const uint32_t (&w)[BITS / 32], const uint32_t (&off)[BITS / 8]) {
-    constexpr int T = BITS / 8;
+__device__ __forceinline__ float lut_score(const uint32_t (&w)[BITS / 32], uint32_t base) {
     float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-    for (int r = 0; r < T; r += 2) {
-        s0 += lds_f32(__byte_perm(w[r >> 2], off[r], 0x7604u | ((uint32_t)(r & 3) << 4)));
-        s1 += lds_f32(__byte_perm(w[(r + 1) >> 2], off[r + 1], 0x7604u | ((uint32_t)((r + 1) & 3) << 4)));
-    }
+    LutTerms<BITS, BITS / 8>::add(w, base, s0, s1);
     return (s0 + s1) + 0.0f;  // + 0 turns a -0 into +0
 }
 
@@ -236,8 +249,8 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
         for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
         if (lane == 0) red[0] = a > 0.0f ? 0.5f / a : 0.0f;
     }
-    // LUT rows: word (v * 64 + copy * T + c) holds LUT_c[v]; lane l fills word l
-    // of each row it owns (copy = l / T, c = l % T), so stores never conflict.
+    // LUT rows: word j of row v holds LUT_{j mod T}[v]; lane l fills words l and
+    // l + 32 (both table l mod T, as 32 is a multiple of T) of the rows it owns.
     {
         const int c = lane % T;
         float qv[8];
@@ -247,7 +260,9 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
             float val = 0.0f;
 #pragma unroll
             for (int u = 0; u < 8; ++u) val += ((v >> u) & 1) ? qv[u] : -qv[u];
-            reinterpret_cast<float *>(lut + v * 256)[lane] = val;
+            float *row = reinterpret_cast<float *>(lut + v * 256);
+            row[lane] = val;
+            row[lane + 32] = val;
         }
     }
     __syncthreads();
@@ -263,12 +278,9 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     const float inv2A = o.inv2A;
 
     // Lane l always handles tokens with t % 32 == l, whose stored bytes are
-    // rotated by rho = l % T (see store_code_rotated): at step r it reads byte r,
-    // which is code byte (r + rho) % T, from table (r + rho) % T in copy l / T.
-    const int rho = lane % T, copy = lane / T;
-    uint32_t off[T];
-#pragma unroll
-    for (int r = 0; r < T; ++r) off[r] = lut_s | 4u * (uint32_t)(copy * T + (rho + r) % T);
+    // rotated by l % T (see store_code_rotated): at step r it reads stored byte
+    // r, which is code byte (r + l) % T, from word l + r of the byte's LUT row.
+    const uint32_t lbase = lut_s | 4u * (uint32_t)lane;  // row address = lbase | byte << 8
 
     const int nloc = (int)(t1 - t0);  // tokens of this CTA (< 2^31)
     // Warp w streams the contiguous range [w R, (w + 1) R) of the CTA's tokens,
@@ -323,7 +335,7 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
         if (i < we) {
             uint32_t w[NW];
             unpack_code<BITS>(code, w);
-            const float s = lut_score<BITS>(w, off);
+            const float s = lut_score<BITS>(w, lbase);
             srow[i] = s;
             bin = score_bin(s, inv2A);
             atomicAdd(&hist[bin], 1u);
