@@ -21,6 +21,19 @@ __device__ unsigned g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }
 
+// Thread-block cluster barrier (every thread of every CTA of the cluster
+// arrives; release / acquire order their memory accesses at cluster scope).
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+    cluster_arrive();
+    cluster_wait();
+}
+
 // Hyperplanes as sign bits: bit (i % 32) of word [j * (d / 32) + i / 32] is set
 // when R[j][i] = -1.  2 KB at bits = d = 128, passed by value as a kernel
 // parameter (constant bank), so no device allocation is needed.

@@ -258,10 +258,23 @@ void launch_encode_d(const dashkv_ctx *ctx, const KV &kv, const int32_t *s, cuda
 template <int BITS, int D>
 void launch_append_bd(const dashkv_ctx *ctx, const KV &kv, const void *kn, const void *vn, int32_t *seq,
                       cudaStream_t st) {
-    int threads = ctx->cfg.num_kv_heads * BITS;
-    if (threads > kAppendThreads) threads = kAppendThreads;
-    launch_pdl(append_keys_kernel<BITS, D>, dim3(ctx->cfg.batch), dim3(threads), 0, st, kv,
-               static_cast<const __nv_bfloat16 *>(kn), static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R);
+    // one cluster of C CTAs per sequence (early start behind the preceding kernel)
+    const int C = ctx->cfg.num_kv_heads < kAppendCluster ? ctx->cfg.num_kv_heads : kAppendCluster;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, ctx->cfg.batch);
+    cfg.blockDim = dim3(kAppendThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, append_keys_kernel<BITS, D>, kv, static_cast<const __nv_bfloat16 *>(kn),
+                       static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R);
 }
 
 template <int D>

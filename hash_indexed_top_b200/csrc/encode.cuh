@@ -109,82 +109,84 @@ encode_keys_kernel(KV kv, const int32_t *__restrict__ seq_lens, const RBits R, i
 }
 
 // ---------------------------------------------------------------------------
-// Decode-step append.  One CTA per sequence: copy the new K/V rows of every kv
-// head into slot seq_lens[b], encode each new key (one thread per
-// (head, hyperplane); the sign bits of a warp are gathered with one ballot),
-// then bump seq_lens[b] once every head is done.
-constexpr int kAppendThreads = 1024;
+// Decode-step append.  One cluster of C = min(Hkv, kAppendCluster) CTAs per
+// sequence; CTA c handles kv heads c, c + C, ...: it copies the new K/V rows
+// into slot seq_lens[b] and encodes the new key (thread j = hyperplane j, one
+// sequential FMA chain over the dims as in the whole-cache encoder; the sign
+// bits of a warp are gathered with one ballot).  After a cluster barrier --
+// every CTA has read seq_lens[b] -- CTA 0 bumps it.
+constexpr int kAppendThreads = 128;
+constexpr int kAppendCluster = 8;
 
 template <int BITS, int D>
 __global__ void __launch_bounds__(kAppendThreads)
 append_keys_kernel(KV kv, const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *__restrict__ v_new,
                    int32_t *seq_lens, const RBits R) {
-    constexpr int WPR = D / 32;                 // R words per hyperplane
-    __shared__ uint32_t Rb[BITS * WPR];         // [j][word]
-    __shared__ float kf[32][D];
-    __shared__ uint32_t code32[32][BITS / 32];
-    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    constexpr int WPR = D / 32;  // R words per hyperplane
+    constexpr int CPR = D / 8;   // 16-byte chunks per row
+    __shared__ float4 kf4[D / 4];
+    __shared__ uint32_t code32[BITS / 32];
+    const int b = blockIdx.y, c = blockIdx.x, C = gridDim.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int Hkv = kv.Hkv;
-    for (int e = tid; e < BITS * WPR; e += blockDim.x) Rb[e] = R.w[e];
+    uint32_t rw[WPR];  // this thread's hyperplane (depends on the context only)
+#pragma unroll
+    for (int w = 0; w < WPR; ++w) rw[w] = tid < BITS ? R.w[tid * WPR + w] : 0u;
 
     griddep_wait();
     griddep_trigger();  // the scorer may start building its LUT meanwhile
-    // every thread checks the slot itself (no extra barrier); thread 0 reports
     const int64_t pos = seq_lens[b];
     bool ok = pos >= 0 && pos < kv.capacity();
     if (ok && kv.page_size) {
         const int32_t p = __ldg(kv.page_table + (int64_t)b * kv.max_pages + pos / kv.page_size);
         ok = p >= 0 && p < kv.num_pages;
-        if (!ok && tid == 0) raise_error(kErrPage);
-    } else if (!ok && tid == 0) {
+        if (!ok && c == 0 && tid == 0) raise_error(kErrPage);
+    } else if (!ok && c == 0 && tid == 0) {
         raise_error(kErrCapacity);
     }
-    constexpr int CPR = D / 8;  // 16-byte chunks per row
     if (ok) {
-        for (int c = tid; c < 2 * Hkv * CPR; c += blockDim.x) {
-            const int isv = c >= Hkv * CPR;
-            const int cc = isv ? c - Hkv * CPR : c;
-            const int h = cc / CPR, part = cc % CPR;
+        for (int h = c; h < Hkv; h += C) {
             const int64_t r = kv.row(b, h, pos);
-            const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + ((int64_t)b * Hkv + h) * D);
-            const uint4 x = __ldg(src + part);
-            reinterpret_cast<uint4 *>((isv ? kv.v : kv.k) + r)[part] = x;
-            if (!isv) {
-                float *dst = &kf[h][8 * part];
-                dst[0] = bf16_lo(x.x); dst[1] = bf16_hi(x.x); dst[2] = bf16_lo(x.y); dst[3] = bf16_hi(x.y);
-                dst[4] = bf16_lo(x.z); dst[5] = bf16_hi(x.z); dst[6] = bf16_lo(x.w); dst[7] = bf16_hi(x.w);
+            for (int e = tid; e < 2 * CPR; e += kAppendThreads) {
+                const int isv = e >= CPR;
+                const int part = isv ? e - CPR : e;
+                const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + ((int64_t)b * Hkv + h) * D);
+                const uint4 x = __ldg(src + part);
+                reinterpret_cast<uint4 *>((isv ? kv.v : kv.k) + r)[part] = x;
+                if (!isv) {
+                    kf4[2 * part] = make_float4(bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y));
+                    kf4[2 * part + 1] = make_float4(bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w));
+                }
             }
-        }
-    }
-    __syncthreads();
-    if (ok) {
-        // thread -> (head, hyperplane): a warp covers 32 consecutive hyperplanes of one head
-        for (int x = tid; x < Hkv * BITS; x += blockDim.x) {
-            const int h = x / BITS, j = x % BITS;
-            uint32_t rw[WPR];
+            __syncthreads();
+            if (tid < BITS) {  // whole warps (BITS is a multiple of 32)
+                float acc = 0.0f;
 #pragma unroll
-            for (int w = 0; w < WPR; ++w) rw[w] = Rb[j * WPR + w];
-            float acc = 0.0f;
+                for (int i4 = 0; i4 < D / 4; ++i4) {
+                    const float4 k4 = kf4[i4];
+                    const float kx[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int i = 0; i < D; ++i) {
-                const float rf = ((rw[i / 32] >> (i % 32)) & 1u) ? -1.0f : 1.0f;
-                acc = fmaf(rf, kf[h][i], acc);
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = 4 * i4 + u;
+                        const float rf = ((rw[i / 32] >> (i % 32)) & 1u) ? -1.0f : 1.0f;
+                        acc = fmaf(rf, kx[u], acc);
+                    }
+                }
+                const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
+                if (lane == 0) code32[tid >> 5] = word;
             }
-            const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
-            if (lane == 0) code32[h][j / 32] = word;
-        }
-    }
-    __syncthreads();
-    if (ok) {
-        for (int h = tid; h < Hkv; h += blockDim.x) {
-            uint32_t w32[BITS / 32];
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t w32[BITS / 32];
 #pragma unroll
-            for (int k = 0; k < BITS / 32; ++k) w32[k] = code32[h][k];
-            store_code_rotated<BITS>(kv.codes + kv.code(b, h, pos), w32, pos);
+                for (int k = 0; k < BITS / 32; ++k) w32[k] = code32[k];
+                store_code_rotated<BITS>(kv.codes + kv.code(b, h, pos), w32, pos);
+            }
+            __syncthreads();  // kf4 and code32 are reused by the next head
         }
     }
-    __syncthreads();
-    if (tid == 0 && ok) seq_lens[b] = (int32_t)(pos + 1);
+    cluster_sync();  // every CTA of this sequence has read seq_lens[b]
+    if (c == 0 && tid == 0 && ok) seq_lens[b] = (int32_t)(pos + 1);
 }
 
 }  // namespace dkv

@@ -734,16 +734,6 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
 constexpr int kInbinMax = 1024;
 constexpr int kMaxCluster = 16;
 
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-    cluster_arrive();
-    cluster_wait();
-}
 // Address, in the cluster's shared window, of the object at `p` (this CTA's
 // shared memory) in the CTA of cluster rank `rank`.
 __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
@@ -756,6 +746,9 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
     uint4 v;
@@ -863,16 +856,24 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     constexpr int NT = kScoreThreads;
     constexpr int NWARP = NT / 32;
     constexpr int CW = 64;  // candidates per warp kept in shared memory (more go to the global segment)
-    constexpr int FB = 8;   // hit chunks whose scores one warp loads per round trip
+    // hit chunks whose scores one warp stages per round trip: [FB][32] floats per
+    // warp in the code ring, which is idle once the scores are written
+    constexpr int FB = (int)(ScoreShape<BITS>::RING_BYTES / (NWARP * 32 * 4)) < 16
+                           ? (int)(ScoreShape<BITS>::RING_BYTES / (NWARP * 32 * 4)) : 16;
+    static_assert(FB >= 1 && (size_t)FB * NWARP * 32 * 4 <= ScoreShape<BITS>::RING_BYTES, "staging exceeds the ring");
+    // the LUT region (64 KB) after scoring: in-bin list | warp candidates | gathered list, or the resolver
+    static_assert(kInbinMax * 16 <= 16384 && NWARP * CW * 8 <= 16384, "fast-path lists exceed their slots");
+    static_assert(sizeof(ResolveSmem<4096>) <= ScoreShape<BITS>::LUT_BYTES, "resolver exceeds the LUT region");
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ int s_warp[32];
     __shared__ int s_thr[4];
     __shared__ int s_misc[4];
     __shared__ float s_theta[2];
     __shared__ uint32_t s_coarse[64];      // this CTA's histogram per super-bin (read by the cluster)
-    __shared__ int s_pub[2];               // this CTA's in-bin entries, definite middle tokens (read by the cluster)
-    __shared__ int s_cinb[kMaxCluster + 1], s_mid[kMaxCluster];
-    __shared__ int s_wcnt[NWARP], s_wdef[NWARP], s_wkeep[NWARP];
+    __shared__ int s_cnt[kMaxCluster][2];  // per CTA of the cluster: in-bin entries, definite middle tokens
+    __shared__ int s_mid[kMaxCluster];
+    __shared__ int s_wkeep[NWARP];
+    __shared__ int s_hlist[NWARP][32];     // per warp: its hit chunks of the current group
     __shared__ int s_ninb;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.y, cta = blockIdx.x;  // cta = rank in the cluster (cluster = the row of CTAs)
@@ -944,12 +945,14 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     }
 
     // ---- fast path.  Warp w owns the 32-token chunks of its range; only the
-    // chunks whose maximum bin reaches T1 are re-read (lane = token, FB chunks
-    // per round trip).  A token is a candidate iff its score >= theta (exactly
-    // bin >= T1) and in the threshold bin iff also score < theta2.  The warp
-    // keeps its candidates in token order with their order keys -- the first CW
-    // in shared memory, the rest in its slice of the global segment -- lists the
-    // in-bin ones for the cluster and counts the definite middle ones.
+    // chunks whose maximum bin reaches T1 are re-read (lane = token, up to FB
+    // chunks per memory round trip, staged in shared memory so that the code
+    // that runs once per step stays a pair of short loops).  A token is a candidate iff its score >=
+    // theta (exactly bin >= T1) and in the threshold bin iff also score <
+    // theta2.  The warp keeps its candidates in token order with their order
+    // keys -- the first CW in shared memory, the rest in its slice of the global
+    // segment -- lists the in-bin ones for the cluster and counts the definite
+    // middle ones.
     uint4 *s_loc = reinterpret_cast<uint4 *>(so.lut);                      // this CTA's in-bin tokens
     uint2 *wcand = reinterpret_cast<uint2 *>(so.lut + 16384) + warp * CW;  // per-warp candidates
     uint4 *s_inb = reinterpret_cast<uint4 *>(so.lut + 32768);              // the cluster's in-bin tokens
@@ -959,137 +962,186 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     const int nch = we > wb ? (we - wb + 31) >> 5 : 0;
     const uint32_t lt = (1u << lane) - 1u;
     int ncand = 0, ndef = 0;
-    for (int cb = 0; cb < nch; cb += 32) {
-        const int gc = (wb >> 5) + cb + lane;
-        const bool hc = cb + lane < nch && (gc >= kCmaxCap || (int)so.cmax[gc] >= T1);
-        uint32_t hm = __ballot_sync(0xffffffffu, hc);
-        while (hm) {
-            float sv[FB];
-            int ci[FB];
-#pragma unroll
-            for (int f = 0; f < FB; ++f) {
-                ci[f] = -1;
-                sv[f] = 0.0f;
-                if (hm) {
-                    ci[f] = cb + __ffs(hm) - 1;
-                    hm &= hm - 1;
-                    const int i = wb + 32 * ci[f] + lane;
-                    if (i < we) sv[f] = __ldcg(srow + t0 + i);
-                }
+    auto chunk_hit = [&](int c) {
+        const int gc = (wb >> 5) + c;
+        return c < nch && (gc >= kCmaxCap || (int)so.cmax[gc] >= T1);
+    };
+    // per-warp staging buffer [FB][32] of scores, in the (now idle) code ring,
+    // and the warp's list of hit chunks of the current group of 32
+    float *fbuf = reinterpret_cast<float *>(so.lut + 65536) + warp * (FB * 32);
+    const uint32_t fbuf_s = (uint32_t)__cvta_generic_to_shared(fbuf);
+    int *hlist = s_hlist[warp];
+    const int wlen = we - wb;  // tokens of this warp
+    for (int g0 = 0; g0 < nch; g0 += 32) {
+        const bool hc = chunk_hit(g0 + lane);
+        const uint32_t hb = __ballot_sync(0xffffffffu, hc);
+        if (hc) hlist[__popc(hb & lt)] = g0 + lane;
+        __syncwarp();
+        const int nh = __popc(hb);
+        for (int h0 = 0; h0 < nh; h0 += FB) {
+            const int nf = min(FB, nh - h0);
+            // stage the scores of chunks h0 .. h0 + nf - 1: 16 bytes per lane, 4 chunks
+            // per instruction, all in flight at once (whole chunks: rows are padded
+            // to 64 tokens, so a chunk never runs past its row)
+#pragma unroll 1
+            for (int q = lane; q < 8 * nf; q += 32) {
+                const int c = hlist[h0 + (q >> 3)];
+                const float *src = srow + t0 + wb + 32 * c + 4 * (q & 7);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(fbuf_s + 16u * (uint32_t)q), "l"(src)
+                             : "memory");
             }
-            // all loads land before any is used: one round trip per FB chunks
-#pragma unroll
-            for (int f = 0; f < FB; ++f) asm volatile("" ::"f"(sv[f]));
-#pragma unroll
-            for (int f = 0; f < FB; ++f) {
-                if (ci[f] < 0) break;
-                const int i = wb + 32 * ci[f] + lane;
-                const bool hit = i < we && sv[f] >= theta;
+            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+            __syncwarp();
+#pragma unroll 1
+            for (int f = 0; f < nf; ++f) {
+                const int li = 32 * hlist[h0 + f] + lane;  // warp-local token
+                const float sv = fbuf[32 * f + lane];
+                const bool hit = li < wlen && sv >= theta;
                 const uint32_t ball = __ballot_sync(0xffffffffu, hit);
                 if (hit) {
                     const int j = ncand + __popc(ball & lt);
-                    const int t = (int)(t0 + i);
-                    const uint32_t key = float_key(sv[f]);
+                    const int t = (int)(t0 + wb + li);
+                    const uint32_t key = float_key(sv);
                     if (j < CW) wcand[j] = make_uint2((uint32_t)t, key);
                     else { cand[t0 + wb + j] = t; ckey[t0 + wb + j] = key; }
-                    if (sv[f] < theta2) {
+                    if (sv < theta2) {
                         const int slot = atomicAdd(&s_ninb, 1);
-                        if (slot < kInbinMax) s_loc[slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, 0u);
+                        if (slot < kInbinMax)
+                            s_loc[slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, (uint32_t)warp);
                     } else if (t >= s_end && t < w_beg) {
                         ++ndef;
                     }
                 }
                 ncand += __popc(ball);
             }
+            __syncwarp();  // the buffer is refilled by the next batch
         }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
-    if (lane == 0) { s_wcnt[warp] = ncand; s_wdef[warp] = ndef; }
+    if (lane == 0) s_wkeep[warp] = ndef;  // kept candidates of the warp: + its selected in-bin ones
     __syncthreads();
     if (warp == 0) {
-        int d = s_wdef[lane];
+        // publish (in-bin entries, definite middle tokens) into every CTA's s_cnt[cta]
+        int d = s_wkeep[lane];
 #pragma unroll
         for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        if (lane == 0) { s_pub[0] = min(s_ninb, kInbinMax); s_pub[1] = d; }
-    }
-    cluster_sync();  // (2): every CTA's in-bin list and counts are published
-
-    // ---- gather the cluster's in-bin lists (their sizes sum to cnt_T1)
-    if (warp == 0) {
-        int ni = 0, nd = 0;
+        const int ni = min(s_ninb, kInbinMax);
         if (lane < nctas) {
-            ni = (int)ld_cluster_u32(cluster_addr(&s_pub[0], lane));
-            nd = (int)ld_cluster_u32(cluster_addr(&s_pub[1], lane));
+            st_cluster_u32(cluster_addr(&s_cnt[cta][0], lane), (uint32_t)ni);
+            st_cluster_u32(cluster_addr(&s_cnt[cta][1], lane), (uint32_t)d);
         }
+    }
+    cluster_sync();  // (2): every CTA's in-bin list is complete and its counts delivered
+
+    // ---- gather the cluster's in-bin lists (their sizes sum to cnt_T1 <= NT):
+    // thread e copies entry e from the CTA whose list holds it
+    const int c1 = cnt_T1;
+    if (warp * 32 < c1) {
+        const int ni = lane < nctas ? s_cnt[lane][0] : 0;
         int incl = ni;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        if (lane < nctas) { s_cinb[lane] = incl - ni; s_mid[lane] = nd; }
-        if (lane == nctas - 1) s_cinb[nctas] = incl;
-    }
-    __syncthreads();
-    const int c1 = min(s_cinb[nctas], kInbinMax);  // == cnt_T1
-    for (int e = tid; e < c1; e += NT) {
+        const int excl = incl - ni;
         int r = 0;
-        while (r + 1 < nctas && s_cinb[r + 1] <= e) ++r;
-        s_inb[e] = ld_cluster_v4(cluster_addr(s_loc + (e - s_cinb[r]), r));
+        for (int q = 1; q < nctas; ++q) r = __shfl_sync(0xffffffffu, excl, q) <= tid ? q : r;
+        const int off = tid - __shfl_sync(0xffffffffu, excl, r);
+        if (tid < c1) s_inb[tid] = ld_cluster_v4(cluster_addr(s_loc + off, r));
     }
-    if (tid == 0) { s_misc[0] = 0; s_misc[1] = 0x7fffffff; }
     __syncthreads();
     cluster_arrive();  // (3): done with the other CTAs' shared memory
 
-    // ---- rank the in-bin list (every CTA, redundantly; it is short)
+    // ---- rank the in-bin list (score desc, token asc): the need1-th entry
+    // (Tkey, IT) is the last one selected.  Credit the selected middle ones to
+    // their CTA (output offsets) and, for this CTA's, to their warp.
     const int need1 = (int)kk - above1;  // 1 <= need1 <= c1
-    if (need1 < c1) {
-        for (int e = tid; e < c1; e += NT) {
-            const uint32_t ke = s_inb[e].x, ie = s_inb[e].y;
-            int rank = 0;
-            for (int f = 0; f < c1; ++f) {
-                const uint32_t kf = s_inb[f].x;
-                rank += (kf > ke) || (kf == ke && s_inb[f].y < ie);
+    if (c1 <= 32) {
+        if (warp == 0) {  // one warp, entry e in lane e
+            const uint4 en = lane < c1 ? s_inb[lane] : make_uint4(0u, 0u, 0u, 0u);
+            uint32_t Tkey = 0u;
+            int IT = 0x7fffffff;
+            if (need1 < c1) {
+                int rank = 0;
+                for (int f = 0; f < c1; ++f) {
+                    const uint32_t kf = __shfl_sync(0xffffffffu, en.x, f);
+                    const uint32_t tf = __shfl_sync(0xffffffffu, en.y, f);
+                    rank += (kf > en.x) || (kf == en.x && tf < en.y);
+                }
+                const int src = __ffs(__ballot_sync(0xffffffffu, lane < c1 && rank == need1 - 1)) - 1;
+                Tkey = __shfl_sync(0xffffffffu, en.x, src);
+                IT = (int)__shfl_sync(0xffffffffu, en.y, src);
             }
-            if (rank == need1 - 1) { s_misc[0] = (int)ke; s_misc[1] = (int)ie; }
+            const int t = (int)en.y;
+            const bool sel = lane < c1 && t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT));
+            int mid = 0;  // lane r < nctas: selected middle tokens of CTA r
+            for (int r = 0; r < nctas; ++r) {
+                const int cr = __popc(__ballot_sync(0xffffffffu, sel && (int)en.z == r));
+                if (lane == r) mid = s_cnt[r][1] + cr;
+            }
+            if (sel && (int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
+            int before = lane < cta ? mid : 0, total = mid;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                before += __shfl_xor_sync(0xffffffffu, before, o);
+                total += __shfl_xor_sync(0xffffffffu, total, o);
+            }
+            if (lane == 0) { s_misc[0] = (int)Tkey; s_misc[1] = IT; s_misc[2] = before; s_misc[3] = total; }
+        }
+    } else {  // a long list: every thread ranks its entries
+        if (tid == 0) { s_misc[0] = 0; s_misc[1] = 0x7fffffff; }
+        if (tid < nctas) s_mid[tid] = s_cnt[tid][1];
+        __syncthreads();
+        if (need1 < c1) {
+            for (int e = tid; e < c1; e += NT) {
+                const uint32_t ke = s_inb[e].x, ie = s_inb[e].y;
+                int rank = 0;
+                for (int f = 0; f < c1; ++f) {
+                    const uint32_t kf = s_inb[f].x;
+                    rank += (kf > ke) || (kf == ke && s_inb[f].y < ie);
+                }
+                if (rank == need1 - 1) { s_misc[0] = (int)ke; s_misc[1] = (int)ie; }
+            }
         }
         __syncthreads();
+        const uint32_t Tkey = (uint32_t)s_misc[0];
+        const int IT = s_misc[1];
+        for (int e = tid; e < c1; e += NT) {
+            const uint4 en = s_inb[e];
+            const int t = (int)en.y;
+            if (t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT))) {
+                atomicAdd(&s_mid[en.z], 1);
+                if ((int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int before = 0, total = 0;
+            for (int r = 0; r < nctas; ++r) {
+                before += r < cta ? s_mid[r] : 0;
+                total += s_mid[r];
+            }
+            s_misc[2] = before;
+            s_misc[3] = total;
+        }
     }
+    __syncthreads();
     const uint32_t Tkey = (uint32_t)s_misc[0];
     const int IT = s_misc[1];
+    const int total_mid = s_misc[3];
     auto keep = [&](int t, uint32_t key) {
         if (t < s_end || t >= w_beg) return false;
         return key_to_float(key) >= theta2 || key > Tkey || (key == Tkey && t <= IT);
     };
-    // selected in-bin tokens in the middle range, credited to their CTA
-    for (int e = tid; e < c1; e += NT) {
-        const int t = (int)s_inb[e].y;
-        const uint32_t key = s_inb[e].x;
-        if (t >= s_end && t < w_beg && (key > Tkey || (key == Tkey && t <= IT))) atomicAdd(&s_mid[s_inb[e].z], 1);
-    }
-    __syncthreads();
-    int before = 0, total_mid = 0;
-    for (int r = 0; r < nctas; ++r) {
-        before += r < cta ? s_mid[r] : 0;
-        total_mid += s_mid[r];
-    }
-    // ---- each warp: kept count, prefix over warps, ordered emission
+    // ---- ordered emission: warp w writes its kept candidates from offset
+    // s_end + (this CTA's offset) + (kept candidates of warps < w)
     auto cand_at = [&](int j, int &t, uint32_t &key) {
         if (j < CW) { const uint2 c = wcand[j]; t = (int)c.x; key = c.y; }
         else { t = __ldcg(cand + t0 + wb + j); key = __ldcg(ckey + t0 + wb + j); }
     };
-    int nkeep = 0;
-    for (int j = lane; j < ncand; j += 32) {
-        int t; uint32_t key;
-        cand_at(j, t, key);
-        nkeep += keep(t, key);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) nkeep += __shfl_xor_sync(0xffffffffu, nkeep, o);
-    if (lane == 0) s_wkeep[warp] = nkeep;
-    __syncthreads();
-    int wpos = s_end + before;
+    int wpos = s_end + s_misc[2];
     for (int w2 = 0; w2 < warp; ++w2) wpos += s_wkeep[w2];
     for (int jb = 0; jb < ncand; jb += 32) {
         const int j = jb + lane;
