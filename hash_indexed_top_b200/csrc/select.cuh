@@ -734,31 +734,6 @@ collect_kernel(SelWS ws, int nctas, int S, int W, int cap_sel, int32_t *sel_idx,
 constexpr int kInbinMax = 1024;
 constexpr int kMaxCluster = 16;
 
-// Address, in the cluster's shared window, of the object at `p` (this CTA's
-// shared memory) in the CTA of cluster rank `rank`.
-__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
-    const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
 // Threshold of the cluster's summed histogram, computed by one full warp from
 // the CTAs' super-bin counts (coarse[64], super-bin s = bins [64 s, 64 s + 64))
 // and histograms (hist[kBins]), both read in place in every CTA's shared
