@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <type_traits>
 
 #include "../../include/dashkv.h"
@@ -416,6 +417,40 @@ void launch_decode_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
 
 }  // namespace
 
+// ---------------------------------------------------------------------------- static scratch
+// Scratch of dashkv_select_static: one fixed array in this library's device
+// image (per device), for callers that may not allocate device memory.  No
+// call here allocates: the address comes from cudaGetSymbolAddress.
+constexpr size_t kStaticScratchBytes = (size_t)24 << 20;  // 24 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+constexpr int kMaxStaticDevices = 64;
+void *g_static_addr[kMaxStaticDevices];  // device address of the scratch, once set up
+std::mutex g_static_mu;
+
+// First use on a device: look the scratch up and zero it (its histogram and
+// counter words must start at zero; every successful selection leaves them
+// so).  The memset and the device synchronisation cannot be captured, so this
+// refuses to run while `st` is capturing.
+dashkv_status static_scratch(int dev, cudaStream_t st, void **out) {
+    if (dev < 0 || dev >= kMaxStaticDevices) return DASHKV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return DASHKV_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return DASHKV_ERR_INVALID_ARG;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DASHKV_ERR_CUDA;
+        if (cudaMemset(p, 0, kStaticScratchBytes) != cudaSuccess) return DASHKV_ERR_CUDA;
+        if (cudaDeviceSynchronize() != cudaSuccess) return DASHKV_ERR_CUDA;
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return DASHKV_OK;
+}
+}  // namespace
+
 // ============================================================================ C ABI
 extern "C" {
 
@@ -572,6 +607,21 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     tr.after();
     copy_scores();
     return launch_status();
+}
+
+// dashkv_select on the library's static scratch (see static_scratch above):
+// for callers that cannot allocate the workspace themselves.
+dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
+                                   const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
+                                   void *stream) {
+    if (!ctx) return DASHKV_ERR_INVALID_ARG;
+    const dashkv_status v = check_view(ctx, kv, false, true);
+    if (v != DASHKV_OK) return v;
+    if (ws_layout(ctx->cfg, view_capacity(ctx, kv)).total > kStaticScratchBytes) return DASHKV_ERR_WORKSPACE;
+    void *w = nullptr;
+    const dashkv_status s = static_scratch(ctx->device, static_cast<cudaStream_t>(stream), &w);
+    if (s != DASHKV_OK) return s;
+    return dashkv_select(ctx, kv, q, seq_lens, sel_idx, sel_cnt, scores, w, kStaticScratchBytes, stream);
 }
 
 dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,

@@ -26,7 +26,8 @@ FLAG_TWO_KERNEL_SELECT = 1
 
 SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_encode_keys",
            "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
-           "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str")
+           "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str",
+           "dashkv_select_static")
 
 
 class DashKVError(RuntimeError):
@@ -69,6 +70,7 @@ def lib() -> ctypes.CDLL:
         L.dashkv_append_keys.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P]
         L.dashkv_select.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
         L.dashkv_sparse_decode.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
+        L.dashkv_select_static.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P]
         L.dashkv_get_error.argtypes = [P]
         L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
         L.dashkv_set_trace.argtypes = [P, P, I32]
@@ -77,7 +79,7 @@ def lib() -> ctypes.CDLL:
         L.dashkv_status_str.argtypes = [ctypes.c_int]
         L.dashkv_status_str.restype = ctypes.c_char_p
         for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode",
-                  "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace"):
+                  "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -223,6 +225,17 @@ class DashKV:
         _check("dashkv_select", lib().dashkv_select(self._ctx, ctypes.byref(v), _ptr(q), _ptr(seq_lens),
                                                     _ptr(sel_idx), _ptr(sel_cnt), _ptr(scores), _ptr(ws),
                                                     ws.numel(), _stream(stream)))
+
+    def select_static(self, cache: KVCache, q: torch.Tensor, seq_lens: torch.Tensor, sel_idx: torch.Tensor,
+                      sel_cnt: torch.Tensor, scores: Optional[torch.Tensor] = None, stream=None) -> None:
+        """dashkv_select on the library's fixed 24 MiB device scratch: for callers
+        that may not allocate device memory (e.g. inside CUDA graph capture,
+        where cudaMalloc is not allowed).  The first call on a device must not be
+        captured; overlapping calls on one device race (one shared scratch)."""
+        v = cache.view()
+        _check("dashkv_select_static", lib().dashkv_select_static(self._ctx, ctypes.byref(v), _ptr(q),
+                                                                  _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt),
+                                                                  _ptr(scores), _stream(stream)))
 
     def sparse_decode(self, cache: KVCache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
                       out: torch.Tensor, lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,

@@ -160,6 +160,26 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
                             float *scores, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/* Allocation-free variant of dashkv_select.  The pages have no counterpart
+ * of this call: it is an interface convenience, not part of the method.
+ * For callers that may not allocate device memory at all -- e.g. code that
+ * runs while a CUDA graph is being captured (cudaMalloc cannot be captured)
+ * or a host runtime that owns every device allocation -- it uses, instead of
+ * a caller workspace, one scratch array compiled into this library: 24 MiB
+ * (25165824 bytes) per device, the limit.  Inputs whose
+ * dashkv_workspace_size(ctx, capacity) exceeds it are rejected with
+ * DASHKV_ERR_WORKSPACE before anything is launched.  It allocates nothing.
+ * The first call on a device looks the scratch up (cudaGetSymbolAddress)
+ * and zero-fills it with a synchronising memset: that first call must come
+ * before any stream capture (during capture it returns
+ * DASHKV_ERR_INVALID_ARG); later calls may be captured.  All calls on a
+ * device share the one scratch: calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller.
+ * Arguments and results are those of dashkv_select. */
+dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
+                                   const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
+                                   float *scores, void *stream);
+
 /* Stage 4.  Exact softmax attention of every query head over the rows its
  * KV head selected: out (device fp32 [B][Hq][d]); lse (optional, device
  * fp32 [B][Hq]) receives log sum_t exp(q.K_t / sqrt(d)) (-inf when nothing
