@@ -16,6 +16,7 @@ the max-over-ranks of the timings.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -44,6 +45,38 @@ def measured_peaks() -> dict:
             d = json.load(f)
         return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
     return dict(hbm_gbs=6650.0, source="fallback")
+
+
+def kernel_sources_sha() -> str:
+    """sha256 over the library's CUDA sources (name and bytes, sorted by name)."""
+    d = os.path.join(ROOT, "hash_indexed_top_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(d)):
+        if n.endswith((".cu", ".cuh")):
+            h.update(n.encode())
+            with open(os.path.join(d, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    summary of this workload, or None when that summary was taken from other
+    kernel sources than the ones built now (the counters would be stale)."""
+    p = os.path.join(ROOT, "profiles", "c128k_step_kernels_full.txt")
+    if not os.path.exists(p):
+        return None
+    sha, traffic = None, {}
+    with open(p) as f:
+        for ln in f:
+            if ln.startswith("kernel sources sha256:"):
+                sha = ln.split(":", 1)[1].strip()
+            elif ln.startswith("traffic_per_launch "):
+                _, name, val = ln.split()
+                traffic[name] = int(val)
+    if sha != kernel_sources_sha():
+        return None
+    return traffic.get(kernel + "_kernel")
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -356,7 +389,8 @@ def run_dashkv(args, cfg, world, rank, local):
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": score_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": score_gbs / peaks["hbm_gbs"],
                          "peak_source": peaks["source"], "frac_of_8tbs": score_gbs / SPEC_HBM_GBS,
-                         "algorithmic_bytes_per_launch": code_bytes, "traffic": None},
+                         "algorithmic_bytes_per_launch": code_bytes,
+                         "traffic": recorded_traffic(dom) if cfg.name == "c128k" else None},
             "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_gbs,
                               "frac": step_gbs / peaks["hbm_gbs"], "frac_of_8tbs": step_gbs / SPEC_HBM_GBS,
                               "code_bytes": code_bytes, "selected_kv_bytes": kv_bytes, "q_out_bytes": qo_bytes},
