@@ -229,17 +229,20 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
         qsum[i] = s;
     }
     __syncthreads();
-    // Qp_j: four threads per hyperplane, each a quarter of the dims.
-    if (tid < 4 * BITS) {
-        const int j = tid >> 2, part = tid & 3;
+    // Qp_j = sum_i R[j][i] qsum[i]: warp w takes hyperplanes w, w + NWARPS, ...
+    // and lane l the dims l, l + 32, ...; a whole warp then reads the same word of
+    // R at a time (a broadcast from the parameter block), and a shuffle tree sums
+    // the lanes.
+    for (int j = warp; j < BITS; j += NWARPS) {
         float acc = 0.0f;
-        for (int i = part * (D / 4); i < (part + 1) * (D / 4); ++i) {
-            float rf = ((R.w[j * (D / 32) + i / 32] >> (i % 32)) & 1u) ? -1.0f : 1.0f;
-            acc = fmaf(rf, qsum[i], acc);
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) {
+            const uint32_t rw = R.w[j * (D / 32) + k];
+            acc = fmaf(((rw >> lane) & 1u) ? -1.0f : 1.0f, qsum[32 * k + lane], acc);
         }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (part == 0) Qp[j] = acc;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) Qp[j] = acc;
     }
     __syncthreads();
     if (warp == 0) {
@@ -250,17 +253,28 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
         if (lane == 0) red[0] = a > 0.0f ? 0.5f / a : 0.0f;
     }
     // LUT rows: word j of row v holds LUT_{j mod T}[v]; lane l fills words l and
-    // l + 32 (both table l mod T, as 32 is a multiple of T) of the rows it owns.
+    // l + 32 (both table l mod T, as 32 is a multiple of T).  Warp w owns the
+    // 256 / NWARPS consecutive rows from v0 = w * 256 / NWARPS (low bits zero):
+    // row v0 is the full signed sum, each other row adds 2 qv[u] for the low
+    // bits u it sets.
     {
+        static_assert(256 % NWARPS == 0 && (256 / NWARPS) <= 8, "rows per warp");
+        constexpr int RPW = 256 / NWARPS;
         const int c = lane % T;
         float qv[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) qv[u] = Qp[8 * c + u];
-        for (int v = warp; v < 256; v += NWARPS) {
-            float val = 0.0f;
+        const int v0 = warp * RPW;
+        float base = 0.0f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) val += ((v >> u) & 1) ? qv[u] : -qv[u];
-            float *row = reinterpret_cast<float *>(lut + v * 256);
+        for (int u = 0; u < 8; ++u) base += ((v0 >> u) & 1) ? qv[u] : -qv[u];
+#pragma unroll
+        for (int d = 0; d < RPW; ++d) {
+            float val = base;
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+                if ((d >> u) & 1) val += 2.0f * qv[u];
+            float *row = reinterpret_cast<float *>(lut + (v0 + d) * 256);
             row[lane] = val;
             row[lane + 32] = val;
         }
