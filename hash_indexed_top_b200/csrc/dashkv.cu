@@ -260,10 +260,15 @@ template <int BITS, int D>
 void launch_append_bd(const dashkv_ctx *ctx, const KV &kv, const void *kn, const void *vn, int32_t *seq,
                       cudaStream_t st) {
     // one cluster of C CTAs per sequence (early start behind the preceding kernel)
-    const int C = ctx->cfg.num_kv_heads < kAppendCluster ? ctx->cfg.num_kv_heads : kAppendCluster;
+    const int Hkv = ctx->cfg.num_kv_heads;
+    int C = (Hkv * BITS + kAppendSpan - 1) / kAppendSpan;
+    if (C > kAppendCluster) C = kAppendCluster;
+    if (C > Hkv) C = Hkv;
+    const int hpc = (Hkv + C - 1) / C;  // <= 1024 / BITS heads per CTA (Hkv * BITS <= 8 * 512)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C, ctx->cfg.batch);
-    cfg.blockDim = dim3(kAppendThreads);
+    cfg.blockDim = dim3(hpc * BITS);
+    cfg.dynamicSmemBytes = (size_t)hpc * (D * 4 + BITS / 8);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -275,7 +280,7 @@ void launch_append_bd(const dashkv_ctx *ctx, const KV &kv, const void *kn, const
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     cudaLaunchKernelEx(&cfg, append_keys_kernel<BITS, D>, kv, static_cast<const __nv_bfloat16 *>(kn),
-                       static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R);
+                       static_cast<const __nv_bfloat16 *>(vn), seq, ctx->R, hpc);
 }
 
 template <int D>

@@ -315,47 +315,40 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     if (!s_last) return;
     __threadfence();
     const float *pbase = ws.part + (int64_t)bh * kMaxSplits * G * (D + 2);
-    // per-(split, head) scale 2^(m_s - M_g) and the total sum L_g, then the
-    // weighted sum of the accumulators with all split loads in flight
-    float *s_c = s_acc;                  // [splits][G] (the CTA states are no longer needed)
-    float *s_L = s_acc + kMaxSplits * G; // [G]
-    float *s_M = s_L + G;                // [G]
-    for (int x = tid; x < splits * G; x += kAttnThreads) {
-        const int sp = x / G, g = x % G;
-        s_c[x] = __ldcg(pbase + (sp * G + g) * (D + 2) + D);      // m_s
-        s_c[kMaxSplits * G + 2 * G + x] = __ldcg(pbase + (sp * G + g) * (D + 2) + D + 1);  // l_s
-    }
-    __syncthreads();
-    if (tid < G) {
-        const int g = tid;
-        float M = -INFINITY;
-        for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, s_c[sp * G + g]);
-        float L = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) {
-            const float c = M == -INFINITY ? 0.0f : fast_exp2(s_c[sp * G + g] - M);
-            L = fmaf(s_c[kMaxSplits * G + 2 * G + sp * G + g], c, L);
-            s_c[sp * G + g] = c;
-        }
-        s_L[g] = L;
-        s_M[g] = M;
-    }
-    __syncthreads();
+    // each output element: every split's (m, l, acc) loaded at once (one round
+    // trip), then the log-sum-exp merge in registers
+    constexpr int MS = 16;  // splits merged per pass (all loads of a pass in flight)
     for (int x = tid; x < G * D; x += kAttnThreads) {
         const int g = x / D, i = x % D;
-        float Acc = 0.0f;
-        int sp = 0;
-        for (; sp + 8 <= splits; sp += 8) {
-            float a[8];
+        float M = -INFINITY, L = 0.0f, Acc = 0.0f;
+        for (int s0 = 0; s0 < splits; s0 += MS) {
+            float pm[MS], pl[MS], pa[MS];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) a[u] = __ldcg(pbase + ((sp + u) * G + g) * (D + 2) + i);
+            for (int u = 0; u < MS; ++u) {
+                const float *ps = pbase + ((s0 + u) * G + g) * (D + 2);
+                const bool in = s0 + u < splits;
+                pm[u] = in ? __ldcg(ps + D) : -INFINITY;
+                pl[u] = in ? __ldcg(ps + D + 1) : 0.0f;
+                pa[u] = in ? __ldcg(ps + i) : 0.0f;
+            }
+            float Mn = M;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) Acc = fmaf(a[u], s_c[(sp + u) * G + g], Acc);
+            for (int u = 0; u < MS; ++u) Mn = fmaxf(Mn, pm[u]);
+            if (Mn == -INFINITY) continue;
+            const float cM = fast_exp2(M - Mn);  // 0 when M = -inf
+            L *= cM;
+            Acc *= cM;
+#pragma unroll
+            for (int u = 0; u < MS; ++u) {
+                const float c = fast_exp2(pm[u] - Mn);  // 0 for empty splits (m = -inf)
+                L = fmaf(pl[u], c, L);
+                Acc = fmaf(pa[u], c, Acc);
+            }
+            M = Mn;
         }
-        for (; sp < splits; ++sp) Acc = fmaf(__ldcg(pbase + (sp * G + g) * (D + 2) + i), s_c[sp * G + g], Acc);
-        const float L = s_L[g];
         const int64_t oq = (int64_t)b * Hq + h * G + g;
         out[oq * D + i] = L > 0.0f ? Acc / L : 0.0f;
-        if (i == 0 && lse) lse[oq] = L > 0.0f ? (s_M[g] + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        if (i == 0 && lse) lse[oq] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
     if (tid == 0) ws.arrive[(int64_t)kSyncStride * bh] = 0;
 }

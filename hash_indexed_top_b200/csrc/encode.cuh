@@ -109,32 +109,48 @@ encode_keys_kernel(KV kv, const int32_t *__restrict__ seq_lens, const RBits R, i
 }
 
 // ---------------------------------------------------------------------------
-// Decode-step append.  One cluster of C = min(Hkv, kAppendCluster) CTAs per
-// sequence; CTA c handles kv heads c, c + C, ...: it copies the new K/V rows
-// into slot seq_lens[b] and encodes the new key (thread j = hyperplane j, one
-// sequential FMA chain over the dims as in the whole-cache encoder; the sign
-// bits of a warp are gathered with one ballot).  After a cluster barrier --
-// every CTA has read seq_lens[b] -- CTA 0 bumps it.
-constexpr int kAppendThreads = 128;
+// Decode-step append.  One cluster of C CTAs per sequence (C = ceil(Hkv * bits
+// / kAppendSpan)): CTA c handles hpc = ceil(Hkv / C) consecutive kv heads,
+// with one thread per (head, hyperplane).  It copies the new K/V rows into
+// slot seq_lens[b] and encodes the new keys (one sequential FMA chain over the
+// dims per hyperplane, as in the whole-cache encoder; the sign bits of a warp,
+// 32 hyperplanes of one head, are gathered with one ballot).  After a cluster
+// barrier -- every CTA has read seq_lens[b] -- CTA 0 bumps it.  Few, wide
+// CTAs: the append runs while the scorer's CTAs (one per SM) are being
+// placed, and every SM it holds is one they cannot use until it ends.
+constexpr int kAppendSpan = 512;     // (head, hyperplane) pairs per CTA
 constexpr int kAppendCluster = 8;
 
 template <int BITS, int D>
-__global__ void __launch_bounds__(kAppendThreads)
+__global__ void __launch_bounds__(1024)
 append_keys_kernel(KV kv, const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *__restrict__ v_new,
-                   int32_t *seq_lens, const RBits R) {
+                   int32_t *seq_lens, const RBits R, int hpc) {
     constexpr int WPR = D / 32;  // R words per hyperplane
     constexpr int CPR = D / 8;   // 16-byte chunks per row
-    __shared__ float4 kf4[D / 4];
-    __shared__ uint32_t code32[BITS / 32];
-    const int b = blockIdx.y, c = blockIdx.x, C = gridDim.x;
+    extern __shared__ float4 kf4[];                                    // [hpc][D / 4]
+    uint32_t *code32 = reinterpret_cast<uint32_t *>(kf4 + hpc * (D / 4));  // [hpc][BITS / 32]
+    const int b = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31;
     const int Hkv = kv.Hkv;
-    uint32_t rw[WPR];  // this thread's hyperplane (depends on the context only)
+    const int h0 = c * hpc, nh = min(hpc, Hkv - h0);  // this CTA's heads [h0, h0 + nh)
+    const int hl = tid / BITS, j = tid % BITS;       // this thread's (head, hyperplane)
+    uint32_t rw[WPR];  // its hyperplane (depends on the context only)
 #pragma unroll
-    for (int w = 0; w < WPR; ++w) rw[w] = tid < BITS ? R.w[tid * WPR + w] : 0u;
+    for (int w = 0; w < WPR; ++w) rw[w] = R.w[j * WPR + w];
 
     griddep_wait();
     griddep_trigger();  // the scorer may start building its LUT meanwhile
+    // thread e < 2 nh CPR copies 16-byte chunk e of this CTA's new K (then V)
+    // rows; its load does not depend on the position, so it is issued together
+    // with the position's (2 * hpc * CPR <= hpc * BITS = blockDim.x)
+    const int e = tid;
+    const int isv = e >= nh * CPR;
+    const int ee = isv ? e - nh * CPR : e;
+    const int hh = ee / CPR, part = ee % CPR;
+    const bool copies = e < 2 * nh * CPR;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (copies)
+        x = __ldg(reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + ((int64_t)b * Hkv + h0 + hh) * D) + part);
     const int64_t pos = seq_lens[b];
     bool ok = pos >= 0 && pos < kv.capacity();
     if (ok && kv.page_size) {
@@ -144,45 +160,37 @@ append_keys_kernel(KV kv, const __nv_bfloat16 *__restrict__ k_new, const __nv_bf
     } else if (!ok && c == 0 && tid == 0) {
         raise_error(kErrCapacity);
     }
-    if (ok) {
-        for (int h = c; h < Hkv; h += C) {
-            const int64_t r = kv.row(b, h, pos);
-            for (int e = tid; e < 2 * CPR; e += kAppendThreads) {
-                const int isv = e >= CPR;
-                const int part = isv ? e - CPR : e;
-                const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + ((int64_t)b * Hkv + h) * D);
-                const uint4 x = __ldg(src + part);
-                reinterpret_cast<uint4 *>((isv ? kv.v : kv.k) + r)[part] = x;
-                if (!isv) {
-                    kf4[2 * part] = make_float4(bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y));
-                    kf4[2 * part + 1] = make_float4(bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w));
-                }
+    if (ok && nh > 0) {
+        if (copies) {
+            const int64_t r = kv.row(b, h0 + hh, pos);
+            reinterpret_cast<uint4 *>((isv ? kv.v : kv.k) + r)[part] = x;
+            if (!isv) {
+                kf4[hh * (D / 4) + 2 * part] = make_float4(bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y));
+                kf4[hh * (D / 4) + 2 * part + 1] = make_float4(bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w));
             }
-            __syncthreads();
-            if (tid < BITS) {  // whole warps (BITS is a multiple of 32)
-                float acc = 0.0f;
+        }
+        __syncthreads();
+        if (hl < nh) {  // whole warps: a warp is 32 hyperplanes of one head
+            const float4 *kh = kf4 + hl * (D / 4);
+            float acc = 0.0f;
 #pragma unroll
-                for (int i4 = 0; i4 < D / 4; ++i4) {
-                    const float4 k4 = kf4[i4];
-                    const float kx[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = 4 * i4 + u;
-                        const float rf = ((rw[i / 32] >> (i % 32)) & 1u) ? -1.0f : 1.0f;
-                        acc = fmaf(rf, kx[u], acc);
-                    }
-                }
-                const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
-                if (lane == 0) code32[tid >> 5] = word;
+            for (int i4 = 0; i4 < D / 4; ++i4) {
+                const float4 k4 = kh[i4];
+                const uint32_t wbits = rw[i4 / 8] >> (4 * (i4 % 8));
+                acc = fmaf((wbits & 1u) ? -1.0f : 1.0f, k4.x, acc);
+                acc = fmaf((wbits & 2u) ? -1.0f : 1.0f, k4.y, acc);
+                acc = fmaf((wbits & 4u) ? -1.0f : 1.0f, k4.z, acc);
+                acc = fmaf((wbits & 8u) ? -1.0f : 1.0f, k4.w, acc);
             }
-            __syncthreads();
-            if (tid == 0) {
-                uint32_t w32[BITS / 32];
+            const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
+            if (lane == 0) code32[hl * (BITS / 32) + j / 32] = word;
+        }
+        __syncthreads();
+        if (tid < nh) {
+            uint32_t w32[BITS / 32];
 #pragma unroll
-                for (int k = 0; k < BITS / 32; ++k) w32[k] = code32[k];
-                store_code_rotated<BITS>(kv.codes + kv.code(b, h, pos), w32, pos);
-            }
-            __syncthreads();  // kf4 and code32 are reused by the next head
+            for (int k = 0; k < BITS / 32; ++k) w32[k] = code32[tid * (BITS / 32) + k];
+            store_code_rotated<BITS>(kv.codes + kv.code(b, h0 + tid, pos), w32, pos);
         }
     }
     cluster_sync();  // every CTA of this sequence has read seq_lens[b]

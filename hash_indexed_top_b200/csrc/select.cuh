@@ -221,6 +221,14 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.y, b = bh / kv.Hkv, h = bh % kv.Hkv;
 
+    // this warp's words of R (hyperplanes warp + NWARPS m): issued first, so their
+    // parameter-block misses overlap the loads of q
+    static_assert(BITS % NWARPS == 0, "hyperplanes per warp");
+    uint32_t rw[BITS / NWARPS][D / 32];
+#pragma unroll
+    for (int m = 0; m < BITS / NWARPS; ++m)
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) rw[m][k] = R.w[(warp + NWARPS * m) * (D / 32) + k];
     for (int i = tid; i < kBins; i += kScoreThreads) hist[i] = 0;
     for (int i = tid; i < D; i += kScoreThreads) {
         const __nv_bfloat16 *qh = q + ((int64_t)b * Hq + (int64_t)h * G) * D + i;
@@ -233,16 +241,14 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     // and lane l the dims l, l + 32, ...; a whole warp then reads the same word of
     // R at a time (a broadcast from the parameter block), and a shuffle tree sums
     // the lanes.
-    for (int j = warp; j < BITS; j += NWARPS) {
+#pragma unroll
+    for (int m = 0; m < BITS / NWARPS; ++m) {
         float acc = 0.0f;
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k) {
-            const uint32_t rw = R.w[j * (D / 32) + k];
-            acc = fmaf(((rw >> lane) & 1u) ? -1.0f : 1.0f, qsum[32 * k + lane], acc);
-        }
+        for (int k = 0; k < D / 32; ++k) acc = fmaf(((rw[m][k] >> lane) & 1u) ? -1.0f : 1.0f, qsum[32 * k + lane], acc);
 #pragma unroll
         for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) Qp[j] = acc;
+        if (lane == 0) Qp[warp + NWARPS * m] = acc;
     }
     __syncthreads();
     if (warp == 0) {
