@@ -117,21 +117,23 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     // q is an input of the step; the selection comes from the preceding kernel
     griddep_wait();
     griddep_trigger();
+    // The splits divide the capacity of the selection (not its count), so the
+    // first ids load together with the count instead of after it; rows past the
+    // count are masked.
     int cnt = sel_cnt[bh];
-    if (cnt > cap_sel) cnt = cap_sel;
-    if (cnt < 0) cnt = 0;
-    const int per = (cnt + splits - 1) / splits;
+    const int per = (cap_sel + splits - 1) / splits;
     const int r0 = split * per;
-    const int r1 = r0 + per < cnt ? r0 + per : cnt;
+    const int r1 = r0 + per < cap_sel ? r0 + per : cap_sel;
 
     const int32_t *ids = sel_idx + (int64_t)bh * cap_sel;
     __nv_bfloat16 *wstage = stage + (size_t)warp * STAGES * TROWS * 2 * D;
     // Token of row `base + lane` of a tile (lanes < TROWS), -1 when the row is
-    // outside the slice or its id lies outside the cache.
+    // outside the slice or past the count, or its id lies outside the cache.
     auto tile_token = [&](int base) -> int {
         const int r = base + lane;
         if (lane >= TROWS || r >= r1) return -1;
         const int t = __ldg(ids + r);
+        if (r >= cnt) return -1;
         if (t < 0 || t >= cap_tokens) {
             raise_error(kErrCapacity);
             return -1;

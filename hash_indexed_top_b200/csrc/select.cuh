@@ -757,9 +757,10 @@ constexpr int kMaxCluster = 16;
 // Threshold of the cluster's summed histogram, computed by one full warp from
 // the CTAs' super-bin counts (coarse[64], super-bin s = bins [64 s, 64 s + 64))
 // and histograms (hist[kBins]), both read in place in every CTA's shared
-// memory.  out = {T1, tokens above T1, tokens in T1} as threshold_bin.
-__device__ __forceinline__ void cluster_threshold(const uint32_t *coarse, const uint32_t *hist, int nranks,
-                                                  int64_t kk, int *out) {
+// memory.  Returns T1 to every lane; out (when not null) = {T1, tokens above
+// T1, tokens in T1} as threshold_bin.
+__device__ __forceinline__ int cluster_threshold(const uint32_t *coarse, const uint32_t *hist, int nranks,
+                                                 int64_t kk, int *out) {
     const int lane = threadIdx.x & 31;
     // lane l holds super-bins 63 - 2l (upper) and 62 - 2l (lower): lane 0 the top
     uint32_t cu = 0, cl = 0;
@@ -799,10 +800,13 @@ __device__ __forceinline__ void cluster_threshold(const uint32_t *coarse, const 
     }
     const int64_t fexcl = above + fincl - fu - fl;
     fincl += above;
-    if (fexcl < kk && kk <= fincl) {
+    const bool hit = fexcl < kk && kk <= fincl;
+    const int t1 = hit ? (fexcl + fu >= kk ? bu : bl) : 0;
+    if (hit && out) {
         if (fexcl + fu >= kk) { out[0] = bu; out[1] = (int)fexcl; out[2] = (int)fu; }
         else { out[0] = bl; out[1] = (int)(fexcl + fu); out[2] = (int)fl; }
     }
+    return __shfl_sync(0xffffffffu, t1, __ffs(__ballot_sync(0xffffffffu, hit)) - 1);
 }
 
 // Smallest finite float s with score_bin(s, inv2A) >= T, or +inf if there is
@@ -888,13 +892,10 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     if (tid == 0) { s_thr[0] = kBins; s_thr[1] = 0; s_thr[2] = 0; s_ninb = 0; }
     cluster_sync();  // (1): every histogram of the cluster is complete
     const float inv2A = so.inv2A;
-    if (normal && warp == 0) {
-        cluster_threshold(s_coarse, hist, nctas, kk, s_thr);
-        __syncwarp();
-        const int T1w = s_thr[0];
-        const float th = bin_floor_value(T1w, inv2A);
-        const float th2 = bin_floor_value(T1w + 1, inv2A);
-        if (lane == 0) { s_theta[0] = th; s_theta[1] = th2; }
+    if (normal && warp < 2) {  // both find T1; warp 0 then theta(T1), warp 1 theta(T1 + 1)
+        const int T1w = cluster_threshold(s_coarse, hist, nctas, kk, warp == 0 ? s_thr : nullptr);
+        const float th = bin_floor_value(T1w + warp, inv2A);
+        if (lane == 0) s_theta[warp] = th;
     }
     __syncthreads();
     const int T1 = s_thr[0], above1 = s_thr[1], cnt_T1 = s_thr[2];
@@ -1150,15 +1151,22 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
         }
         wpos += __popc(ball);
     }
-    if (cta == 0) {
-        for (int t = tid; t < s_end; t += NT) out[t] = t;
+    {   // the sinks, the window and the padding, spread over the cluster's CTAs
         const int wpos0 = s_end + total_mid;
-        for (int t = w_beg + tid; t < n; t += NT)
-            if (wpos0 + (t - w_beg) < cap_sel) out[wpos0 + (t - w_beg)] = t;
-        int total = wpos0 + (int)(n - w_beg);
-        if (total > cap_sel) total = cap_sel;
-        for (int r = total + tid; r < cap_sel; r += NT) out[r] = -1;
-        if (tid == 0) sel_cnt[bh] = total;
+        const int nwin = (int)(n - w_beg);
+        const int total = min(wpos0 + nwin, cap_sel);
+        const int nall = s_end + nwin + (cap_sel - total);
+        for (int x = cta * NT + tid; x < nall; x += nctas * NT) {
+            if (x < s_end) {
+                out[x] = x;
+            } else if (x < s_end + nwin) {
+                const int tw = x - s_end;
+                if (wpos0 + tw < cap_sel) out[wpos0 + tw] = w_beg + tw;
+            } else {
+                out[total + (x - s_end - nwin)] = -1;
+            }
+        }
+        if (cta == 0 && tid == 0) sel_cnt[bh] = total;
     }
     cluster_wait();  // (3): no CTA leaves while another may still read its shared memory
 }
