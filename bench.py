@@ -265,7 +265,7 @@ def run_dashkv(args, cfg, world, rank, local):
             eng.select(cache, w.q[s], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
             if e is not None:
                 eng.set_trace(e[8:10])
-            eng.sparse_decode(cache, w.q[s], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+            eng.sparse_decode(cache, w.q[s], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws, seq_lens=seq)
             if e is not None:
                 eng.set_trace(None)
         return g
@@ -357,7 +357,7 @@ def run_dashkv(args, cfg, world, rank, local):
             dvn.copy_(hv[s], non_blocking=True)
             eng.append_keys(cache, dkn, dvn, seq)
             eng.select(cache, dq, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
-            eng.sparse_decode(cache, dq, buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws)
+            eng.sparse_decode(cache, dq, buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws, seq_lens=seq)
             h_out.copy_(buf["out"], non_blocking=True)
             h_lse.copy_(buf["lse"], non_blocking=True)
             eev[i][1].record(stream)

@@ -187,7 +187,7 @@ int attn_splits(const dashkv_ctx *ctx) {
     int64_t n = (2 * ctx->sm_count) / BH;  // one wave of two CTAs per SM
     const int64_t by_rows = ceil_div(cap_sel, 64);
     if (n > by_rows) n = by_rows;
-    if (n > kMaxSplits) n = kMaxSplits;
+    if (n > kMaxSplits - 1) n = kMaxSplits - 1;  // one slot stays for the window CTA
     return n < 1 ? 1 : (int)n;
 }
 
@@ -397,26 +397,39 @@ void launch_score_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const in
     }
 }
 
+// Window CTAs (one per (b, h), leading rows of the decode grid) when the
+// lengths are given and they fit on the SMs the fused selection leaves free
+// (two decode CTAs per SM), so that they run while it streams.
+int window_rows(const dashkv_ctx *ctx, int64_t cap, const int32_t *seq_lens, int splits) {
+    if (!seq_lens || !use_fused(ctx)) return 0;
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int64_t sel_ctas = (int64_t)fused_cluster(ctx, cap) * BH;
+    if (sel_ctas >= ctx->sm_count || BH > 2 * (ctx->sm_count - sel_ctas)) return 0;
+    return (BH + splits - 1) / splits;
+}
+
 template <int D, int G>
 void launch_decode_dg(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *si, const int32_t *sc,
-                      float *out, float *lse, const AttnWS &ws, cudaStream_t st) {
+                      float *out, float *lse, const AttnWS &ws, const int32_t *seq_lens, int64_t cap,
+                      cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int splits = attn_splits(ctx);
+    const int wy = window_rows(ctx, cap, seq_lens, splits);
     const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    launch_pdl(sparse_decode_kernel<D, G>, dim3(splits, BH), dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st, kv,
-               static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws, splits,
-               scale_log2);
+    launch_pdl(sparse_decode_kernel<D, G>, dim3(splits, BH + wy), dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st,
+               kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws,
+               splits, scale_log2, seq_lens, ctx->cfg.sink, ctx->cfg.window, ctx->cfg.topk, wy);
 }
 
 template <int D>
 void launch_decode_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *si, const int32_t *sc,
-                     float *out, float *lse, const AttnWS &ws, cudaStream_t st) {
+                     float *out, float *lse, const AttnWS &ws, const int32_t *seq, int64_t cap, cudaStream_t st) {
     switch (ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads) {
-        case 1: launch_decode_dg<D, 1>(ctx, kv, q, si, sc, out, lse, ws, st); break;
-        case 2: launch_decode_dg<D, 2>(ctx, kv, q, si, sc, out, lse, ws, st); break;
-        case 4: launch_decode_dg<D, 4>(ctx, kv, q, si, sc, out, lse, ws, st); break;
-        default: launch_decode_dg<D, 8>(ctx, kv, q, si, sc, out, lse, ws, st); break;
+        case 1: launch_decode_dg<D, 1>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
+        case 2: launch_decode_dg<D, 2>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
+        case 4: launch_decode_dg<D, 4>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
+        default: launch_decode_dg<D, 8>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
     }
 }
 
@@ -630,8 +643,9 @@ dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
 }
 
 dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
-                                   const int32_t *sel_idx, const int32_t *sel_cnt, float *out, float *lse,
-                                   void *workspace, size_t workspace_bytes, void *stream) {
+                                   const int32_t *seq_lens, const int32_t *sel_idx, const int32_t *sel_cnt,
+                                   float *out, float *lse, void *workspace, size_t workspace_bytes,
+                                   void *stream) {
     if (!ctx || !q || !sel_idx || !sel_cnt || !out || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
     dashkv_status s = check_view(ctx, kv, true, false);
     if (s != DASHKV_OK) return s;
@@ -646,8 +660,9 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Tracer tr(ctx, st);
     tr.before();
-    if (ctx->cfg.head_dim == 64) launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, st);
-    else launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, st);
+    const int64_t cap = view_capacity(ctx, kv);
+    if (ctx->cfg.head_dim == 64) launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
+    else launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
     tr.after();
     return launch_status();
 }

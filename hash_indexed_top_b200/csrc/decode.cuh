@@ -3,15 +3,16 @@
 // top-k the indexer picked; DASH-KV page, section "技术架构：动态混合精度机制":
 // the tokens that matter are attended in full precision).
 //
-// Gathered split-K flash-decode: grid = (splits, B * Hkv).  Each CTA takes a
-// contiguous slice of one (b, kv head)'s selected ids.  A lane group of LPR
+// Gathered split-K flash-decode: grid = (splits, wy + B * Hkv).  Each of the
+// last B * Hkv rows' CTAs takes a contiguous slice of one (b, kv head)'s
+// selected ids; the optional first wy rows hold window CTAs (see the kernel).  A lane group of LPR
 // lanes owns one row at a time (DPL = d / LPR dims per lane), gathers its K and
 // V slices with 16-byte loads once, and serves all G query heads of the group
 // from them.  Rows are processed in tiles of RT per lane group: the logits of
 // the tile are formed first, then one running-max update and one rescale of
 // the accumulators per tile (fp32, base-2 exponentials).  Each CTA merges its
 // lane groups' states in shared memory and writes one partial; the last CTA of
-// the (b, h) (atomic arrival counter, no waiting) merges the partials with a
+// the (b, h) to arrive (atomic counter, no waiting) merges the partials with a
 // log-sum-exp reduction and writes out / lse.
 #pragma once
 #include "common.cuh"
@@ -19,7 +20,7 @@
 namespace dkv {
 
 constexpr int kAttnThreads = 256;
-constexpr int kMaxSplits = 256;
+constexpr int kMaxSplits = 256;  // partial slots per (b, h): top-k splits + the window CTA
 
 struct AttnWS {
     float *part;        // [BH][kMaxSplits][G][D + 2]  (acc[D], m, l)
@@ -76,7 +77,8 @@ template <int D, int G>
 __global__ void __launch_bounds__(kAttnThreads, 2)
 sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                      const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt, int cap_sel,
-                     float *__restrict__ out, float *__restrict__ lse, AttnWS ws, int splits, float scale_log2) {
+                     float *__restrict__ out, float *__restrict__ lse, AttnWS ws, int splits, float scale_log2,
+                     const int32_t *__restrict__ seq_lens, int n_sink, int n_window, int topk, int wy) {
     using S = DecodeShape<D, G>;
     constexpr int DPL = S::DPL, LPR = S::LPR, RPW = S::RPW, NST = S::NST, RT = S::RT;
     constexpr int TROWS = S::TROWS, CPR = S::CPR, NWARP = S::NWARP, STAGES = S::STAGES;
@@ -89,8 +91,19 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = lane / LPR, li = lane % LPR;
-    const int bh = blockIdx.y, b = bh / kv.Hkv, h = bh % kv.Hkv;
-    const int split = blockIdx.x;
+    // Roles.  With wy > 0 the first wy rows of the grid hold one window CTA per
+    // (b, h): it attends over the sinks and the window, which every selection
+    // contains, straight from the token range, so it does not wait for the
+    // selection and runs while the scorer still streams (on the SMs the scorer
+    // leaves free).  The other CTAs take the top-k (middle) part of the list,
+    // split `splits` ways.  With wy = 0 they take the whole list.
+    const int BH = (int)gridDim.y - wy;
+    const bool win = (int)blockIdx.y < wy;
+    const int bh = win ? (int)(blockIdx.y * splits + blockIdx.x) : (int)blockIdx.y - wy;
+    if (bh >= BH) return;  // spare window slots
+    const int split = win ? splits : (int)blockIdx.x;  // partial slot
+    const int nparts = splits + (wy > 0 ? 1 : 0);
+    const int b = bh / kv.Hkv, h = bh % kv.Hkv;
     const int64_t cap_tokens = kv.capacity();
 
     // this lane's slice of every query head of the group
@@ -115,15 +128,37 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     }
 
     // q is an input of the step; the selection comes from the preceding kernel
-    griddep_wait();
+    // (the window CTAs need none of it: the lengths and rows they read were
+    // written before the selection started)
+    if (!win) griddep_wait();
     griddep_trigger();
-    // The splits divide the capacity of the selection (not its count), so the
-    // first ids load together with the count instead of after it; rows past the
-    // count are masked.
-    int cnt = sel_cnt[bh];
-    const int per = (cap_sel + splits - 1) / splits;
-    const int r0 = split * per;
-    const int r1 = r0 + per < cap_sel ? r0 + per : cap_sel;
+    // The splits divide the capacity of their part of the list (not its count),
+    // so the first ids load together with the count instead of after it; rows
+    // past the count are masked.
+    int64_t n = 0;
+    if (wy > 0) {
+        n = __ldcg(seq_lens + b);
+        n = n < 0 ? 0 : (n > cap_tokens ? cap_tokens : n);
+    }
+    const int s_end = (int)(n_sink < n ? n_sink : n);
+    const int w_beg = (int)(n - n_window > s_end ? n - n_window : s_end);
+    const int nwin = (int)n - w_beg;
+    const int cnt = win ? 0 : sel_cnt[bh];
+    int r0, r1, rend;  // rows [r0, r1) of this CTA, valid below rend
+    if (win) {
+        r0 = 0;
+        r1 = rend = s_end + nwin;
+    } else if (wy > 0) {  // the middle: list positions [n_sink, n_sink + topk), valid below cnt - nwin
+        const int per = (topk + splits - 1) / splits;
+        r0 = n_sink + split * per;
+        r1 = min(r0 + per, n_sink + topk);
+        rend = cnt - nwin;
+    } else {
+        const int per = (cap_sel + splits - 1) / splits;
+        r0 = split * per;
+        r1 = min(r0 + per, cap_sel);
+        rend = cnt;
+    }
 
     const int32_t *ids = sel_idx + (int64_t)bh * cap_sel;
     __nv_bfloat16 *wstage = stage + (size_t)warp * STAGES * TROWS * 2 * D;
@@ -132,8 +167,8 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     auto tile_token = [&](int base) -> int {
         const int r = base + lane;
         if (lane >= TROWS || r >= r1) return -1;
-        const int t = __ldg(ids + r);
-        if (r >= cnt) return -1;
+        const int t = win ? (r < s_end ? r : w_beg + (r - s_end)) : __ldg(ids + r);
+        if (r >= rend) return -1;
         if (t < 0 || t >= cap_tokens) {
             raise_error(kErrCapacity);
             return -1;
@@ -312,7 +347,7 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     // the last CTA of this (b, h) merges the splits
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(ws.arrive + (int64_t)kSyncStride * bh, 1u) == (unsigned)(splits - 1);
+    if (tid == 0) s_last = atomicAdd(ws.arrive + (int64_t)kSyncStride * bh, 1u) == (unsigned)(nparts - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
@@ -323,12 +358,12 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     for (int x = tid; x < G * D; x += kAttnThreads) {
         const int g = x / D, i = x % D;
         float M = -INFINITY, L = 0.0f, Acc = 0.0f;
-        for (int s0 = 0; s0 < splits; s0 += MS) {
+        for (int s0 = 0; s0 < nparts; s0 += MS) {
             float pm[MS], pl[MS], pa[MS];
 #pragma unroll
             for (int u = 0; u < MS; ++u) {
                 const float *ps = pbase + ((s0 + u) * G + g) * (D + 2);
-                const bool in = s0 + u < splits;
+                const bool in = s0 + u < nparts;
                 pm[u] = in ? __ldcg(ps + D) : -INFINITY;
                 pl[u] = in ? __ldcg(ps + D + 1) : 0.0f;
                 pa[u] = in ? __ldcg(ps + i) : 0.0f;

@@ -199,10 +199,13 @@ struct ScoreOut {
     int R;               // tokens per warp range (multiple of 32)
     float inv2A;
     unsigned char *lut;  // 64 KB LUT region, free for reuse once scoring is done
-    uint16_t *cmax;      // [kCmaxCap] largest bin per 32-token chunk (CMAX only)
+    uint16_t *cmax;      // [kCmaxCap] largest bin per 32-token chunk (FUSED only)
 };
 
-template <int BITS, int D, bool PAGED, bool CMAX = false>
+// FUSED: the fused selection -- record the chunk maxima, and let the dependent
+// launch (the sparse decode, whose window CTAs need nothing from the selection)
+// start right after the wait on the preceding kernel.
+template <int BITS, int D, bool PAGED, bool FUSED = false>
 __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                                                 const int32_t *__restrict__ seq_lens, const RBits &R,
                                                 const SelWS &ws, int nctas, unsigned char *smem) {
@@ -292,6 +295,7 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     o.cmax = reinterpret_cast<uint16_t *>(smem + S::SCRATCH_BYTES);
     // everything above depends on q only; codes and lengths come from the append
     griddep_wait();
+    if constexpr (FUSED) griddep_trigger();
     o.n = clamp_len(kv, seq_lens, b);
     cta_range(o.n, blockIdx.x, nctas, o.t0, o.t1);
     const int64_t t0 = o.t0, t1 = o.t1;
@@ -360,7 +364,7 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
             bin = score_bin(s, inv2A);
             atomicAdd(&hist[bin], 1u);
         }
-        if constexpr (CMAX) {
+        if constexpr (FUSED) {
             const unsigned m = __reduce_max_sync(0xffffffffu, (unsigned)bin);
             const int c = (wb >> 5) + k;  // chunk of local tokens [32 c, 32 c + 32)
             if (lane == 0 && c < kCmaxCap) o.cmax[c] = (uint16_t)m;
@@ -879,7 +883,6 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     const int nctas = gridDim.x;
     const ScoreOut so = score_phase<BITS, D, PAGED, true>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
     const uint32_t *hist = reinterpret_cast<const uint32_t *>(smem);
-    griddep_trigger();
     {   // super-bin counts: 16 threads per super-bin, 4 bins each
         uint32_t c = hist[4 * tid] + hist[4 * tid + 1] + hist[4 * tid + 2] + hist[4 * tid + 3];
 #pragma unroll

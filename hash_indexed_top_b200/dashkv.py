@@ -69,7 +69,7 @@ def lib() -> ctypes.CDLL:
         L.dashkv_encode_keys.argtypes = [P, ctypes.POINTER(KVView), P, P]
         L.dashkv_append_keys.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P]
         L.dashkv_select.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
-        L.dashkv_sparse_decode.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
+        L.dashkv_sparse_decode.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, P, SZ, P]
         L.dashkv_select_static.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P]
         L.dashkv_get_error.argtypes = [P]
         L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
@@ -239,12 +239,15 @@ class DashKV:
 
     def sparse_decode(self, cache: KVCache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
                       out: torch.Tensor, lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                      stream=None) -> None:
+                      stream=None, seq_lens: Optional[torch.Tensor] = None) -> None:
+        """seq_lens (optional): the lengths sel_idx was selected for; given, the
+        sinks and the window are attended from the token range by CTAs that do
+        not wait for the selection."""
         ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
         v = cache.view()
         _check("dashkv_sparse_decode", lib().dashkv_sparse_decode(self._ctx, ctypes.byref(v), _ptr(q),
-                                                                  _ptr(sel_idx), _ptr(sel_cnt), _ptr(out),
-                                                                  _ptr(lse), _ptr(ws), ws.numel(),
+                                                                  _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt),
+                                                                  _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                                                   _stream(stream)))
 
     def select_kernels(self, max_tokens: int) -> int:

@@ -184,10 +184,15 @@ dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
  * KV head selected: out (device fp32 [B][Hq][d]); lse (optional, device
  * fp32 [B][Hq]) receives log sum_t exp(q.K_t / sqrt(d)) (-inf when nothing
  * is selected, out = 0 then).  sel_idx / sel_cnt as dashkv_select writes
- * them; ids must be < seq_lens[b]. */
+ * them; ids must be < seq_lens[b].  seq_lens (optional, device int32 [B]):
+ * NULL attends over exactly the rows of sel_idx.  When given, sel_idx /
+ * sel_cnt must be dashkv_select's output for these lengths: the sinks and the
+ * window (which every selection contains, at the two ends of the list) are
+ * then read from the token range directly by extra CTAs that need nothing
+ * from the selection and may run while it is still being computed. */
 dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
-                                   const int32_t *sel_idx, const int32_t *sel_cnt,
-                                   float *out, float *lse, void *workspace,
+                                   const int32_t *seq_lens, const int32_t *sel_idx,
+                                   const int32_t *sel_cnt, float *out, float *lse, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
 /* Synchronise `stream`, then read and clear the current device's error

@@ -17,8 +17,10 @@ ATOL, RTOL = 1e-3, 8e-3
 
 
 class GpuRun:
-    def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED, two_kernel: bool = False):
+    def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED, two_kernel: bool = False,
+                 window: bool = True):
         self.cfg, self.w = cfg, w
+        self.window = window  # decode given the lengths (window CTAs) or the plain list
         dev = w.K.device
         self.eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
                              cfg.page_size if w.paged else 0, seed, two_kernel_select=two_kernel)
@@ -37,7 +39,8 @@ class GpuRun:
     def select_decode(self, q: torch.Tensor):
         b = self.buf
         self.eng.select(self.cache, q, self.seq, b["sel_idx"], b["sel_cnt"], self.scores)
-        self.eng.sparse_decode(self.cache, q, b["sel_idx"], b["sel_cnt"], b["out"], b["lse"])
+        self.eng.sparse_decode(self.cache, q, b["sel_idx"], b["sel_cnt"], b["out"], b["lse"],
+                               seq_lens=self.seq if self.window else None)
 
     def error(self) -> int:
         return self.eng.get_error()
@@ -106,13 +109,13 @@ def compare_step(g: GpuRun, o: OracleRun, r: dict, what: str = "") -> dict:
 
 
 def run_parity(cfg: W.Config, steps: int, device="cuda", w: W.Workload | None = None, mutate=None,
-               two_kernel: bool = False) -> list:
+               two_kernel: bool = False, window: bool = True) -> list:
     """Encode, then `steps` x (append, select, decode) on GPU and oracle, comparing every step."""
     if w is None:
         w = W.make_workload(cfg, device="cpu", steps=steps)
     if mutate is not None:
         w = mutate(w)
-    g = GpuRun(cfg, w.to(device), two_kernel=two_kernel)
+    g = GpuRun(cfg, w.to(device), two_kernel=two_kernel, window=window)
     o = OracleRun(cfg, w)
     g.encode()
     diags = []

@@ -36,14 +36,18 @@ def built():
     build.build()
 
 
-PATHS = {"fused": False, "two_kernel": True}
+# selection path x decode mode: the fused selection with the decode's window
+# CTAs (lengths given), the same selection with a plain list decode, and the
+# two-kernel selection
+PATHS = {"fused": dict(two_kernel=False, window=True), "fused_list_decode": dict(two_kernel=False, window=False),
+         "two_kernel": dict(two_kernel=True, window=True)}
 
 
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(CASES))
 def test_parity(name, path):
     cfg, steps = CASES[name]
-    diags = run_parity(cfg, steps, two_kernel=PATHS[path])
+    diags = run_parity(cfg, steps, **PATHS[path])
     assert len(diags) == steps
 
 
@@ -51,14 +55,14 @@ def test_parity(name, path):
 def test_topk_covers_everything_is_dense_attention(path):
     cfg = W.Config("allk", B=2, Hq=8, Hkv=2, d=128, N=700, n_min=300, bits=64, topk=5000, sink=4, window=16,
                    steps=1, needles=2, seed=80)
-    run_parity(cfg, 1, two_kernel=PATHS[path])
+    run_parity(cfg, 1, **PATHS[path])
 
 
 @pytest.mark.parametrize("path", list(PATHS))
 def test_sinks_and_window_overlap_short_sequences(path):
     cfg = W.Config("overlap", B=4, Hq=4, Hkv=1, d=64, N=60, n_min=1, bits=32, topk=5, sink=20, window=50,
                    steps=2, needles=0, seed=81)
-    run_parity(cfg, 2, two_kernel=PATHS[path])
+    run_parity(cfg, 2, **PATHS[path])
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -71,7 +75,7 @@ def test_zero_query_all_scores_tie(path):
     def mutate(w):
         w.q.zero_()
         return w
-    run_parity(cfg, 1, mutate=mutate, two_kernel=PATHS[path])
+    run_parity(cfg, 1, mutate=mutate, **PATHS[path])
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -85,7 +89,7 @@ def test_repeated_keys_heavy_ties(path):
         idx = torch.arange(w.K.shape[2]) % 3
         w.K[:] = pat[:, :, idx]
         return w
-    run_parity(cfg, 1, mutate=mutate, two_kernel=PATHS[path])
+    run_parity(cfg, 1, mutate=mutate, **PATHS[path])
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -95,7 +99,7 @@ def test_empty_sequence_selects_nothing(path):
     w = W.make_workload(cfg, steps=0)
     w.seq_lens[1] = 0
     from pipeline import GpuRun, OracleRun, compare_step
-    g = GpuRun(cfg, w.to("cuda"), two_kernel=PATHS[path])
+    g = GpuRun(cfg, w.to("cuda"), **PATHS[path])
     o = OracleRun(cfg, w)
     g.encode()
     q = torch.zeros((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16)
@@ -114,7 +118,7 @@ def test_repeat_calls_are_deterministic_and_leave_workspace_clean(path):
     cfg, _ = CASES["c128k_small"]
     w = W.make_workload(cfg, steps=1).to("cuda")
     from pipeline import GpuRun
-    g = GpuRun(cfg, w, two_kernel=PATHS[path])
+    g = GpuRun(cfg, w, **PATHS[path])
     g.encode()
     g.append(0)
     outs = []
