@@ -352,40 +352,58 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     if (!s_last) return;
     __threadfence();
     const float *pbase = ws.part + (int64_t)bh * kMaxSplits * G * (D + 2);
-    // each output element: every split's (m, l, acc) loaded at once (one round
-    // trip), then the log-sum-exp merge in registers
-    constexpr int MS = 16;  // splits merged per pass (all loads of a pass in flight)
-    for (int x = tid; x < G * D; x += kAttnThreads) {
-        const int g = x / D, i = x % D;
-        float M = -INFINITY, L = 0.0f, Acc = 0.0f;
+    // each output element: every part's (m, l, acc) loaded at once -- for all
+    // the elements of this thread (EPT) in one round trip -- then the
+    // log-sum-exp merge in registers
+    constexpr int MS = 16;  // parts merged per pass (all loads of a pass in flight)
+    constexpr int EPT0 = (G * D + kAttnThreads - 1) / kAttnThreads;  // elements per thread
+    constexpr int EPT = EPT0 < 2 ? EPT0 : 2;                           // of them per round trip
+    for (int x0 = tid; x0 < G * D; x0 += EPT * kAttnThreads) {
+        float M[EPT], L[EPT], Acc[EPT];
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) { M[e] = -INFINITY; L[e] = 0.0f; Acc[e] = 0.0f; }
         for (int s0 = 0; s0 < nparts; s0 += MS) {
-            float pm[MS], pl[MS], pa[MS];
+            float pm[EPT][MS], pl[EPT][MS], pa[EPT][MS];
 #pragma unroll
-            for (int u = 0; u < MS; ++u) {
-                const float *ps = pbase + ((s0 + u) * G + g) * (D + 2);
-                const bool in = s0 + u < nparts;
-                pm[u] = in ? __ldcg(ps + D) : -INFINITY;
-                pl[u] = in ? __ldcg(ps + D + 1) : 0.0f;
-                pa[u] = in ? __ldcg(ps + i) : 0.0f;
+            for (int e = 0; e < EPT; ++e) {
+                const int x = x0 + e * kAttnThreads;
+                const int g = x / D, i = x % D;
+#pragma unroll
+                for (int u = 0; u < MS; ++u) {
+                    const float *ps = pbase + ((s0 + u) * G + g) * (D + 2);
+                    const bool in = x < G * D && s0 + u < nparts;
+                    pm[e][u] = in ? __ldcg(ps + D) : -INFINITY;
+                    pl[e][u] = in ? __ldcg(ps + D + 1) : 0.0f;
+                    pa[e][u] = in ? __ldcg(ps + i) : 0.0f;
+                }
             }
-            float Mn = M;
 #pragma unroll
-            for (int u = 0; u < MS; ++u) Mn = fmaxf(Mn, pm[u]);
-            if (Mn == -INFINITY) continue;
-            const float cM = fast_exp2(M - Mn);  // 0 when M = -inf
-            L *= cM;
-            Acc *= cM;
+            for (int e = 0; e < EPT; ++e) {
+                float Mn = M[e];
 #pragma unroll
-            for (int u = 0; u < MS; ++u) {
-                const float c = fast_exp2(pm[u] - Mn);  // 0 for empty splits (m = -inf)
-                L = fmaf(pl[u], c, L);
-                Acc = fmaf(pa[u], c, Acc);
+                for (int u = 0; u < MS; ++u) Mn = fmaxf(Mn, pm[e][u]);
+                if (Mn == -INFINITY) continue;
+                const float cM = fast_exp2(M[e] - Mn);  // 0 when M = -inf
+                L[e] *= cM;
+                Acc[e] *= cM;
+#pragma unroll
+                for (int u = 0; u < MS; ++u) {
+                    const float c = fast_exp2(pm[e][u] - Mn);  // 0 for empty parts (m = -inf)
+                    L[e] = fmaf(pl[e][u], c, L[e]);
+                    Acc[e] = fmaf(pa[e][u], c, Acc[e]);
+                }
+                M[e] = Mn;
             }
-            M = Mn;
         }
-        const int64_t oq = (int64_t)b * Hq + h * G + g;
-        out[oq * D + i] = L > 0.0f ? Acc / L : 0.0f;
-        if (i == 0 && lse) lse[oq] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+            const int x = x0 + e * kAttnThreads;
+            if (x >= G * D) continue;
+            const int g = x / D, i = x % D;
+            const int64_t oq = (int64_t)b * Hq + h * G + g;
+            out[oq * D + i] = L[e] > 0.0f ? Acc[e] / L[e] : 0.0f;
+            if (i == 0 && lse) lse[oq] = L[e] > 0.0f ? (M[e] + log2f(L[e])) * 0.6931471805599453f : -INFINITY;
+        }
     }
     if (tid == 0) ws.arrive[(int64_t)kSyncStride * bh] = 0;
 }

@@ -991,7 +991,7 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
             }
             asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
             __syncwarp();
-#pragma unroll 1
+#pragma unroll 2
             for (int f = 0; f < nf; ++f) {
                 const int li = 32 * hlist[h0 + f] + lane;  // warp-local token
                 const float sv = fbuf[32 * f + lane];
@@ -1003,17 +1003,36 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                     const uint32_t key = float_key(sv);
                     if (j < CW) wcand[j] = make_uint2((uint32_t)t, key);
                     else { cand[t0 + wb + j] = t; ckey[t0 + wb + j] = key; }
-                    if (sv < theta2) {
-                        const int slot = atomicAdd(&s_ninb, 1);
-                        if (slot < kInbinMax)
-                            s_loc[slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, (uint32_t)warp);
-                    } else if (t >= s_end && t < w_beg) {
-                        ++ndef;
-                    }
                 }
                 ncand += __popc(ball);
             }
             __syncwarp();  // the buffer is refilled by the next batch
+        }
+    }
+    auto cand_at = [&](int j, int &t, uint32_t &key) {
+        if (j < CW) { const uint2 c = wcand[j]; t = (int)c.x; key = c.y; }
+        else { t = __ldcg(cand + t0 + wb + j); key = __ldcg(ckey + t0 + wb + j); }
+    };
+    __syncwarp();
+    // classify the warp's candidates, 32 at a time: in the threshold bin (score <
+    // theta2: listed for the cluster, one reservation per group) or definite
+    // (counted when in the middle range)
+    const uint32_t key2 = float_key(theta2);  // order keys follow scores
+    for (int jb = 0; jb < ncand; jb += 32) {
+        const int j = jb + lane;
+        int t = 0;
+        uint32_t key = 0;
+        if (j < ncand) cand_at(j, t, key);
+        const bool inb = j < ncand && key < key2;
+        const bool def = j < ncand && !inb && t >= s_end && t < w_beg;
+        ndef += __popc(__ballot_sync(0xffffffffu, def)) * (lane == 0);
+        const uint32_t ib = __ballot_sync(0xffffffffu, inb);
+        if (ib) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&s_ninb, __popc(ib));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int slot = base + __popc(ib & lt);
+            if (inb && slot < kInbinMax) s_loc[slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, (uint32_t)warp);
         }
     }
 #pragma unroll
@@ -1136,10 +1155,6 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     };
     // ---- ordered emission: warp w writes its kept candidates from offset
     // s_end + (this CTA's offset) + (kept candidates of warps < w)
-    auto cand_at = [&](int j, int &t, uint32_t &key) {
-        if (j < CW) { const uint2 c = wcand[j]; t = (int)c.x; key = c.y; }
-        else { t = __ldcg(cand + t0 + wb + j); key = __ldcg(ckey + t0 + wb + j); }
-    };
     int wpos = s_end + s_misc[2];
     for (int w2 = 0; w2 < warp; ++w2) wpos += s_wkeep[w2];
     for (int jb = 0; jb < ncand; jb += 32) {
