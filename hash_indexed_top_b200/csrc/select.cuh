@@ -325,6 +325,9 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     const unsigned char *ring = lut + 65536 + tid * VB;
     const Vec *dense = reinterpret_cast<const Vec *>(kv.codes) + ((int64_t)bh * kv.n_cap + t0);
     float *srow = ws.scores + (int64_t)bh * ws.ld + t0;
+    // Step k copies token wb + 32 k + lane into ring slot k % STAGES; the loop
+    // is unrolled by STAGES so every slot (and its shared address) is a
+    // compile-time constant, and the positions advance by 32 tokens per step.
     auto issue = [&](int k, int slot) {  // copy the code of token wb + 32 k + lane into `slot`
         const int i = wb + 32 * k + lane;
         const void *src = dense;
@@ -347,27 +350,29 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     };
 #pragma unroll
     for (int k = 0; k < STAGES - 1; ++k) issue(k, k);
-    int slot = 0, islot = STAGES - 1;
-    for (int k = 0; k < nk; ++k) {
-        issue(k + STAGES - 1, islot);
-        islot = islot == STAGES - 1 ? 0 : islot + 1;
-        asm volatile("cp.async.wait_group %0;" ::"n"(STAGES - 1) : "memory");
-        const int i = wb + 32 * k + lane;
-        const Vec code = *reinterpret_cast<const Vec *>(ring + slot * NT * VB);
-        slot = slot == STAGES - 1 ? 0 : slot + 1;
-        int bin = 0;
-        if (i < we) {
-            uint32_t w[NW];
-            unpack_code<BITS>(code, w);
-            const float s = lut_score<BITS>(w, lbase);
-            srow[i] = s;
-            bin = score_bin(s, inv2A);
-            atomicAdd(&hist[bin], 1u);
-        }
-        if constexpr (FUSED) {
-            const unsigned m = __reduce_max_sync(0xffffffffu, (unsigned)bin);
-            const int c = (wb >> 5) + k;  // chunk of local tokens [32 c, 32 c + 32)
-            if (lane == 0 && c < kCmaxCap) o.cmax[c] = (uint16_t)m;
+    for (int k0 = 0; k0 < nk; k0 += STAGES) {
+#pragma unroll
+        for (int u = 0; u < STAGES; ++u) {
+            const int k = k0 + u;
+            if (k >= nk) break;
+            issue(k + STAGES - 1, (u + STAGES - 1) % STAGES);
+            asm volatile("cp.async.wait_group %0;" ::"n"(STAGES - 1) : "memory");
+            const int i = wb + 32 * k + lane;
+            const Vec code = *reinterpret_cast<const Vec *>(ring + u * NT * VB);
+            int bin = 0;
+            if (i < we) {
+                uint32_t w[NW];
+                unpack_code<BITS>(code, w);
+                const float sc = lut_score<BITS>(w, lbase);
+                srow[i] = sc;
+                bin = score_bin(sc, inv2A);
+                atomicAdd(&hist[bin], 1u);
+            }
+            if constexpr (FUSED) {
+                const unsigned m = __reduce_max_sync(0xffffffffu, (unsigned)bin);
+                const int c = (wb >> 5) + k;  // chunk of local tokens [32 c, 32 c + 32)
+                if (lane == 0 && c < kCmaxCap) o.cmax[c] = (uint16_t)m;
+            }
         }
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
