@@ -47,15 +47,41 @@ def measured_peaks() -> dict:
     return dict(hbm_gbs=6650.0, source="fallback")
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed (string
+    literals are kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"':
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_sources_sha() -> str:
-    """sha256 over the library's CUDA sources (name and bytes, sorted by name)."""
+    """sha256 over the library's CUDA sources (name and code without comments
+    or layout, sorted by name): it changes when the kernels do, not when only
+    their comments do."""
     d = os.path.join(ROOT, "hash_indexed_top_b200", "csrc")
     h = hashlib.sha256()
     for n in sorted(os.listdir(d)):
         if n.endswith((".cu", ".cuh")):
             h.update(n.encode())
-            with open(os.path.join(d, n), "rb") as f:
-                h.update(f.read())
+            with open(os.path.join(d, n), encoding="utf-8") as f:
+                h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

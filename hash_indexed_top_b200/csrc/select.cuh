@@ -18,17 +18,24 @@
 // tokens): top-k over all N tokens ordered by (score desc, index asc), united
 // with [0, S) and [N - W, N), written ascending.
 //
-// Kernels (grid = (ctas per (b, h), B * Hkv)):
-//   score_hist_kernel : LUT prologue, stream the codes, write fp32 scores, build
-//                       a 4096-bin histogram of the scores over [-A, A]
-//                       (A = sum_j |Qp_j| bounds every |s_t|); the last CTA of a
-//                       (b, h) finds the bin T1 holding the k-th largest score.
-//   collect_kernel    : ordered compaction of the tokens whose bin is >= T1
-//                       into per-CTA segments; the last CTA of a (b, h) resolves
-//                       the exact threshold inside bin T1 (score, then index)
-//                       and writes the final ascending selection.
-// No kernel waits on another CTA: "last CTA" is decided by an atomic arrival
-// counter, which the last CTA resets, so the workspace is left clean.
+// Kernels (grid = (CTAs per (b, h), B * Hkv)):
+//   select_fused_kernel (default): one thread-block cluster per (b, h).  Each
+//                       CTA streams its range of codes (LUT scorer, fp32
+//                       scores, 4096-bin histogram over [-A, A] with
+//                       A = sum_j |Qp_j| bounding every |s_t|, per-chunk maximum
+//                       bins); the cluster then finds the bin T1 holding the
+//                       k-th largest score from its histograms in distributed
+//                       shared memory, keeps the tokens with bin >= T1, ranks
+//                       the ones in T1 exactly (score, then index) and writes
+//                       the ascending selection.  CTAs wait for one another only
+//                       at hardware cluster barriers.
+//   score_hist_kernel + collect_kernel (without cluster launch support, or on
+//                       request): the same scoring, then the last CTA of a
+//                       (b, h) (atomic arrival counter, which it resets: the
+//                       workspace is left clean) finds T1; the collect kernel
+//                       compacts the tokens with bin >= T1 into per-CTA
+//                       segments and its last CTA resolves the threshold bin
+//                       and writes the selection.  No CTA waits for another.
 #pragma once
 #include "common.cuh"
 
