@@ -16,7 +16,7 @@ from oracle import oracle as O
 ATOL, RTOL = 1e-3, 8e-3
 
 
-class GpuRun:
+class DeviceRun:
     def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED, two_kernel: bool = False,
                  window: bool = True):
         self.cfg, self.w = cfg, w
@@ -82,7 +82,7 @@ def within_tol(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
     return both_inf | (err <= ATOL + RTOL * np.abs(ref))
 
 
-def compare_step(g: GpuRun, o: OracleRun, r: dict, what: str = "") -> dict:
+def compare_step(g: DeviceRun, o: OracleRun, r: dict, what: str = "") -> dict:
     """Assert parity of one step; returns a few diagnostics."""
     gc = dk.canonical_codes(g.cache.codes, o.cfg.bits).cpu().numpy().view(np.uint64)
     assert np.array_equal(gc, o.codes), f"{what}: codes differ at {np.argwhere(gc != o.codes)[:5].tolist()}"
@@ -115,7 +115,7 @@ def run_parity(cfg: W.Config, steps: int, device="cuda", w: W.Workload | None = 
         w = W.make_workload(cfg, device="cpu", steps=steps)
     if mutate is not None:
         w = mutate(w)
-    g = GpuRun(cfg, w.to(device), two_kernel=two_kernel, window=window)
+    g = DeviceRun(cfg, w.to(device), two_kernel=two_kernel, window=window)
     o = OracleRun(cfg, w)
     g.encode()
     diags = []

@@ -98,8 +98,8 @@ def test_empty_sequence_selects_nothing(path):
                    steps=0, needles=0, seed=84)
     w = W.make_workload(cfg, steps=0)
     w.seq_lens[1] = 0
-    from pipeline import GpuRun, OracleRun, compare_step
-    g = GpuRun(cfg, w.to("cuda"), **PATHS[path])
+    from pipeline import DeviceRun, OracleRun, compare_step
+    g = DeviceRun(cfg, w.to("cuda"), **PATHS[path])
     o = OracleRun(cfg, w)
     g.encode()
     q = torch.zeros((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16)
@@ -117,8 +117,8 @@ def test_empty_sequence_selects_nothing(path):
 def test_repeat_calls_are_deterministic_and_leave_workspace_clean(path):
     cfg, _ = CASES["c128k_small"]
     w = W.make_workload(cfg, steps=1).to("cuda")
-    from pipeline import GpuRun
-    g = GpuRun(cfg, w, **PATHS[path])
+    from pipeline import DeviceRun
+    g = DeviceRun(cfg, w, **PATHS[path])
     g.encode()
     g.append(0)
     outs = []
@@ -136,8 +136,8 @@ def test_needle_recall_reported():
     # quality number, not a parity gate: planted needles close to the query
     cfg = W.CONFIGS["c32k"].scaled(name="recall", N=16384, steps=1)
     w = W.make_workload(cfg, steps=1).to("cuda")
-    from pipeline import GpuRun
-    g = GpuRun(cfg, w)
+    from pipeline import DeviceRun
+    g = DeviceRun(cfg, w)
     g.encode()
     g.append(0)
     g.select_decode(w.q[0])
