@@ -1,0 +1,89 @@
+"""Full-size parity: every configured long-context workload at its full size,
+one decode step in the launch configuration the benchmark times (the fused
+selection, the decode given the lengths), checked against the oracle on whole
+sampled (sequence, kv head) pairs: all of a pair's codes and scores, its
+selection, and the attention output and lse of its query heads.
+
+The oracle recomputes a pair from its own encode of the pair's keys (no GPU
+value enters it); the pairs are the first and the last of the grid."""
+import numpy as np
+import pytest
+import torch
+
+from hash_indexed_top_b200 import dashkv as dk
+from hash_indexed_top_b200 import workloads as W
+from oracle import oracle as O
+
+from pipeline import within_tol
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["c32k", "c128k", "ragged_paged", "c1m"]
+
+
+def _pair_rows(x: torch.Tensor, w: W.Workload, b: int, h: int, n: int) -> torch.Tensor:
+    """Rows [0, n) of kv head h of sequence b: [n, ...] (dense or through the page table)."""
+    if not w.paged:
+        return x[b, h, :n]
+    ps = w.cfg.page_size
+    t = torch.arange(n, device=x.device)
+    pages = w.page_table[b].long()[t // ps]
+    return x[pages, t % ps, h]
+
+
+def _pair_codes(codes: torch.Tensor, w: W.Workload, b: int, h: int, n: int) -> torch.Tensor:
+    if not w.paged:
+        return codes[b, h, :n]
+    ps = w.cfg.page_size
+    t = torch.arange(n, device=codes.device)
+    pages = w.page_table[b].long()[t // ps]
+    return codes[pages, h, t % ps]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_step_on_sampled_pairs(name):
+    cfg = W.CONFIGS[name]
+    dev = torch.device("cuda")
+    w = W.make_workload(cfg, device=dev, steps=1)
+    eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
+                    cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED)
+    try:
+        cache = dk.KVCache(w.K, w.V, dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged), w.page_table)
+        seq = w.seq_lens.clone()
+        eng.encode_keys(cache, seq)
+        eng.append_keys(cache, w.k_new[0], w.v_new[0], seq)
+        buf = eng.alloc_step(dev)
+        scores = torch.full((cfg.B, cfg.Hkv, cache.capacity), float("nan"), device=dev)
+        ws = eng.workspace(cache.capacity, dev)
+        eng.select(cache, w.q[0], seq, buf["sel_idx"], buf["sel_cnt"], scores, ws)
+        eng.sparse_decode(cache, w.q[0], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws, seq_lens=seq)
+        torch.cuda.synchronize()
+        assert eng.get_error() == 0
+        gcodes = dk.canonical_codes(cache.codes, cfg.bits)
+        R = O.hyperplanes(W.HYPERPLANE_SEED, cfg.bits, cfg.d)
+        G = cfg.G
+        for b, h in [(0, 0), (cfg.B - 1, cfg.Hkv - 1)]:
+            n = int(seq[b])
+            K = _pair_rows(w.K, w, b, h, n).double().cpu().numpy().reshape(1, 1, n, cfg.d)
+            V = _pair_rows(w.V, w, b, h, n).double().cpu().numpy().reshape(1, 1, n, cfg.d)
+            L = O.Layout(1, 1, cfg.d, cfg.bits, n_cap=n)
+            sl = np.array([n], dtype=np.int32)
+            oc = O.encode(L, K, sl, R)
+            gc = _pair_codes(gcodes, w, b, h, n).cpu().numpy().view(np.uint64)
+            assert np.array_equal(gc, oc[0, 0]), f"{name} ({b},{h}): codes differ at {np.argwhere(gc != oc[0, 0])[:3]}"
+            q = w.q[0][b, h * G:(h + 1) * G].double().cpu().numpy().reshape(1, G, cfg.d)
+            r = O.decode_step(L, G, q, K, V, oc, sl, R, cfg.topk, cfg.sink, cfg.window)
+            gs = scores[b, h, :n].cpu().numpy()
+            es = r["scores"][0, 0, :n].astype(np.float32)
+            assert np.array_equal(gs.view(np.uint32), es.view(np.uint32)), \
+                f"{name} ({b},{h}): scores differ at {np.argwhere(gs != es)[:3].ravel()}"
+            cnt = int(buf["sel_cnt"][b, h])
+            assert cnt == int(r["sel_cnt"][0, 0]), f"{name} ({b},{h}): sel_cnt {cnt} vs {int(r['sel_cnt'][0, 0])}"
+            assert np.array_equal(buf["sel_idx"][b, h].cpu().numpy(), r["sel_idx"][0, 0]), \
+                f"{name} ({b},{h}): selection differs"
+            out = buf["out"][b, h * G:(h + 1) * G].double().cpu().numpy()
+            lse = buf["lse"][b, h * G:(h + 1) * G].double().cpu().numpy()
+            assert within_tol(out, r["out"][0]).all(), f"{name} ({b},{h}): out err {np.abs(out - r['out'][0]).max()}"
+            assert within_tol(lse, r["lse"][0]).all(), f"{name} ({b},{h}): lse err {np.abs(lse - r['lse'][0]).max()}"
+    finally:
+        eng.close()
