@@ -16,22 +16,18 @@ def test_strip_comments_keeps_code_and_string_literals():
     assert bench._strip_comments(src) == 'int a = 1; const char *p = "x//y/*z*/"; int b;'
 
 
-def _copy_tree(tmp_path):
-    for sub in ("hash_indexed_top_b200/csrc", "profiles"):
-        shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub)
-    return tmp_path
-
-
 def test_recorded_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
-    root = _copy_tree(tmp_path)
-    monkeypatch.setattr(bench, "ROOT", str(root))
-    summary = root / "profiles" / "c128k_step_kernels_full.txt"
-    recorded = [ln for ln in summary.read_text().splitlines() if ln.startswith("traffic_per_launch select_fused")]
-    assert recorded, "the summary records the select kernel's traffic"
-    expect = int(recorded[0].split()[2])
-    assert bench.recorded_traffic("select_fused") == expect  # committed summary matches the committed code
-    src = root / "hash_indexed_top_b200" / "csrc" / "select.cuh"
+    shutil.copytree(os.path.join(ROOT, "hash_indexed_top_b200", "csrc"), tmp_path / "hash_indexed_top_b200" / "csrc")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    summary = tmp_path / "profiles" / "c128k_step_kernels_full.txt"
+    assert bench.recorded_traffic("select_fused") is None  # no summary, no figure
+    summary.write_text(f"kernel sources sha256: {bench.kernel_sources_sha()}\n"
+                       "traffic_per_launch select_fused_kernel 123456\n")
+    assert bench.recorded_traffic("select_fused") == 123456  # taken from these kernels
+    assert bench.recorded_traffic("score_hist") is None  # not measured
+    src = tmp_path / "hash_indexed_top_b200" / "csrc" / "select.cuh"
     src.write_text("// a comment-only change\n" + src.read_text())
-    assert bench.recorded_traffic("select_fused") == expect  # comments do not make the counters stale
+    assert bench.recorded_traffic("select_fused") == 123456  # comments do not make the counters stale
     src.write_text(src.read_text() + "\nstatic int changed_code = 1;\n")
     assert bench.recorded_traffic("select_fused") is None  # a code change does
