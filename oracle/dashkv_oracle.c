@@ -316,3 +316,82 @@ void dko_attend(int B, int Hq, int Hkv, int d, int64_t n_cap,
             free(logit);
         }
 }
+
+/* ------------------------------------------------------- block summaries */
+/*
+ * CSA-style two-level index (DeepSeek DSA->CSA/HCA page, CSA section: every m
+ * history tokens are compressed into one summary entry and the top-k is taken
+ * over the summaries; section on the compressed KV cache versus the state
+ * cache: tokens of a block that is not yet complete -- the page's example has
+ * 2 of m = 4 -- wait in the state cache until the block fills up).
+ *
+ * The pages' compressor is learned; none is available here.  The summary of
+ * block i (tokens [i*m, (i+1)*m)) is therefore the hash code of the block's
+ * summed key: the sign of a projection of the block's mean key is the sign of
+ * the projection of its sum.  Only complete blocks, i < floor(N / m), have a
+ * summary.  Attention stays exact: it runs over every token of the selected
+ * blocks, the sinks, the window and the incomplete tail (the state cache).
+ *
+ * block codes: dense [B][Hkv][nb_cap][W64], canonical bit order.
+ */
+void dko_encode_blocks(int B, int Hkv, int d, int bits, int64_t n_cap,
+                       const int32_t *page_table, int max_pages, int page,
+                       const double *K, const int32_t *seq_lens, int block,
+                       const int8_t *R, int64_t nb_cap, uint64_t *block_codes) {
+    dko_layout L = make_layout(B, Hkv, d, bits, n_cap, page_table, max_pages, page);
+    int w64 = bits / 64 > 0 ? bits / 64 : 1;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            int64_t nb = seq_lens[b] / block;
+#pragma omp parallel for schedule(static)
+            for (int64_t i = 0; i < nb; ++i) {
+                double *ksum = (double *)calloc((size_t)d, sizeof(double));
+                for (int64_t t = i * block; t < (i + 1) * block; ++t) {
+                    const double *k = K + row_index(&L, b, h, t);
+                    for (int e = 0; e < d; ++e) ksum[e] += k[e];
+                }
+                encode_one(ksum, R, bits, d, block_codes + (((int64_t)b * Hkv + h) * nb_cap + i) * w64);
+                free(ksum);
+            }
+        }
+}
+
+/* Token selection from block scores.  block_scores: [B][Hkv][nb_cap], valid
+ * for blocks i < floor(seq_lens[b] / block).  Per (b, kv head): the
+ * topk_blocks best complete blocks (score desc, block index asc; all of them
+ * when fewer exist), every token of each, united with the sinks [0, S), the
+ * window [N-W, N) and the tail [m*floor(N/m), N).  Output as dko_select:
+ * ascending ids, -1 padded to cap.  Returns 0, or -1 when cap is too small. */
+int dko_select_blocks(int B, int Hkv, int64_t nb_cap, const int32_t *seq_lens, int block,
+                      const double *block_scores, int topk_blocks, int sink, int window,
+                      int32_t *sel_idx, int32_t *sel_cnt, int cap) {
+    int rc = 0;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            int64_t n = seq_lens[b];
+            int64_t nb = n / block;
+            const double *s = block_scores + ((int64_t)b * Hkv + h) * nb_cap;
+            scored *all = (scored *)malloc(sizeof(scored) * (size_t)(nb > 0 ? nb : 1));
+            for (int64_t i = 0; i < nb; ++i) { all[i].s = s[i]; all[i].t = i; }
+            qsort(all, (size_t)nb, sizeof(scored), by_score_desc_index_asc);
+            int64_t kk = topk_blocks < nb ? topk_blocks : nb;
+            char *in = (char *)calloc((size_t)(n > 0 ? n : 1), 1);
+            for (int64_t r = 0; r < kk; ++r)
+                for (int64_t t = all[r].t * block; t < (all[r].t + 1) * block; ++t) in[t] = 1;
+            for (int64_t t = 0; t < n && t < sink; ++t) in[t] = 1;
+            for (int64_t t = n - window; t < n; ++t) if (t >= 0) in[t] = 1;
+            for (int64_t t = nb * block; t < n; ++t) in[t] = 1;
+            int64_t c = 0;
+            int32_t *out = sel_idx + ((int64_t)b * Hkv + h) * cap;
+            for (int64_t t = 0; t < n; ++t)
+                if (in[t]) {
+                    if (c < cap) out[c] = (int32_t)t; else rc = -1;
+                    ++c;
+                }
+            for (int64_t r = c; r < cap; ++r) out[r] = -1;
+            sel_cnt[(int64_t)b * Hkv + h] = (int32_t)c;
+            free(in);
+            free(all);
+        }
+    return rc;
+}

@@ -54,6 +54,9 @@ def lib():
         L.dko_select.argtypes = [I, I, I64, P, P, I, I, I, P, P, I]
         L.dko_select.restype = I
         L.dko_attend.argtypes = [I, I, I, I, I64, P, I, I, P, P, P, P, P, I, P, P]
+        L.dko_encode_blocks.argtypes = [I, I, I, I, I64, P, I, I, P, P, I, P, I64, P]
+        L.dko_select_blocks.argtypes = [I, I, I64, P, I, P, I, I, I, P, P, I]
+        L.dko_select_blocks.restype = I
         L.dko_set_threads.argtypes = [I]
         L.dko_get_threads.restype = I
         _lib = L
@@ -174,3 +177,54 @@ def decode_step(layout: Layout, Hq, q, K, V, codes, seq_lens, R, topk, sink, win
     idx, cnt = select(sc, seq_lens, topk, sink, window)
     out, lse = attend(layout, Hq, q, K, V, idx, cnt)
     return dict(scores=sc, bound=bound, sel_idx=idx, sel_cnt=cnt, out=out, lse=lse)
+
+
+# ---------------------------------------------------------------- block summaries
+# CSA-style two-level index (DeepSeek DSA->CSA/HCA page, CSA section and the
+# section on the compressed versus the state cache): the summary of each
+# complete block of m tokens is the code of the block's summed key, the top
+# blocks are selected by the same asymmetric score, and attention runs exactly
+# over their tokens, the sinks, the window and the incomplete tail.
+
+def block_capacity(n_cap: int, block: int) -> int:
+    """Blocks a cache of n_cap tokens can hold (complete blocks only)."""
+    return int(n_cap) // int(block)
+
+
+def encode_blocks(layout: Layout, K, seq_lens, block: int, R, nb_cap: int) -> np.ndarray:
+    """Summary codes [B, Hkv, nb_cap, W64] (uint64, canonical bit order) of the
+    complete blocks [0, seq_lens[b] // block); other entries 0."""
+    codes = np.zeros((layout.B, layout.Hkv, int(nb_cap), layout.w64), dtype=np.uint64)
+    lib().dko_encode_blocks(*layout.args(), _p(_f64(K)), _p(_i32(seq_lens)), int(block),
+                            _p(np.ascontiguousarray(R, dtype=np.int8)), int(nb_cap), _p(codes))
+    return codes
+
+
+def block_scores(layout: Layout, Hq, q, block_codes, seq_lens, block: int, R):
+    """(scores [B, Hkv, nb_cap] float64 of the complete blocks (NaN beyond), bound):
+    the asymmetric score of each block's summary code."""
+    nb_cap = int(block_codes.shape[2])
+    L = Layout(layout.B, layout.Hkv, layout.d, layout.bits, n_cap=nb_cap)
+    return scores(L, Hq, q, block_codes, _i32(seq_lens) // int(block), R)
+
+
+def select_blocks(bscores, seq_lens, block: int, topk_blocks: int, sink: int, window: int, cap: int):
+    """(sel_idx [B, Hkv, cap] int32 ascending token ids, -1 padded; sel_cnt [B, Hkv])."""
+    s = _f64(bscores)
+    B, Hkv, nb_cap = s.shape
+    idx = np.empty((B, Hkv, int(cap)), dtype=np.int32)
+    cnt = np.empty((B, Hkv), dtype=np.int32)
+    rc = lib().dko_select_blocks(B, Hkv, nb_cap, _p(_i32(seq_lens)), int(block), _p(s), int(topk_blocks),
+                                 int(sink), int(window), _p(idx), _p(cnt), int(cap))
+    if rc != 0:
+        raise ValueError("selection larger than cap")
+    return idx, cnt
+
+
+def decode_step_blocks(layout: Layout, Hq, q, K, V, block_codes, seq_lens, R, block, topk_blocks, sink, window,
+                       cap):
+    """Block score -> block select -> exact attention for one decode query batch."""
+    bs, bound = block_scores(layout, Hq, q, block_codes, seq_lens, block, R)
+    idx, cnt = select_blocks(bs, seq_lens, block, topk_blocks, sink, window, cap)
+    out, lse = attend(layout, Hq, q, K, V, idx, cnt)
+    return dict(block_scores=bs, bound=bound, sel_idx=idx, sel_cnt=cnt, out=out, lse=lse)
