@@ -198,9 +198,11 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ----------------------------------------------------------------------------- oracle leg
 def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
-    """Time the CPU oracle's decode step (score + select + attend) on one
-    sequence of the workload (all its KV / query heads), after one untimed
-    oracle encode of that sequence's cache."""
+    """Time the CPU oracle's decode step (score + select + attend; with block
+    summaries: block score + block select + attend) on one sequence of the
+    workload (all its KV / query heads), after one untimed oracle encode of that
+    sequence's cache.  Appends (and the summary of a block an append completes)
+    are untimed too."""
     from oracle import oracle as O
     one = cfg.scaled(B=1, steps=n_steps + 1)
     w = W.make_workload(one, device="cpu", steps=n_steps + 1)
@@ -210,22 +212,44 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
     V = w.V.double().numpy()
     seq = w.seq_lens.numpy().astype(np.int32).copy()
     codes = O.encode(L, K, seq, R)
+    m = cfg.block
+    if m:
+        nb_cap = w.n_cap // m
+        bcodes = O.encode_blocks(L, K, seq, m, R, nb_cap)
+
+    def append(s):
+        O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
+        n = int(seq[0])
+        if m and n % m == 0:  # the block this append completed
+            Lb = O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=m)
+            last = np.ascontiguousarray(K[:, :, n - m:n])
+            bcodes[:, :, n // m - 1] = O.encode_blocks(Lb, last, np.array([m], np.int32), m, R, 1)[:, :, 0]
+
+    def decode(s):
+        q = w.q[s].double().numpy()
+        if m:
+            O.decode_step_blocks(L, cfg.Hq, q, K, V, bcodes, seq, R, m, cfg.topk // m, cfg.sink, cfg.window,
+                                 cap=cfg.sel_cap)
+        else:
+            O.decode_step(L, cfg.Hq, q, K, V, codes, seq, R, cfg.topk, cfg.sink, cfg.window)
+
     times = []
     for s in range(n_steps):
-        O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
+        append(s)
         t0 = time.perf_counter()
-        O.decode_step(L, cfg.Hq, w.q[s].double().numpy(), K, V, codes, seq, R, cfg.topk, cfg.sink, cfg.window)
+        decode(s)
         times.append(time.perf_counter() - t0)
     cores = O.get_threads()
     # one more step on a single thread, for reference
-    O.append(L, K, V, codes, seq, w.k_new[n_steps].double().numpy(), w.v_new[n_steps].double().numpy(), R)
+    append(n_steps)
     O.set_threads(1)
     t0 = time.perf_counter()
-    O.decode_step(L, cfg.Hq, w.q[n_steps].double().numpy(), K, V, codes, seq, R, cfg.topk, cfg.sink, cfg.window)
+    decode(n_steps)
     one_thread_s = time.perf_counter() - t0
     O.set_threads(cores)
+    how = f", blocks of {m}" if m else ""
     return dict(times=times, cores=cores, one_thread_s=one_thread_s,
-                sample=f"sequence {seq_index} of {cfg.B} (N={cfg.N}, all {cfg.Hkv} KV / {cfg.Hq} query heads), "
+                sample=f"sequence {seq_index} of {cfg.B} (N={cfg.N}, all {cfg.Hkv} KV / {cfg.Hq} query heads{how}), "
                        f"{n_steps} decode steps, oracle encode untimed")
 
 
@@ -242,7 +266,7 @@ def run_reference(args, cfg, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
                    "bits": cfg.bits, "topk": cfg.topk, "sink": cfg.sink, "window": cfg.window,
-                   "per_step_sample": "one sequence's decode query"},
+                   "block": cfg.block or None, "per_step_sample": "one sequence's decode query"},
         "cpu_baseline": {"value": value, "unit": "queries/s", "cores": r["cores"], "kind": "oracle",
                          "sample": r["sample"], "one_thread_value": 1.0 / r["one_thread_s"]},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -274,6 +298,10 @@ def run_dashkv(args, cfg, world, rank, local):
     flush = W.L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     eng.encode_keys(cache, seq)
+    index = None
+    if cfg.block:  # block summaries of the prefilled cache (untimed, like the key codes)
+        index = dk.BlockIndex.empty_for(cache, cfg.B, cfg.bits, cfg.block)
+        eng.encode_blocks(cache, index, seq)
     torch.cuda.synchronize(dev)
     assert eng.get_error() == 0
     # the prefill encode, timed on its own (a second, identical call: cold L2, kernel already loaded)
@@ -301,26 +329,45 @@ def run_dashkv(args, cfg, world, rank, local):
     K = args.steps
     T = min(K, args.trace_steps)
     n_sel_kernels = eng.select_kernels(cache.capacity)
-    dom = "select_fused" if n_sel_kernels == 1 else "score_hist"  # the kernel that streams the codes
+    sel_names = ["select_fused"] if n_sel_kernels == 1 else ["score_hist", "collect_select"]
+    dom = sel_names[0]  # the kernel that streams the codes (of the tokens, or of the block summaries)
+    # the kernels of one step, in launch order, and the calls that launch them
+    calls = [("append_keys", ["append_keys"])]
+    if cfg.block:
+        calls += [("append_blocks", ["append_blocks"]), ("select_blocks", sel_names + ["expand_blocks"])]
+    else:
+        calls += [("select", sel_names)]
+    calls += [("sparse_decode", ["sparse_decode"])]
+    kernels = [k for _, ks in calls for k in ks]
     n_graph = args.warmup + K + T
+
+    def step(q, kn, vn, out, lse, e=None):
+        """Enqueue one decode step; with events e, trace pair 1 + j around kernel j."""
+        j = 1
+        for name, ks in calls:
+            if e is not None:
+                eng.set_trace(e[2 * j:2 * (j + len(ks))])
+            if name == "append_keys":
+                eng.append_keys(cache, kn, vn, seq)
+            elif name == "append_blocks":
+                eng.append_blocks(cache, index, seq)
+            elif name == "select_blocks":
+                eng.select_blocks(cache, index, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            elif name == "select":
+                eng.select(cache, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            else:
+                eng.sparse_decode(cache, q, buf["sel_idx"], buf["sel_cnt"], out, lse, ws, seq_lens=seq)
+            j += len(ks)
+        if e is not None:
+            eng.set_trace(None)
 
     def capture(s, e=None):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            if e is not None:
-                eng.set_trace(e[2:4])
-            eng.append_keys(cache, w.k_new[s], w.v_new[s], seq)
-            if e is not None:
-                eng.set_trace(e[4:8])
-            eng.select(cache, w.q[s], seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
-            if e is not None:
-                eng.set_trace(e[8:10])
-            eng.sparse_decode(cache, w.q[s], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws, seq_lens=seq)
-            if e is not None:
-                eng.set_trace(None)
+            step(w.q[s], w.k_new[s], w.v_new[s], buf["out"], buf["lse"], e)
         return g
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(n_graph)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + 2 * len(kernels))] for _ in range(n_graph)]
     for e in ev:  # materialise the CUDA events (torch creates them on first record)
         for x in e:
             x.record(stream)
@@ -357,13 +404,8 @@ def run_dashkv(args, cfg, world, rank, local):
                     traced[i].replay()
                 torch.cuda.synchronize(dev)
                 tb = args.warmup + K
-                kern = {"append_keys": [ev[tb + i][2].elapsed_time(ev[tb + i][3]) for i in range(T)]}
-                if n_sel_kernels == 1:
-                    kern["select_fused"] = [ev[tb + i][4].elapsed_time(ev[tb + i][5]) for i in range(T)]
-                else:
-                    kern["score_hist"] = [ev[tb + i][4].elapsed_time(ev[tb + i][5]) for i in range(T)]
-                    kern["collect_select"] = [ev[tb + i][6].elapsed_time(ev[tb + i][7]) for i in range(T)]
-                kern["sparse_decode"] = [ev[tb + i][8].elapsed_time(ev[tb + i][9]) for i in range(T)]
+                kern = {k: [ev[tb + i][2 + 2 * j].elapsed_time(ev[tb + i][3 + 2 * j]) for i in range(T)]
+                        for j, k in enumerate(kernels)}
     # back-to-back replays of the same steps without the L2 flush (warm; reported
     # for reference only, labelled as such)
     for i in range(K):
@@ -381,9 +423,11 @@ def run_dashkv(args, cfg, world, rank, local):
     ms_per_step = sum_ms / K
     value = world * cfg.B * K / (sum_ms / 1e3)
 
-    # ---- algorithmic bytes (codes of every cached key + selected K/V rows + q in / out)
+    # ---- algorithmic bytes (codes of every cached key -- or of every complete
+    # block -- + selected K/V rows + q in / out)
     lens_mid = n_before.double() + 1 + (K - 1) / 2.0  # mean cache length over the timed steps
-    code_bytes = float(lens_mid.sum()) * cfg.Hkv * cfg.bits / 8
+    scanned = lens_mid / cfg.block if cfg.block else lens_mid  # codes the scan reads per sequence
+    code_bytes = float(scanned.sum()) * cfg.Hkv * cfg.bits / 8
     sel_rows = float(buf["sel_cnt"].sum())
     kv_bytes = sel_rows * 2 * cfg.d * 2
     qo_bytes = cfg.B * cfg.Hq * cfg.d * (2 + 4)
@@ -423,9 +467,7 @@ def run_dashkv(args, cfg, world, rank, local):
         torch.cuda.synchronize(dev)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            eng.append_keys(cache, dkn, dvn, seq)
-            eng.select(cache, dq, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
-            eng.sparse_decode(cache, dq, buf["sel_idx"], buf["sel_cnt"], out_v, lse_v, ws, seq_lens=seq)
+            step(dq, dkn, dvn, out_v, lse_v)
         g.replay()  # upload the graph (one more appended token; the capacity covers it)
         torch.cuda.synchronize(dev)
         eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(E)]
@@ -445,8 +487,8 @@ def run_dashkv(args, cfg, world, rank, local):
         e2e = {"value": world * cfg.B * E / (e_ms / 1e3), "unit": "queries/s",
                "h2d_bytes_per_step": hin[0].numel() * hin.element_size(),
                "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": E,
-               "how": "per step: one pinned H2D copy of (q | k_new | v_new), a CUDA graph of the append, "
-                      "select and decode calls, one D2H copy of (out | lse); L2 flushed before each step"}
+               "how": "per step: one pinned H2D copy of (q | k_new | v_new), a CUDA graph of the step's calls "
+                      f"({', '.join(n for n, _ in calls)}), one D2H copy of (out | lse); L2 flushed before each step"}
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_steps > 0:
@@ -462,7 +504,7 @@ def run_dashkv(args, cfg, world, rank, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
                        "bits": cfg.bits, "topk": cfg.topk, "sink": cfg.sink, "window": cfg.window,
-                       "layout": "paged" if w.paged else "dense", "l2": "flushed before every step: 2 x L2 write, then 2 x L2 clean read (no pending write-backs)",
+                       "block": cfg.block or None, "layout": "paged" if w.paged else "dense", "l2": "flushed before every step: 2 x L2 write, then 2 x L2 clean read (no pending write-backs)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": score_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": score_gbs / peaks["hbm_gbs"],
@@ -477,10 +519,10 @@ def run_dashkv(args, cfg, world, rank, local):
             "per_head_queries_per_s": value * cfg.Hq,
             "warm_ms_per_step": warm_ms,
             "encode": encode,
-            "codes_scanned_per_s": float(lens_mid.sum()) * cfg.Hkv / (ms_per_step * 1e-3),
+            "codes_scanned_per_s": float(scanned.sum()) * cfg.Hkv / (ms_per_step * 1e-3),
             "selected_kv_bytes_per_s": kv_bytes / (ms_per_step * 1e-3),
-            "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": (2 + n_sel_kernels) * K, "clocks": clk,
-            "timing": "one CUDA graph per step (append, select, decode; programmatic dependent launches); events around each replay; kernels_ms from separately traced replays",
+            "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": len(kernels) * K, "clocks": clk,
+            "timing": f"one CUDA graph per step ({', '.join(n for n, _ in calls)}; programmatic dependent launches); events around each replay; kernels_ms from separately traced replays",
             "wall_s_timed_region": wall,
         }
         print(json.dumps(line), flush=True)

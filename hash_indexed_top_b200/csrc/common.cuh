@@ -84,6 +84,7 @@ struct KV {
     int32_t Hkv;
     int32_t d;
     int32_t W;                 // 64-bit code words per key
+    int32_t len_shift;         // entries per sequence = seq_lens[b] >> len_shift (block summaries: log2 m)
 
     __host__ __device__ int64_t capacity() const {
         return page_size ? (int64_t)max_pages * page_size : n_cap;
@@ -114,9 +115,10 @@ struct KV {
     }
 };
 
-// Sequence length clamped to the capacity (error word set when it exceeds it).
+// Entries of sequence b (tokens, or complete blocks of a block-summary view)
+// clamped to the capacity (error word set when they exceed it).
 __device__ __forceinline__ int64_t clamp_len(const KV &kv, const int32_t *seq_lens, int b) {
-    int64_t n = __ldg(seq_lens + b);
+    int64_t n = __ldg(seq_lens + b) >> kv.len_shift;
     int64_t cap = kv.capacity();
     if (n > cap) {
         raise_error(kErrCapacity);

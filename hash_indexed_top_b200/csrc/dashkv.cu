@@ -1,6 +1,7 @@
 // dashkv.cu -- the C ABI declared in include/dashkv.h: host-side validation,
 // context, workspace carving and kernel launches.  Every stage of the decode
-// step runs in the kernels of encode.cuh, select.cuh and decode.cuh; this file
+// step runs in the kernels of encode.cuh, select.cuh, decode.cuh and
+// blocks.cuh; this file
 // only checks arguments and enqueues them.  The library allocates no device
 // memory: the caller passes every buffer, including the workspace.
 #include <math.h>
@@ -11,6 +12,7 @@
 #include <type_traits>
 
 #include "../../include/dashkv.h"
+#include "blocks.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "encode.cuh"
@@ -114,6 +116,44 @@ KV make_kv(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
     o.Hkv = ctx->cfg.num_kv_heads;
     o.d = ctx->cfg.head_dim;
     o.W = ctx->cfg.bits >= 64 ? ctx->cfg.bits / 64 : 1;
+    o.len_shift = 0;
+    return o;
+}
+
+// log2 of a power of two in [1, 1024], else -1.
+int block_shift(int32_t m) {
+    for (int s = 0; s <= 10; ++s)
+        if (m == (1 << s)) return s;
+    return -1;
+}
+
+// Block summaries: the codes and block size are valid, and the block capacity
+// lies in [1, token capacity] (so the selection workspace laid out for the
+// token capacity also serves the block selection).
+dashkv_status check_blocks(const dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk) {
+    if (!blk || !blk->codes || block_shift(blk->block) < 0 || blk->reserved) return DASHKV_ERR_INVALID_ARG;
+    if (!aligned(blk->codes, ctx->cfg.bits == 128 ? 16 : 8)) return DASHKV_ERR_INVALID_ARG;
+    const int64_t cap = ctx->cfg.page_size ? (int64_t)kv->max_pages * ctx->cfg.page_size : kv->n_cap;
+    if (blk->nb_cap < 1 || blk->nb_cap > cap) return DASHKV_ERR_INVALID_ARG;
+    return DASHKV_OK;
+}
+
+// The block codes as a dense cache of N >> log2(m) entries per sequence (no
+// keys or values behind it).
+KV make_blk(const dashkv_ctx *ctx, const dashkv_block_view *blk) {
+    KV o;
+    o.k = nullptr;
+    o.v = nullptr;
+    o.codes = blk->codes;
+    o.n_cap = blk->nb_cap;
+    o.page_table = nullptr;
+    o.max_pages = 0;
+    o.num_pages = 0;
+    o.page_size = 0;
+    o.Hkv = ctx->cfg.num_kv_heads;
+    o.d = ctx->cfg.head_dim;
+    o.W = ctx->cfg.bits >= 64 ? ctx->cfg.bits / 64 : 1;
+    o.len_shift = block_shift(blk->block);
     return o;
 }
 
@@ -121,9 +161,9 @@ int64_t view_capacity(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
     return ctx->cfg.page_size ? (int64_t)kv->max_pages * ctx->cfg.page_size : kv->n_cap;
 }
 
-// ---- workspace: [scores | cand | ckey | hist | state | arrive(3 x BH lines) | seg_cnt | partials]
+// ---- workspace: [scores | cand | ckey | hist | state | arrive(3 x BH lines) | seg_cnt | partials | block ids]
 struct WsLayout {
-    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, total;
+    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, blk, total;
 };
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -145,6 +185,7 @@ WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
     L.arrive = o;  o = align_up(o + 3 * BH * kSyncStride * 4);
     L.seg_cnt = o; o = align_up(o + BH * kMaxSelCtas * 4);
     L.part = o;    o = align_up(o + BH * kMaxSplits * G * (c.head_dim + 2) * 4);
+    L.blk = o;     o = align_up(o + BH * ((size_t)c.topk + 1) * 4);  // selected block ids + counts
     L.total = o;
     return L;
 }
@@ -210,6 +251,8 @@ bool score_layout_ok() {
 template <int BITS, int D>
 void set_attrs_bd() {
     cudaFuncSetAttribute(encode_keys_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)EncodeShape<BITS, D>::SMEM);
+    cudaFuncSetAttribute(encode_blocks_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)EncodeShape<BITS, D>::SMEM);
     cudaFuncSetAttribute(score_hist_kernel<BITS, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)ScoreShape<BITS>::SMEM);
@@ -293,14 +336,21 @@ void launch_append_d(const dashkv_ctx *ctx, const KV &kv, const void *kn, const 
     }
 }
 
+// What one selection takes: k (top-k), S sinks, W window, the row length of
+// sel_idx.  The token selection uses the context's values; the block selection
+// takes k blocks and no sinks or window.
+struct SelArgs {
+    int topk, sink, window, cap_sel;
+};
+
 template <int BITS, int D>
 void launch_score_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
-                     int nctas, cudaStream_t st) {
+                     int nctas, int topk, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
     auto kern = kv.page_size ? score_hist_kernel<BITS, D, true> : score_hist_kernel<BITS, D, false>;
     launch_pdl(kern, dim3(nctas, BH), dim3(kScoreThreads), ScoreShape<BITS>::SMEM, st, kv,
-               static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, ctx->cfg.topk, nctas);
+               static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R, ws, topk, nctas);
 }
 
 // Fused selection whenever cluster launches are available (and not disabled).
@@ -354,10 +404,9 @@ int pick_cluster(const dashkv_ctx *ctx) {
 // per (b, h)) that may also start early behind the preceding kernel.
 template <int BITS, int D>
 void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
-                     int nctas, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
+                     int nctas, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
-    const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     auto kern = kv.page_size ? select_fused_kernel<BITS, D, true> : select_fused_kernel<BITS, D, false>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nctas, BH);
@@ -374,26 +423,26 @@ void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     cudaLaunchKernelEx(&cfg, kern, kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R,
-                       ws, ctx->cfg.topk, ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
+                       ws, a.topk, a.sink, a.window, a.cap_sel, sel_idx, sel_cnt);
 }
 
 template <int D>
 void launch_fused_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
-                    int nctas, int32_t *si, int32_t *sc, cudaStream_t st) {
+                    int nctas, const SelArgs &a, int32_t *si, int32_t *sc, cudaStream_t st) {
     switch (ctx->cfg.bits) {
-        case 32: launch_fused_bd<32, D>(ctx, kv, q, seq, ws, nctas, si, sc, st); break;
-        case 64: launch_fused_bd<64, D>(ctx, kv, q, seq, ws, nctas, si, sc, st); break;
-        default: launch_fused_bd<128, D>(ctx, kv, q, seq, ws, nctas, si, sc, st); break;
+        case 32: launch_fused_bd<32, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
+        case 64: launch_fused_bd<64, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
+        default: launch_fused_bd<128, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
     }
 }
 
 template <int D>
 void launch_score_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
-                    int nctas, cudaStream_t st) {
+                    int nctas, int topk, cudaStream_t st) {
     switch (ctx->cfg.bits) {
-        case 32: launch_score_bd<32, D>(ctx, kv, q, seq, ws, nctas, st); break;
-        case 64: launch_score_bd<64, D>(ctx, kv, q, seq, ws, nctas, st); break;
-        default: launch_score_bd<128, D>(ctx, kv, q, seq, ws, nctas, st); break;
+        case 32: launch_score_bd<32, D>(ctx, kv, q, seq, ws, nctas, topk, st); break;
+        case 64: launch_score_bd<64, D>(ctx, kv, q, seq, ws, nctas, topk, st); break;
+        default: launch_score_bd<128, D>(ctx, kv, q, seq, ws, nctas, topk, st); break;
     }
 }
 
@@ -433,6 +482,87 @@ void launch_decode_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
     }
 }
 
+
+// One selection over `k` (the token cache, or the block codes): the fused
+// kernel, or score + collect; then the optional copy of the scores (rows of
+// length cap).  The workspace is carved as L lays it out.
+void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout &L, char *w, const void *q,
+                const int32_t *seq_lens, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
+                Tracer &tr, cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    SelWS ws;
+    ws.scores = reinterpret_cast<float *>(w + L.scores);
+    ws.ld = row_ld(cap);
+    ws.scores_out = scores;
+    ws.ld_out = cap;
+    ws.cand = reinterpret_cast<int32_t *>(w + L.cand);
+    ws.ckey = reinterpret_cast<uint32_t *>(w + L.ckey);
+    ws.hist = reinterpret_cast<uint32_t *>(w + L.hist);
+    ws.state = reinterpret_cast<SelState *>(w + L.state);
+    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive);
+    ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
+    const int nscore = sel_ctas(ctx, cap, 1);    // score kernel: one 1024-thread CTA per SM
+    const int ncollect = sel_ctas(ctx, cap, 2);  // collect kernel: two 512-thread CTAs per SM
+    auto copy_scores = [&]() {
+        if (!scores) return;
+        const int gx = (int)((cap + 255) / 256 < 64 ? (cap + 255) / 256 : 64);
+        launch_pdl(copy_scores_kernel, dim3(gx > 0 ? gx : 1, BH), dim3(256), 0, st,
+                   (const float *)ws.scores, ws.ld, scores, ws.ld_out, seq_lens, ctx->cfg.num_kv_heads, cap,
+                   (int)k.len_shift);
+    };
+    if (use_fused(ctx)) {
+        const int nc = fused_cluster(ctx, cap);
+        tr.before();
+        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nc, a, sel_idx, sel_cnt, st);
+        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nc, a, sel_idx, sel_cnt, st);
+        tr.after();
+        copy_scores();
+        return;
+    }
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_score_d<64>(ctx, k, q, seq_lens, ws, nscore, a.topk, st);
+    else launch_score_d<128>(ctx, k, q, seq_lens, ws, nscore, a.topk, st);
+    tr.after();
+    tr.before();
+    launch_pdl(collect_kernel, dim3(ncollect, BH), dim3(kSelThreads), sizeof(CollectSmem), st, ws, ncollect, a.sink,
+               a.window, a.cap_sel, sel_idx, sel_cnt);
+    tr.after();
+    copy_scores();
+}
+
+// ---- block summaries
+template <int BITS, int D>
+void launch_encode_blocks_bd(const dashkv_ctx *ctx, const KV &kv, const KV &blk, const int32_t *seq_lens,
+                             cudaStream_t st) {
+    using S = EncodeShape<BITS, D>;
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int64_t tiles = ceil_div(blk.n_cap, S::KT);
+    int64_t gx = ceil_div(8 * ctx->sm_count, BH);
+    if (gx > tiles) gx = tiles;
+    if (gx < 1) gx = 1;
+    encode_blocks_kernel<BITS, D><<<dim3((unsigned)gx, BH), S::THREADS, S::SMEM, st>>>(kv, blk, seq_lens, ctx->R,
+                                                                                      tiles);
+}
+
+template <int BITS, int D>
+void launch_append_blocks_bd(const dashkv_ctx *ctx, const KV &kv, const KV &blk, const int32_t *seq_lens,
+                             cudaStream_t st) {
+    const int Hkv = ctx->cfg.num_kv_heads;
+    const int C = (Hkv * BITS + 1023) / 1024;  // CTAs per sequence
+    const int hpc = (Hkv + C - 1) / C;         // heads per CTA: hpc * BITS <= 1024
+    launch_pdl(append_blocks_kernel<BITS, D>, dim3(C, ctx->cfg.batch), dim3(hpc * BITS),
+               (size_t)hpc * (D * 4 + BITS / 8), st, kv, blk, seq_lens, ctx->R, hpc);
+}
+
+template <int D>
+void launch_blocks_d(const dashkv_ctx *ctx, bool whole, const KV &kv, const KV &blk, const int32_t *s,
+                     cudaStream_t st) {
+    switch (ctx->cfg.bits) {
+        case 32: whole ? launch_encode_blocks_bd<32, D>(ctx, kv, blk, s, st) : launch_append_blocks_bd<32, D>(ctx, kv, blk, s, st); break;
+        case 64: whole ? launch_encode_blocks_bd<64, D>(ctx, kv, blk, s, st) : launch_append_blocks_bd<64, D>(ctx, kv, blk, s, st); break;
+        default: whole ? launch_encode_blocks_bd<128, D>(ctx, kv, blk, s, st) : launch_append_blocks_bd<128, D>(ctx, kv, blk, s, st); break;
+    }
+}
 }  // namespace
 
 // ---------------------------------------------------------------------------- static scratch
@@ -581,49 +711,12 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     const int64_t cap = view_capacity(ctx, kv);
     const WsLayout L = ws_layout(ctx->cfg, cap);
     if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
-    char *w = static_cast<char *>(workspace);
-    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
-    SelWS ws;
-    ws.scores = reinterpret_cast<float *>(w + L.scores);
-    ws.ld = row_ld(cap);
-    ws.scores_out = scores;
-    ws.ld_out = cap;
-    ws.cand = reinterpret_cast<int32_t *>(w + L.cand);
-    ws.ckey = reinterpret_cast<uint32_t *>(w + L.ckey);
-    ws.hist = reinterpret_cast<uint32_t *>(w + L.hist);
-    ws.state = reinterpret_cast<SelState *>(w + L.state);
-    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive);
-    ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
-    const KV k = make_kv(ctx, kv);
+    const SelArgs a{ctx->cfg.topk, ctx->cfg.sink, ctx->cfg.window,
+                    ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int nscore = sel_ctas(ctx, cap, 1);    // score kernel: one 1024-thread CTA per SM
-    const int ncollect = sel_ctas(ctx, cap, 2);  // collect kernel: two 512-thread CTAs per SM
     Tracer tr(ctx, st);
-    auto copy_scores = [&]() {
-        if (!scores) return;
-        const int gx = (int)((cap + 255) / 256 < 64 ? (cap + 255) / 256 : 64);
-        launch_pdl(copy_scores_kernel, dim3(gx > 0 ? gx : 1, BH), dim3(256), 0, st,
-                   (const float *)ws.scores, ws.ld, scores, ws.ld_out, seq_lens, ctx->cfg.num_kv_heads, cap);
-    };
-    if (use_fused(ctx)) {
-        const int nc = fused_cluster(ctx, cap);
-        tr.before();
-        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nc, sel_idx, sel_cnt, st);
-        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nc, sel_idx, sel_cnt, st);
-        tr.after();
-        copy_scores();
-        return launch_status();
-    }
-    tr.before();
-    if (ctx->cfg.head_dim == 64) launch_score_d<64>(ctx, k, q, seq_lens, ws, nscore, st);
-    else launch_score_d<128>(ctx, k, q, seq_lens, ws, nscore, st);
-    tr.after();
-    const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
-    tr.before();
-    launch_pdl(collect_kernel, dim3(ncollect, BH), dim3(kSelThreads), sizeof(CollectSmem), st, ws, ncollect,
-               ctx->cfg.sink, ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
-    tr.after();
-    copy_scores();
+    run_select(ctx, make_kv(ctx, kv), cap, L, static_cast<char *>(workspace), q, seq_lens, a, sel_idx, sel_cnt,
+               scores, tr, st);
     return launch_status();
 }
 
@@ -663,6 +756,69 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
     const int64_t cap = view_capacity(ctx, kv);
     if (ctx->cfg.head_dim == 64) launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
     else launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_encode_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk,
+                                   const int32_t *seq_lens, void *stream) {
+    if (!ctx || !seq_lens) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, false);
+    if (s == DASHKV_OK) s = check_blocks(ctx, kv, blk);
+    if (s != DASHKV_OK) return s;
+    const KV k = make_kv(ctx, kv), b = make_blk(ctx, blk);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_blocks_d<64>(ctx, true, k, b, seq_lens, st);
+    else launch_blocks_d<128>(ctx, true, k, b, seq_lens, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_append_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk,
+                                   const int32_t *seq_lens, void *stream) {
+    if (!ctx || !seq_lens) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, false);
+    if (s == DASHKV_OK) s = check_blocks(ctx, kv, blk);
+    if (s != DASHKV_OK) return s;
+    const KV k = make_kv(ctx, kv), b = make_blk(ctx, blk);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_blocks_d<64>(ctx, false, k, b, seq_lens, st);
+    else launch_blocks_d<128>(ctx, false, k, b, seq_lens, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_select_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk,
+                                   const void *q, const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
+                                   float *block_scores, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!ctx || !q || !seq_lens || !sel_idx || !sel_cnt || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, false, false);
+    if (s == DASHKV_OK) s = check_blocks(ctx, kv, blk);
+    if (s != DASHKV_OK) return s;
+    const int shift = block_shift(blk->block);
+    const int kb = ctx->cfg.topk >> shift;  // blocks whose tokens fill the top-k budget
+    if (kb < 1 || ctx->cfg.window < blk->block - 1) return DASHKV_ERR_UNSUPPORTED;
+    const int64_t cap = view_capacity(ctx, kv);
+    const WsLayout L = ws_layout(ctx->cfg, cap);
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
+    char *w = static_cast<char *>(workspace);
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    int32_t *blk_idx = reinterpret_cast<int32_t *>(w + L.blk);
+    int32_t *blk_cnt = blk_idx + (size_t)BH * kb;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    // top kb blocks by the score of their summary codes (no sinks, no window)
+    run_select(ctx, make_blk(ctx, blk), blk->nb_cap, L, w, q, seq_lens, SelArgs{kb, 0, 0, kb}, blk_idx, blk_cnt,
+               block_scores, tr, st);
+    const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
+    tr.before();
+    launch_pdl(expand_blocks_kernel, dim3(BH), dim3(kExpandThreads), 0, st, (const int32_t *)blk_idx,
+               (const int32_t *)blk_cnt, kb, seq_lens, cap, ctx->cfg.num_kv_heads, shift, ctx->cfg.sink,
+               ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
     tr.after();
     return launch_status();
 }

@@ -387,12 +387,13 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     return o;
 }
 
-// Optional user copy of the scores: entries [0, seq_lens[b]) of every row.
+// Optional user copy of the scores: entries [0, seq_lens[b] >> len_shift) of
+// every row.
 __global__ void copy_scores_kernel(const float *__restrict__ src, int64_t ld, float *__restrict__ dst, int64_t ld_out,
-                                   const int32_t *__restrict__ seq_lens, int Hkv, int64_t cap) {
+                                   const int32_t *__restrict__ seq_lens, int Hkv, int64_t cap, int len_shift) {
     griddep_wait();
     const int bh = blockIdx.y;
-    int64_t n = seq_lens[bh / Hkv];
+    int64_t n = seq_lens[bh / Hkv] >> len_shift;
     if (n > cap) n = cap;
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x)
         dst[(int64_t)bh * ld_out + t] = src[(int64_t)bh * ld + t];

@@ -27,7 +27,7 @@ FLAG_TWO_KERNEL_SELECT = 1
 SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_encode_keys",
            "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
            "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str",
-           "dashkv_select_static")
+           "dashkv_select_static", "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks")
 
 
 class DashKVError(RuntimeError):
@@ -47,6 +47,11 @@ class KVView(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("n_cap", ctypes.c_int64), ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32)]
+
+
+class BlockView(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("nb_cap", ctypes.c_int64), ("block", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 _lib = None
@@ -71,6 +76,10 @@ def lib() -> ctypes.CDLL:
         L.dashkv_select.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
         L.dashkv_sparse_decode.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, P, SZ, P]
         L.dashkv_select_static.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P]
+        L.dashkv_encode_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P]
+        L.dashkv_append_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P]
+        L.dashkv_select_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P, P, P, P, P,
+                                           SZ, P]
         L.dashkv_get_error.argtypes = [P]
         L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
         L.dashkv_set_trace.argtypes = [P, P, I32]
@@ -79,7 +88,8 @@ def lib() -> ctypes.CDLL:
         L.dashkv_status_str.argtypes = [ctypes.c_int]
         L.dashkv_status_str.restype = ctypes.c_char_p
         for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode",
-                  "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_static"):
+                  "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_static",
+                  "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -166,6 +176,30 @@ class KVCache:
         return torch.zeros((B, Hkv, n_cap, W), dtype=torch.int64, device=k.device)
 
 
+@dataclasses.dataclass
+class BlockIndex:
+    """Summary codes of the complete blocks of `block` tokens of a cache:
+    codes [B, Hkv, nb_cap, W] int64 on the device (block i at index i, stored
+    like token codes; canonical_codes() undoes the rotation)."""
+    codes: torch.Tensor
+    block: int
+
+    @property
+    def capacity(self) -> int:
+        return int(self.codes.shape[2])
+
+    def view(self) -> BlockView:
+        return BlockView(self.codes.data_ptr(), self.capacity, int(self.block), 0)
+
+    @staticmethod
+    def empty_for(cache: KVCache, batch: int, bits: int, block: int) -> "BlockIndex":
+        """Zeroed codes for every complete block the cache can hold."""
+        Hkv = int(cache.k.shape[2] if cache.paged else cache.k.shape[1])
+        nb_cap = max(1, cache.capacity // int(block))
+        W = max(1, bits // 64)
+        return BlockIndex(torch.zeros((batch, Hkv, nb_cap, W), dtype=torch.int64, device=cache.k.device), int(block))
+
+
 class DashKV:
     """One problem configuration (shapes, bits, k, S, W, layout, seed)."""
 
@@ -249,6 +283,29 @@ class DashKV:
                                                                   _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt),
                                                                   _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                                                   _stream(stream)))
+
+    # ---- block summaries (CSA-style two-level index)
+    def encode_blocks(self, cache: KVCache, index: BlockIndex, seq_lens: torch.Tensor, stream=None) -> None:
+        v, bv = cache.view(), index.view()
+        _check("dashkv_encode_blocks", lib().dashkv_encode_blocks(self._ctx, ctypes.byref(v), ctypes.byref(bv),
+                                                                  _ptr(seq_lens), _stream(stream)))
+
+    def append_blocks(self, cache: KVCache, index: BlockIndex, seq_lens: torch.Tensor, stream=None) -> None:
+        """After append_keys: encode the block the append completed, if any."""
+        v, bv = cache.view(), index.view()
+        _check("dashkv_append_blocks", lib().dashkv_append_blocks(self._ctx, ctypes.byref(v), ctypes.byref(bv),
+                                                                  _ptr(seq_lens), _stream(stream)))
+
+    def select_blocks(self, cache: KVCache, index: BlockIndex, q: torch.Tensor, seq_lens: torch.Tensor,
+                      sel_idx: torch.Tensor, sel_cnt: torch.Tensor, block_scores: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+        """Top topk // block blocks by summary score, as a token list in select()'s format."""
+        ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
+        v, bv = cache.view(), index.view()
+        _check("dashkv_select_blocks", lib().dashkv_select_blocks(self._ctx, ctypes.byref(v), ctypes.byref(bv),
+                                                                  _ptr(q), _ptr(seq_lens), _ptr(sel_idx),
+                                                                  _ptr(sel_cnt), _ptr(block_scores), _ptr(ws),
+                                                                  ws.numel(), _stream(stream)))
 
     def select_kernels(self, max_tokens: int) -> int:
         """1 when dashkv_select runs the fused kernel for this cache size, 2 for score + collect."""

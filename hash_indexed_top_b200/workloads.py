@@ -51,6 +51,7 @@ class Config:
     page_size: int = 0     # 0 = dense layout
     n_min: int = 0         # ragged: lower bound of the length draw (0 = fixed N)
     seed: int = 1234
+    block: int = 0         # > 0: select through summaries of blocks of this many tokens
 
     @property
     def G(self) -> int:
@@ -76,6 +77,11 @@ CONFIGS = {
     "c1m": Config("c1m", B=1, Hq=64, Hkv=8, d=128, N=1048576, bits=128, topk=4096, sink=4, window=1024,
                   steps=16, needles=64, seed=1238),
 }
+# the same workloads selected through block summaries of 4 tokens (the
+# compression ratio of the DeepSeek DSA->CSA/HCA page's CSA example): the
+# top topk / 4 blocks give the same top-k token budget
+CONFIGS["c128k_blocks4"] = CONFIGS["c128k"].scaled(name="c128k_blocks4", block=4)
+CONFIGS["c1m_blocks4"] = CONFIGS["c1m"].scaled(name="c1m_blocks4", block=4)
 
 
 def grid(x: torch.Tensor) -> torch.Tensor:

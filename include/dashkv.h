@@ -195,6 +195,59 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    const int32_t *sel_cnt, float *out, float *lse, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Block summaries: a CSA-style two-level index.
+ *
+ * DeepSeek DSA->CSA/HCA page, section CSA: every m history tokens are
+ * compressed into one summary entry and the top-k is taken over the
+ * summaries, while a sliding window keeps the recent tokens exact; section on
+ * the compressed KV cache versus the state cache: the tokens of a block that
+ * is not yet complete wait in the state cache until m have arrived.
+ *
+ * Without the pages' learned compressor, the summary of block i (tokens
+ * [i m, (i + 1) m) of a sequence) is the code of the block's summed key,
+ * bit_j = [ sum_i R[j][i] (sum_t k_t)[i] >= 0 ], stored like a token code.
+ * Only complete blocks, i < seq_lens[b] / m, have one.  Selection scores the
+ * summaries with the query exactly as dashkv_select scores keys, takes the
+ * top kb = topk / m blocks (ties to the lower block), and lists every token of
+ * those blocks united with the sinks and the window; the window must cover
+ * the incomplete tail (window >= m - 1).  dashkv_sparse_decode then attends
+ * exactly over that list.  The scan reads one code per m tokens.
+ * ------------------------------------------------------------------------ */
+typedef struct dashkv_block_view {
+    uint64_t *codes;   /* device u64 [B][Hkv][nb_cap][W]: summary of block i at
+                          index i, stored (rotated by i mod T) like token codes */
+    int64_t nb_cap;    /* blocks per (b, kv head); 1 <= nb_cap <= token capacity */
+    int32_t block;     /* m, tokens per block: a power of two in [1, 1024]      */
+    int32_t reserved;  /* must be 0                                              */
+} dashkv_block_view;
+
+/* Summaries of every complete block [0, seq_lens[b] / m) of every (b, kv
+ * head) from kv->k (dense or paged), written to blk->codes.  Blocks beyond
+ * nb_cap set the capacity error word and are skipped. */
+dashkv_status dashkv_encode_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk,
+                                   const int32_t *seq_lens, void *stream);
+
+/* Decode-step update, to be called after dashkv_append_keys with the lengths
+ * it incremented: for every sequence whose length is now a multiple of m, the
+ * summary of the block that the append completed (seq_lens[b] / m - 1) is
+ * encoded from kv->k.  Other sequences are left alone (their new token waits
+ * in the tail).  Idempotent. */
+dashkv_status dashkv_append_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk,
+                                   const int32_t *seq_lens, void *stream);
+
+/* Stages 2 and 3 over the summaries.  Writes sel_idx / sel_cnt exactly as
+ * dashkv_select does (ascending, duplicate-free, rows of topk + sink + window,
+ * -1 after the count; sinks first, window last), for the token set
+ *   { tokens of the top topk / m complete blocks } U [0, S) U [N - W, N).
+ * block_scores (optional): device fp32 [B][Hkv][nb_cap] receives the summary
+ * scores of blocks i < seq_lens[b] / m.  Requires topk >= m and window >= m-1
+ * (else DASHKV_ERR_UNSUPPORTED).  The workspace is dashkv_select's (same size
+ * for the token capacity); reads blk->codes, kv only for its capacity. */
+dashkv_status dashkv_select_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_block_view *blk,
+                                   const void *q, const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
+                                   float *block_scores, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Synchronise `stream`, then read and clear the current device's error
  * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, or DASHKV_ERR_CUDA
  * when the stream reports an error. */

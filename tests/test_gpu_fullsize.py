@@ -87,3 +87,62 @@ def test_full_size_step_on_sampled_pairs(name):
             assert within_tol(lse, r["lse"][0]).all(), f"{name} ({b},{h}): lse err {np.abs(lse - r['lse'][0]).max()}"
     finally:
         eng.close()
+
+
+BLOCK_FULL = ["c128k_blocks4", "c1m_blocks4"]
+
+
+@pytest.mark.parametrize("name", BLOCK_FULL)
+def test_full_size_block_step_on_sampled_pairs(name):
+    # one step through block summaries as the benchmark runs it (append,
+    # summary update, block selection, decode given the lengths); the oracle
+    # encodes the pair's summaries from its keys
+    cfg = W.CONFIGS[name]
+    m = cfg.block
+    dev = torch.device("cuda")
+    w = W.make_workload(cfg, device=dev, steps=1)
+    eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
+                    cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED)
+    try:
+        cache = dk.KVCache(w.K, w.V, dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged), w.page_table)
+        seq = w.seq_lens.clone()
+        eng.encode_keys(cache, seq)
+        index = dk.BlockIndex.empty_for(cache, cfg.B, cfg.bits, m)
+        eng.encode_blocks(cache, index, seq)
+        eng.append_keys(cache, w.k_new[0], w.v_new[0], seq)
+        eng.append_blocks(cache, index, seq)
+        buf = eng.alloc_step(dev)
+        bsc = torch.full((cfg.B, cfg.Hkv, index.capacity), float("nan"), device=dev)
+        ws = eng.workspace(cache.capacity, dev)
+        eng.select_blocks(cache, index, w.q[0], seq, buf["sel_idx"], buf["sel_cnt"], bsc, ws)
+        eng.sparse_decode(cache, w.q[0], buf["sel_idx"], buf["sel_cnt"], buf["out"], buf["lse"], ws, seq_lens=seq)
+        torch.cuda.synchronize()
+        assert eng.get_error() == 0
+        gcodes = dk.canonical_codes(index.codes, cfg.bits)
+        R = O.hyperplanes(W.HYPERPLANE_SEED, cfg.bits, cfg.d)
+        G = cfg.G
+        for b, h in [(0, 0), (cfg.B - 1, cfg.Hkv - 1)]:
+            n = int(seq[b])
+            nb = n // m
+            K = _pair_rows(w.K, w, b, h, n).double().cpu().numpy().reshape(1, 1, n, cfg.d)
+            V = _pair_rows(w.V, w, b, h, n).double().cpu().numpy().reshape(1, 1, n, cfg.d)
+            L = O.Layout(1, 1, cfg.d, cfg.bits, n_cap=n)
+            sl = np.array([n], dtype=np.int32)
+            oc = O.encode_blocks(L, K, sl, m, R, nb_cap=max(1, nb))
+            gc = gcodes[b, h, :nb].cpu().numpy().view(np.uint64)
+            assert np.array_equal(gc, oc[0, 0, :nb]), f"{name} ({b},{h}): summaries differ"
+            q = w.q[0][b, h * G:(h + 1) * G].double().cpu().numpy().reshape(1, G, cfg.d)
+            r = O.decode_step_blocks(L, G, q, K, V, oc, sl, R, m, cfg.topk // m, cfg.sink, cfg.window,
+                                     cap=cfg.sel_cap)
+            gs = bsc[b, h, :nb].cpu().numpy()
+            es = r["block_scores"][0, 0, :nb].astype(np.float32)
+            assert np.array_equal(gs.view(np.uint32), es.view(np.uint32)), f"{name} ({b},{h}): block scores differ"
+            assert int(buf["sel_cnt"][b, h]) == int(r["sel_cnt"][0, 0])
+            assert np.array_equal(buf["sel_idx"][b, h].cpu().numpy(), r["sel_idx"][0, 0]), \
+                f"{name} ({b},{h}): selection differs"
+            out = buf["out"][b, h * G:(h + 1) * G].double().cpu().numpy()
+            lse = buf["lse"][b, h * G:(h + 1) * G].double().cpu().numpy()
+            assert within_tol(out, r["out"][0]).all(), f"{name} ({b},{h}): out err {np.abs(out - r['out'][0]).max()}"
+            assert within_tol(lse, r["lse"][0]).all(), f"{name} ({b},{h}): lse err {np.abs(lse - r['lse'][0]).max()}"
+    finally:
+        eng.close()
