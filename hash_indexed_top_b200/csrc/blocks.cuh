@@ -208,8 +208,11 @@ expand_blocks_kernel(const int32_t *__restrict__ blk_idx, const int32_t *__restr
                      const int32_t *__restrict__ seq_lens, int64_t cap_tokens, int Hkv, int len_shift, int S, int W,
                      int cap_sel, int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_cnt) {
     __shared__ int s_warp[32];
-    griddep_wait();  // the block selection is complete
+    // The decode may launch now: its window CTAs read only what the append
+    // wrote (complete before the selection, which this kernel follows, began),
+    // its other CTAs wait for this kernel to complete.
     griddep_trigger();
+    griddep_wait();  // the block selection is complete
     const int bh = blockIdx.x, b = bh / Hkv, tid = threadIdx.x;
     int64_t n = seq_lens[b];
     n = n < 0 ? 0 : (n > cap_tokens ? cap_tokens : n);

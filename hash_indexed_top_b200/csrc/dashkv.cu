@@ -228,7 +228,7 @@ int attn_splits(const dashkv_ctx *ctx) {
     int64_t n = (2 * ctx->sm_count) / BH;  // one wave of two CTAs per SM
     const int64_t by_rows = ceil_div(cap_sel, 64);
     if (n > by_rows) n = by_rows;
-    if (n > kMaxSplits - 1) n = kMaxSplits - 1;  // one slot stays for the window CTA
+    if (n > kMaxSplits - 1) n = kMaxSplits - 1;  // at least one slot stays for a window CTA
     return n < 1 ? 1 : (int)n;
 }
 
@@ -446,15 +446,23 @@ void launch_score_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const in
     }
 }
 
-// Window CTAs (one per (b, h), leading rows of the decode grid) when the
-// lengths are given and they fit on the SMs the fused selection leaves free
-// (two decode CTAs per SM), so that they run while it streams.
-int window_rows(const dashkv_ctx *ctx, int64_t cap, const int32_t *seq_lens, int splits) {
+// Window CTAs per (b, h) (leading rows of the decode grid) when the lengths
+// are given and at least one per (b, h) fits on the SMs the fused selection
+// leaves free (two decode CTAs per SM), so that they run while it streams: as
+// many as make a window CTA's share of the sinks + window about a top-k
+// split's, as long as all of them fit there.  0: no window CTAs.
+int window_ctas(const dashkv_ctx *ctx, int64_t cap, const int32_t *seq_lens, int splits) {
     if (!seq_lens || !use_fused(ctx)) return 0;
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int64_t sel_ctas = (int64_t)fused_cluster(ctx, cap) * BH;
-    if (sel_ctas >= ctx->sm_count || BH > 2 * (ctx->sm_count - sel_ctas)) return 0;
-    return (BH + splits - 1) / splits;
+    if (sel_ctas >= ctx->sm_count) return 0;
+    const int64_t slots = 2 * (ctx->sm_count - sel_ctas);
+    if (BH > slots) return 0;
+    const int64_t per_split = ceil_div(ctx->cfg.topk, splits);
+    int64_t nw = ceil_div((int64_t)ctx->cfg.sink + ctx->cfg.window, per_split);
+    if (nw > slots / BH) nw = slots / BH;
+    if (nw > kMaxSplits - splits) nw = kMaxSplits - splits;
+    return nw < 1 ? 1 : (int)nw;
 }
 
 template <int D, int G>
@@ -463,12 +471,13 @@ void launch_decode_dg(const dashkv_ctx *ctx, const KV &kv, const void *q, const 
                       cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int splits = attn_splits(ctx);
-    const int wy = window_rows(ctx, cap, seq_lens, splits);
+    const int nw = window_ctas(ctx, cap, seq_lens, splits);
+    const int wy = (BH * nw + splits - 1) / splits;  // grid rows of window CTAs
     const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     launch_pdl(sparse_decode_kernel<D, G>, dim3(splits, BH + wy), dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st,
                kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws,
-               splits, scale_log2, seq_lens, ctx->cfg.sink, ctx->cfg.window, ctx->cfg.topk, wy);
+               splits, scale_log2, seq_lens, ctx->cfg.sink, ctx->cfg.window, ctx->cfg.topk, wy, nw > 0 ? nw : 1);
 }
 
 template <int D>

@@ -20,7 +20,7 @@
 namespace dkv {
 
 constexpr int kAttnThreads = 256;
-constexpr int kMaxSplits = 256;  // partial slots per (b, h): top-k splits + the window CTA
+constexpr int kMaxSplits = 256;  // partial slots per (b, h): top-k splits + the window CTAs
 
 struct AttnWS {
     float *part;        // [BH][kMaxSplits][G][D + 2]  (acc[D], m, l)
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                      const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt, int cap_sel,
                      float *__restrict__ out, float *__restrict__ lse, AttnWS ws, int splits, float scale_log2,
-                     const int32_t *__restrict__ seq_lens, int n_sink, int n_window, int topk, int wy) {
+                     const int32_t *__restrict__ seq_lens, int n_sink, int n_window, int topk, int wy, int nw) {
     using S = DecodeShape<D, G>;
     constexpr int DPL = S::DPL, LPR = S::LPR, RPW = S::RPW, NST = S::NST, RT = S::RT;
     constexpr int TROWS = S::TROWS, CPR = S::CPR, NWARP = S::NWARP, STAGES = S::STAGES;
@@ -91,18 +91,20 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = lane / LPR, li = lane % LPR;
-    // Roles.  With wy > 0 the first wy rows of the grid hold one window CTA per
-    // (b, h): it attends over the sinks and the window, which every selection
-    // contains, straight from the token range, so it does not wait for the
-    // selection and runs while the scorer still streams (on the SMs the scorer
-    // leaves free).  The other CTAs take the top-k (middle) part of the list,
-    // split `splits` ways.  With wy = 0 they take the whole list.
+    // Roles.  With wy > 0 the first wy rows of the grid hold nw window CTAs per
+    // (b, h): between them they attend over the sinks and the window, which
+    // every selection contains, straight from the token range, so they do not
+    // wait for the selection and run while the scorer still streams (on the SMs
+    // the scorer leaves free).  The other CTAs take the top-k (middle) part of
+    // the list, split `splits` ways.  With wy = 0 they take the whole list.
     const int BH = (int)gridDim.y - wy;
     const bool win = (int)blockIdx.y < wy;
-    const int bh = win ? (int)(blockIdx.y * splits + blockIdx.x) : (int)blockIdx.y - wy;
+    const int wid = win ? (int)(blockIdx.y * splits + blockIdx.x) : 0;  // window CTA number
+    const int bh = win ? wid / nw : (int)blockIdx.y - wy;
     if (bh >= BH) return;  // spare window slots
-    const int split = win ? splits : (int)blockIdx.x;  // partial slot
-    const int nparts = splits + (wy > 0 ? 1 : 0);
+    const int piece = wid % nw;  // this window CTA's share of the sinks + window
+    const int split = win ? splits + piece : (int)blockIdx.x;  // partial slot
+    const int nparts = splits + (wy > 0 ? nw : 0);
     const int b = bh / kv.Hkv, h = bh % kv.Hkv;
     const int64_t cap_tokens = kv.capacity();
 
@@ -145,9 +147,11 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     const int nwin = (int)n - w_beg;
     const int cnt = win ? 0 : sel_cnt[bh];
     int r0, r1, rend;  // rows [r0, r1) of this CTA, valid below rend
-    if (win) {
-        r0 = 0;
-        r1 = rend = s_end + nwin;
+    if (win) {  // the pieces divide the capacity n_sink + n_window of this part
+        const int per = (n_sink + n_window + nw - 1) / nw;
+        r0 = piece * per;
+        r1 = r0 + per;
+        rend = s_end + nwin;
     } else if (wy > 0) {  // the middle: list positions [n_sink, n_sink + topk), valid below cnt - nwin
         const int per = (topk + splits - 1) / splits;
         r0 = n_sink + split * per;
