@@ -395,3 +395,68 @@ int dko_select_blocks(int B, int Hkv, int64_t nb_cap, const int32_t *seq_lens, i
         }
     return rc;
 }
+
+/* ---------------------------------------------------------- radius scaling */
+/*
+ * Radius-scaled scores (Spherical KV page, section 2.1 ADA: the compact key
+ * keeps a quantized radius r~ beside its angle code, and the logit is
+ * estimated as |q| * r~ * f_b(angle codes); f_b is played here by the
+ * asymmetric code score s_t, and |q| is one constant per query, so the
+ * ranking only needs s'_t = r~_t * s_t).
+ *
+ * The page does not fix the quantizer.  Reading used: 8 bits, uniform in the
+ * key norm with step 1/4 and midpoint reconstruction,
+ *   c_t  = min(255, floor(4 * sqrtf(sum_i k_i^2)))   sum in fp32, i ascending,
+ *   r~_t = (c_t + 1/2) / 4.
+ * Single precision is part of the definition, so that the integer c_t is
+ * decided the same way by any implementation (sqrtf is correctly rounded).
+ * On keys of the 1/64 grid the sum is exact.  s'_t is the fp32 product of
+ * r~_t and the fp32 score s_t (one rounding: the double product of the two
+ * is exact), returned widened to double.
+ *
+ * radius codes: dense [B][Hkv][n_cap], paged [P][Hkv][page] (the codes'
+ * layout without the word axis), uint8.
+ */
+static int64_t radius_index(const dko_layout *L, int b, int h, int64_t t) {
+    if (L->page == 0)
+        return ((int64_t)b * L->Hkv + h) * L->n_cap + t;
+    int64_t p = L->page_table[(int64_t)b * L->max_pages + t / L->page];
+    return (p * L->Hkv + h) * L->page + t % L->page;
+}
+
+uint8_t dko_radius_code(const double *k, int d) {
+    float s = 0.0f;
+    for (int i = 0; i < d; ++i) {
+        float x = (float)k[i];
+        s += x * x;
+    }
+    float c = floorf(4.0f * sqrtf(s));
+    return c >= 255.0f ? (uint8_t)255 : (uint8_t)c;
+}
+
+double dko_radius_value(uint8_t c) { return ((double)c + 0.5) / 4.0; }
+
+/* Radius codes of tokens [0, seq_lens[b]) of every (b, kv head). */
+void dko_radius_codes(int B, int Hkv, int d, int64_t n_cap, const int32_t *page_table, int max_pages, int page,
+                      const double *K, const int32_t *seq_lens, uint8_t *rc) {
+    dko_layout L = make_layout(B, Hkv, d, 64, n_cap, page_table, max_pages, page);
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h)
+            for (int64_t t = 0; t < seq_lens[b]; ++t)
+                rc[radius_index(&L, b, h, t)] = dko_radius_code(K + row_index(&L, b, h, t), d);
+}
+
+/* s'[b][h][t] = fp32(r~_t * s[b][h][t]) for t < seq_lens[b] (scores rows of
+ * length n_cap, as dko_scores writes them); other entries untouched. */
+void dko_radius_scale(int B, int Hkv, int64_t n_cap, const int32_t *page_table, int max_pages, int page,
+                      const int32_t *seq_lens, const uint8_t *rc, const double *scores, double *out) {
+    dko_layout L = make_layout(B, Hkv, 1, 64, n_cap, page_table, max_pages, page);
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h)
+            for (int64_t t = 0; t < seq_lens[b]; ++t) {
+                int64_t i = ((int64_t)b * Hkv + h) * n_cap + t;
+                float st = (float)scores[i];  /* the token path's fp32 score */
+                float prod = (float)(dko_radius_value(rc[radius_index(&L, b, h, t)]) * (double)st);
+                out[i] = (double)prod + 0.0;
+            }
+}

@@ -57,6 +57,12 @@ def lib():
         L.dko_encode_blocks.argtypes = [I, I, I, I, I64, P, I, I, P, P, I, P, I64, P]
         L.dko_select_blocks.argtypes = [I, I, I64, P, I, P, I, I, I, P, P, I]
         L.dko_select_blocks.restype = I
+        L.dko_radius_code.argtypes = [P, I]
+        L.dko_radius_code.restype = ctypes.c_uint8
+        L.dko_radius_value.argtypes = [ctypes.c_uint8]
+        L.dko_radius_value.restype = ctypes.c_double
+        L.dko_radius_codes.argtypes = [I, I, I, I64, P, I, I, P, P, P]
+        L.dko_radius_scale.argtypes = [I, I, I64, P, I, I, P, P, P, P]
         L.dko_set_threads.argtypes = [I]
         L.dko_get_threads.restype = I
         _lib = L
@@ -228,3 +234,51 @@ def decode_step_blocks(layout: Layout, Hq, q, K, V, block_codes, seq_lens, R, bl
     idx, cnt = select_blocks(bs, seq_lens, block, topk_blocks, sink, window, cap)
     out, lse = attend(layout, Hq, q, K, V, idx, cnt)
     return dict(block_scores=bs, bound=bound, sel_idx=idx, sel_cnt=cnt, out=out, lse=lse)
+
+
+# ---------------------------------------------------------------- radius scaling
+# Spherical KV page, section 2.1 ADA: a quantized key radius r~ beside the
+# angle code, logits estimated as |q| r~ f_b(codes).  Here s'_t = r~_t s_t (the
+# constant |q| does not change the ranking); 8-bit radius codes, step 1/4.
+
+def radius_code(k) -> int:
+    """c = min(255, floor(4 sqrtf(sum k_i^2))) (fp32 sum, i ascending)."""
+    k = _f64(k)
+    return int(lib().dko_radius_code(_p(k), int(k.shape[-1])))
+
+
+def radius_value(c: int) -> float:
+    """r~ = (c + 1/2) / 4."""
+    return float(lib().dko_radius_value(int(c)))
+
+
+def radius_codes(layout: Layout, K, seq_lens) -> np.ndarray:
+    """uint8 radius codes of tokens [0, seq_lens[b]): dense [B, Hkv, n_cap],
+    paged [P, Hkv, page] (zero elsewhere)."""
+    K = _f64(K)
+    if layout.page:
+        rc = np.zeros((K.shape[0], layout.Hkv, layout.page), dtype=np.uint8)
+    else:
+        rc = np.zeros((layout.B, layout.Hkv, layout.n_cap), dtype=np.uint8)
+    lib().dko_radius_codes(layout.B, layout.Hkv, layout.d, layout.n_cap, _p(layout.page_table), layout.max_pages,
+                           layout.page, _p(K), _p(_i32(seq_lens)), _p(rc))
+    return rc
+
+
+def radius_scale(layout: Layout, scores_arr, seq_lens, rc) -> np.ndarray:
+    """s' = fp32(r~_t * fp32(s_t)) for t < seq_lens[b] (NaN elsewhere), float64."""
+    s = _f64(scores_arr)
+    out = np.full_like(s, np.nan)
+    B, Hkv, n_cap = s.shape
+    lib().dko_radius_scale(B, Hkv, n_cap, _p(layout.page_table), layout.max_pages, layout.page,
+                           _p(_i32(seq_lens)), _p(np.ascontiguousarray(rc, dtype=np.uint8)), _p(s), _p(out))
+    return out
+
+
+def decode_step_radius(layout: Layout, Hq, q, K, V, codes, rc, seq_lens, R, topk, sink, window):
+    """Score -> radius scale -> select -> attend for one decode query batch."""
+    sc, bound = scores(layout, Hq, q, codes, seq_lens, R)
+    ss = radius_scale(layout, sc, seq_lens, rc)
+    idx, cnt = select(ss, seq_lens, topk, sink, window)
+    out, lse = attend(layout, Hq, q, K, V, idx, cnt)
+    return dict(scores=ss, unscaled=sc, bound=bound, sel_idx=idx, sel_cnt=cnt, out=out, lse=lse)
