@@ -197,6 +197,18 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ----------------------------------------------------------------------------- oracle leg
+def oracle_block_update(L, K: np.ndarray, bcodes: np.ndarray, n: int, m: int, R) -> None:
+    """After an oracle append that made sequence 0 n tokens long: when n is a
+    multiple of m, encode the summary of the block the append completed (the
+    oracle's whole-cache summary encode applied to that block's m rows)."""
+    from oracle import oracle as O
+    if n == 0 or n % m:
+        return
+    Lb = O.Layout(1, L.Hkv, L.d, L.bits, n_cap=m)
+    last = np.ascontiguousarray(K[:, :, n - m:n])
+    bcodes[:, :, n // m - 1] = O.encode_blocks(Lb, last, np.array([m], np.int32), m, R, 1)[:, :, 0]
+
+
 def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
     """Time the CPU oracle's decode step (score + select + attend; with block
     summaries: block score + block select + attend) on one sequence of the
@@ -219,11 +231,8 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
 
     def append(s):
         O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
-        n = int(seq[0])
-        if m and n % m == 0:  # the block this append completed
-            Lb = O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=m)
-            last = np.ascontiguousarray(K[:, :, n - m:n])
-            bcodes[:, :, n // m - 1] = O.encode_blocks(Lb, last, np.array([m], np.int32), m, R, 1)[:, :, 0]
+        if m:
+            oracle_block_update(L, K, bcodes, int(seq[0]), m, R)
 
     def decode(s):
         q = w.q[s].double().numpy()

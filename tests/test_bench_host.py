@@ -31,3 +31,29 @@ def test_recorded_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
     assert bench.recorded_traffic("select_fused") == 123456  # comments do not make the counters stale
     src.write_text(src.read_text() + "\nstatic int changed_code = 1;\n")
     assert bench.recorded_traffic("select_fused") is None  # a code change does
+
+
+def test_oracle_block_update_matches_a_whole_cache_encode():
+    # the bench's CPU-baseline leg keeps block summaries up to date one append
+    # at a time; after every step they must equal a from-scratch encode
+    import numpy as np
+    from hash_indexed_top_b200 import workloads as W
+    from oracle import oracle as O
+    cfg = W.CONFIGS["tiny"].scaled(name="tiny_b8", N=101, block=8)
+    steps = 20
+    w = W.make_workload(cfg, device="cpu", steps=steps)
+    R = O.hyperplanes(W.HYPERPLANE_SEED, cfg.bits, cfg.d)
+    L = O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=w.n_cap)
+    K = w.K.double().numpy().copy()
+    V = w.V.double().numpy().copy()
+    seq = w.seq_lens.numpy().astype(np.int32).copy()
+    codes = O.encode(L, K, seq, R)
+    nb_cap = w.n_cap // cfg.block
+    bcodes = O.encode_blocks(L, K, seq, cfg.block, R, nb_cap)
+    completed = 0
+    for s in range(steps):
+        O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
+        bench.oracle_block_update(L, K, bcodes, int(seq[0]), cfg.block, R)
+        completed += int(seq[0]) % cfg.block == 0
+        assert np.array_equal(bcodes, O.encode_blocks(L, K, seq, cfg.block, R, nb_cap)), s
+    assert completed >= 2

@@ -5,7 +5,9 @@ sampled (sequence, kv head) pairs: all of a pair's codes and scores, its
 selection, and the attention output and lse of its query heads.
 
 The oracle recomputes a pair from its own encode of the pair's keys (no GPU
-value enters it); the pairs are the first and the last of the grid."""
+value enters it); the pairs are the first and the last of the grid.  The
+block-summary workloads are checked the same way, summaries and block scores
+included."""
 import numpy as np
 import pytest
 import torch
