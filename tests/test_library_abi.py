@@ -70,6 +70,7 @@ def _cfg(**kw):
     (dict(head_dim=96), 2), (dict(bits=48), 2), (dict(bits=256), 2), (dict(num_q_heads=12, num_kv_heads=1), 2),
     (dict(num_q_heads=6, num_kv_heads=4), 1), (dict(topk=0), 1), (dict(sink=-1), 1), (dict(page_size=48), 2),
     (dict(batch=0), 1), (dict(flags=6), 1), (dict(num_q_heads=64, num_kv_heads=64), 2),
+    (dict(page_size=1056), 2), (dict(window=-1), 1), (dict(topk=2**30, sink=2**29, window=2**29), 1),
 ])
 def test_create_rejects_bad_configs(kw, status):
     h = ctypes.c_void_p()
@@ -101,3 +102,22 @@ def test_canonical_codes_undoes_the_storage_rotation(bits):
     st = torch.from_numpy(stored.copy()).view(torch.int64).reshape(2, 3, 70, W)
     back = dk.canonical_codes(st, bits).view(torch.uint8).reshape(2, 3, 70, W * 8).numpy()
     assert np.array_equal(back, orig)
+
+
+def test_block_view_layout_and_index_shapes():
+    # dashkv_block_view: { uint64_t *codes; int64_t nb_cap; int32_t block; int32_t reserved; }
+    assert ctypes.sizeof(dk.BlockView) == 24
+    assert [dk.BlockView.codes.offset, dk.BlockView.nb_cap.offset, dk.BlockView.block.offset,
+            dk.BlockView.reserved.offset] == [0, 8, 16, 20]
+    # summaries for every complete block the cache holds: dense and paged
+    K = torch.zeros((3, 2, 1001, 64), dtype=torch.bfloat16)
+    dense = dk.KVCache(K, K, dk.KVCache.empty_codes_like(K, 128, False))
+    idx = dk.BlockIndex.empty_for(dense, 3, 128, 8)
+    assert tuple(idx.codes.shape) == (3, 2, 125, 2) and idx.capacity == 125
+    v = idx.view()
+    assert v.nb_cap == 125 and v.block == 8 and v.reserved == 0
+    Kp = torch.zeros((10, 64, 4, 128), dtype=torch.bfloat16)
+    pt = torch.zeros((2, 7), dtype=torch.int32)
+    paged = dk.KVCache(Kp, Kp, dk.KVCache.empty_codes_like(Kp, 64, True), pt)
+    idx = dk.BlockIndex.empty_for(paged, 2, 64, 16)
+    assert tuple(idx.codes.shape) == (2, 4, 7 * 64 // 16, 1)
