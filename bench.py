@@ -233,10 +233,18 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
         O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
         if m:
             oracle_block_update(L, K, bcodes, int(seq[0]), m, R)
+        if cfg.radius:  # the appended token's radius code
+            n = int(seq[0])
+            rc[:, :, n - 1] = O.radius_codes(O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=1),
+                                             np.ascontiguousarray(K[:, :, n - 1:n]), np.array([1], np.int32))[:, :, 0]
+
+    rc = O.radius_codes(L, K, seq) if cfg.radius else None
 
     def decode(s):
         q = w.q[s].double().numpy()
-        if m:
+        if cfg.radius:
+            O.decode_step_radius(L, cfg.Hq, q, K, V, codes, rc, seq, R, cfg.topk, cfg.sink, cfg.window)
+        elif m:
             O.decode_step_blocks(L, cfg.Hq, q, K, V, bcodes, seq, R, m, cfg.topk // m, cfg.sink, cfg.window,
                                  cap=cfg.sel_cap)
         else:
@@ -256,7 +264,7 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
     decode(n_steps)
     one_thread_s = time.perf_counter() - t0
     O.set_threads(cores)
-    how = f", blocks of {m}" if m else ""
+    how = f", blocks of {m}" if m else (", radius-scaled scores" if cfg.radius else "")
     return dict(times=times, cores=cores, one_thread_s=one_thread_s,
                 sample=f"sequence {seq_index} of {cfg.B} (N={cfg.N}, all {cfg.Hkv} KV / {cfg.Hq} query heads{how}), "
                        f"{n_steps} decode steps, oracle encode untimed")
@@ -307,10 +315,13 @@ def run_dashkv(args, cfg, world, rank, local):
     flush = W.L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     eng.encode_keys(cache, seq)
-    index = None
+    index = radius = None
     if cfg.block:  # block summaries of the prefilled cache (untimed, like the key codes)
         index = dk.BlockIndex.empty_for(cache, cfg.B, cfg.bits, cfg.block)
         eng.encode_blocks(cache, index, seq)
+    if cfg.radius:  # radius codes of the prefilled cache (untimed)
+        radius = dk.KVCache.empty_radius_like(w.K, w.paged)
+        eng.encode_radius(cache, radius, seq)
     torch.cuda.synchronize(dev)
     assert eng.get_error() == 0
     # the prefill encode, timed on its own (a second, identical call: cold L2, kernel already loaded)
@@ -344,6 +355,8 @@ def run_dashkv(args, cfg, world, rank, local):
     calls = [("append_keys", ["append_keys"])]
     if cfg.block:
         calls += [("append_blocks", ["append_blocks"]), ("select_blocks", sel_names + ["expand_blocks"])]
+    elif cfg.radius:
+        calls += [("append_radius", ["append_radius"]), ("select_radius", ["select_fused"])]
     else:
         calls += [("select", sel_names)]
     calls += [("sparse_decode", ["sparse_decode"])]
@@ -362,6 +375,10 @@ def run_dashkv(args, cfg, world, rank, local):
                 eng.append_blocks(cache, index, seq)
             elif name == "select_blocks":
                 eng.select_blocks(cache, index, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            elif name == "append_radius":
+                eng.append_radius(cache, radius, seq)
+            elif name == "select_radius":
+                eng.select_radius(cache, radius, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
             elif name == "select":
                 eng.select(cache, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
             else:
@@ -513,7 +530,8 @@ def run_dashkv(args, cfg, world, rank, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
                        "bits": cfg.bits, "topk": cfg.topk, "sink": cfg.sink, "window": cfg.window,
-                       "block": cfg.block or None, "layout": "paged" if w.paged else "dense", "l2": "flushed before every step: 2 x L2 write, then 2 x L2 clean read (no pending write-backs)",
+                       "block": cfg.block or None, "radius": cfg.radius or None,
+                       "layout": "paged" if w.paged else "dense", "l2": "flushed before every step: 2 x L2 write, then 2 x L2 clean read (no pending write-backs)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": score_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": score_gbs / peaks["hbm_gbs"],

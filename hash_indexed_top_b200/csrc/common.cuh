@@ -85,6 +85,7 @@ struct KV {
     int32_t d;
     int32_t W;                 // 64-bit code words per key
     int32_t len_shift;         // entries per sequence = seq_lens[b] >> len_shift (block summaries: log2 m)
+    const uint8_t *radius;     // optional 8-bit key-norm codes (layout of radius_index), or null
 
     __host__ __device__ int64_t capacity() const {
         return page_size ? (int64_t)max_pages * page_size : n_cap;
@@ -105,6 +106,14 @@ struct KV {
         int64_t p = page_of(b, t);
         if (p < 0) return -1;
         return ((p * page_size + t % page_size) * Hkv + h) * (int64_t)d;
+    }
+    // Byte offset of the radius code of (b, h, t) -- dense [B][Hkv][n_cap], paged
+    // [P][Hkv][page] (the codes' layout without the word axis) -- or -1.
+    __device__ __forceinline__ int64_t radius_index(int b, int h, int64_t t) const {
+        if (!page_size) return ((int64_t)b * Hkv + h) * n_cap + t;
+        int64_t p = page_of(b, t);
+        if (p < 0) return -1;
+        return (p * Hkv + h) * page_size + t % page_size;
     }
     // Word offset of the code of (b, h, t), or -1.
     __device__ __forceinline__ int64_t code(int b, int h, int64_t t) const {

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "encode.cuh"
+#include "radius.cuh"
 #include "select.cuh"
 
 using namespace dkv;
@@ -117,6 +118,7 @@ KV make_kv(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
     o.d = ctx->cfg.head_dim;
     o.W = ctx->cfg.bits >= 64 ? ctx->cfg.bits / 64 : 1;
     o.len_shift = 0;
+    o.radius = nullptr;
     return o;
 }
 
@@ -154,6 +156,7 @@ KV make_blk(const dashkv_ctx *ctx, const dashkv_block_view *blk) {
     o.d = ctx->cfg.head_dim;
     o.W = ctx->cfg.bits >= 64 ? ctx->cfg.bits / 64 : 1;
     o.len_shift = block_shift(blk->block);
+    o.radius = nullptr;
     return o;
 }
 
@@ -238,11 +241,13 @@ int attn_splits(const dashkv_ctx *ctx) {
 // leave room for the low region below 64 KB.
 template <int BITS, int D>
 bool score_layout_ok() {
-    cudaFuncAttributes a[4];
+    cudaFuncAttributes a[6];
     cudaFuncGetAttributes(&a[0], score_hist_kernel<BITS, D, false>);
     cudaFuncGetAttributes(&a[1], score_hist_kernel<BITS, D, true>);
     cudaFuncGetAttributes(&a[2], select_fused_kernel<BITS, D, false>);
     cudaFuncGetAttributes(&a[3], select_fused_kernel<BITS, D, true>);
+    cudaFuncGetAttributes(&a[4], select_fused_kernel<BITS, D, false, true>);
+    cudaFuncGetAttributes(&a[5], select_fused_kernel<BITS, D, true, true>);
     for (auto &x : a)
         if (x.sharedSizeBytes + 1024 + ScoreShape<BITS>::LOW_BYTES > 65536) return false;
     return true;
@@ -262,6 +267,12 @@ void set_attrs_bd() {
                          (int)ScoreShape<BITS>::SMEM);
     cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
 }
 
 template <int D, int G>
@@ -407,7 +418,9 @@ void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
                      int nctas, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
-    auto kern = kv.page_size ? select_fused_kernel<BITS, D, true> : select_fused_kernel<BITS, D, false>;
+    auto kern = kv.radius ? (kv.page_size ? select_fused_kernel<BITS, D, true, true>
+                                          : select_fused_kernel<BITS, D, false, true>)
+                          : (kv.page_size ? select_fused_kernel<BITS, D, true> : select_fused_kernel<BITS, D, false>);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nctas, BH);
     cfg.blockDim = dim3(kScoreThreads);
@@ -561,6 +574,21 @@ void launch_append_blocks_bd(const dashkv_ctx *ctx, const KV &kv, const KV &blk,
     const int hpc = (Hkv + C - 1) / C;         // heads per CTA: hpc * BITS <= 1024
     launch_pdl(append_blocks_kernel<BITS, D>, dim3(C, ctx->cfg.batch), dim3(hpc * BITS),
                (size_t)hpc * (D * 4 + BITS / 8), st, kv, blk, seq_lens, ctx->R, hpc);
+}
+
+template <int D>
+void launch_radius_d(const dashkv_ctx *ctx, bool whole, const KV &kv, const int32_t *seq_lens, uint8_t *out,
+                     cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    if (whole) {
+        int64_t gx = ceil_div(kv.capacity(), kRadiusThreads);
+        const int64_t cap_x = ceil_div(8 * ctx->sm_count, BH);
+        if (gx > cap_x) gx = cap_x;
+        if (gx < 1) gx = 1;
+        radius_codes_kernel<D><<<dim3((unsigned)gx, BH), kRadiusThreads, 0, st>>>(kv, seq_lens, out);
+    } else {
+        launch_pdl(append_radius_kernel<D>, dim3(ctx->cfg.batch), dim3(32), 0, st, kv, seq_lens, out);
+    }
 }
 
 template <int D>
@@ -829,6 +857,56 @@ dashkv_status dashkv_select_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                (const int32_t *)blk_cnt, kb, seq_lens, cap, ctx->cfg.num_kv_heads, shift, ctx->cfg.sink,
                ctx->cfg.window, cap_sel, sel_idx, sel_cnt);
     tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_encode_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, const int32_t *seq_lens,
+                                   uint8_t *radius, void *stream) {
+    if (!ctx || !seq_lens || !radius) return DASHKV_ERR_INVALID_ARG;
+    const dashkv_status s = check_view(ctx, kv, true, false);
+    if (s != DASHKV_OK) return s;
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_radius_d<64>(ctx, true, k, seq_lens, radius, st);
+    else launch_radius_d<128>(ctx, true, k, seq_lens, radius, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_append_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, const int32_t *seq_lens,
+                                   uint8_t *radius, void *stream) {
+    if (!ctx || !seq_lens || !radius) return DASHKV_ERR_INVALID_ARG;
+    const dashkv_status s = check_view(ctx, kv, true, false);
+    if (s != DASHKV_OK) return s;
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    if (ctx->cfg.head_dim == 64) launch_radius_d<64>(ctx, false, k, seq_lens, radius, st);
+    else launch_radius_d<128>(ctx, false, k, seq_lens, radius, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_select_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, const uint8_t *radius, const void *q,
+                                   const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
+                                   void *workspace, size_t workspace_bytes, void *stream) {
+    if (!ctx || !radius || !q || !seq_lens || !sel_idx || !sel_cnt || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
+    const dashkv_status s = check_view(ctx, kv, false, true);
+    if (s != DASHKV_OK) return s;
+    if (!use_fused(ctx)) return DASHKV_ERR_UNSUPPORTED;  // the fused selection only
+    const int64_t cap = view_capacity(ctx, kv);
+    const WsLayout L = ws_layout(ctx->cfg, cap);
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
+    KV k = make_kv(ctx, kv);
+    k.radius = radius;
+    const SelArgs a{ctx->cfg.topk, ctx->cfg.sink, ctx->cfg.window,
+                    ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    run_select(ctx, k, cap, L, static_cast<char *>(workspace), q, seq_lens, a, sel_idx, sel_cnt, scores, tr, st);
     return launch_status();
 }
 

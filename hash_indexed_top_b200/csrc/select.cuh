@@ -42,6 +42,7 @@
 namespace dkv {
 
 constexpr int kBins = 4096;
+constexpr float kRadiusMax = 63.875f;  // largest radius r~ = (255 + 1/2) / 4
 constexpr int kSelThreads = 512;
 constexpr int kMaxSelCtas = 512;
 constexpr int kCandSmem = 2048;   // in-bin candidates ranked in shared memory
@@ -212,7 +213,11 @@ struct ScoreOut {
 // FUSED: the fused selection -- record the chunk maxima, and let the dependent
 // launch (the sparse decode, whose window CTAs need nothing from the selection)
 // start right after the wait on the preceding kernel.
-template <int BITS, int D, bool PAGED, bool FUSED = false>
+// RADIUS: radius-scaled scores s' = r~ s (Spherical KV page, section 2.1 ADA: a
+// quantized key radius beside the angle code scales the logit), r~ = (c + 1/2)/4
+// from the token's 8-bit code c in kv.radius; the bins span r~_max times the
+// unscaled range.
+template <int BITS, int D, bool PAGED, bool FUSED = false, bool RADIUS = false>
 __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                                                 const int32_t *__restrict__ seq_lens, const RBits &R,
                                                 const SelWS &ws, int nctas, unsigned char *smem) {
@@ -266,6 +271,7 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
         for (int j = lane; j < BITS; j += 32) a += fabsf(Qp[j]);
 #pragma unroll
         for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (RADIUS) a *= kRadiusMax;
         if (lane == 0) red[0] = a > 0.0f ? 0.5f / a : 0.0f;
     }
     // LUT rows: word j of row v holds LUT_{j mod T}[v]; lane l fills words l and
@@ -355,6 +361,15 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
             asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
+    // r~ of token wb + 32 k + lane (read one step ahead of its use), 0 outside
+    auto radius_of = [&](int k) -> float {
+        const int i = wb + 32 * k + lane;
+        if (k >= nk || i >= we) return 0.0f;
+        const int64_t r = kv.radius_index(b, h, t0 + i);
+        return r >= 0 ? ((float)__ldg(kv.radius + r) + 0.5f) * 0.25f : 0.0f;
+    };
+    float rnext = 0.0f;
+    if constexpr (RADIUS) rnext = radius_of(0);
 #pragma unroll
     for (int k = 0; k < STAGES - 1; ++k) issue(k, k);
     for (int k0 = 0; k0 < nk; k0 += STAGES) {
@@ -363,6 +378,11 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
             const int k = k0 + u;
             if (k >= nk) break;
             issue(k + STAGES - 1, (u + STAGES - 1) % STAGES);
+            float rcur = 0.0f;
+            if constexpr (RADIUS) {
+                rcur = rnext;
+                rnext = radius_of(k + 1);
+            }
             asm volatile("cp.async.wait_group %0;" ::"n"(STAGES - 1) : "memory");
             const int i = wb + 32 * k + lane;
             const Vec code = *reinterpret_cast<const Vec *>(ring + u * NT * VB);
@@ -370,7 +390,8 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
             if (i < we) {
                 uint32_t w[NW];
                 unpack_code<BITS>(code, w);
-                const float sc = lut_score<BITS>(w, lbase);
+                float sc = lut_score<BITS>(w, lbase);
+                if constexpr (RADIUS) sc = __fmul_rn(sc, rcur);  // one rounding, as the definition
                 srow[i] = sc;
                 bin = score_bin(sc, inv2A);
                 atomicAdd(&hist[bin], 1u);
@@ -864,7 +885,7 @@ __device__ __forceinline__ float bin_floor_value(int T, float inv2A) {
     return key_to_float((uint32_t)lo);     // `none` maps to +inf
 }
 
-template <int BITS, int D, bool PAGED>
+template <int BITS, int D, bool PAGED, bool RADIUS = false>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                     const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int S, int W,
@@ -894,7 +915,7 @@ select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.y, cta = blockIdx.x;  // cta = rank in the cluster (cluster = the row of CTAs)
     const int nctas = gridDim.x;
-    const ScoreOut so = score_phase<BITS, D, PAGED, true>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
+    const ScoreOut so = score_phase<BITS, D, PAGED, true, RADIUS>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
     const uint32_t *hist = reinterpret_cast<const uint32_t *>(smem);
     {   // super-bin counts: 16 threads per super-bin, 4 bins each
         uint32_t c = hist[4 * tid] + hist[4 * tid + 1] + hist[4 * tid + 2] + hist[4 * tid + 3];

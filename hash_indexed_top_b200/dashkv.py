@@ -27,7 +27,8 @@ FLAG_TWO_KERNEL_SELECT = 1
 SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_encode_keys",
            "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
            "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str",
-           "dashkv_select_static", "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks")
+           "dashkv_select_static", "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks",
+           "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius")
 
 
 class DashKVError(RuntimeError):
@@ -80,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.dashkv_append_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P]
         L.dashkv_select_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P, P, P, P, P,
                                            SZ, P]
+        L.dashkv_encode_radius.argtypes = [P, ctypes.POINTER(KVView), P, P, P]
+        L.dashkv_append_radius.argtypes = [P, ctypes.POINTER(KVView), P, P, P]
+        L.dashkv_select_radius.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, P, SZ, P]
         L.dashkv_get_error.argtypes = [P]
         L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
         L.dashkv_set_trace.argtypes = [P, P, I32]
@@ -89,7 +93,8 @@ def lib() -> ctypes.CDLL:
         L.dashkv_status_str.restype = ctypes.c_char_p
         for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode",
                   "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_static",
-                  "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks"):
+                  "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks",
+                  "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -165,6 +170,15 @@ class KVCache:
                           self.page_table.data_ptr(), int(self.page_table.shape[1]), int(self.k.shape[0]))
         return KVView(self.k.data_ptr(), self.v.data_ptr(), self.codes.data_ptr(), int(self.k.shape[2]),
                       None, 0, 0)
+
+    @staticmethod
+    def empty_radius_like(k: torch.Tensor, paged: bool) -> torch.Tensor:
+        """Zeroed uint8 radius codes: dense [B,Hkv,n_cap], paged [P,Hkv,page]."""
+        if paged:
+            P, ps, Hkv, _ = k.shape
+            return torch.zeros((P, Hkv, ps), dtype=torch.uint8, device=k.device)
+        B, Hkv, n_cap, _ = k.shape
+        return torch.zeros((B, Hkv, n_cap), dtype=torch.uint8, device=k.device)
 
     @staticmethod
     def empty_codes_like(k: torch.Tensor, bits: int, paged: bool) -> torch.Tensor:
@@ -306,6 +320,29 @@ class DashKV:
                                                                   _ptr(q), _ptr(seq_lens), _ptr(sel_idx),
                                                                   _ptr(sel_cnt), _ptr(block_scores), _ptr(ws),
                                                                   ws.numel(), _stream(stream)))
+
+    # ---- radius-scaled scores (8-bit key-norm codes)
+    def encode_radius(self, cache: KVCache, radius: torch.Tensor, seq_lens: torch.Tensor, stream=None) -> None:
+        v = cache.view()
+        _check("dashkv_encode_radius", lib().dashkv_encode_radius(self._ctx, ctypes.byref(v), _ptr(seq_lens),
+                                                                  _ptr(radius), _stream(stream)))
+
+    def append_radius(self, cache: KVCache, radius: torch.Tensor, seq_lens: torch.Tensor, stream=None) -> None:
+        """After append_keys: the radius code of each sequence's newest token."""
+        v = cache.view()
+        _check("dashkv_append_radius", lib().dashkv_append_radius(self._ctx, ctypes.byref(v), _ptr(seq_lens),
+                                                                  _ptr(radius), _stream(stream)))
+
+    def select_radius(self, cache: KVCache, radius: torch.Tensor, q: torch.Tensor, seq_lens: torch.Tensor,
+                      sel_idx: torch.Tensor, sel_cnt: torch.Tensor, scores: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+        """select() on the radius-scaled scores r~ s."""
+        ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
+        v = cache.view()
+        _check("dashkv_select_radius", lib().dashkv_select_radius(self._ctx, ctypes.byref(v), _ptr(radius), _ptr(q),
+                                                                  _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt),
+                                                                  _ptr(scores), _ptr(ws), ws.numel(),
+                                                                  _stream(stream)))
 
     def select_kernels(self, max_tokens: int) -> int:
         """1 when dashkv_select runs the fused kernel for this cache size, 2 for score + collect."""

@@ -52,6 +52,7 @@ class Config:
     n_min: int = 0         # ragged: lower bound of the length draw (0 = fixed N)
     seed: int = 1234
     block: int = 0         # > 0: select through summaries of blocks of this many tokens
+    radius: bool = False   # select on radius-scaled scores (8-bit key-norm codes)
 
     @property
     def G(self) -> int:
@@ -82,6 +83,8 @@ CONFIGS = {
 # top topk / 4 blocks give the same top-k token budget
 CONFIGS["c128k_blocks4"] = CONFIGS["c128k"].scaled(name="c128k_blocks4", block=4)
 CONFIGS["c1m_blocks4"] = CONFIGS["c1m"].scaled(name="c1m_blocks4", block=4)
+# the 128K workload selected on radius-scaled scores
+CONFIGS["c128k_radius"] = CONFIGS["c128k"].scaled(name="c128k_radius", radius=True)
 
 
 def grid(x: torch.Tensor) -> torch.Tensor:

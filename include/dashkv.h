@@ -248,6 +248,39 @@ dashkv_status dashkv_select_blocks(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    const void *q, const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
                                    float *block_scores, void *workspace, size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Radius-scaled scores.
+ *
+ * Spherical KV page, section 2.1 ADA: a compact key keeps a quantized radius
+ * r~ beside its angle code, and the logit is estimated as |q| r~ f_b(codes).
+ * Here the selection may rank s'_t = r~_t s_t (s_t the score of
+ * dashkv_select; |q| is one constant per query).  The radius code of a key is
+ *   c = min(255, floor(4 sqrt(sum_i k_i^2)))   (fp32, i ascending, every
+ *                                               operation rounded once),
+ *   r~ = (c + 1/2) / 4,
+ * stored as one byte per token and kv head: dense [B][Hkv][n_cap], paged
+ * [num_pages][Hkv][page_size] (the codes' layout without the word axis).
+ * s' is the fp32 product of r~ and the fp32 score (one rounding).
+ * ------------------------------------------------------------------------ */
+
+/* Radius codes of tokens [0, seq_lens[b]) of every (b, kv head) from kv->k,
+ * written to `radius` (device, layout above). */
+dashkv_status dashkv_encode_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, const int32_t *seq_lens,
+                                   uint8_t *radius, void *stream);
+
+/* Decode-step update, after dashkv_append_keys with the lengths it
+ * incremented: the radius code of token seq_lens[b] - 1 of every kv head. */
+dashkv_status dashkv_append_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, const int32_t *seq_lens,
+                                   uint8_t *radius, void *stream);
+
+/* dashkv_select on the radius-scaled scores: same arguments and outputs
+ * (scores, when given, receives s'), plus the radius codes.  Runs the fused
+ * selection only: DASHKV_ERR_UNSUPPORTED without cluster launch support or
+ * with DASHKV_FLAG_TWO_KERNEL_SELECT. */
+dashkv_status dashkv_select_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, const uint8_t *radius, const void *q,
+                                   const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
 /* Synchronise `stream`, then read and clear the current device's error
  * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, or DASHKV_ERR_CUDA
  * when the stream reports an error. */
