@@ -341,7 +341,17 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     // Step k copies token wb + 32 k + lane into ring slot k % STAGES; the loop
     // is unrolled by STAGES so every slot (and its shared address) is a
     // compile-time constant, and the positions advance by 32 tokens per step.
-    auto issue = [&](int k, int slot) {  // copy the code of token wb + 32 k + lane into `slot`
+    // PAGED: a step's 32 tokens lie in one page (t0 and the warp ranges are
+    // multiples of 32, pages hold a multiple of 32 tokens), so its physical page
+    // is one warp-wide load, made one step before the copy that needs it.
+    auto page_of_step = [&](int k) -> int64_t {  // -1: no tokens; -2: page id out of range
+        const int i = wb + 32 * k;
+        if (k >= nk || i >= we) return -1;
+        const int64_t t = t0 + i;
+        const int32_t p = __ldg(kv.page_table + (int64_t)b * kv.max_pages + t / kv.page_size);
+        return (p < 0 || p >= kv.num_pages) ? -2 : (int64_t)p;
+    };
+    auto issue = [&](int k, int slot, int64_t pg) {  // copy the code of token wb + 32 k + lane into `slot`
         const int i = wb + 32 * k + lane;
         const void *src = dense;
         int bytes = 0;
@@ -349,9 +359,12 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
             if (!PAGED) {
                 src = dense + i;
                 bytes = VB;
-            } else {
-                const int64_t c = kv.code(b, h, t0 + i);
-                if (c >= 0) { src = kv.codes + c; bytes = VB; }
+            } else if (pg >= 0) {
+                const int64_t t = t0 + i;
+                src = kv.codes + ((pg * kv.Hkv + h) * kv.page_size + t % kv.page_size) * kv.W;
+                bytes = VB;
+            } else if (pg == -2) {
+                raise_error(kErrPage);
             }
         }
         const uint32_t dst = ring_s + (uint32_t)(slot * NT * VB);
@@ -371,13 +384,16 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     float rnext = 0.0f;
     if constexpr (RADIUS) rnext = radius_of(0);
 #pragma unroll
-    for (int k = 0; k < STAGES - 1; ++k) issue(k, k);
+    for (int k = 0; k < STAGES - 1; ++k) issue(k, k, PAGED ? page_of_step(k) : 0);
+    int64_t pg_next = PAGED ? page_of_step(STAGES - 1) : 0;  // page of the next step to be issued
     for (int k0 = 0; k0 < nk; k0 += STAGES) {
 #pragma unroll
         for (int u = 0; u < STAGES; ++u) {
             const int k = k0 + u;
             if (k >= nk) break;
-            issue(k + STAGES - 1, (u + STAGES - 1) % STAGES);
+            const int64_t pg = pg_next;
+            if constexpr (PAGED) pg_next = page_of_step(k + STAGES);
+            issue(k + STAGES - 1, (u + STAGES - 1) % STAGES, pg);
             float rcur = 0.0f;
             if constexpr (RADIUS) {
                 rcur = rnext;
