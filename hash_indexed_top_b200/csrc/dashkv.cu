@@ -611,28 +611,63 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 namespace {
 constexpr int kMaxStaticDevices = 64;
-void *g_static_addr[kMaxStaticDevices];  // device address of the scratch, once set up
+// Per device: the scratch's device address (once set up) and the regions of
+// the last selection layout whose counter words are known to be zero.  The
+// histogram and arrival words sit at offsets that depend on B * Hkv and the
+// capacity, so a call with another layout may find rows an earlier call left
+// there; those words are zeroed again (on the call's stream) whenever the
+// layout changes or after a call that failed.
+struct StaticScratch {
+    void *addr;
+    size_t hist_off, hist_bytes, arrive_off, arrive_bytes;  // all 0: nothing known to be zero
+};
+StaticScratch g_static[kMaxStaticDevices];
 std::mutex g_static_mu;
 
-// First use on a device: look the scratch up and zero it (its histogram and
-// counter words must start at zero; every successful selection leaves them
-// so).  The memset and the device synchronisation cannot be captured, so this
-// refuses to run while `st` is capturing.
-dashkv_status static_scratch(int dev, cudaStream_t st, void **out) {
-    if (dev < 0 || dev >= kMaxStaticDevices) return DASHKV_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_addr[dev]) {
-        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return DASHKV_ERR_CUDA;
-        if (cs != cudaStreamCaptureStatusNone) return DASHKV_ERR_INVALID_ARG;
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DASHKV_ERR_CUDA;
-        if (cudaMemset(p, 0, kStaticScratchBytes) != cudaSuccess) return DASHKV_ERR_CUDA;
-        if (cudaDeviceSynchronize() != cudaSuccess) return DASHKV_ERR_CUDA;
-        g_static_addr[dev] = p;
-    }
-    *out = g_static_addr[dev];
+// First use on a device: look the scratch up and zero it whole.  The memset
+// and the device synchronisation cannot be captured, so this refuses to run
+// while `st` is capturing.  The caller holds g_static_mu.
+dashkv_status static_scratch_setup(int dev, cudaStream_t st) {
+    if (g_static[dev].addr) return DASHKV_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return DASHKV_ERR_INVALID_ARG;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DASHKV_ERR_CUDA;
+    if (cudaMemset(p, 0, kStaticScratchBytes) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return DASHKV_ERR_CUDA;
+    g_static[dev] = StaticScratch{p, 0, 0, 0, 0};
     return DASHKV_OK;
+}
+
+// Make the counter words of layout L zero before a selection on `st`: nothing
+// to do when the previous successful call used the same regions (it left them
+// zero); otherwise they are cleared with stream-ordered (capturable) memsets.
+// Under capture the record is not updated, since the graph may never run.
+dashkv_status static_scratch_prepare(int dev, const WsLayout &L, size_t hist_bytes, size_t arrive_bytes,
+                                     cudaStream_t st) {
+    StaticScratch &s = g_static[dev];
+    if (s.hist_off == L.hist && s.hist_bytes == hist_bytes && s.arrive_off == L.arrive &&
+        s.arrive_bytes == arrive_bytes)
+        return DASHKV_OK;
+    char *w = static_cast<char *>(s.addr);
+    if (cudaMemsetAsync(w + L.hist, 0, hist_bytes, st) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (cudaMemsetAsync(w + L.arrive, 0, arrive_bytes, st) != cudaSuccess) return DASHKV_ERR_CUDA;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusNone) {
+        s.hist_off = L.hist;
+        s.hist_bytes = hist_bytes;
+        s.arrive_off = L.arrive;
+        s.arrive_bytes = arrive_bytes;
+    }
+    return DASHKV_OK;
+}
+
+// After a failed call nothing is known about the counter words any more.
+void static_scratch_forget(int dev) {
+    StaticScratch &s = g_static[dev];
+    s.hist_off = s.hist_bytes = s.arrive_off = s.arrive_bytes = 0;
 }
 }  // namespace
 
@@ -757,7 +792,7 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
     return launch_status();
 }
 
-// dashkv_select on the library's static scratch (see static_scratch above):
+// dashkv_select on the library's static scratch (see StaticScratch above):
 // for callers that cannot allocate the workspace themselves.
 dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
                                    const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
@@ -765,11 +800,23 @@ dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
     if (!ctx) return DASHKV_ERR_INVALID_ARG;
     const dashkv_status v = check_view(ctx, kv, false, true);
     if (v != DASHKV_OK) return v;
-    if (ws_layout(ctx->cfg, view_capacity(ctx, kv)).total > kStaticScratchBytes) return DASHKV_ERR_WORKSPACE;
-    void *w = nullptr;
-    const dashkv_status s = static_scratch(ctx->device, static_cast<cudaStream_t>(stream), &w);
-    if (s != DASHKV_OK) return s;
-    return dashkv_select(ctx, kv, q, seq_lens, sel_idx, sel_cnt, scores, w, kStaticScratchBytes, stream);
+    const WsLayout L = ws_layout(ctx->cfg, view_capacity(ctx, kv));
+    if (L.total > kStaticScratchBytes) return DASHKV_ERR_WORKSPACE;
+    // the scratch address belongs to the current device: it must be the context's
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (cur != ctx->device) return DASHKV_ERR_INVALID_ARG;
+    if (cur < 0 || cur >= kMaxStaticDevices) return DASHKV_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t BH = (size_t)ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    dashkv_status s = static_scratch_setup(cur, st);
+    if (s == DASHKV_OK) s = static_scratch_prepare(cur, L, BH * kBins * 4, 3 * BH * kSyncStride * 4, st);
+    if (s == DASHKV_OK)
+        s = dashkv_select(ctx, kv, q, seq_lens, sel_idx, sel_cnt, scores, g_static[cur].addr, kStaticScratchBytes,
+                          stream);
+    if (s != DASHKV_OK && g_static[cur].addr) static_scratch_forget(cur);
+    return s;
 }
 
 dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,

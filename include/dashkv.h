@@ -169,13 +169,18 @@ dashkv_status dashkv_select(dashkv_ctx *ctx, const dashkv_kv_view *kv, const voi
  * (25165824 bytes) per device, the limit.  Inputs whose
  * dashkv_workspace_size(ctx, capacity) exceeds it are rejected with
  * DASHKV_ERR_WORKSPACE before anything is launched.  It allocates nothing.
- * The first call on a device looks the scratch up (cudaGetSymbolAddress)
- * and zero-fills it with a synchronising memset: that first call must come
- * before any stream capture (during capture it returns
- * DASHKV_ERR_INVALID_ARG); later calls may be captured.  All calls on a
- * device share the one scratch: calls that overlap on the GPU (other
- * streams, other threads) race and must be serialised by the caller.
- * Arguments and results are those of dashkv_select. */
+ * The device current at the call must be the context's (else
+ * DASHKV_ERR_INVALID_ARG).  The first call on a device looks the scratch up
+ * (cudaGetSymbolAddress) and zero-fills it with a synchronising memset: that
+ * first call must come before any stream capture (during capture it returns
+ * DASHKV_ERR_INVALID_ARG).  A later call whose problem shape lays the scratch
+ * out differently from the previous successful call's, or that follows a
+ * failed call, first clears the selection's counter words with
+ * cudaMemsetAsync on `stream` (stream-ordered, so it may be captured).  All
+ * calls on a device share the one scratch and it keeps the last call's
+ * contents: calls that overlap on the GPU (other streams, other threads)
+ * race and must be serialised by the caller.  Arguments and results are
+ * those of dashkv_select. */
 dashkv_status dashkv_select_static(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q,
                                    const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
                                    float *scores, void *stream);

@@ -4,7 +4,11 @@ device scratch) against dashkv_select with a caller workspace.
 Collected last on purpose: the static scratch lives for the whole process,
 so these checks must hold both alone and after every other test has used the
 library.  Two steps in a row (append, then both selections) also check that
-each call leaves the scratch ready for the next.
+each call leaves the scratch ready for the next; a sequence of problems with
+different capacities and batch shapes checks that a call whose scratch layout
+differs from the previous one's does not read counters the previous call left
+in its rows (both selection paths: the two-kernel path reads histogram and
+arrival words that must start at zero).
 """
 import pytest
 import torch
@@ -22,20 +26,21 @@ CASES = {
 }
 
 
-def _engine(cfg, w):
+def _engine(cfg, w, two_kernel=False):
     eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
-                    cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED)
+                    cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED, two_kernel_select=two_kernel)
     codes = dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged)
     return eng, dk.KVCache(w.K, w.V, codes, w.page_table)
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("two_kernel", [False, True], ids=["fused", "two_kernel"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_static_select_matches_workspace_select(name):
+def test_static_select_matches_workspace_select(name, two_kernel):
     cfg = CASES[name]
     dev = torch.device("cuda")
     w = W.make_workload(cfg, device=dev, steps=cfg.steps)
-    eng, cache = _engine(cfg, w)
+    eng, cache = _engine(cfg, w, two_kernel)
     try:
         assert eng.workspace_size(cache.capacity) <= STATIC_SCRATCH_BYTES
         seq = w.seq_lens.clone()
@@ -62,6 +67,49 @@ def test_static_select_matches_workspace_select(name):
             assert int(cb.min()) > 0
     finally:
         eng.close()
+
+
+# Problems whose scratch layouts differ (capacity and B * Hkv), run in this
+# order in one process: large, small, large again.
+LAYOUTS = [
+    W.Config("ns_large", B=2, Hq=16, Hkv=8, d=64, N=9000, bits=64, topk=400, sink=4, window=64, steps=1,
+             needles=4, seed=4201),
+    W.Config("ns_small", B=1, Hq=8, Hkv=2, d=128, N=3000, bits=128, topk=150, sink=2, window=16, steps=1,
+             needles=4, seed=4202),
+    W.Config("ns_large2", B=2, Hq=16, Hkv=8, d=64, N=9000, bits=64, topk=400, sink=4, window=64, steps=1,
+             needles=4, seed=4203),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("two_kernel", [False, True], ids=["fused", "two_kernel"])
+def test_static_select_across_layout_changes(two_kernel):
+    dev = torch.device("cuda")
+    for cfg in LAYOUTS:
+        w = W.make_workload(cfg, device=dev, steps=1)
+        eng, cache = _engine(cfg, w, two_kernel)
+        try:
+            seq = w.seq_lens.clone()
+            eng.encode_keys(cache, seq)
+            eng.append_keys(cache, w.k_new[0], w.v_new[0], seq)
+            cap_sel = cfg.topk + cfg.sink + cfg.window
+            res = {}
+            for kind in ("static", "fresh"):
+                idx = torch.full((cfg.B, cfg.Hkv, cap_sel), -7, dtype=torch.int32, device=dev)
+                cnt = torch.full((cfg.B, cfg.Hkv), -7, dtype=torch.int32, device=dev)
+                if kind == "static":
+                    eng.select_static(cache, w.q[0], seq, idx, cnt)
+                else:  # a freshly zeroed caller workspace
+                    ws = torch.zeros(eng.workspace_size(cache.capacity), dtype=torch.uint8, device=dev)
+                    eng.select(cache, w.q[0], seq, idx, cnt, None, ws)
+                torch.cuda.synchronize()
+                assert eng.get_error() == 0
+                res[kind] = (idx.cpu(), cnt.cpu())
+            assert torch.equal(res["static"][1], res["fresh"][1]), cfg.name
+            assert torch.equal(res["static"][0], res["fresh"][0]), cfg.name
+            assert int(res["static"][1].min()) > 0
+        finally:
+            eng.close()
 
 
 @pytest.mark.gpu
