@@ -85,24 +85,35 @@ def kernel_sources_sha() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
-    summary of this workload, or None when that summary was taken from other
-    kernel sources than the ones built now (the counters would be stale)."""
-    p = os.path.join(ROOT, "profiles", "c128k_step_kernels_full.txt")
-    if not os.path.exists(p):
+def recorded_traffic(workload: str, kernel: str, algorithmic_bytes: float = 0.0):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from a
+    committed ncu summary under profiles/ -- a text file with the lines
+    ``workload: <name>``, ``kernel sources sha256: <sha>`` and
+    ``traffic_per_launch <kernel> <bytes>`` -- or None when there is no summary
+    for this workload taken from the kernel sources built now (the counters
+    would be stale).  `algorithmic_bytes` is unused; it documents what the
+    figure is compared with."""
+    del algorithmic_bytes
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
         return None
-    sha, traffic = None, {}
-    with open(p) as f:
-        for ln in f:
-            if ln.startswith("kernel sources sha256:"):
-                sha = ln.split(":", 1)[1].strip()
-            elif ln.startswith("traffic_per_launch "):
-                _, name, val = ln.split()
-                traffic[name] = int(val)
-    if sha != kernel_sources_sha():
-        return None
-    return traffic.get(kernel + "_kernel")
+    sha_now = kernel_sources_sha()
+    for name in sorted(os.listdir(d)):
+        if not name.endswith(".txt"):
+            continue
+        wl, sha, traffic = None, None, {}
+        with open(os.path.join(d, name)) as f:
+            for ln in f:
+                if ln.startswith("workload:"):
+                    wl = ln.split(":", 1)[1].strip()
+                elif ln.startswith("kernel sources sha256:"):
+                    sha = ln.split(":", 1)[1].strip()
+                elif ln.startswith("traffic_per_launch "):
+                    parts = ln.split()
+                    traffic[parts[1]] = int(parts[2])
+        if wl == workload and sha == sha_now and kernel in traffic:
+            return traffic[kernel]
+    return None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -349,17 +360,24 @@ def run_dashkv(args, cfg, world, rank, local):
     K = args.steps
     T = min(K, args.trace_steps)
     n_sel_kernels = eng.select_kernels(cache.capacity)
-    sel_names = ["select_fused"] if n_sel_kernels == 1 else ["score_hist", "collect_select"]
-    dom = sel_names[0]  # the kernel that streams the codes (of the tokens, or of the block summaries)
+    sel_names = ["select_step"] if n_sel_kernels == 1 else ["score_hist", "collect_select"]
+    # the whole step as one clustered launch (dashkv_decode_step) for token
+    # selection on the clustered path; the separate calls otherwise
+    fused = not (cfg.block or cfg.radius or args.split_step or n_sel_kernels != 1)
     # the kernels of one step, in launch order, and the calls that launch them
-    calls = [("append_keys", ["append_keys"])]
-    if cfg.block:
-        calls += [("append_blocks", ["append_blocks"]), ("select_blocks", sel_names + ["expand_blocks"])]
-    elif cfg.radius:
-        calls += [("append_radius", ["append_radius"]), ("select_radius", ["select_fused"])]
+    if fused:
+        calls = [("decode_step", ["decode_step"])]
+        dom = "decode_step"
     else:
-        calls += [("select", sel_names)]
-    calls += [("sparse_decode", ["sparse_decode"])]
+        dom = sel_names[0]  # the kernel that streams the codes (of the tokens, or of the block summaries)
+        calls = [("append_keys", ["append_keys"])]
+        if cfg.block:
+            calls += [("append_blocks", ["append_blocks"]), ("select_blocks", sel_names + ["expand_blocks"])]
+        elif cfg.radius:
+            calls += [("append_radius", ["append_radius"]), ("select_radius", sel_names)]
+        else:
+            calls += [("select", sel_names)]
+        calls += [("sparse_decode", ["sparse_decode"])]
     kernels = [k for _, ks in calls for k in ks]
     n_graph = args.warmup + K + T
 
@@ -369,7 +387,9 @@ def run_dashkv(args, cfg, world, rank, local):
         for name, ks in calls:
             if e is not None:
                 eng.set_trace(e[2 * j:2 * (j + len(ks))])
-            if name == "append_keys":
+            if name == "decode_step":
+                eng.decode_step(cache, q, kn, vn, seq, buf["sel_idx"], buf["sel_cnt"], out, lse, ws)
+            elif name == "append_keys":
                 eng.append_keys(cache, kn, vn, seq)
             elif name == "append_blocks":
                 eng.append_blocks(cache, index, seq)
@@ -460,8 +480,13 @@ def run_dashkv(args, cfg, world, rank, local):
     step_bytes = code_bytes + kv_bytes + qo_bytes
     peaks = measured_peaks()
     kms = {k: statistics.mean(v) for k, v in kern.items()}
-    score_gbs = code_bytes / (kms[dom] * 1e-3) / 1e9
-    decode_gbs = kv_bytes / (kms["sparse_decode"] * 1e-3) / 1e9
+    # the roofline kernel: the fused step kernel moves every byte of the step;
+    # on the split path the selection kernel moves the codes
+    dom_bytes = step_bytes if fused else code_bytes
+    dom_gbs = dom_bytes / (kms[dom] * 1e-3) / 1e9
+    kernel_gbs = {dom: dom_gbs}
+    if "sparse_decode" in kms:
+        kernel_gbs["sparse_decode"] = kv_bytes / (kms["sparse_decode"] * 1e-3) / 1e9
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed.
@@ -533,16 +558,16 @@ def run_dashkv(args, cfg, world, rank, local):
                        "block": cfg.block or None, "radius": cfg.radius or None,
                        "layout": "paged" if w.paged else "dense", "l2": "flushed before every step: 2 x L2 write, then 2 x L2 clean read (no pending write-backs)",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": score_gbs,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": score_gbs / peaks["hbm_gbs"],
-                         "peak_source": peaks["source"], "frac_of_8tbs": score_gbs / SPEC_HBM_GBS,
-                         "algorithmic_bytes_per_launch": code_bytes,
-                         "traffic": recorded_traffic(dom) if cfg.name == "c128k" else None},
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dom_gbs / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"], "frac_of_8tbs": dom_gbs / SPEC_HBM_GBS,
+                         "algorithmic_bytes_per_launch": dom_bytes,
+                         "traffic": recorded_traffic(cfg.name, dom, dom_bytes)},
             "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_gbs,
                               "frac": step_gbs / peaks["hbm_gbs"], "frac_of_8tbs": step_gbs / SPEC_HBM_GBS,
                               "code_bytes": code_bytes, "selected_kv_bytes": kv_bytes, "q_out_bytes": qo_bytes},
             "kernels_ms": kms,
-            "kernel_gbs": {dom: score_gbs, "sparse_decode": decode_gbs},
+            "kernel_gbs": kernel_gbs,
             "per_head_queries_per_s": value * cfg.Hq,
             "warm_ms_per_step": warm_ms,
             "encode": encode,
@@ -566,7 +591,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-steps", type=int, default=2)
     ap.add_argument("--two-kernel-select", action="store_true",
-                    help="use the two-kernel selection path")
+                    help="use the two-kernel selection path (and the separate calls)")
+    ap.add_argument("--split-step", action="store_true",
+                    help="time append_keys + select + sparse_decode instead of the one-launch decode step")
     ap.add_argument("--trace-steps", type=int, default=10,
                     help="extra traced steps for the per-kernel durations")
     ap.add_argument("--clock-reps", type=int, default=20,

@@ -16,8 +16,11 @@ constexpr int kSmCountFallback = 148;
 constexpr int kSyncStride = 32;
 
 // Device error word (one per device that loads the library).  Bits:
-enum : unsigned { kErrCapacity = 1u, kErrPage = 2u };
-__device__ unsigned g_error_word;
+// kErrTimeout: a bounded wait on a shared-memory barrier gave up (a bulk copy
+// did not complete in time); the affected results are not valid.
+enum : unsigned { kErrCapacity = 1u, kErrPage = 2u, kErrTimeout = 4u };
+// Defined once, in dashkv.cu (the library is built with relocatable device code).
+extern __device__ unsigned g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }
 
@@ -62,6 +65,49 @@ __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
                  : "r"(addr)
                  : "memory");
     return v;
+}
+
+// ---- shared-memory barriers and bulk copies (global -> this CTA's shared
+// memory, completion counted in bytes on an mbarrier; never multicast).
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+// Make barrier initialisation visible to the async proxy (bulk copies).
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+// Copy `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
+// memory into this CTA's shared memory; completion is signalled on `mbar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+// Bounded wait for the phase of parity `parity` of `mbar` to complete.  Gives
+// up after about kMbarSpins polls (each may suspend for up to kMbarSuspendNs),
+// sets the timeout bit of the error word and returns false.
+constexpr int kMbarSpins = 1 << 20;
+constexpr uint32_t kMbarSuspendNs = 256;
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+    for (int it = 0; it < kMbarSpins; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity), "r"(kMbarSuspendNs)
+            : "memory");
+        if (done) return true;
+    }
+    raise_error(kErrTimeout);
+    return false;
 }
 
 // Hyperplanes as sign bits: bit (i % 32) of word [j * (d / 32) + i / 32] is set
@@ -171,15 +217,21 @@ __device__ __forceinline__ void rotate_bytes(uint32_t (&w)[NW], bool by8, bool b
 // in byte j/8 bit j%8) is stored with its bytes rotated by t mod T: stored byte
 // p holds code byte (p + t mod T) mod T.  The scorer's lane that handles token t
 // reads its bytes in exactly that order, so the swizzle replaces a per-token
-// register rotation.  w: the code as BITS/32 little-endian 32-bit words.
+// register rotation.  w: the code as BITS/32 little-endian 32-bit words;
+// rotate_code() turns them into the stored order in registers.
+template <int BITS>
+__device__ __forceinline__ void rotate_code(uint32_t (&w)[BITS / 32], int64_t t) {
+    constexpr int NW = BITS / 32;
+    const int rho = (int)(t % (BITS / 8));
+    rotate_bytes<NW>(w, (rho & 8) != 0, (rho & 4) != 0, 8u * (uint32_t)(rho & 3));
+}
 template <int BITS>
 __device__ __forceinline__ void store_code_rotated(uint64_t *dst, const uint32_t (&w)[BITS / 32], int64_t t) {
     constexpr int NW = BITS / 32;
-    const int rho = (int)(t % (BITS / 8));
     uint32_t r[NW];
 #pragma unroll
     for (int k = 0; k < NW; ++k) r[k] = w[k];
-    rotate_bytes<NW>(r, (rho & 8) != 0, (rho & 4) != 0, 8u * (uint32_t)(rho & 3));
+    rotate_code<BITS>(r, t);
     if constexpr (NW == 1) {
         dst[0] = (uint64_t)r[0];
     } else {

@@ -18,6 +18,11 @@
 #include "encode.cuh"
 #include "radius.cuh"
 #include "select.cuh"
+#include "step_args.cuh"
+
+namespace dkv {
+__device__ unsigned g_error_word;  // the device error word (declared in common.cuh)
+}  // namespace dkv
 
 using namespace dkv;
 
@@ -26,7 +31,8 @@ struct dashkv_ctx {
     RBits R;
     int device;
     int sm_count;
-    int cluster_max;  // CTAs per (b, h) cluster of the fused selection; 0: no cluster launch
+    int cluster_max;  // CTAs per (b, h) cluster of the clustered step kernel; 0: no cluster launch
+    int step_smem;    // dynamic shared memory of a step-kernel launch (the opt-in maximum minus static)
     int force_two_kernel;
     void **trace;   // optional cudaEvent_t pairs around each kernel of a call
     int n_trace;
@@ -164,9 +170,10 @@ int64_t view_capacity(const dashkv_ctx *ctx, const dashkv_kv_view *kv) {
     return ctx->cfg.page_size ? (int64_t)kv->max_pages * ctx->cfg.page_size : kv->n_cap;
 }
 
-// ---- workspace: [scores | cand | ckey | hist | state | arrive(3 x BH lines) | seg_cnt | partials | block ids]
+// ---- workspace: [scores | cand | ckey | hist | state | arrive(3 x BH lines) | seg_cnt | partials | block ids |
+// per-sequence arrival lines]
 struct WsLayout {
-    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, blk, total;
+    size_t scores, cand, ckey, hist, state, arrive, seg_cnt, part, blk, seqarr, total;
 };
 
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -189,6 +196,7 @@ WsLayout ws_layout(const dashkv_config &c, int64_t max_tokens) {
     L.seg_cnt = o; o = align_up(o + BH * kMaxSelCtas * 4);
     L.part = o;    o = align_up(o + BH * kMaxSplits * G * (c.head_dim + 2) * 4);
     L.blk = o;     o = align_up(o + BH * ((size_t)c.topk + 1) * 4);  // selected block ids + counts
+    L.seqarr = o;  o = align_up(o + (size_t)c.batch * kSyncStride * 4);  // decode step: clusters done with a length
     L.total = o;
     return L;
 }
@@ -241,16 +249,59 @@ int attn_splits(const dashkv_ctx *ctx) {
 // leave room for the low region below 64 KB.
 template <int BITS, int D>
 bool score_layout_ok() {
-    cudaFuncAttributes a[6];
+    cudaFuncAttributes a[2];
     cudaFuncGetAttributes(&a[0], score_hist_kernel<BITS, D, false>);
     cudaFuncGetAttributes(&a[1], score_hist_kernel<BITS, D, true>);
-    cudaFuncGetAttributes(&a[2], select_fused_kernel<BITS, D, false>);
-    cudaFuncGetAttributes(&a[3], select_fused_kernel<BITS, D, true>);
-    cudaFuncGetAttributes(&a[4], select_fused_kernel<BITS, D, false, true>);
-    cudaFuncGetAttributes(&a[5], select_fused_kernel<BITS, D, true, true>);
     for (auto &x : a)
         if (x.sharedSizeBytes + 1024 + ScoreShape<BITS>::LOW_BYTES > 65536) return false;
     return true;
+}
+
+// ---- the clustered step kernel (instantiated in step_inst.cu)
+StepKern step_kern(int bits, int d, int G, bool paged, bool radius) {
+    if (d == 64) {
+        if (bits == 32) return step_kern_32_64(G, paged, radius);
+        if (bits == 64) return step_kern_64_64(G, paged, radius);
+        return step_kern_128_64(G, paged, radius);
+    }
+    if (bits == 32) return step_kern_32_128(G, paged, radius);
+    if (bits == 64) return step_kern_64_128(G, paged, radius);
+    return step_kern_128_128(G, paged, radius);
+}
+
+// Dynamic shared memory of the context's step kernels (the device's per-block
+// opt-in maximum minus their static part; the kernels lay out what they get),
+// with the attributes their launches need; 0 when a kernel cannot get enough.
+int setup_step_kernels(const dashkv_ctx *c) {
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
+    int smem = optin;
+    StepKern ks[6];
+    int nk = 0;
+    for (int paged = 0; paged < 2; ++paged) {
+        ks[nk++] = step_kern(c->cfg.bits, c->cfg.head_dim, 0, paged, false);
+        ks[nk++] = step_kern(c->cfg.bits, c->cfg.head_dim, 0, paged, true);
+        ks[nk++] = step_kern(c->cfg.bits, c->cfg.head_dim, G, paged, false);
+    }
+    for (int i = 0; i < nk; ++i) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, ks[i]) != cudaSuccess) { cudaGetLastError(); return 0; }
+        if (optin - (int)fa.sharedSizeBytes < smem) smem = optin - (int)fa.sharedSizeBytes;
+    }
+    // the layout needs the low region below the LUT's 64 KB boundary, the LUT, the
+    // code ring and some candidate room above it
+    const int ring = kStepWarps * kRingStages * 32 * (c->cfg.bits >= 64 ? c->cfg.bits / 8 : 8);
+    if (smem < 2 * 65536 + ring + 4096) return 0;
+    for (int i = 0; i < nk; ++i) {
+        cudaFuncSetAttribute(ks[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaFuncSetAttribute(ks[i], cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    }
+    if (cudaGetLastError() != cudaSuccess) return 0;
+    return smem;
 }
 
 template <int BITS, int D>
@@ -263,16 +314,6 @@ void set_attrs_bd() {
                          (int)ScoreShape<BITS>::SMEM);
     cudaFuncSetAttribute(score_hist_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)ScoreShape<BITS>::SMEM);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)ScoreShape<BITS>::SMEM);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)ScoreShape<BITS>::SMEM);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)ScoreShape<BITS>::SMEM);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)ScoreShape<BITS>::SMEM);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
 }
 
 template <int D, int G>
@@ -376,25 +417,23 @@ int fused_cluster(const dashkv_ctx *ctx, int64_t cap) {
 }
 
 // Largest cluster size C <= kMaxCluster for which all B * Hkv clusters of the
-// fused selection are resident at once (one wave, one CTA per SM); 1 when
-// even single CTAs need several waves; 0 without cluster launch support.
-template <int BITS, int D>
+// step kernel are resident at once (one wave, one CTA per SM); 1 when even
+// single CTAs need several waves; 0 without cluster launch support.
 int pick_cluster(const dashkv_ctx *ctx) {
     int ok = 0;
-    if (cudaDeviceGetAttribute(&ok, cudaDevAttrClusterLaunch, ctx->device) != cudaSuccess || !ok) {
+    if (!ctx->step_smem || cudaDeviceGetAttribute(&ok, cudaDevAttrClusterLaunch, ctx->device) != cudaSuccess || !ok) {
         cudaGetLastError();
         return 0;
     }
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    const StepKern kern = step_kern(ctx->cfg.bits, ctx->cfg.head_dim, 0, false, false);
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     int c = ctx->sm_count / BH;
     if (c > kMaxCluster) c = kMaxCluster;
     for (; c > 1; --c) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(c, BH);
-        cfg.blockDim = dim3(kScoreThreads);
-        cfg.dynamicSmemBytes = ScoreShape<BITS>::SMEM;
+        cfg.blockDim = dim3(kStepThreads);
+        cfg.dynamicSmemBytes = ctx->step_smem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = c;
@@ -403,28 +442,20 @@ int pick_cluster(const dashkv_ctx *ctx) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, select_fused_kernel<BITS, D, false>, &cfg) == cudaSuccess &&
-            nclusters >= BH)
-            break;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess && nclusters >= BH) break;
         cudaGetLastError();
     }
     return c < 1 ? 1 : c;
 }
 
-// Fused selection: a grid of (C, B * Hkv) CTAs in clusters of C (one cluster
-// per (b, h)) that may also start early behind the preceding kernel.
-template <int BITS, int D>
-void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
-                     int nctas, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
+// The step kernel on a grid of (C, B * Hkv) CTAs in clusters of C (one
+// cluster per (b, h)), allowed to start early behind the preceding kernel.
+void launch_step(const dashkv_ctx *ctx, StepKern kern, int nctas, const StepArgs &args, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
-    const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
-    auto kern = kv.radius ? (kv.page_size ? select_fused_kernel<BITS, D, true, true>
-                                          : select_fused_kernel<BITS, D, false, true>)
-                          : (kv.page_size ? select_fused_kernel<BITS, D, true> : select_fused_kernel<BITS, D, false>);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nctas, BH);
-    cfg.blockDim = dim3(kScoreThreads);
-    cfg.dynamicSmemBytes = ScoreShape<BITS>::SMEM;
+    cfg.blockDim = dim3(kStepThreads);
+    cfg.dynamicSmemBytes = ctx->step_smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -435,18 +466,36 @@ void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaLaunchKernelEx(&cfg, kern, kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R,
-                       ws, a.topk, a.sink, a.window, a.cap_sel, sel_idx, sel_cnt);
+    cudaLaunchKernelEx(&cfg, kern, args, ctx->R);
 }
 
-template <int D>
-void launch_fused_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
-                    int nctas, const SelArgs &a, int32_t *si, int32_t *sc, cudaStream_t st) {
-    switch (ctx->cfg.bits) {
-        case 32: launch_fused_bd<32, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
-        case 64: launch_fused_bd<64, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
-        default: launch_fused_bd<128, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
-    }
+// Arguments of a selection-only step launch over `kv` (token codes or block
+// summaries).
+StepArgs select_args(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                     const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, float *scores, int64_t ld_out) {
+    StepArgs s = {};
+    s.kv = kv;
+    s.q = static_cast<const __nv_bfloat16 *>(q);
+    s.Hq = ctx->cfg.num_q_heads;
+    s.G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
+    s.seq_lens = const_cast<int32_t *>(seq);  // not written without an append
+    s.k_new = nullptr;
+    s.v_new = nullptr;
+    s.ws = ws;
+    s.topk = a.topk;
+    s.S = a.sink;
+    s.W = a.window;
+    s.cap_sel = a.cap_sel;
+    s.sel_idx = sel_idx;
+    s.sel_cnt = sel_cnt;
+    s.scores_out = scores;
+    s.ld_out = ld_out;
+    s.out = nullptr;
+    s.lse = nullptr;
+    s.scale_log2 = 0.0f;
+    s.seq_arrive = nullptr;
+    s.smem_bytes = ctx->step_smem;
+    return s;
 }
 
 template <int D>
@@ -505,13 +554,8 @@ void launch_decode_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const i
 }
 
 
-// One selection over `k` (the token cache, or the block codes): the fused
-// kernel, or score + collect; then the optional copy of the scores (rows of
-// length cap).  The workspace is carved as L lays it out.
-void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout &L, char *w, const void *q,
-                const int32_t *seq_lens, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
-                Tracer &tr, cudaStream_t st) {
-    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+// The selection's view of a workspace laid out by L for rows of `cap` tokens.
+SelWS carve_selws(const WsLayout &L, char *w, int64_t cap, float *scores) {
     SelWS ws;
     ws.scores = reinterpret_cast<float *>(w + L.scores);
     ws.ld = row_ld(cap);
@@ -523,6 +567,17 @@ void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout 
     ws.state = reinterpret_cast<SelState *>(w + L.state);
     ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive);
     ws.seg_cnt = reinterpret_cast<int32_t *>(w + L.seg_cnt);
+    return ws;
+}
+
+// One selection over `k` (the token cache, or the block codes): the clustered
+// step kernel (selection only), or score + collect followed by the optional
+// copy of the scores (rows of length cap).  The workspace is carved as L lays it out.
+void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout &L, char *w, const void *q,
+                const int32_t *seq_lens, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
+                Tracer &tr, cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const SelWS ws = carve_selws(L, w, cap, scores);
     const int nscore = sel_ctas(ctx, cap, 1);    // score kernel: one 1024-thread CTA per SM
     const int ncollect = sel_ctas(ctx, cap, 2);  // collect kernel: two 512-thread CTAs per SM
     auto copy_scores = [&]() {
@@ -534,11 +589,11 @@ void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout 
     };
     if (use_fused(ctx)) {
         const int nc = fused_cluster(ctx, cap);
+        const StepArgs s = select_args(ctx, k, q, seq_lens, ws, a, sel_idx, sel_cnt, scores, cap);
         tr.before();
-        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nc, a, sel_idx, sel_cnt, st);
-        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nc, a, sel_idx, sel_cnt, st);
+        launch_step(ctx, step_kern(ctx->cfg.bits, ctx->cfg.head_dim, 0, k.page_size != 0, k.radius != nullptr), nc, s,
+                    st);
         tr.after();
-        copy_scores();
         return;
     }
     tr.before();
@@ -684,6 +739,7 @@ const char *dashkv_status_str(dashkv_status s) {
         case DASHKV_ERR_CUDA: return "CUDA error";
         case DASHKV_ERR_DEVICE: return "page id out of range";
         case DASHKV_ERR_NO_DEVICE: return "no CUDA device";
+        case DASHKV_ERR_TIMEOUT: return "a bounded wait in a kernel gave up";
     }
     return "unknown status";
 }
@@ -717,10 +773,8 @@ dashkv_status dashkv_create(const dashkv_config *cfg, dashkv_ctx **out) {
     c->force_two_kernel = (cfg->flags & DASHKV_FLAG_TWO_KERNEL_SELECT) != 0;
     build_rbits(cfg->seed, cfg->bits, cfg->head_dim, &c->R);
     set_attrs();
-    c->cluster_max =
-        cfg->head_dim == 64
-            ? (cfg->bits == 32 ? pick_cluster<32, 64>(c) : cfg->bits == 64 ? pick_cluster<64, 64>(c) : pick_cluster<128, 64>(c))
-            : (cfg->bits == 32 ? pick_cluster<32, 128>(c) : cfg->bits == 64 ? pick_cluster<64, 128>(c) : pick_cluster<128, 128>(c));
+    c->step_smem = setup_step_kernels(c);
+    c->cluster_max = pick_cluster(c);
     const bool layout_ok =
         cfg->head_dim == 64
             ? (cfg->bits == 32 ? score_layout_ok<32, 64>() : cfg->bits == 64 ? score_layout_ok<64, 64>() : score_layout_ok<128, 64>())
@@ -840,6 +894,46 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
     const int64_t cap = view_capacity(ctx, kv);
     if (ctx->cfg.head_dim == 64) launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
     else launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
+    tr.after();
+    return launch_status();
+}
+
+dashkv_status dashkv_decode_step(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q, const void *k_new,
+                                 const void *v_new, int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
+                                 float *out, float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!ctx || !q || !k_new || !v_new || !seq_lens || !sel_idx || !sel_cnt || !out || !aligned(q, 16) ||
+        !aligned(k_new, 16) || !aligned(v_new, 16))
+        return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, true);
+    if (s != DASHKV_OK) return s;
+    const int64_t cap = view_capacity(ctx, kv);
+    const WsLayout L = ws_layout(ctx->cfg, cap);
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
+    if (!use_fused(ctx)) {  // the three calls, one after the other
+        s = dashkv_append_keys(ctx, kv, k_new, v_new, seq_lens, stream);
+        if (s == DASHKV_OK)
+            s = dashkv_select(ctx, kv, q, seq_lens, sel_idx, sel_cnt, nullptr, workspace, workspace_bytes, stream);
+        if (s == DASHKV_OK)
+            s = dashkv_sparse_decode(ctx, kv, q, seq_lens, sel_idx, sel_cnt, out, lse, workspace, workspace_bytes,
+                                     stream);
+        return s;
+    }
+    char *w = static_cast<char *>(workspace);
+    const SelArgs a{ctx->cfg.topk, ctx->cfg.sink, ctx->cfg.window, ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window};
+    StepArgs args = select_args(ctx, make_kv(ctx, kv), q, seq_lens, carve_selws(L, w, cap, nullptr), a, sel_idx,
+                                sel_cnt, nullptr, cap);
+    args.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    args.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    args.out = out;
+    args.lse = lse;
+    args.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
+    args.seq_arrive = reinterpret_cast<uint32_t *>(w + L.seqarr);
+    const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    launch_step(ctx, step_kern(ctx->cfg.bits, ctx->cfg.head_dim, G, ctx->cfg.page_size != 0, false),
+                fused_cluster(ctx, cap), args, st);
     tr.after();
     return launch_status();
 }
@@ -976,6 +1070,7 @@ dashkv_status dashkv_get_error(void *stream) {
     unsigned w = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return DASHKV_ERR_CUDA;
     if (w && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return DASHKV_ERR_CUDA;
+    if (w & kErrTimeout) return DASHKV_ERR_TIMEOUT;
     if (w & kErrPage) return DASHKV_ERR_DEVICE;
     if (w & kErrCapacity) return DASHKV_ERR_CAPACITY;
     return DASHKV_OK;

@@ -1,0 +1,926 @@
+// step.cuh -- one decode step in one kernel: (append the step's key) -> score
+// every cached key from its code -> exact top-k united with sinks and window
+// -> (exact attention over the selection).
+//
+// DASH-KV page, "DASH-KV的核心创新：非对称深度哈希" (the query stays in full
+// precision, keys are hashed) and "从平方到线性" (hash codes, then top-K
+// candidate pruning); Spherical KV page, section 2.1 ADA (logits straight from
+// the packed codes); DeepSeek DSA->CSA/HCA page, "从 DSA 说起" (an indexer
+// scores the whole history, attention runs on the top-k only) and the SWA
+// paragraph of its CSA section (a recent window stays exact); DySCO page, Q3
+// (attention sinks).
+//
+// Grid: one thread-block cluster of C CTAs (1024 threads, one per SM) per
+// (sequence, kv head); CTA c owns a contiguous, 64-aligned token range and
+// warp w of it a contiguous, 32-aligned sub-range.
+//
+//  stream   every warp streams its codes through a private ring of 32-token
+//           chunks filled by bulk copies (cp.async.bulk, completion on an
+//           mbarrier, issued by lane 0 a few chunks ahead); lane l scores the
+//           tokens t = l (mod 32) with the byte-LUT of the query (the codes are
+//           stored byte-rotated by t mod T, see store_code_rotated).  A token
+//           whose histogram bin reaches the CTA's running threshold is kept
+//           with its exact order key in the warp's candidate list in shared
+//           memory and counted in the CTA histogram; the running threshold is
+//           the bin of the CTA's k-th largest score so far (never above the
+//           final one), so every token that can be selected is kept and the
+//           histogram is exact for every bin at or above the final threshold.
+//  select   the cluster sums its histograms through distributed shared
+//           memory and finds the bin T1 holding the k-th largest score; the
+//           warps classify their candidates, rank the few of bin T1 exactly
+//           (score desc, index asc) and write the ascending selection.  Heavy
+//           ties (more than kInbinMax tokens in T1) or a full candidate list
+//           take an exact slow path (re-score into the workspace, CTA 0 runs
+//           the two-kernel path's resolver).
+//  attend   (G > 0) every CTA takes an equal slice of the emitted list, bulk
+//           copies the K and V rows into shared memory (two tiles in flight
+//           per warp) and runs an online softmax in fp32; the CTAs' partial
+//           states are merged through distributed shared memory.
+//  append   (k_new given) the CTA that owns position seq_lens[b] encodes the
+//           new key, writes its code and K/V rows there and scores it from
+//           the code it computed; the last cluster of a sequence to pass its
+//           first cluster barrier increments seq_lens[b].
+#pragma once
+#include "decode.cuh"
+#include "select.cuh"
+#include "step_args.cuh"
+
+namespace dkv {
+
+// Bin of the CTA's kk-th largest counted score from its super-bin and bin
+// counts (one full warp; 0 when fewer than kk are counted).  Counts only grow
+// while this runs, so a stale read can only give a lower bin.
+__device__ __forceinline__ int local_threshold(const uint32_t *sup, const uint32_t *hist, int64_t kk) {
+    const int lane = threadIdx.x & 31;
+    const volatile uint32_t *vs = sup;
+    const volatile uint32_t *vh = hist;
+    const uint32_t cu = vs[63 - 2 * lane], cl = vs[62 - 2 * lane];
+    int64_t incl = (int64_t)cu + cl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int64_t excl = incl - cu - cl;
+    const bool here = excl < kk && kk <= incl;
+    const uint32_t hb = __ballot_sync(0xffffffffu, here);
+    if (!hb) return 0;
+    int sb = 0;
+    int64_t above = 0;
+    if (here) {
+        if (excl + cu >= kk) { sb = 63 - 2 * lane; above = excl; }
+        else { sb = 62 - 2 * lane; above = excl + cu; }
+    }
+    const int src = __ffs(hb) - 1;
+    sb = __shfl_sync(0xffffffffu, sb, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    const int bu = 64 * sb + 63 - 2 * lane, bl = bu - 1;
+    const uint32_t fu = vh[bu], fl = vh[bl];
+    int64_t fincl = (int64_t)fu + fl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, fincl, o);
+        if (lane >= o) fincl += y;
+    }
+    const int64_t fexcl = above + fincl - fu - fl;
+    fincl += above;
+    const bool hit = fexcl < kk && kk <= fincl;
+    const uint32_t hm = __ballot_sync(0xffffffffu, hit);
+    if (!hm) return 64 * sb;  // counts moved under the read: the super-bin's floor is still a lower bound
+    const int t = hit ? (fexcl + fu >= kk ? bu : bl) : 0;
+    return __shfl_sync(0xffffffffu, t, __ffs(hm) - 1);
+}
+
+// fp32 LUT score of one token's (rotated) code words for a token t (any lane):
+// lane offset t mod 32 keeps the table order right (t mod T = lane mod T).
+template <int BITS>
+__device__ __forceinline__ float lut_score_any(const uint32_t (&w)[BITS / 32], uint32_t lut_s, int64_t t) {
+    return lut_score<BITS>(w, lut_s | (4u * (uint32_t)(t & 31)));
+}
+
+// Code words of token t of (b, h) loaded with a plain load (slow paths), or
+// false when its page is out of range.
+template <int BITS>
+__device__ __forceinline__ bool load_code_plain(const KV &kv, int b, int h, int64_t t, uint32_t (&w)[BITS / 32]) {
+    const int64_t c = kv.code(b, h, t);
+    if (c < 0) return false;
+    if constexpr (BITS == 128) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(kv.codes + c));
+        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+    } else if constexpr (BITS == 64) {
+        const uint2 x = __ldg(reinterpret_cast<const uint2 *>(kv.codes + c));
+        w[0] = x.x; w[1] = x.y;
+    } else {
+        w[0] = __ldg(reinterpret_cast<const uint32_t *>(kv.codes + c));
+    }
+    return true;
+}
+
+// r~ = (c + 1/2) / 4 of token t's radius code (radius-scaled scores).
+__device__ __forceinline__ float radius_of_token(const KV &kv, int b, int h, int64_t t) {
+    const int64_t r = kv.radius_index(b, h, t);
+    return r >= 0 ? ((float)__ldg(kv.radius + r) + 0.5f) * 0.25f : 0.0f;
+}
+
+template <int BITS, int D, int G, bool PAGED, bool RADIUS>
+__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, const RBits R) {
+    using SS = StepShape<BITS>;
+    constexpr int NS = kRingStages;
+    constexpr int NWARP = kStepWarps, NT = kStepThreads;
+    constexpr int CODE_B = SS::CODE_B, CHUNK_B = SS::CHUNK_B;
+    constexpr int T = BITS / 8;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const KV &kv = a.kv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.y, cta = blockIdx.x, nctas = gridDim.x;
+    const int b = bh / kv.Hkv, h = bh % kv.Hkv;
+    const uint32_t lt = (1u << lane) - 1u;
+
+    const uint32_t smem_s = (uint32_t)__cvta_generic_to_shared(smem);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + StepLow::HIST);
+    uint32_t *sup = reinterpret_cast<uint32_t *>(smem + StepLow::SUP);
+    float *qsum = reinterpret_cast<float *>(smem + StepLow::QSUM);
+    float *Qp = reinterpret_cast<float *>(smem + StepLow::QP);
+    float *knew = reinterpret_cast<float *>(smem + StepLow::KNEW);
+    int *misc = reinterpret_cast<int *>(smem + StepLow::MISC);
+    uint32_t *newc = reinterpret_cast<uint32_t *>(smem + StepLow::NEWC);
+    uint32_t *newr = reinterpret_cast<uint32_t *>(smem + StepLow::NEWR);
+    int *s_wkeep = reinterpret_cast<int *>(smem + StepLow::WKEEP);
+    int (*s_cnt)[2] = reinterpret_cast<int (*)[2]>(smem + StepLow::CNT);
+    int *s_mid = reinterpret_cast<int *>(smem + StepLow::MID);
+    const uint32_t mbar_ring = smem_s + StepLow::MBAR + 8u * (uint32_t)(warp * NS);
+    const uint32_t mbar_att = smem_s + StepLow::MBAR_ATT + 8u * (uint32_t)(warp * 2);
+    const uint32_t lut_s = (smem_s + StepLow::END + 65535u) & ~65535u;  // 64 KB aligned
+    unsigned char *lut = smem + (lut_s - smem_s);
+    const uint32_t ring_s = lut_s + 65536u;
+    unsigned char *ring = lut + 65536;
+    const uint32_t end_s = smem_s + (uint32_t)a.smem_bytes;
+    // candidate list of this warp: cap_lo entries below the LUT, cap_hi above the ring
+    const int cap_lo = (int)((lut_s - (smem_s + StepLow::END)) / (8u * NWARP));
+    const int cap_hi = end_s > ring_s + SS::RING_B ? (int)((end_s - ring_s - SS::RING_B) / (8u * NWARP)) : 0;
+    uint2 *cand_lo = reinterpret_cast<uint2 *>(smem + StepLow::END) + warp * cap_lo;
+    uint2 *cand_hi = reinterpret_cast<uint2 *>(ring + SS::RING_B) + warp * cap_hi;
+    const int cap = cap_lo + cap_hi;
+    auto cand_ref = [&](int j) -> uint2 & { return j < cap_lo ? cand_lo[j] : cand_hi[j - cap_lo]; };
+
+    // ---- set-up: counters, barriers, this warp's hyperplane words
+    for (int i = tid; i < kBins; i += NT) hist[i] = 0;
+    if (tid < 64) { sup[tid] = 0; misc[tid] = 0; }
+    if (tid < NWARP * NS) mbar_init(smem_s + StepLow::MBAR + 8u * tid, 1);
+    if (tid < NWARP * 2) mbar_init(smem_s + StepLow::MBAR_ATT + 8u * tid, 1);
+    if (tid < NWARP * NS || tid < NWARP * 2) fence_mbar_init();
+    static_assert(BITS % NWARP == 0, "hyperplanes per warp");
+    uint32_t rw[BITS / NWARP][D / 32];
+#pragma unroll
+    for (int m = 0; m < BITS / NWARP; ++m)
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) rw[m][k] = R.w[(warp + NWARP * m) * (D / 32) + k];
+
+    // everything the kernel reads may come from the preceding kernel of the stream
+    griddep_wait();
+    griddep_trigger();
+
+    // ---- lengths (and the append's position)
+    const bool appending = a.k_new != nullptr;
+    const int64_t capn = kv.capacity();
+    int64_t pos = -1;  // position of the appended token, or -1
+    int64_t n;
+    bool app_ok = false;
+    if (appending) {
+        const int64_t p0 = __ldcg(a.seq_lens + b);
+        app_ok = p0 >= 0 && p0 < capn;
+        if (app_ok && PAGED) {
+            const int32_t pg = __ldg(kv.page_table + (int64_t)b * kv.max_pages + p0 / kv.page_size);
+            app_ok = pg >= 0 && pg < kv.num_pages;
+            if (!app_ok && cta == 0 && tid == 0) raise_error(kErrPage);
+        } else if (!app_ok && cta == 0 && tid == 0) {
+            raise_error(kErrCapacity);
+        }
+        if (app_ok) pos = p0;
+        n = app_ok ? p0 + 1 : (p0 < 0 ? 0 : (p0 > capn ? capn : p0));
+    } else {
+        n = clamp_len(kv, a.seq_lens, b);
+    }
+    int64_t t0, t1;
+    cta_range(n, cta, nctas, t0, t1);
+    const int nloc = (int)(t1 - t0);
+    const int wlen = (int)(ceil_div(ceil_div(nloc, NWARP), 32) * 32);
+    const int wb = warp * wlen;
+    const int we = min(nloc, wb + wlen);
+    const int nk = we > wb ? (we - wb + 31) / 32 : 0;  // chunks of this warp
+    const bool own_new = pos >= t0 && pos < t1;
+
+    // ---- issue the first chunks now: their latency overlaps the LUT build
+    const unsigned char *codes_b = reinterpret_cast<const unsigned char *>(kv.codes);
+    const int64_t dense_row = ((int64_t)bh * kv.n_cap + t0 + wb) * CODE_B;  // byte offset of the warp's first code
+    // PAGED: the page ids of the chunks of groups gA, gA + 1 and gA + 2 (lane l
+    // of register pg[i] holds chunk 32 (gA + i) + l), loaded a group ahead of use
+    auto chunk_page = [&](int c) -> int {  // -1: no chunk, -2: page id out of range
+        if (c >= nk) return -1;
+        const int64_t t = t0 + wb + 32 * (int64_t)c;
+        const int32_t p = __ldg(kv.page_table + (int64_t)b * kv.max_pages + t / kv.page_size);
+        if (p < 0 || p >= kv.num_pages) return -2;
+        return p;
+    };
+    int pgA = 0, pgB = 0, pgC = 0, gA = 0;
+    if constexpr (PAGED) {
+        pgA = chunk_page(lane);
+        pgB = chunk_page(32 + lane);
+        pgC = chunk_page(64 + lane);
+    }
+    auto page_of_chunk = [&](int c) -> int {  // every lane calls; c in groups gA .. gA + 2
+        const int g = (c >> 5) - gA;
+        return __shfl_sync(0xffffffffu, g == 0 ? pgA : (g == 1 ? pgB : pgC), c & 31);
+    };
+    // Source of chunk c for a bulk copy, or null when its tokens are read with
+    // plain loads instead (a dense chunk running past the capacity, or an
+    // address that is not 16-byte aligned) or skipped (a bad page id: *bad).
+    // Every lane calls (the page id is shuffled from the lane that holds it).
+    auto chunk_src = [&](int c, bool &bad) -> const unsigned char * {
+        bad = false;
+        const unsigned char *src = nullptr;
+        if constexpr (PAGED) {
+            const int p = page_of_chunk(c);
+            if (p < 0) {
+                bad = true;
+                return nullptr;
+            }
+            const int64_t t = t0 + wb + 32 * (int64_t)c;
+            src = codes_b + (((int64_t)p * kv.Hkv + h) * kv.page_size + t % kv.page_size) * CODE_B;
+        } else {
+            if (t0 + wb + 32 * (int64_t)c + 32 > kv.n_cap) return nullptr;
+            src = codes_b + dense_row + (int64_t)c * CHUNK_B;
+        }
+        return (reinterpret_cast<uintptr_t>(src) & 15u) ? nullptr : src;
+    };
+    auto issue = [&](int c) {
+        const uint32_t mb = mbar_ring + 8u * (uint32_t)(c % NS);
+        const uint32_t dst = ring_s + (uint32_t)((warp * NS + c % NS) * CHUNK_B);
+        if constexpr (PAGED) {
+            if ((c >> 5) == gA + 2) {  // entering group gA + 2: drop gA, load gA + 3
+                gA += 1;
+                pgA = pgB;
+                pgB = pgC;
+                pgC = chunk_page(32 * (gA + 2) + lane);
+            }
+        }
+        bool bad;
+        const unsigned char *src = chunk_src(c, bad);
+        if (lane == 0) {
+            if (bad) raise_error(kErrPage);  // issued chunks exist: a negative id is out of range
+            if (src) {
+                mbar_arrive_expect_tx(mb, CHUNK_B);
+                bulk_g2s(dst, src, CHUNK_B, mb);
+            } else {
+                mbar_arrive(mb);  // completes the phase with no data
+            }
+        }
+    };
+    __syncthreads();  // barriers initialised
+#pragma unroll 1
+    for (int c = 0; c < NS && c < nk; ++c) issue(c);
+
+    // ---- LUT of the group's summed query (as the two-kernel scorer builds it)
+    for (int i = tid; i < D; i += NT) {
+        const __nv_bfloat16 *qh = a.q + ((int64_t)b * a.Hq + (int64_t)h * a.G) * D + i;
+        float s = 0.0f;
+        for (int g = 0; g < a.G; ++g) s += __bfloat162float(qh[(int64_t)g * D]);
+        qsum[i] = s;
+    }
+    if (own_new && tid < D) knew[tid] = __bfloat162float(a.k_new[((int64_t)b * kv.Hkv + h) * D + tid]);
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < BITS / NWARP; ++m) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) acc = fmaf(((rw[m][k] >> lane) & 1u) ? -1.0f : 1.0f, qsum[32 * k + lane], acc);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) Qp[warp + NWARP * m] = acc;
+    }
+    // the appended key's code: thread j < BITS projects it on hyperplane j (one
+    // sequential FMA chain over the dims, as the encoder; exact on grid inputs)
+    if (own_new && tid < BITS) {
+        const int j = tid;
+        float acc = 0.0f;
+#pragma unroll 4
+        for (int i = 0; i < D; ++i) {
+            const uint32_t wbits = R.w[j * (D / 32) + i / 32];
+            acc = fmaf(((wbits >> (i % 32)) & 1u) ? -1.0f : 1.0f, knew[i], acc);
+        }
+        const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
+        if (lane == 0) newc[j / 32] = word;
+    }
+    __syncthreads();
+    float inv2A;
+    {
+        float s = 0.0f;
+        for (int j = lane; j < BITS; j += 32) s += fabsf(Qp[j]);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (RADIUS) s *= kRadiusMax;
+        inv2A = s > 0.0f ? 0.5f / s : 0.0f;
+    }
+    {   // LUT rows: word j of row v holds LUT_{j mod T}[v] (see score_phase)
+        static_assert(256 % NWARP == 0 && (256 / NWARP) <= 8, "rows per warp");
+        constexpr int RPW = 256 / NWARP;
+        const int c = lane % T;
+        float qv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) qv[u] = Qp[8 * c + u];
+        const int v0 = warp * RPW;
+        float base = 0.0f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) base += ((v0 >> u) & 1) ? qv[u] : -qv[u];
+#pragma unroll
+        for (int dd = 0; dd < RPW; ++dd) {
+            float val = base;
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+                if ((dd >> u) & 1) val += 2.0f * qv[u];
+            float *row = reinterpret_cast<float *>(lut + (v0 + dd) * 256);
+            row[lane] = val;
+            row[lane + 32] = val;
+        }
+    }
+    // the appended token: its K / V rows and code go to the cache (the
+    // attention below reads its rows from k_new / v_new, and this kernel
+    // scores it from newc)
+    if (own_new) {
+        if (tid < 2 * (D / 8)) {
+            const bool isv = tid >= D / 8;
+            const int part = isv ? tid - D / 8 : tid;
+            const int64_t r = kv.row(b, h, pos);
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>((isv ? a.v_new : a.k_new) +
+                                                                  ((int64_t)b * kv.Hkv + h) * D) + part);
+            if (r >= 0) reinterpret_cast<uint4 *>((isv ? kv.v : kv.k) + r)[part] = x;
+        }
+        if (tid == 64) {
+            uint32_t w32[BITS / 32];
+#pragma unroll
+            for (int k = 0; k < BITS / 32; ++k) w32[k] = newc[k];
+            const int64_t c = kv.code(b, h, pos);
+            if (c >= 0) store_code_rotated<BITS>(kv.codes + c, w32, pos);
+            rotate_code<BITS>(w32, pos);  // the order the scorer reads codes in
+#pragma unroll
+            for (int k = 0; k < BITS / 32; ++k) newr[k] = w32[k];
+        }
+    }
+    const int64_t kk = a.topk < n ? a.topk : n;
+    const bool normal = n > 0 && kk < n;
+    if (tid == 0) misc[kMTloc] = normal ? 0 : kBins;  // kBins: nothing is kept
+    __syncthreads();  // LUT, newc, tloc ready
+
+    // ---- stream: score every token of the warp's range
+    const uint32_t lbase = lut_s | (4u * (uint32_t)lane);
+    const int upd = (int)(kk / 4 > 256 ? kk / 4 : 256);  // candidates between threshold updates
+    int ncand = 0;
+    bool ovf = false, tmo = false;
+    float *srow_out = a.scores_out ? a.scores_out + (int64_t)bh * a.ld_out + t0 : nullptr;
+    volatile int *vtloc = misc + kMTloc;
+    float rnext = 0.0f;
+    if constexpr (RADIUS) rnext = (wb + lane < we) ? radius_of_token(kv, b, h, t0 + wb + lane) : 0.0f;
+    int j = 0;
+#pragma unroll 1
+    for (; j < nk; ++j) {
+        const int slot = j % NS;
+        if (!mbar_wait(mbar_ring + 8u * slot, (uint32_t)((j / NS) & 1))) { tmo = true; break; }
+        const int i = wb + 32 * j + lane;  // CTA-local token
+        bool valid = i < we;
+        uint32_t w[BITS / 32];
+        bool bad;
+        if (chunk_src(j, bad)) {
+            const unsigned char *src = ring + (warp * NS + slot) * CHUNK_B + lane * CODE_B;
+            if constexpr (BITS == 128) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(src);
+                w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+            } else if constexpr (BITS == 64) {
+                const uint2 x = *reinterpret_cast<const uint2 *>(src);
+                w[0] = x.x; w[1] = x.y;
+            } else {
+                w[0] = *reinterpret_cast<const uint32_t *>(src);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < BITS / 32; ++k) w[k] = 0;
+            if (bad) valid = false;
+            if (valid) valid = load_code_plain<BITS>(kv, b, h, t0 + i, w);
+        }
+        if (t0 + i == pos) {
+#pragma unroll
+            for (int k = 0; k < BITS / 32; ++k) w[k] = newr[k];
+        }
+        // the chunk's codes are in registers: refill its slot
+        __syncwarp();
+        if (j + NS < nk) issue(j + NS);
+        float sc = lut_score<BITS>(w, lbase);
+        if constexpr (RADIUS) {
+            const float rc = rnext;
+            const int i2 = i + 32;
+            rnext = (j + 1 < nk && i2 < we) ? radius_of_token(kv, b, h, t0 + i2) : 0.0f;
+            sc = __fmul_rn(sc, rc);
+        }
+        if (srow_out && valid) srow_out[i] = sc;
+        const int bin = score_bin(sc, inv2A);
+        const bool isc = valid && bin >= *vtloc;
+        const uint32_t ball = __ballot_sync(0xffffffffu, isc);
+        if (ball) {
+            if (isc) {
+                atomicAdd(&hist[bin], 1u);
+                atomicAdd(&sup[bin >> 6], 1u);
+            }
+            const int nb = __popc(ball);
+            if (!ovf && ncand + nb > cap) {
+                // full: raise the threshold to the CTA's current k-th bin and drop what is below
+                const int tnew = local_threshold(sup, hist, kk);
+                if (lane == 0) atomicMax(misc + kMTloc, tnew);
+                __syncwarp();
+                const int tl = *vtloc;
+                int kept = 0;
+                for (int jb = 0; jb < ncand; jb += 32) {
+                    const int jj = jb + lane;
+                    uint2 e = make_uint2(0u, 0u);
+                    if (jj < ncand) e = cand_ref(jj);
+                    const bool keep = jj < ncand && score_bin(key_to_float(e.y), inv2A) >= tl;
+                    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+                    __syncwarp();
+                    if (keep) cand_ref(kept + __popc(kb & lt)) = e;
+                    kept += __popc(kb);
+                    __syncwarp();
+                }
+                ncand = kept;
+                if (ncand + nb > cap) {
+                    ovf = true;
+                    if (lane == 0) misc[kMOvf] = 1;
+                }
+            }
+            if (!ovf) {
+                if (isc) cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)(i - wb), float_key(sc));
+                ncand += nb;
+            }
+            int trig = 0;
+            if (lane == 0) {
+                const int old = atomicAdd(misc + kMIns, nb);
+                trig = (old / upd) != ((old + nb) / upd);
+            }
+            if (__shfl_sync(0xffffffffu, trig, 0)) {
+                const int tnew = local_threshold(sup, hist, kk);
+                if (lane == 0) atomicMax(misc + kMTloc, tnew);
+            }
+        }
+    }
+    if (tmo) {  // give the copies still in flight a bounded chance to land before the buffers are reused
+        for (int c = j; c < nk && c < j + NS; ++c) mbar_wait(mbar_ring + 8u * (c % NS), (uint32_t)((c / NS) & 1));
+        if (lane == 0) misc[kMOvf] = 1;
+        ovf = true;
+    }
+    __syncthreads();  // every warp's list and the histogram are complete
+
+    // ---- the cluster's threshold bin T1 (exact: every CTA counted every token
+    // of every bin at or above it)
+    if (tid == 0) { misc[kMT1] = kBins; misc[kMAbove] = 0; misc[kMCntT1] = 0; misc[kMNinb] = 0; }
+    cluster_sync();  // (1)
+    if (appending && cta == 0 && tid == 0) {
+        // every CTA of this cluster has read seq_lens[b]; the last cluster of
+        // the sequence to get here moves its length on
+        __threadfence();
+        const uint32_t old = atomicAdd(a.seq_arrive + (int64_t)b * kSyncStride, 1u);
+        if (old == (uint32_t)(kv.Hkv - 1)) {
+            a.seq_arrive[(int64_t)b * kSyncStride] = 0;
+            if (app_ok) a.seq_lens[b] = (int32_t)(pos + 1);
+        }
+    }
+    if (normal && warp == 0) cluster_threshold(sup, hist, nctas, kk, misc + kMT1);
+    if (warp == 1) {
+        const int f = lane < nctas ? (int)ld_cluster_u32(cluster_addr(misc + kMOvf, lane)) : 0;
+        const uint32_t any = __ballot_sync(0xffffffffu, f != 0);
+        if (lane == 0) misc[kMAnyOvf] = any != 0;
+    }
+    __syncthreads();
+    const int T1 = misc[kMT1], above1 = misc[kMAbove], cnt_T1 = misc[kMCntT1];
+    const int s_end = (int)(a.S < n ? a.S : n);
+    const int w_beg = (int)(n - a.W > s_end ? n - a.W : s_end);
+    int32_t *out = a.sel_idx + (int64_t)bh * a.cap_sel;
+    bool slow = !normal || misc[kMAnyOvf] != 0 || cnt_T1 > kInbinMax;
+
+    int total_mid = 0;
+    if (!slow) {
+        // ---- fast path: classify this warp's candidates (definite: bin > T1,
+        // in the threshold bin: listed for the cluster)
+        uint4 *s_loc = reinterpret_cast<uint4 *>(ring);              // this CTA's in-bin tokens
+        uint4 *s_inb = reinterpret_cast<uint4 *>(ring) + kInbinMax;  // the cluster's
+        int ndef = 0;
+        for (int jb = 0; jb < ncand; jb += 32) {
+            const int jj = jb + lane;
+            uint2 e = make_uint2(0u, 0u);
+            if (jj < ncand) e = cand_ref(jj);
+            const int t = (int)(t0 + wb + (int)e.x);
+            const int bin = score_bin(key_to_float(e.y), inv2A);
+            const bool inb = jj < ncand && bin == T1;
+            const bool def = jj < ncand && bin > T1 && t >= s_end && t < w_beg;
+            ndef += __popc(__ballot_sync(0xffffffffu, def)) * (lane == 0);
+            const uint32_t ib = __ballot_sync(0xffffffffu, inb);
+            if (ib) {
+                int base = 0;
+                if (lane == 0) base = atomicAdd(misc + kMNinb, __popc(ib));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const int slot = base + __popc(ib & lt);
+                if (inb && slot < kInbinMax) s_loc[slot] = make_uint4(e.y, (uint32_t)t, (uint32_t)cta, (uint32_t)warp);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
+        if (lane == 0) s_wkeep[warp] = ndef;
+        __syncthreads();
+        if (warp == 0) {  // publish (in-bin entries, definite middle tokens) into every CTA's s_cnt[cta]
+            int dsum = s_wkeep[lane];
+#pragma unroll
+            for (int o = 16; o; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+            const int ni = min(misc[kMNinb], kInbinMax);
+            if (lane < nctas) {
+                st_cluster_u32(cluster_addr(&s_cnt[cta][0], lane), (uint32_t)ni);
+                st_cluster_u32(cluster_addr(&s_cnt[cta][1], lane), (uint32_t)dsum);
+            }
+        }
+        cluster_sync();  // (2)
+        const int c1 = cnt_T1;
+        if (warp * 32 < c1) {  // thread e copies in-bin entry e from the CTA whose list holds it
+            const int ni = lane < nctas ? s_cnt[lane][0] : 0;
+            int incl = ni;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int excl = incl - ni;
+            int r = 0;
+            for (int qq = 1; qq < nctas; ++qq) r = __shfl_sync(0xffffffffu, excl, qq) <= tid ? qq : r;
+            const int off = tid - __shfl_sync(0xffffffffu, excl, r);
+            if (tid < c1) s_inb[tid] = ld_cluster_v4(cluster_addr(s_loc + off, r));
+        }
+        __syncthreads();
+        cluster_arrive();  // (3): done with the other CTAs' shared memory
+        // rank the in-bin list: the need1-th (score desc, token asc) is the last selected
+        const int need1 = (int)kk - above1;
+        if (c1 <= 32) {
+            if (warp == 0) {
+                const uint4 en = lane < c1 ? s_inb[lane] : make_uint4(0u, 0u, 0u, 0u);
+                uint32_t Tkey = 0u;
+                int IT = 0x7fffffff;
+                if (need1 < c1) {
+                    int rank = 0;
+                    for (int f = 0; f < c1; ++f) {
+                        const uint32_t kf = __shfl_sync(0xffffffffu, en.x, f);
+                        const uint32_t tf = __shfl_sync(0xffffffffu, en.y, f);
+                        rank += (kf > en.x) || (kf == en.x && tf < en.y);
+                    }
+                    const int src = __ffs(__ballot_sync(0xffffffffu, lane < c1 && rank == need1 - 1)) - 1;
+                    Tkey = __shfl_sync(0xffffffffu, en.x, src);
+                    IT = (int)__shfl_sync(0xffffffffu, en.y, src);
+                }
+                const int t = (int)en.y;
+                const bool sel = lane < c1 && t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT));
+                int mid = 0;
+                for (int r = 0; r < nctas; ++r) {
+                    const int cr = __popc(__ballot_sync(0xffffffffu, sel && (int)en.z == r));
+                    if (lane == r) mid = s_cnt[r][1] + cr;
+                }
+                if (sel && (int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
+                int before = lane < cta ? mid : 0, tot = mid;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    before += __shfl_xor_sync(0xffffffffu, before, o);
+                    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+                }
+                if (lane == 0) { misc[kMTkey] = (int)Tkey; misc[kMIT] = IT; misc[kMBefore] = before; misc[kMTotal] = tot; }
+            }
+        } else {
+            if (tid == 0) { misc[kMTkey] = 0; misc[kMIT] = 0x7fffffff; }
+            if (tid < nctas) s_mid[tid] = s_cnt[tid][1];
+            __syncthreads();
+            if (need1 < c1) {
+                for (int e = tid; e < c1; e += NT) {
+                    const uint32_t ke = s_inb[e].x, ie = s_inb[e].y;
+                    int rank = 0;
+                    for (int f = 0; f < c1; ++f) {
+                        const uint32_t kf = s_inb[f].x;
+                        rank += (kf > ke) || (kf == ke && s_inb[f].y < ie);
+                    }
+                    if (rank == need1 - 1) { misc[kMTkey] = (int)ke; misc[kMIT] = (int)ie; }
+                }
+            }
+            __syncthreads();
+            const uint32_t Tkey = (uint32_t)misc[kMTkey];
+            const int IT = misc[kMIT];
+            for (int e = tid; e < c1; e += NT) {
+                const uint4 en = s_inb[e];
+                const int t = (int)en.y;
+                if (t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT))) {
+                    atomicAdd(&s_mid[en.z], 1);
+                    if ((int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
+                }
+            }
+            __syncthreads();
+            if (tid == 0) {
+                int before = 0, tot = 0;
+                for (int r = 0; r < nctas; ++r) {
+                    before += r < cta ? s_mid[r] : 0;
+                    tot += s_mid[r];
+                }
+                misc[kMBefore] = before;
+                misc[kMTotal] = tot;
+            }
+        }
+        __syncthreads();
+        const uint32_t Tkey = (uint32_t)misc[kMTkey];
+        const int IT = misc[kMIT];
+        total_mid = misc[kMTotal];
+        // ordered emission: warp w writes its kept candidates after those of CTAs
+        // < cta and warps < w
+        int wpos = s_end + misc[kMBefore];
+        for (int w2 = 0; w2 < warp; ++w2) wpos += s_wkeep[w2];
+        for (int jb = 0; jb < ncand; jb += 32) {
+            const int jj = jb + lane;
+            uint2 e = make_uint2(0u, 0u);
+            if (jj < ncand) e = cand_ref(jj);
+            const int t = (int)(t0 + wb + (int)e.x);
+            const int bin = score_bin(key_to_float(e.y), inv2A);
+            const bool keep = jj < ncand && t >= s_end && t < w_beg &&
+                              (bin > T1 || (bin == T1 && (e.y > Tkey || (e.y == Tkey && t <= IT))));
+            const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+            if (keep) {
+                const int p = wpos + __popc(kb & lt);
+                if (p < a.cap_sel) out[p] = t;
+            }
+            wpos += __popc(kb);
+        }
+        {   // the sinks, the window and the padding, spread over the cluster's CTAs
+            const int wpos0 = s_end + total_mid;
+            const int nwin = (int)(n - w_beg);
+            const int total = min(wpos0 + nwin, a.cap_sel);
+            const int nall = s_end + nwin + (a.cap_sel - total);
+            for (int x = cta * NT + tid; x < nall; x += nctas * NT) {
+                if (x < s_end) {
+                    out[x] = x;
+                } else if (x < s_end + nwin) {
+                    const int tw = x - s_end;
+                    if (wpos0 + tw < a.cap_sel) out[wpos0 + tw] = w_beg + tw;
+                } else {
+                    out[total + (x - s_end - nwin)] = -1;
+                }
+            }
+            if (cta == 0 && tid == 0) a.sel_cnt[bh] = total;
+        }
+        cluster_wait();  // (3)
+    } else {
+        // ---- exact slow path (heavy ties, a full candidate list, or all / none
+        // selected): re-score the CTA's range into the workspace rows, list the
+        // tokens of bins >= T1 per CTA, and let CTA 0 resolve and emit.
+        float *srow = a.ws.scores + (int64_t)bh * a.ws.ld;
+        int32_t *cand = a.ws.cand + (int64_t)bh * a.ws.ld;
+        int *s_warp = s_wkeep;  // scratch for the block scan
+        int seg = 0;
+        if (normal) {
+            for (int64_t base = t0; base < t1; base += NT) {
+                const int64_t t = base + warp * 32 + lane;
+                bool flag = false;
+                if (t < t1) {
+                    uint32_t w[BITS / 32];
+                    bool ok = true;
+                    if (t == pos) {
+#pragma unroll
+                        for (int k = 0; k < BITS / 32; ++k) w[k] = newr[k];
+                    } else {
+                        ok = load_code_plain<BITS>(kv, b, h, t, w);
+                    }
+                    float sc = ok ? lut_score_any<BITS>(w, lut_s, t) : 0.0f;
+                    if constexpr (RADIUS) sc = __fmul_rn(sc, radius_of_token(kv, b, h, t));
+                    srow[t] = sc;
+                    flag = ok && score_bin(sc, inv2A) >= T1;
+                }
+                const uint32_t fb = __ballot_sync(0xffffffffu, flag);
+                int tot;
+                const int wex = block_excl_scan<NT>(lane == 0 ? __popc(fb) : 0, s_warp, &tot);
+                const int wbase = __shfl_sync(0xffffffffu, wex, 0);
+                if (flag) cand[t0 + seg + wbase + __popc(fb & lt)] = (int32_t)t;
+                seg += tot;
+            }
+        }
+        if (tid == 0) a.ws.seg_cnt[(int64_t)bh * kMaxSelCtas + cta] = seg;
+        __threadfence();
+        cluster_sync();  // (2s): segments complete
+        if (cta == 0) {
+            SelState st;
+            st.T1 = T1; st.above1 = above1; st.cnt_T1 = cnt_T1;
+            st.flags = n == 0 ? kStateEmpty : (normal ? kStateNormal : kStateAll);
+            st.inv2A = inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
+            resolve_emit<NT, 4096>(a.ws, bh, nctas, st, a.S, a.W, a.cap_sel, a.sel_idx, a.sel_cnt,
+                                   *reinterpret_cast<ResolveSmem<4096> *>(lut));
+        }
+    }
+
+    if constexpr (G > 0) {
+        // ---- attention over the emitted list: CTA c takes an equal slice of it
+        __threadfence();
+        cluster_sync();  // (4): the whole list and its count are written
+        constexpr int HG = G < 4 ? G : 4;   // query heads per warp
+        constexpr int NTEAM = G / HG;       // warp teams, each over every row for its HG heads
+        constexpr int WPT = NWARP / NTEAM;  // warps per team
+        constexpr int SL = 32 / HG;         // lanes per head: dim slices
+        constexpr int DPL = D / SL;         // dims per lane
+        constexpr int TROWS = D == 128 ? 4 : 8;
+        constexpr int ROW_B = D * 2;
+        constexpr int TILE_B = TROWS * 2 * ROW_B;
+        static_assert(DPL % 8 == 0 || DPL == 4 || DPL == 2, "dims per lane");
+        const int team = warp / WPT, wt = warp % WPT;
+        const int gl = lane / SL, sl = lane % SL;
+        const int g = team * HG + gl;
+        float qf[DPL];
+        {
+            const __nv_bfloat16 *qr = a.q + ((int64_t)b * a.Hq + (int64_t)h * G + g) * D + sl * DPL;
+#pragma unroll
+            for (int e = 0; e < DPL; e += 2) {
+                const uint32_t x = *reinterpret_cast<const uint32_t *>(qr + e);
+                qf[e] = bf16_lo(x) * a.scale_log2;
+                qf[e + 1] = bf16_hi(x) * a.scale_log2;
+            }
+        }
+        float m = -INFINITY, l = 0.0f, acc[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = 0.0f;
+        const int cnt = __ldcg(a.sel_cnt + bh);
+        const int32_t *list = a.sel_idx + (int64_t)bh * a.cap_sel;
+        const int per = (cnt + nctas - 1) / nctas;
+        const int r0 = cta * per, r1 = min(cnt, r0 + per);
+        const int ntiles = r1 > r0 ? (r1 - r0 + TROWS - 1) / TROWS : 0;
+        const uint32_t stage_s = lut_s + (uint32_t)(warp * 2 * TILE_B);
+        const unsigned char *stage = lut + warp * 2 * TILE_B;
+        const __nv_bfloat16 *kn_row = appending ? a.k_new + ((int64_t)b * kv.Hkv + h) * D : nullptr;
+        const __nv_bfloat16 *vn_row = appending ? a.v_new + ((int64_t)b * kv.Hkv + h) * D : nullptr;
+        // the rows of tile `tile` into buffer `buf`; returns the valid-row mask
+        auto fetch = [&](int tile, int buf) -> uint32_t {
+            const int r = r0 + tile * TROWS + lane;
+            int64_t off = -1;
+            int tok = -1;
+            if (lane < TROWS && r < r1) {
+                tok = __ldcg(list + r);
+                if (tok < 0 || tok >= capn) {
+                    raise_error(kErrCapacity);
+                    tok = -1;
+                } else if (tok != pos) {
+                    off = kv.row(b, h, tok);
+                    if (off < 0) tok = -1;
+                }
+            }
+            const uint32_t vm = __ballot_sync(0xffffffffu, tok >= 0);
+            const uint32_t mb = mbar_att + 8u * (uint32_t)buf;
+            if (lane == 0) {
+                if (vm) mbar_arrive_expect_tx(mb, (uint32_t)__popc(vm) * 2u * ROW_B);
+                else mbar_arrive(mb);
+            }
+            __syncwarp();
+            if (tok >= 0) {
+                const uint32_t dst = stage_s + (uint32_t)(buf * TILE_B + lane * 2 * ROW_B);
+                const void *ks = tok == pos ? (const void *)kn_row : (const void *)(kv.k + off);
+                const void *vs = tok == pos ? (const void *)vn_row : (const void *)(kv.v + off);
+                bulk_g2s(dst, ks, ROW_B, mb);
+                bulk_g2s(dst + ROW_B, vs, ROW_B, mb);
+            }
+            return vm;
+        };
+        uint32_t vmask[2] = {0u, 0u};
+        int k = 0;
+        if (wt < ntiles) vmask[0] = fetch(wt, 0);
+        if (wt + WPT < ntiles) vmask[1] = fetch(wt + WPT, 1);
+        for (int tile = wt; tile < ntiles; tile += WPT, ++k) {
+            const int buf = k & 1;
+            if (!mbar_wait(mbar_att + 8u * buf, (uint32_t)((k >> 1) & 1))) break;
+            const unsigned char *tb = stage + buf * TILE_B;
+            const uint32_t vm = vmask[buf];
+            float x[TROWS];
+#pragma unroll
+            for (int r = 0; r < TROWS; ++r) {
+                const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(tb + r * 2 * ROW_B) + sl * DPL;
+                float2 d2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int e = 0; e < DPL; e += 8) {
+                    if constexpr (DPL >= 8) {
+                        const uint4 w4 = *reinterpret_cast<const uint4 *>(kr + e);
+                        d2 = ffma2(make_float2(qf[e], qf[e + 1]), bf16x2_to_float2(w4.x), d2);
+                        d2 = ffma2(make_float2(qf[e + 2], qf[e + 3]), bf16x2_to_float2(w4.y), d2);
+                        d2 = ffma2(make_float2(qf[e + 4], qf[e + 5]), bf16x2_to_float2(w4.z), d2);
+                        d2 = ffma2(make_float2(qf[e + 6], qf[e + 7]), bf16x2_to_float2(w4.w), d2);
+                    }
+                }
+                if constexpr (DPL == 4) {
+                    const uint2 w2 = *reinterpret_cast<const uint2 *>(kr);
+                    d2 = ffma2(make_float2(qf[0], qf[1]), bf16x2_to_float2(w2.x), d2);
+                    d2 = ffma2(make_float2(qf[2], qf[3]), bf16x2_to_float2(w2.y), d2);
+                } else if constexpr (DPL == 2) {
+                    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(kr);
+                    d2 = ffma2(make_float2(qf[0], qf[1]), bf16x2_to_float2(w1), d2);
+                }
+                x[r] = d2.x + d2.y;
+            }
+#pragma unroll
+            for (int o = SL / 2; o; o >>= 1)
+#pragma unroll
+                for (int r = 0; r < TROWS; ++r) x[r] += __shfl_xor_sync(0xffffffffu, x[r], o);
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < TROWS; ++r) {
+                x[r] = ((vm >> r) & 1u) ? x[r] : -INFINITY;
+                tmax = fmaxf(tmax, x[r]);
+            }
+            if (tmax != -INFINITY) {
+                const float mn = fmaxf(m, tmax);
+                const float c = fast_exp2(m - mn);
+                m = mn;
+                l *= c;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) acc[e] *= c;
+#pragma unroll
+                for (int r = 0; r < TROWS; ++r) {
+                    // invalid rows were not copied: their staging bytes are stale
+                    if (!((vm >> r) & 1u)) continue;
+                    const float p = fast_exp2(x[r] - mn);
+                    l += p;
+                    const __nv_bfloat16 *vr =
+                        reinterpret_cast<const __nv_bfloat16 *>(tb + r * 2 * ROW_B + ROW_B) + sl * DPL;
+                    const float2 p2 = make_float2(p, p);
+                    if constexpr (DPL >= 8) {
+#pragma unroll
+                        for (int e = 0; e < DPL; e += 8) {
+                            const uint4 w4 = *reinterpret_cast<const uint4 *>(vr + e);
+                            float2 a0 = ffma2(p2, bf16x2_to_float2(w4.x), make_float2(acc[e], acc[e + 1]));
+                            float2 a1 = ffma2(p2, bf16x2_to_float2(w4.y), make_float2(acc[e + 2], acc[e + 3]));
+                            float2 a2 = ffma2(p2, bf16x2_to_float2(w4.z), make_float2(acc[e + 4], acc[e + 5]));
+                            float2 a3 = ffma2(p2, bf16x2_to_float2(w4.w), make_float2(acc[e + 6], acc[e + 7]));
+                            acc[e] = a0.x; acc[e + 1] = a0.y; acc[e + 2] = a1.x; acc[e + 3] = a1.y;
+                            acc[e + 4] = a2.x; acc[e + 5] = a2.y; acc[e + 6] = a3.x; acc[e + 7] = a3.y;
+                        }
+                    } else if constexpr (DPL == 4) {
+                        const uint2 w2 = *reinterpret_cast<const uint2 *>(vr);
+                        float2 a0 = ffma2(p2, bf16x2_to_float2(w2.x), make_float2(acc[0], acc[1]));
+                        float2 a1 = ffma2(p2, bf16x2_to_float2(w2.y), make_float2(acc[2], acc[3]));
+                        acc[0] = a0.x; acc[1] = a0.y; acc[2] = a1.x; acc[3] = a1.y;
+                    } else {
+                        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(vr);
+                        float2 a0 = ffma2(p2, bf16x2_to_float2(w1), make_float2(acc[0], acc[1]));
+                        acc[0] = a0.x; acc[1] = a0.y;
+                    }
+                }
+            }
+            __syncwarp();  // the buffer is refilled next
+            if (tile + 2 * WPT < ntiles) vmask[buf] = fetch(tile + 2 * WPT, buf);
+        }
+        __syncthreads();  // every warp is done with its staging buffers
+        // CTA merge of the warps' states: [warp][HG] (m, l) and [warp][HG][D] acc at the LUT base
+        float *s_acc = reinterpret_cast<float *>(lut);
+        float *s_ml = s_acc + NWARP * HG * D;
+        if (sl == 0) { s_ml[(warp * HG + gl) * 2] = m; s_ml[(warp * HG + gl) * 2 + 1] = l; }
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) s_acc[(warp * HG + gl) * D + sl * DPL + e] = acc[e];
+        __syncthreads();
+        // this CTA's partial (m, l, acc) per query head, in the low region (read by the cluster)
+        float *cpart = reinterpret_cast<float *>(smem + StepLow::END);  // [G][D + 2]
+        for (int x2 = tid; x2 < G * D; x2 += NT) {
+            const int gg = x2 / D, i = x2 % D;
+            const int tm = gg / HG, gq = gg % HG;
+            float M = -INFINITY;
+            for (int w2 = tm * WPT; w2 < (tm + 1) * WPT; ++w2) M = fmaxf(M, s_ml[(w2 * HG + gq) * 2]);
+            float L = 0.0f, A = 0.0f;
+            if (M != -INFINITY) {
+                for (int w2 = tm * WPT; w2 < (tm + 1) * WPT; ++w2) {
+                    const float c = fast_exp2(s_ml[(w2 * HG + gq) * 2] - M);
+                    L = fmaf(s_ml[(w2 * HG + gq) * 2 + 1], c, L);
+                    A = fmaf(s_acc[(w2 * HG + gq) * D + i], c, A);
+                }
+            }
+            cpart[gg * (D + 2) + i] = A;
+            if (i == 0) { cpart[gg * (D + 2) + D] = M; cpart[gg * (D + 2) + D + 1] = L; }
+        }
+        cluster_sync();  // (5): every CTA's partial is complete
+        // the cluster merge, element x handled by CTA x mod C
+        for (int x2 = cta + nctas * tid; x2 < G * D; x2 += nctas * NT) {
+            const int gg = x2 / D, i = x2 % D;
+            float M = -INFINITY;
+            for (int r = 0; r < nctas; ++r) M = fmaxf(M, ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + D, r)));
+            float L = 0.0f, A = 0.0f;
+            if (M != -INFINITY) {
+                for (int r = 0; r < nctas; ++r) {
+                    const float pm = ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + D, r));
+                    const float c = fast_exp2(pm - M);
+                    L = fmaf(ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + D + 1, r)), c, L);
+                    A = fmaf(ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + i, r)), c, A);
+                }
+            }
+            const int64_t oq = (int64_t)b * a.Hq + (int64_t)h * G + gg;
+            a.out[oq * D + i] = L > 0.0f ? A / L : 0.0f;
+            if (i == 0 && a.lse) a.lse[oq] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        }
+        cluster_sync();  // (6): no CTA leaves while another may still read its partial
+    }
+}
+
+}  // namespace dkv

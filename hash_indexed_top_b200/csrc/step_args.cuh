@@ -1,0 +1,78 @@
+// step_args.cuh -- shapes, shared-memory layout and launch arguments of the
+// clustered step kernel (step.cuh), shared with the host code that launches it.
+#pragma once
+#include "common.cuh"
+#include "select.cuh"
+
+namespace dkv {
+
+constexpr int kStepThreads = 1024;
+constexpr int kStepWarps = kStepThreads / 32;
+constexpr int kRingStages = 5;
+
+template <int BITS>
+struct StepShape {
+    static constexpr int CODE_B = BITS >= 64 ? BITS / 8 : 8;  // bytes of one token's code in memory
+    static constexpr int CHUNK_B = 32 * CODE_B;               // one warp step: 32 tokens
+    static constexpr int RING_B = kStepWarps * kRingStages * CHUNK_B;
+};
+
+// Fixed part of the low shared region (byte offsets from the dynamic base).
+struct StepLow {
+    static constexpr int HIST = 0;                                 // u32[kBins]
+    static constexpr int SUP = HIST + kBins * 4;                   // u32[64] super-bin counts
+    static constexpr int QSUM = SUP + 64 * 4;                      // f32[kMaxDim]
+    static constexpr int QP = QSUM + kMaxDim * 4;                  // f32[kMaxBits]
+    static constexpr int KNEW = QP + kMaxBits * 4;                 // f32[kMaxDim] appended key
+    static constexpr int MISC = KNEW + kMaxDim * 4;                // int[64]
+    static constexpr int NEWC = MISC + 64 * 4;                     // u32[4] appended key's code
+    static constexpr int NEWR = NEWC + 16;                         // u32[4] the same in stored (rotated) order
+    static constexpr int MBAR = NEWR + 16;                         // u64[kStepWarps][kRingStages]
+    static constexpr int MBAR_ATT = MBAR + kStepWarps * kRingStages * 8;  // u64[kStepWarps][2]
+    static constexpr int WKEEP = MBAR_ATT + kStepWarps * 2 * 8;    // int[kStepWarps]
+    static constexpr int CNT = WKEEP + kStepWarps * 4;             // int[kMaxCluster][2]
+    static constexpr int MID = CNT + kMaxCluster * 8;              // int[kMaxCluster]
+    static constexpr int WKEY = MID + kMaxCluster * 4;             // unused pad
+    static constexpr int END = (WKEY + 255) / 256 * 256;           // candidate lists start here
+};
+static_assert(StepLow::MBAR % 8 == 0, "mbarriers are 8-byte aligned");
+
+// misc[] slots
+enum : int {
+    kMTloc = 0, kMIns = 1, kMNinb = 2, kMOvf = 3, kMT1 = 4, kMAbove = 5, kMCntT1 = 6,
+    kMTkey = 8, kMIT = 9, kMBefore = 10, kMTotal = 11, kMAnyOvf = 12, kMIbOvf = 13, kMAnyIbOvf = 14
+};
+
+struct StepArgs {
+    KV kv;
+    const __nv_bfloat16 *q;
+    int Hq, G;
+    int32_t *seq_lens;                   // read; incremented when appending
+    const __nv_bfloat16 *k_new, *v_new;  // [B][Hkv][D] (null: no append)
+    SelWS ws;                            // scores / cand / seg_cnt rows for the slow path
+    int topk, S, W, cap_sel;
+    int32_t *sel_idx, *sel_cnt;
+    float *scores_out;                   // optional [B][Hkv][ld_out]
+    int64_t ld_out;
+    float *out, *lse;                    // attention outputs (G > 0)
+    float scale_log2;                    // log2(e) / sqrt(d)
+    uint32_t *seq_arrive;                // [B] x kSyncStride: clusters of a sequence done with its length
+    int smem_bytes;                      // dynamic shared memory of the launch
+};
+
+using StepKern = void (*)(const StepArgs, const RBits);
+
+// The step kernel for (bits, head dim, G, paged, radius); G = 0: selection
+// only, G > 0: append + selection + attention for G query heads per kv head.
+// One getter per (bits, head dim), each defined in its own translation unit
+// (step_inst.cu compiled once per pair).
+#define DKV_STEP_GETTER(BITS, D) StepKern step_kern_##BITS##_##D(int G, bool paged, bool radius);
+DKV_STEP_GETTER(32, 64)
+DKV_STEP_GETTER(32, 128)
+DKV_STEP_GETTER(64, 64)
+DKV_STEP_GETTER(64, 128)
+DKV_STEP_GETTER(128, 64)
+DKV_STEP_GETTER(128, 128)
+#undef DKV_STEP_GETTER
+
+}  // namespace dkv

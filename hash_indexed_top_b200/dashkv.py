@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libdashkv.so")
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace missing or too small",
     4: "sequence length beyond cache capacity", 5: "CUDA error", 6: "page id out of range", 7: "no CUDA device",
+    8: "a bounded wait in a kernel gave up",
 }
 
 FLAG_TWO_KERNEL_SELECT = 1
@@ -28,7 +29,7 @@ SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_e
            "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
            "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str",
            "dashkv_select_static", "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks",
-           "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius")
+           "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius", "dashkv_decode_step")
 
 
 class DashKVError(RuntimeError):
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.dashkv_select.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, SZ, P]
         L.dashkv_sparse_decode.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, P, SZ, P]
         L.dashkv_select_static.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P]
+        L.dashkv_decode_step.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, P, P, P, SZ, P]
         L.dashkv_encode_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P]
         L.dashkv_append_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P]
         L.dashkv_select_blocks.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(BlockView), P, P, P, P, P, P,
@@ -91,10 +93,10 @@ def lib() -> ctypes.CDLL:
         L.dashkv_select_kernels.restype = I32
         L.dashkv_status_str.argtypes = [ctypes.c_int]
         L.dashkv_status_str.restype = ctypes.c_char_p
-        for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode",
+        for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_decode_step",
                   "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_static",
                   "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks",
-                  "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius"):
+                  "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius", "dashkv_decode_step"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -297,6 +299,18 @@ class DashKV:
                                                                   _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt),
                                                                   _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                                                   _stream(stream)))
+
+    def decode_step(self, cache: KVCache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                    seq_lens: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor, out: torch.Tensor,
+                    lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+        """append_keys + select + sparse_decode (given the lengths) in one launch."""
+        ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
+        v = cache.view()
+        _check("dashkv_decode_step", lib().dashkv_decode_step(self._ctx, ctypes.byref(v), _ptr(q), _ptr(k_new),
+                                                              _ptr(v_new), _ptr(seq_lens), _ptr(sel_idx),
+                                                              _ptr(sel_cnt), _ptr(out), _ptr(lse), _ptr(ws),
+                                                              ws.numel(), _stream(stream)))
 
     # ---- block summaries (CSA-style two-level index)
     def encode_blocks(self, cache: KVCache, index: BlockIndex, seq_lens: torch.Tensor, stream=None) -> None:

@@ -78,15 +78,19 @@ typedef enum dashkv_status {
     DASHKV_ERR_CAPACITY = 4,     /* device error word: a sequence outgrew its cache   */
     DASHKV_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, sync, copy)   */
     DASHKV_ERR_DEVICE = 6,       /* device error word: bad page id in page_table      */
-    DASHKV_ERR_NO_DEVICE = 7     /* no usable CUDA device                             */
+    DASHKV_ERR_NO_DEVICE = 7,    /* no usable CUDA device                             */
+    DASHKV_ERR_TIMEOUT = 8       /* device error word: a bounded wait in a kernel gave
+                                    up (a bulk copy did not land); results invalid    */
 } dashkv_status;
 
-/* Selection path.  By default dashkv_select runs one kernel with one
- * thread-block cluster per (sequence, kv head): its CTAs (one per SM, up to
- * 16 per cluster) exchange histograms and boundary tokens through distributed
- * shared memory and hardware cluster barriers.  Without cluster launch
- * support, or with this flag, it runs two ordinary kernels instead.  Both give
- * identical results. */
+/* Selection path.  By default dashkv_select (and dashkv_decode_step) runs one
+ * kernel with one thread-block cluster per (sequence, kv head): its CTAs (one
+ * per SM, up to 16 per cluster) stream the codes through bulk-copy rings, keep
+ * the candidates in shared memory and exchange histograms and boundary tokens
+ * through distributed shared memory and hardware cluster barriers.  Without
+ * cluster launch support, or with this flag, the selection runs two ordinary
+ * kernels instead (and dashkv_decode_step the three separate calls).  All
+ * give identical selections. */
 #define DASHKV_FLAG_TWO_KERNEL_SELECT 1
 
 /* Problem description.  Supported: head_dim in {64, 128}; bits in
@@ -200,6 +204,24 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    const int32_t *sel_cnt, float *out, float *lse, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* The whole decode step in one launch: dashkv_append_keys, dashkv_select and
+ * dashkv_sparse_decode (given the lengths) fused into one kernel of one
+ * thread-block cluster per (sequence, kv head), with the same results as those
+ * three calls made in that order: k_new / v_new (device bf16 [B][Hkv][d]) are
+ * written at position seq_lens[b] of every (b, kv head) with their codes, the
+ * selection (over the cache including them) goes to sel_idx / sel_cnt, the
+ * attention output to out (and lse when not NULL), and seq_lens[b] is
+ * incremented on the device.  Pages above: DASH-KV page (hashing, asymmetric
+ * scoring), DeepSeek DSA->CSA/HCA page "从 DSA 说起" (indexer, top-k, attention
+ * on the top-k), the SWA paragraph of its CSA section and the DySCO page, Q3
+ * (window and sinks).  The workspace is dashkv_select's (zero-filled once;
+ * every successful call leaves it ready for the next).  Without the clustered
+ * path (see DASHKV_FLAG_TWO_KERNEL_SELECT) the three calls run one after the
+ * other. */
+dashkv_status dashkv_decode_step(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q, const void *k_new,
+                                 const void *v_new, int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt,
+                                 float *out, float *lse, void *workspace, size_t workspace_bytes, void *stream);
+
 /* ------------------------------------------------------------------------
  * Block summaries: a CSA-style two-level index.
  *
@@ -287,8 +309,9 @@ dashkv_status dashkv_select_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* Synchronise `stream`, then read and clear the current device's error
- * word: DASHKV_OK, DASHKV_ERR_CAPACITY, DASHKV_ERR_DEVICE, or DASHKV_ERR_CUDA
- * when the stream reports an error. */
+ * word: DASHKV_OK, DASHKV_ERR_TIMEOUT, DASHKV_ERR_DEVICE, DASHKV_ERR_CAPACITY
+ * (in that order of precedence), or DASHKV_ERR_CUDA when the stream reports an
+ * error. */
 dashkv_status dashkv_get_error(void *stream);
 
 /* The hyperplanes a context built with (seed, bits, d) uses, as int8 +1/-1

@@ -14,13 +14,28 @@ from hash_indexed_top_b200 import workloads as W
 from oracle import oracle as O
 
 ATOL, RTOL = 1e-3, 8e-3
+# Scores are compared bit for bit because on 1/64-grid inputs every partial sum
+# of the fp32 scorer is a multiple of 1/64 bounded by A = sum_j |Qp_j| (the
+# oracle's `bound`); fp32 holds all of them exactly while 64 A < 2^24.
+EXACT_BOUND = 2.0 ** 18
+
+
+def assert_exact_scoring(bound: float, what: str = "") -> None:
+    assert bound < EXACT_BOUND, f"{what}: score bound {bound} breaks the exactness precondition (< 2^18)"
 
 
 class DeviceRun:
+    """The device side of a parity run.  fused_step: each step is one
+    dashkv_decode_step call (append + select + attention in one launch, no
+    scores output); otherwise append_keys, select (with its scores) and
+    sparse_decode, given the lengths (window) or the plain list."""
+
     def __init__(self, cfg: W.Config, w: W.Workload, seed: int = W.HYPERPLANE_SEED, two_kernel: bool = False,
-                 window: bool = True):
+                 window: bool = True, fused_step: bool = False):
         self.cfg, self.w = cfg, w
         self.window = window  # decode given the lengths (window CTAs) or the plain list
+        self.fused_step = fused_step
+        self.pending = None   # fused step: the step whose append is still to run
         dev = w.K.device
         self.eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
                              cfg.page_size if w.paged else 0, seed, two_kernel_select=two_kernel)
@@ -34,10 +49,23 @@ class DeviceRun:
         self.eng.encode_keys(self.cache, self.seq)
 
     def append(self, s: int):
+        if self.fused_step:
+            self.pending = s
+            return
         self.eng.append_keys(self.cache, self.w.k_new[s], self.w.v_new[s], self.seq)
+
+    @property
+    def has_scores(self) -> bool:
+        return not self.fused_step
 
     def select_decode(self, q: torch.Tensor):
         b = self.buf
+        if self.fused_step:
+            assert self.pending is not None, "the fused step appends: call append(s) first"
+            s, self.pending = self.pending, None
+            self.eng.decode_step(self.cache, q, self.w.k_new[s], self.w.v_new[s], self.seq, b["sel_idx"],
+                                 b["sel_cnt"], b["out"], b["lse"])
+            return
         self.eng.select(self.cache, q, self.seq, b["sel_idx"], b["sel_cnt"], self.scores)
         self.eng.sparse_decode(self.cache, q, b["sel_idx"], b["sel_cnt"], b["out"], b["lse"],
                                seq_lens=self.seq if self.window else None)
@@ -84,16 +112,21 @@ def within_tol(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
 
 def compare_step(g: DeviceRun, o: OracleRun, r: dict, what: str = "") -> dict:
     """Assert parity of one step; returns a few diagnostics."""
+    assert_exact_scoring(r["bound"], what)
     gc = dk.canonical_codes(g.cache.codes, o.cfg.bits).cpu().numpy().view(np.uint64)
     assert np.array_equal(gc, o.codes), f"{what}: codes differ at {np.argwhere(gc != o.codes)[:5].tolist()}"
     assert np.array_equal(g.seq.cpu().numpy(), o.seq), f"{what}: seq_lens differ"
-    gs = g.scores.cpu().numpy()
-    os_ = r["scores"].astype(np.float32)
-    for b in range(o.cfg.B):
-        n = int(o.seq[b])
-        a, e = gs[b, :, :n], os_[b, :, :n]
-        assert np.array_equal(a.view(np.uint32), e.view(np.uint32)), \
-            f"{what}: scores differ (b={b}) at {np.argwhere(a != e)[:5].tolist()}"
+    if g.fused_step:  # the step wrote the appended rows itself
+        assert np.array_equal(g.cache.k.cpu().double().numpy(), o.K), f"{what}: cached keys differ"
+        assert np.array_equal(g.cache.v.cpu().double().numpy(), o.V), f"{what}: cached values differ"
+    if g.has_scores:
+        gs = g.scores.cpu().numpy()
+        os_ = r["scores"].astype(np.float32)
+        for b in range(o.cfg.B):
+            n = int(o.seq[b])
+            a, e = gs[b, :, :n], os_[b, :, :n]
+            assert np.array_equal(a.view(np.uint32), e.view(np.uint32)), \
+                f"{what}: scores differ (b={b}) at {np.argwhere(a != e)[:5].tolist()}"
     gi = g.buf["sel_idx"].cpu().numpy()
     gn = g.buf["sel_cnt"].cpu().numpy()
     assert np.array_equal(gn, r["sel_cnt"]), f"{what}: sel_cnt {gn.ravel()[:8]} vs {r['sel_cnt'].ravel()[:8]}"
@@ -109,13 +142,13 @@ def compare_step(g: DeviceRun, o: OracleRun, r: dict, what: str = "") -> dict:
 
 
 def run_parity(cfg: W.Config, steps: int, device="cuda", w: W.Workload | None = None, mutate=None,
-               two_kernel: bool = False, window: bool = True) -> list:
+               two_kernel: bool = False, window: bool = True, fused_step: bool = False) -> list:
     """Encode, then `steps` x (append, select, decode) on GPU and oracle, comparing every step."""
     if w is None:
         w = W.make_workload(cfg, device="cpu", steps=steps)
     if mutate is not None:
         w = mutate(w)
-    g = DeviceRun(cfg, w.to(device), two_kernel=two_kernel, window=window)
+    g = DeviceRun(cfg, w.to(device), two_kernel=two_kernel, window=window, fused_step=fused_step)
     o = OracleRun(cfg, w)
     g.encode()
     diags = []

@@ -20,17 +20,19 @@ def test_recorded_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
     shutil.copytree(os.path.join(ROOT, "hash_indexed_top_b200", "csrc"), tmp_path / "hash_indexed_top_b200" / "csrc")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    summary = tmp_path / "profiles" / "c128k_step_kernels_full.txt"
-    assert bench.recorded_traffic("select_fused") is None  # no summary, no figure
-    summary.write_text(f"kernel sources sha256: {bench.kernel_sources_sha()}\n"
-                       "traffic_per_launch select_fused_kernel 123456\n")
-    assert bench.recorded_traffic("select_fused") == 123456  # taken from these kernels
-    assert bench.recorded_traffic("score_hist") is None  # not measured
-    src = tmp_path / "hash_indexed_top_b200" / "csrc" / "select.cuh"
+    summary = tmp_path / "profiles" / "decode_step_c128k.txt"
+    assert bench.recorded_traffic("c128k", "decode_step") is None  # no summary, no figure
+    summary.write_text("workload: c128k\n"
+                       f"kernel sources sha256: {bench.kernel_sources_sha()}\n"
+                       "traffic_per_launch decode_step 123456\n")
+    assert bench.recorded_traffic("c128k", "decode_step") == 123456  # taken from these kernels
+    assert bench.recorded_traffic("c1m", "decode_step") is None  # another workload
+    assert bench.recorded_traffic("c128k", "score_hist") is None  # not measured
+    src = tmp_path / "hash_indexed_top_b200" / "csrc" / "step.cuh"
     src.write_text("// a comment-only change\n" + src.read_text())
-    assert bench.recorded_traffic("select_fused") == 123456  # comments do not make the counters stale
+    assert bench.recorded_traffic("c128k", "decode_step") == 123456  # comments do not make the counters stale
     src.write_text(src.read_text() + "\nstatic int changed_code = 1;\n")
-    assert bench.recorded_traffic("select_fused") is None  # a code change does
+    assert bench.recorded_traffic("c128k", "decode_step") is None  # a code change does
 
 
 def test_oracle_block_update_matches_a_whole_cache_encode():

@@ -1,13 +1,19 @@
-"""Full-size parity: every configured long-context workload at its full size,
-one decode step in the launch configuration the benchmark times (the fused
-selection, the decode given the lengths), checked against the oracle on whole
-sampled (sequence, kv head) pairs: all of a pair's codes and scores, its
-selection, and the attention output and lse of its query heads.
+"""Full-size parity: every configured long-context workload at its full size.
 
-The oracle recomputes a pair from its own encode of the pair's keys (no GPU
-value enters it); the pairs are the first and the last of the grid.  The
-block-summary workloads are checked the same way, summaries and block scores
-included."""
+test_full_size_decode_steps_every_pair runs the configured number of decode
+steps exactly as the benchmark times them -- each step one
+dashkv_decode_step call captured in a CUDA graph and replayed -- and checks
+every (sequence, kv head) pair of every step against the oracle: selection
+(bit for bit), attention output and lse of the pair's query heads (within
+tolerance), and at the end the pair's codes, cached keys and values.  The
+oracle starts from its own encode of a copy of the prefilled cache taken
+before the GPU ran and appends the step inputs itself (no GPU value enters
+it); pairs are checked one at a time so host memory holds one pair.
+
+test_full_size_select_scores_on_sampled_pairs checks the selection call with
+its scores output (fp32 scores bit for bit) on the first and last pair, and
+the block-summary workloads are checked the same way, summaries and block
+scores included."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +22,7 @@ from hash_indexed_top_b200 import dashkv as dk
 from hash_indexed_top_b200 import workloads as W
 from oracle import oracle as O
 
-from pipeline import within_tol
+from pipeline import assert_exact_scoring, within_tol
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +49,74 @@ def _pair_codes(codes: torch.Tensor, w: W.Workload, b: int, h: int, n: int) -> t
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_step_on_sampled_pairs(name):
+def test_full_size_decode_steps_every_pair(name):
+    cfg = W.CONFIGS[name]
+    steps = cfg.steps
+    dev = torch.device("cuda")
+    w = W.make_workload(cfg, device=dev, steps=steps)
+    K0, V0 = w.K.clone(), w.V.clone()  # the prefilled cache, for the oracle
+    eng = dk.DashKV(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.bits, cfg.topk, cfg.sink, cfg.window,
+                    cfg.page_size if w.paged else 0, W.HYPERPLANE_SEED)
+    rec = []
+    try:
+        cache = dk.KVCache(w.K, w.V, dk.KVCache.empty_codes_like(w.K, cfg.bits, w.paged), w.page_table)
+        seq = w.seq_lens.clone()
+        eng.encode_keys(cache, seq)
+        buf = eng.alloc_step(dev)
+        ws = eng.workspace(cache.capacity, dev)
+        torch.cuda.synchronize()
+        for s in range(steps):  # one captured graph per step, as the benchmark replays them
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                eng.decode_step(cache, w.q[s], w.k_new[s], w.v_new[s], seq, buf["sel_idx"], buf["sel_cnt"],
+                                buf["out"], buf["lse"], ws)
+            g.replay()
+            torch.cuda.synchronize()
+            rec.append({k: v.cpu() for k, v in buf.items()})
+            del g
+        assert eng.get_error() == 0
+        gcodes = dk.canonical_codes(cache.codes, cfg.bits)
+        R = O.hyperplanes(W.HYPERPLANE_SEED, cfg.bits, cfg.d)
+        G = cfg.G
+        assert torch.equal(seq.cpu(), w.seq_lens.cpu() + steps)
+        for b in range(cfg.B):
+            n0 = int(w.seq_lens[b])
+            for h in range(cfg.Hkv):
+                cap = n0 + steps
+                L = O.Layout(1, 1, cfg.d, cfg.bits, n_cap=cap)
+                K = np.zeros((1, 1, cap, cfg.d))
+                V = np.zeros((1, 1, cap, cfg.d))
+                K[0, 0, :n0] = _pair_rows(K0, w, b, h, n0).double().cpu().numpy()
+                V[0, 0, :n0] = _pair_rows(V0, w, b, h, n0).double().cpu().numpy()
+                sl = np.array([n0], dtype=np.int32)
+                oc = O.encode(L, K, sl, R)
+                for s in range(steps):
+                    O.append(L, K, V, oc, sl, w.k_new[s][b:b + 1, h:h + 1].double().cpu().numpy(),
+                             w.v_new[s][b:b + 1, h:h + 1].double().cpu().numpy(), R)
+                    q = w.q[s][b, h * G:(h + 1) * G].double().cpu().numpy().reshape(1, G, cfg.d)
+                    r = O.decode_step(L, G, q, K, V, oc, sl, R, cfg.topk, cfg.sink, cfg.window)
+                    what = f"{name} step {s} ({b},{h})"
+                    assert_exact_scoring(r["bound"], what)
+                    got = rec[s]
+                    assert int(got["sel_cnt"][b, h]) == int(r["sel_cnt"][0, 0]), f"{what}: sel_cnt"
+                    assert np.array_equal(got["sel_idx"][b, h].numpy(), r["sel_idx"][0, 0]), f"{what}: selection"
+                    out = got["out"][b, h * G:(h + 1) * G].double().numpy()
+                    lse = got["lse"][b, h * G:(h + 1) * G].double().numpy()
+                    assert within_tol(out, r["out"][0]).all(), f"{what}: out err {np.abs(out - r['out'][0]).max()}"
+                    assert within_tol(lse, r["lse"][0]).all(), f"{what}: lse err {np.abs(lse - r['lse'][0]).max()}"
+                n = int(sl[0])
+                gc = _pair_codes(gcodes, w, b, h, n).cpu().numpy().view(np.uint64)
+                assert np.array_equal(gc, oc[0, 0, :n]), f"{name} ({b},{h}): codes differ"
+                assert np.array_equal(_pair_rows(w.K, w, b, h, n).double().cpu().numpy(), K[0, 0, :n]), \
+                    f"{name} ({b},{h}): cached keys differ"
+                assert np.array_equal(_pair_rows(w.V, w, b, h, n).double().cpu().numpy(), V[0, 0, :n]), \
+                    f"{name} ({b},{h}): cached values differ"
+    finally:
+        eng.close()
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_select_scores_on_sampled_pairs(name):
     cfg = W.CONFIGS[name]
     dev = torch.device("cuda")
     w = W.make_workload(cfg, device=dev, steps=1)
@@ -75,6 +148,7 @@ def test_full_size_step_on_sampled_pairs(name):
             assert np.array_equal(gc, oc[0, 0]), f"{name} ({b},{h}): codes differ at {np.argwhere(gc != oc[0, 0])[:3]}"
             q = w.q[0][b, h * G:(h + 1) * G].double().cpu().numpy().reshape(1, G, cfg.d)
             r = O.decode_step(L, G, q, K, V, oc, sl, R, cfg.topk, cfg.sink, cfg.window)
+            assert_exact_scoring(r["bound"], f"{name} ({b},{h})")
             gs = scores[b, h, :n].cpu().numpy()
             es = r["scores"][0, 0, :n].astype(np.float32)
             assert np.array_equal(gs.view(np.uint32), es.view(np.uint32)), \

@@ -36,11 +36,14 @@ def built():
     build.build()
 
 
-# selection path x decode mode: the fused selection with the decode's window
-# CTAs (lengths given), the same selection with a plain list decode, and the
-# two-kernel selection
+# selection path x decode mode: the clustered selection with the decode's
+# window CTAs (lengths given), the same selection with a plain list decode, the
+# two-kernel selection, and the whole step as one clustered launch
+# (dashkv_decode_step: append, selection and attention in one kernel)
 PATHS = {"fused": dict(two_kernel=False, window=True), "fused_list_decode": dict(two_kernel=False, window=False),
-         "two_kernel": dict(two_kernel=True, window=True)}
+         "two_kernel": dict(two_kernel=True, window=True), "step": dict(fused_step=True)}
+# the paths whose select and decode can run without an append before them
+SPLIT_PATHS = {k: v for k, v in PATHS.items() if k != "step"}
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -92,7 +95,7 @@ def test_repeated_keys_heavy_ties(path):
     run_parity(cfg, 1, mutate=mutate, **PATHS[path])
 
 
-@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("path", list(SPLIT_PATHS))
 def test_empty_sequence_selects_nothing(path):
     cfg = W.Config("empty", B=3, Hq=4, Hkv=2, d=64, N=200, bits=64, topk=10, sink=2, window=2,
                    steps=0, needles=0, seed=84)
@@ -113,7 +116,7 @@ def test_empty_sequence_selects_nothing(path):
     g.close()
 
 
-@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("path", list(SPLIT_PATHS))
 def test_repeat_calls_are_deterministic_and_leave_workspace_clean(path):
     cfg, _ = CASES["c128k_small"]
     w = W.make_workload(cfg, steps=1).to("cuda")
