@@ -89,11 +89,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar)
                  : "memory");
 }
-// Bounded wait for the phase of parity `parity` of `mbar` to complete.  Gives
-// up after about kMbarSpins polls (each may suspend for up to kMbarSuspendNs),
-// sets the timeout bit of the error word and returns false.
-constexpr int kMbarSpins = 1 << 20;
-constexpr uint32_t kMbarSuspendNs = 256;
+// Bounded wait for the phase of parity `parity` of `mbar` to complete.  Each
+// poll suspends the warp until the phase completes or kMbarSuspendNs pass (a
+// suspended warp takes no issue slots from the warps that have work); after
+// kMbarSpins polls (about a second at most) it gives up, sets the timeout bit
+// of the error word and returns false.
+constexpr int kMbarSpins = 1 << 12;
+constexpr uint32_t kMbarSuspendNs = 250000;
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
     for (int it = 0; it < kMbarSpins; ++it) {
         uint32_t done;

@@ -155,9 +155,9 @@ __device__ __forceinline__ void unpack_code(const typename ScoreShape<BITS>::Vec
     }
 }
 
-// Shared-memory load from a 32-bit shared address.  Not volatile: its address
-// always depends on code words loaded after the barrier that publishes the LUT,
-// so it cannot be scheduled before that barrier.
+// Shared-memory load from a 32-bit shared address plus the byte offset IMM.
+// Not volatile: its address always depends on code words loaded after the
+// barrier that publishes the LUT, so it cannot be scheduled before it.
 template <int IMM>
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
     float v;
@@ -165,29 +165,45 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
-// Terms r = 0 .. R - 1 of a score (even r into s0, odd r into s1, ascending).
+// Packed fp32 add (two lanes of fp32 per instruction on sm_100), each lane
+// rounded once like a scalar add.
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return *reinterpret_cast<float2 *>(&d);
+}
+
+// Table entry of stored byte r of a (rotated) code for the lane whose row
+// address base is `base` (see the scorer below).
+template <int BITS, int r>
+__device__ __forceinline__ float lut_term(const uint32_t (&w)[BITS / 32], uint32_t base) {
+    return lds_f32<4 * r>(__byte_perm(w[r >> 2], base, 0x7604u | ((uint32_t)(r & 3) << 4)));
+}
+
+// Terms (r, r + 1) for r = 0, 2, .. R - 2 of a score: even bytes into s.x, odd
+// bytes into s.y (each chain ascending), one packed add per pair.
 template <int BITS, int R>
-struct LutTerms {
-    static __device__ __forceinline__ void add(const uint32_t (&w)[BITS / 32], uint32_t base, float &s0, float &s1) {
-        LutTerms<BITS, R - 1>::add(w, base, s0, s1);
-        constexpr int r = R - 1;
-        const float v = lds_f32<4 * r>(__byte_perm(w[r >> 2], base, 0x7604u | ((uint32_t)(r & 3) << 4)));
-        if (r % 2 == 0) s0 += v; else s1 += v;
+struct LutPairs {
+    static __device__ __forceinline__ void add(const uint32_t (&w)[BITS / 32], uint32_t base, float2 &s) {
+        LutPairs<BITS, R - 2>::add(w, base, s);
+        s = fadd2(s, make_float2(lut_term<BITS, R - 2>(w, base), lut_term<BITS, R - 1>(w, base)));
     }
 };
 template <int BITS>
-struct LutTerms<BITS, 0> {
-    static __device__ __forceinline__ void add(const uint32_t (&)[BITS / 32], uint32_t, float &, float &) {}
+struct LutPairs<BITS, 0> {
+    static __device__ __forceinline__ void add(const uint32_t (&)[BITS / 32], uint32_t, float2 &) {}
 };
 
-// Score of one (rotated) code: sum over its T bytes of the lane's table entries.
+// Score of one (rotated) code: sum over its T bytes of the lane's table
+// entries, the even and the odd bytes in two chains, then the chains added.
 template <int BITS>
 __device__ __forceinline__ float lut_score(const uint32_t (&w)[BITS / 32], uint32_t base) {
-    float s0 = 0.0f, s1 = 0.0f;
-    LutTerms<BITS, BITS / 8>::add(w, base, s0, s1);
-    return (s0 + s1) + 0.0f;  // + 0 turns a -0 into +0
+    float2 s = make_float2(0.0f, 0.0f);
+    LutPairs<BITS, BITS / 8>::add(w, base, s);
+    return (s.x + s.y) + 0.0f;  // + 0 turns a -0 into +0
 }
-
 
 // ---------------------------------------------------------------------------
 // Score phase shared by the fused and the two-kernel selection: LUT prologue

@@ -11,12 +11,14 @@
 // (attention sinks).
 //
 // Grid: one thread-block cluster of C CTAs (1024 threads, one per SM) per
-// (sequence, kv head); CTA c owns a contiguous, 64-aligned token range and
-// warp w of it a contiguous, 32-aligned sub-range.
+// (sequence, kv head); CTA c owns a contiguous, 64-aligned token range.
 //
-//  stream   every warp streams its codes through a private ring of 32-token
-//           chunks filled by bulk copies (cp.async.bulk, completion on an
-//           mbarrier, issued by lane 0 a few chunks ahead); lane l scores the
+//  stream   the CTA streams its codes in stages of 16 KB through a ring in
+//           shared memory: dense caches by one bulk copy per stage
+//           (cp.async.bulk, completion counted in bytes on the stage's
+//           mbarrier, issued by the last warp to finish with the slot), paged
+//           caches by per-thread cp.async of each thread's own tokens.  Warp w
+//           takes a 32- or 64-token slice of every stage and lane l scores the
 //           tokens t = l (mod 32) with the byte-LUT of the query (the codes are
 //           stored byte-rotated by t mod T, see store_code_rotated).  A token
 //           whose histogram bin reaches the CTA's running threshold is kept
@@ -28,7 +30,8 @@
 //  select   the cluster sums its histograms through distributed shared
 //           memory and finds the bin T1 holding the k-th largest score; the
 //           warps classify their candidates, rank the few of bin T1 exactly
-//           (score desc, index asc) and write the ascending selection.  Heavy
+//           (score desc, index asc), mark the kept tokens in a bitmap of the
+//           CTA's range and write them in order.  Heavy
 //           ties (more than kInbinMax tokens in T1) or a full candidate list
 //           take an exact slow path (re-score into the workspace, CTA 0 runs
 //           the two-kernel path's resolver).
@@ -38,8 +41,8 @@
 //           states are merged through distributed shared memory.
 //  append   (k_new given) the CTA that owns position seq_lens[b] encodes the
 //           new key, writes its code and K/V rows there and scores it from
-//           the code it computed; the last cluster of a sequence to pass its
-//           first cluster barrier increments seq_lens[b].
+//           the code it computed; the last cluster of a sequence to finish
+//           increments seq_lens[b] (every CTA read it at its start).
 #pragma once
 #include "decode.cuh"
 #include "select.cuh"
@@ -91,6 +94,30 @@ __device__ __forceinline__ int local_threshold(const uint32_t *sup, const uint32
     return __shfl_sync(0xffffffffu, t, __ffs(hm) - 1);
 }
 
+// Drop from a warp's candidate list (entries j < ncand, the first cap_lo in
+// lo[], the rest in hi[]) the ones whose bin is below tl, keeping their order;
+// returns the new count.  One full warp; out of line (rare).
+static __device__ __noinline__ int compact_candidates(uint2 *lo, uint2 *hi, int cap_lo, int ncand, int tl, float inv2A) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    int kept = 0;
+    for (int jb = 0; jb < ncand; jb += 32) {
+        const int jj = jb + lane;
+        uint2 e = make_uint2(0u, 0u);
+        if (jj < ncand) e = jj < cap_lo ? lo[jj] : hi[jj - cap_lo];
+        const bool keep = jj < ncand && score_bin(key_to_float(e.y), inv2A) >= tl;
+        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+        __syncwarp();
+        if (keep) {
+            const int d = kept + __popc(kb & lt);
+            if (d < cap_lo) lo[d] = e; else hi[d - cap_lo] = e;
+        }
+        kept += __popc(kb);
+        __syncwarp();
+    }
+    return kept;
+}
+
 // fp32 LUT score of one token's (rotated) code words for a token t (any lane):
 // lane offset t mod 32 keeps the table order right (t mod T = lane mod T).
 template <int BITS>
@@ -127,7 +154,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     using SS = StepShape<BITS>;
     constexpr int NS = kRingStages;
     constexpr int NWARP = kStepWarps, NT = kStepThreads;
-    constexpr int CODE_B = SS::CODE_B, CHUNK_B = SS::CHUNK_B;
+    constexpr int CODE_B = SS::CODE_B, TPL = SS::TPL, STG_TOK = SS::STG_TOK, STG_B = SS::STG_B;
     constexpr int T = BITS / 8;
     extern __shared__ __align__(1024) unsigned char smem[];
     const KV &kv = a.kv;
@@ -145,10 +172,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     int *misc = reinterpret_cast<int *>(smem + StepLow::MISC);
     uint32_t *newc = reinterpret_cast<uint32_t *>(smem + StepLow::NEWC);
     uint32_t *newr = reinterpret_cast<uint32_t *>(smem + StepLow::NEWR);
-    int *s_wkeep = reinterpret_cast<int *>(smem + StepLow::WKEEP);
+    uint32_t *stg_cnt = reinterpret_cast<uint32_t *>(smem + StepLow::STG_CNT);
+    int *s_wdef = reinterpret_cast<int *>(smem + StepLow::WDEF);
     int (*s_cnt)[2] = reinterpret_cast<int (*)[2]>(smem + StepLow::CNT);
     int *s_mid = reinterpret_cast<int *>(smem + StepLow::MID);
-    const uint32_t mbar_ring = smem_s + StepLow::MBAR + 8u * (uint32_t)(warp * NS);
+    int *s_warp = reinterpret_cast<int *>(smem + StepLow::WARPSCAN);
+    const uint32_t mbar_full = smem_s + StepLow::MBAR;  // [NS]
     const uint32_t mbar_att = smem_s + StepLow::MBAR_ATT + 8u * (uint32_t)(warp * 2);
     const uint32_t lut_s = (smem_s + StepLow::END + 65535u) & ~65535u;  // 64 KB aligned
     unsigned char *lut = smem + (lut_s - smem_s);
@@ -166,9 +195,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     // ---- set-up: counters, barriers, this warp's hyperplane words
     for (int i = tid; i < kBins; i += NT) hist[i] = 0;
     if (tid < 64) { sup[tid] = 0; misc[tid] = 0; }
-    if (tid < NWARP * NS) mbar_init(smem_s + StepLow::MBAR + 8u * tid, 1);
-    if (tid < NWARP * 2) mbar_init(smem_s + StepLow::MBAR_ATT + 8u * tid, 1);
-    if (tid < NWARP * NS || tid < NWARP * 2) fence_mbar_init();
+    if (tid < 4) newc[tid] = 0;
+    if (tid < NS) { mbar_init(mbar_full + 8u * tid, 1); stg_cnt[tid] = 0; }
+    if (tid >= 32 && tid < 32 + NWARP * 2) mbar_init(smem_s + StepLow::MBAR_ATT + 8u * (tid - 32), 1);
+    if (tid < 32 + NWARP * 2) fence_mbar_init();
     static_assert(BITS % NWARP == 0, "hyperplanes per warp");
     uint32_t rw[BITS / NWARP][D / 32];
 #pragma unroll
@@ -204,81 +234,86 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     int64_t t0, t1;
     cta_range(n, cta, nctas, t0, t1);
     const int nloc = (int)(t1 - t0);
-    const int wlen = (int)(ceil_div(ceil_div(nloc, NWARP), 32) * 32);
-    const int wb = warp * wlen;
-    const int we = min(nloc, wb + wlen);
-    const int nk = we > wb ? (we - wb + 31) / 32 : 0;  // chunks of this warp
+    const int nstg = (nloc + STG_TOK - 1) / STG_TOK;  // stages of this CTA
     const bool own_new = pos >= t0 && pos < t1;
+    const int pos_loc = own_new ? (int)(pos - t0) : -1;
 
-    // ---- issue the first chunks now: their latency overlaps the LUT build
+    // ---- the code ring.  Dense: stage s is one bulk copy of the stage's codes
+    // (when they lie inside the capacity at a 16-byte aligned address; else its
+    // tokens are read with plain loads), issued by whichever warp is the last
+    // to finish with the slot.  Paged: every thread copies its own tokens of the
+    // stage with cp.async (a stage's 32-token warp slices lie in single pages
+    // for pages of 64 or more tokens) and reads only what it copied.
     const unsigned char *codes_b = reinterpret_cast<const unsigned char *>(kv.codes);
-    const int64_t dense_row = ((int64_t)bh * kv.n_cap + t0 + wb) * CODE_B;  // byte offset of the warp's first code
-    // PAGED: the page ids of the chunks of groups gA, gA + 1 and gA + 2 (lane l
-    // of register pg[i] holds chunk 32 (gA + i) + l), loaded a group ahead of use
-    auto chunk_page = [&](int c) -> int {  // -1: no chunk, -2: page id out of range
-        if (c >= nk) return -1;
-        const int64_t t = t0 + wb + 32 * (int64_t)c;
-        const int32_t p = __ldg(kv.page_table + (int64_t)b * kv.max_pages + t / kv.page_size);
-        if (p < 0 || p >= kv.num_pages) return -2;
-        return p;
+    const unsigned char *dense_base = codes_b + ((int64_t)bh * kv.n_cap + t0) * CODE_B;
+    auto stage_tokens = [&](int s) { return min(STG_TOK, nloc - s * STG_TOK); };
+    // bytes of dense stage s's bulk copy, or 0 when it is read with plain loads
+    auto stage_bulk_bytes = [&](int s) -> uint32_t {
+        if constexpr (PAGED) return 0u;
+        const int cnt = stage_tokens(s);
+        const uint32_t bytes = ((uint32_t)(cnt * CODE_B) + 15u) & ~15u;
+        const unsigned char *src = dense_base + (int64_t)s * STG_B;
+        const bool inside = (t0 + (int64_t)s * STG_TOK) * CODE_B + bytes <= kv.n_cap * CODE_B;
+        return (inside && !(reinterpret_cast<uintptr_t>(src) & 15u)) ? bytes : 0u;
     };
-    int pgA = 0, pgB = 0, pgC = 0, gA = 0;
-    if constexpr (PAGED) {
-        pgA = chunk_page(lane);
-        pgB = chunk_page(32 + lane);
-        pgC = chunk_page(64 + lane);
-    }
-    auto page_of_chunk = [&](int c) -> int {  // every lane calls; c in groups gA .. gA + 2
-        const int g = (c >> 5) - gA;
-        return __shfl_sync(0xffffffffu, g == 0 ? pgA : (g == 1 ? pgB : pgC), c & 31);
-    };
-    // Source of chunk c for a bulk copy, or null when its tokens are read with
-    // plain loads instead (a dense chunk running past the capacity, or an
-    // address that is not 16-byte aligned) or skipped (a bad page id: *bad).
-    // Every lane calls (the page id is shuffled from the lane that holds it).
-    auto chunk_src = [&](int c, bool &bad) -> const unsigned char * {
-        bad = false;
-        const unsigned char *src = nullptr;
-        if constexpr (PAGED) {
-            const int p = page_of_chunk(c);
-            if (p < 0) {
-                bad = true;
-                return nullptr;
-            }
-            const int64_t t = t0 + wb + 32 * (int64_t)c;
-            src = codes_b + (((int64_t)p * kv.Hkv + h) * kv.page_size + t % kv.page_size) * CODE_B;
+    auto issue_dense = [&](int s) {  // one thread
+        const uint32_t mb = mbar_full + 8u * (uint32_t)(s % NS);
+        const uint32_t bytes = stage_bulk_bytes(s);
+        if (bytes) {
+            mbar_arrive_expect_tx(mb, bytes);
+            bulk_g2s(ring_s + (uint32_t)((s % NS) * STG_B), dense_base + (int64_t)s * STG_B, bytes, mb);
         } else {
-            if (t0 + wb + 32 * (int64_t)c + 32 > kv.n_cap) return nullptr;
-            src = codes_b + dense_row + (int64_t)c * CHUNK_B;
-        }
-        return (reinterpret_cast<uintptr_t>(src) & 15u) ? nullptr : src;
-    };
-    auto issue = [&](int c) {
-        const uint32_t mb = mbar_ring + 8u * (uint32_t)(c % NS);
-        const uint32_t dst = ring_s + (uint32_t)((warp * NS + c % NS) * CHUNK_B);
-        if constexpr (PAGED) {
-            if ((c >> 5) == gA + 2) {  // entering group gA + 2: drop gA, load gA + 3
-                gA += 1;
-                pgA = pgB;
-                pgB = pgC;
-                pgC = chunk_page(32 * (gA + 2) + lane);
-            }
-        }
-        bool bad;
-        const unsigned char *src = chunk_src(c, bad);
-        if (lane == 0) {
-            if (bad) raise_error(kErrPage);  // issued chunks exist: a negative id is out of range
-            if (src) {
-                mbar_arrive_expect_tx(mb, CHUNK_B);
-                bulk_g2s(dst, src, CHUNK_B, mb);
-            } else {
-                mbar_arrive(mb);  // completes the phase with no data
-            }
+            mbar_arrive(mb);  // completes the phase with no data
         }
     };
+    // PAGED: physical page of this lane's token u of stage s (-1: none, -2: out of range)
+    auto lane_page = [&](int s, int u) -> int {
+        const int i = s * STG_TOK + warp * 32 * TPL + 32 * u + lane;
+        if (s >= nstg || i >= nloc) return -1;
+        const int32_t p = __ldg(kv.page_table + (int64_t)b * kv.max_pages + (t0 + i) / kv.page_size);
+        return (p < 0 || p >= kv.num_pages) ? -2 : p;
+    };
+    uint32_t pbad = 0;  // PAGED: bit (slot * TPL + u) set when that token's page is out of range
+    auto issue_paged = [&](int s, const int (&pg)[TPL]) {  // every thread, one commit group per stage
+        const int slot = s % NS;
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int li = warp * 32 * TPL + 32 * u + lane;  // token within the stage
+            const int i = s * STG_TOK + li;
+            const void *src = codes_b;
+            uint32_t sz = 0;
+            const uint32_t bit = 1u << (slot * TPL + u);
+            pbad &= ~bit;
+            if (pg[u] >= 0) {
+                src = codes_b + (((int64_t)pg[u] * kv.Hkv + h) * kv.page_size + (t0 + i) % kv.page_size) * CODE_B;
+                sz = CODE_B;
+            } else if (pg[u] == -2) {
+                raise_error(kErrPage);
+                pbad |= bit;
+            }
+            const uint32_t dst = ring_s + (uint32_t)(slot * STG_B + li * CODE_B);
+            if constexpr (CODE_B == 16)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
+            else
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    int pgn[TPL];  // PAGED: pages of this lane's tokens of the next stage to issue
     __syncthreads();  // barriers initialised
-#pragma unroll 1
-    for (int c = 0; c < NS && c < nk; ++c) issue(c);
+    if constexpr (PAGED) {
+        for (int s = 0; s < NS; ++s) {
+            int pg[TPL];
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) pg[u] = lane_page(s, u);
+            issue_paged(s, pg);
+        }
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) pgn[u] = lane_page(NS, u);
+    } else {
+        if (tid == 0)
+            for (int s = 0; s < NS && s < nstg; ++s) issue_dense(s);
+    }
 
     // ---- LUT of the group's summed query (as the two-kernel scorer builds it)
     for (int i = tid; i < D; i += NT) {
@@ -289,27 +324,29 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     }
     if (own_new && tid < D) knew[tid] = __bfloat162float(a.k_new[((int64_t)b * kv.Hkv + h) * D + tid]);
     __syncthreads();
+    // Qp_j = sum_i R[j][i] qsum[i] (and, in the CTA that appends, the new key's
+    // projections): warp w takes hyperplanes w, w + 32, ... and lane l the dims
+    // l, l + 32, ...; a shuffle tree sums the lanes.  Exact on grid inputs.
 #pragma unroll
     for (int m = 0; m < BITS / NWARP; ++m) {
-        float acc = 0.0f;
+        float acc = 0.0f, kacc = 0.0f;
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k) acc = fmaf(((rw[m][k] >> lane) & 1u) ? -1.0f : 1.0f, qsum[32 * k + lane], acc);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) Qp[warp + NWARP * m] = acc;
-    }
-    // the appended key's code: thread j < BITS projects it on hyperplane j (one
-    // sequential FMA chain over the dims, as the encoder; exact on grid inputs)
-    if (own_new && tid < BITS) {
-        const int j = tid;
-        float acc = 0.0f;
-#pragma unroll 4
-        for (int i = 0; i < D; ++i) {
-            const uint32_t wbits = R.w[j * (D / 32) + i / 32];
-            acc = fmaf(((wbits >> (i % 32)) & 1u) ? -1.0f : 1.0f, knew[i], acc);
+        for (int k = 0; k < D / 32; ++k) {
+            const float sg = ((rw[m][k] >> lane) & 1u) ? -1.0f : 1.0f;
+            acc = fmaf(sg, qsum[32 * k + lane], acc);
+            if (own_new) kacc = fmaf(sg, knew[32 * k + lane], kacc);
         }
-        const uint32_t word = __ballot_sync(0xffffffffu, acc >= 0.0f);
-        if (lane == 0) newc[j / 32] = word;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            kacc += __shfl_xor_sync(0xffffffffu, kacc, o);
+        }
+        if (lane == 0) {
+            Qp[warp + NWARP * m] = acc;
+            // hyperplane j = warp + NWARP m is bit j % 32 of code word j / 32 (a tie at 0 gives 1)
+            const int j = warp + NWARP * m;
+            if (own_new && kacc >= 0.0f) atomicOr(newc + (j >> 5), 1u << (j & 31));
+        }
     }
     __syncthreads();
     float inv2A;
@@ -322,8 +359,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         inv2A = s > 0.0f ? 0.5f / s : 0.0f;
     }
     {   // LUT rows: word j of row v holds LUT_{j mod T}[v] (see score_phase)
-        static_assert(256 % NWARP == 0 && (256 / NWARP) <= 8, "rows per warp");
+        static_assert(256 % NWARP == 0 && (256 / NWARP) <= 16, "rows per warp");
         constexpr int RPW = 256 / NWARP;
+        constexpr int RB = RPW >= 16 ? 4 : (RPW >= 8 ? 3 : (RPW >= 4 ? 2 : (RPW >= 2 ? 1 : 0)));  // log2 RPW
         const int c = lane % T;
         float qv[8];
 #pragma unroll
@@ -336,7 +374,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         for (int dd = 0; dd < RPW; ++dd) {
             float val = base;
 #pragma unroll
-            for (int u = 0; u < 3; ++u)
+            for (int u = 0; u < RB; ++u)
                 if ((dd >> u) & 1) val += 2.0f * qv[u];
             float *row = reinterpret_cast<float *>(lut + (v0 + dd) * 256);
             row[lane] = val;
@@ -345,7 +383,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     }
     // the appended token: its K / V rows and code go to the cache (the
     // attention below reads its rows from k_new / v_new, and this kernel
-    // scores it from newc)
+    // scores it from newr)
     if (own_new) {
         if (tid < 2 * (D / 8)) {
             const bool isv = tid >= D / 8;
@@ -369,108 +407,154 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     const int64_t kk = a.topk < n ? a.topk : n;
     const bool normal = n > 0 && kk < n;
     if (tid == 0) misc[kMTloc] = normal ? 0 : kBins;  // kBins: nothing is kept
-    __syncthreads();  // LUT, newc, tloc ready
+    __syncthreads();  // LUT, newr, tloc ready
 
-    // ---- stream: score every token of the warp's range
+    // ---- stream: score every token of the CTA's range, stage by stage
     const uint32_t lbase = lut_s | (4u * (uint32_t)lane);
-    const int upd = (int)(kk / 4 > 256 ? kk / 4 : 256);  // candidates between threshold updates
+
+    const int wsl = warp * 32 * TPL;                      // this warp's slice of a stage
     int ncand = 0;
     bool ovf = false, tmo = false;
     float *srow_out = a.scores_out ? a.scores_out + (int64_t)bh * a.ld_out + t0 : nullptr;
     volatile int *vtloc = misc + kMTloc;
-    float rnext = 0.0f;
-    if constexpr (RADIUS) rnext = (wb + lane < we) ? radius_of_token(kv, b, h, t0 + wb + lane) : 0.0f;
-    int j = 0;
+    float rad[TPL];
+#pragma unroll
+    for (int u = 0; u < TPL; ++u) rad[u] = 0.0f;
+    auto load_radius = [&](int s) {
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int i = s * STG_TOK + wsl + 32 * u + lane;
+            rad[u] = (s < nstg && i < nloc) ? radius_of_token(kv, b, h, t0 + i) : 0.0f;
+        }
+    };
+    if constexpr (RADIUS) load_radius(0);
+    // every stage but the last is full: one check covers them (the alignment of
+    // a stage is that of the first, and the last full one is the one nearest
+    // the capacity)
+    const bool bulk_mid = nstg > 1 && stage_bulk_bytes(nstg - 2) != 0u;
+    const bool bulk_last = nstg > 0 && stage_bulk_bytes(nstg - 1) != 0u;
+    int s = 0, slot = 0;
+    uint32_t phase = 0;
 #pragma unroll 1
-    for (; j < nk; ++j) {
-        const int slot = j % NS;
-        if (!mbar_wait(mbar_ring + 8u * slot, (uint32_t)((j / NS) & 1))) { tmo = true; break; }
-        const int i = wb + 32 * j + lane;  // CTA-local token
-        bool valid = i < we;
-        uint32_t w[BITS / 32];
-        bool bad;
-        if (chunk_src(j, bad)) {
-            const unsigned char *src = ring + (warp * NS + slot) * CHUNK_B + lane * CODE_B;
-            if constexpr (BITS == 128) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(src);
-                w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
-            } else if constexpr (BITS == 64) {
-                const uint2 x = *reinterpret_cast<const uint2 *>(src);
-                w[0] = x.x; w[1] = x.y;
-            } else {
-                w[0] = *reinterpret_cast<const uint32_t *>(src);
-            }
+    for (; s < nstg; ++s) {
+        bool bulk_bytes = false;
+        if constexpr (PAGED) {
+            asm volatile("cp.async.wait_group %0;" ::"n"(NS - 1) : "memory");
         } else {
-#pragma unroll
-            for (int k = 0; k < BITS / 32; ++k) w[k] = 0;
-            if (bad) valid = false;
-            if (valid) valid = load_code_plain<BITS>(kv, b, h, t0 + i, w);
+            if (!mbar_wait(mbar_full + 8u * slot, phase)) { tmo = true; break; }
+            bulk_bytes = s + 1 < nstg ? bulk_mid : bulk_last;
         }
-        if (t0 + i == pos) {
+        float rnow[TPL];
 #pragma unroll
-            for (int k = 0; k < BITS / 32; ++k) w[k] = newr[k];
+        for (int u = 0; u < TPL; ++u) rnow[u] = rad[u];
+        if constexpr (RADIUS) load_radius(s + 1);
+        // the stage's codes of this lane, then their scores (independent chains)
+        uint32_t w[TPL][BITS / 32];
+        bool valid[TPL];
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int li = wsl + 32 * u + lane;  // token within the stage
+            const int i = s * STG_TOK + li;      // CTA-local token
+            valid[u] = i < nloc;
+            if (PAGED || bulk_bytes) {
+                const unsigned char *src = ring + slot * STG_B + li * CODE_B;
+                if constexpr (BITS == 128) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(src);
+                    w[u][0] = x.x; w[u][1] = x.y; w[u][2] = x.z; w[u][3] = x.w;
+                } else if constexpr (BITS == 64) {
+                    const uint2 x = *reinterpret_cast<const uint2 *>(src);
+                    w[u][0] = x.x; w[u][1] = x.y;
+                } else {
+                    w[u][0] = *reinterpret_cast<const uint32_t *>(src);
+                }
+                if constexpr (PAGED) valid[u] = valid[u] && !((pbad >> (slot * TPL + u)) & 1u);
+            } else {
+#pragma unroll
+                for (int k = 0; k < BITS / 32; ++k) w[u][k] = 0;
+                if (valid[u]) valid[u] = load_code_plain<BITS>(kv, b, h, t0 + i, w[u]);
+            }
+            if (i == pos_loc) {
+#pragma unroll
+                for (int k = 0; k < BITS / 32; ++k) w[u][k] = newr[k];
+            }
         }
-        // the chunk's codes are in registers: refill its slot
+        float sc[TPL];
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            sc[u] = lut_score<BITS>(w[u], lbase);
+            if constexpr (RADIUS) sc[u] = __fmul_rn(sc[u], rnow[u]);
+        }
+        const int tl = *vtloc;
+        int bins[TPL];
+        bool isc[TPL];
+        bool mine = false;
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int i = s * STG_TOK + wsl + 32 * u + lane;
+            if (srow_out && valid[u]) srow_out[i] = sc[u];
+            bins[u] = score_bin(sc[u], inv2A);
+            isc[u] = valid[u] && bins[u] >= tl;
+            mine |= isc[u];
+        }
+        if (__any_sync(0xffffffffu, mine)) {
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                const uint32_t ball = __ballot_sync(0xffffffffu, isc[u]);
+                if (!ball) continue;
+                const int i = s * STG_TOK + wsl + 32 * u + lane;
+                if (isc[u]) {  // results unused: reductions, no round trip
+                    atomicAdd(&hist[bins[u]], 1u);
+                    atomicAdd(&sup[bins[u] >> 6], 1u);
+                }
+                const int nb = __popc(ball);
+                if (!ovf && ncand + nb > cap) {
+                    // full: raise the threshold to the CTA's current k-th bin and drop what is below
+                    const int tnew = local_threshold(sup, hist, kk);
+                    if (lane == 0) atomicMax(misc + kMTloc, tnew);
+                    __syncwarp();
+                    ncand = compact_candidates(cand_lo, cand_hi, cap_lo, ncand, *vtloc, inv2A);
+                    if (ncand + nb > cap) {
+                        ovf = true;
+                        if (lane == 0) misc[kMOvf] = 1;
+                    }
+                }
+                if (!ovf) {
+                    if (isc[u]) cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)i, float_key(sc[u]));
+                    ncand += nb;
+                }
+            }
+        }
+        // once per stage one warp (in turn) moves the CTA's threshold up to the
+        // bin of its current k-th largest counted score
+        if (warp == (s % NWARP) && tl < kBins) {
+            const int tnew = local_threshold(sup, hist, kk);
+            if (lane == 0 && tnew > tl) atomicMax(misc + kMTloc, tnew);
+        }
+        // release the slot and refill it with stage s + NS
         __syncwarp();
-        if (j + NS < nk) issue(j + NS);
-        float sc = lut_score<BITS>(w, lbase);
-        if constexpr (RADIUS) {
-            const float rc = rnext;
-            const int i2 = i + 32;
-            rnext = (j + 1 < nk && i2 < we) ? radius_of_token(kv, b, h, t0 + i2) : 0.0f;
-            sc = __fmul_rn(sc, rc);
-        }
-        if (srow_out && valid) srow_out[i] = sc;
-        const int bin = score_bin(sc, inv2A);
-        const bool isc = valid && bin >= *vtloc;
-        const uint32_t ball = __ballot_sync(0xffffffffu, isc);
-        if (ball) {
-            if (isc) {
-                atomicAdd(&hist[bin], 1u);
-                atomicAdd(&sup[bin >> 6], 1u);
-            }
-            const int nb = __popc(ball);
-            if (!ovf && ncand + nb > cap) {
-                // full: raise the threshold to the CTA's current k-th bin and drop what is below
-                const int tnew = local_threshold(sup, hist, kk);
-                if (lane == 0) atomicMax(misc + kMTloc, tnew);
-                __syncwarp();
-                const int tl = *vtloc;
-                int kept = 0;
-                for (int jb = 0; jb < ncand; jb += 32) {
-                    const int jj = jb + lane;
-                    uint2 e = make_uint2(0u, 0u);
-                    if (jj < ncand) e = cand_ref(jj);
-                    const bool keep = jj < ncand && score_bin(key_to_float(e.y), inv2A) >= tl;
-                    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-                    __syncwarp();
-                    if (keep) cand_ref(kept + __popc(kb & lt)) = e;
-                    kept += __popc(kb);
-                    __syncwarp();
-                }
-                ncand = kept;
-                if (ncand + nb > cap) {
-                    ovf = true;
-                    if (lane == 0) misc[kMOvf] = 1;
-                }
-            }
-            if (!ovf) {
-                if (isc) cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)(i - wb), float_key(sc));
-                ncand += nb;
-            }
-            int trig = 0;
+        if constexpr (PAGED) {
+            int pg[TPL];
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) pg[u] = pgn[u];
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) pgn[u] = lane_page(s + NS + 1, u);
+            issue_paged(s + NS, pg);
+        } else {
             if (lane == 0) {
-                const int old = atomicAdd(misc + kMIns, nb);
-                trig = (old / upd) != ((old + nb) / upd);
+                // the last of the warps to finish with the slot refills it (the
+                // count only grows: every NWARP arrivals are one use of the slot)
+                const uint32_t old = atomicAdd(stg_cnt + slot, 1u);
+                if ((old + 1u) % NWARP == 0u && s + NS < nstg) issue_dense(s + NS);
             }
-            if (__shfl_sync(0xffffffffu, trig, 0)) {
-                const int tnew = local_threshold(sup, hist, kk);
-                if (lane == 0) atomicMax(misc + kMTloc, tnew);
-            }
+        }
+        if (++slot == NS) {
+            slot = 0;
+            phase ^= 1u;
         }
     }
+    if constexpr (PAGED) asm volatile("cp.async.wait_group 0;" ::: "memory");
     if (tmo) {  // give the copies still in flight a bounded chance to land before the buffers are reused
-        for (int c = j; c < nk && c < j + NS; ++c) mbar_wait(mbar_ring + 8u * (c % NS), (uint32_t)((c / NS) & 1));
+        for (int c = s; c < nstg && c < s + NS; ++c) mbar_wait(mbar_full + 8u * (c % NS), (uint32_t)((c / NS) & 1));
         if (lane == 0) misc[kMOvf] = 1;
         ovf = true;
     }
@@ -478,18 +562,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
 
     // ---- the cluster's threshold bin T1 (exact: every CTA counted every token
     // of every bin at or above it)
-    if (tid == 0) { misc[kMT1] = kBins; misc[kMAbove] = 0; misc[kMCntT1] = 0; misc[kMNinb] = 0; }
+    if (tid == 0) { misc[kMT1] = kBins; misc[kMAbove] = 0; misc[kMCntT1] = 0; misc[kMNinb] = 0; misc[kMKept] = 0; }
     cluster_sync();  // (1)
-    if (appending && cta == 0 && tid == 0) {
-        // every CTA of this cluster has read seq_lens[b]; the last cluster of
-        // the sequence to get here moves its length on
-        __threadfence();
-        const uint32_t old = atomicAdd(a.seq_arrive + (int64_t)b * kSyncStride, 1u);
-        if (old == (uint32_t)(kv.Hkv - 1)) {
-            a.seq_arrive[(int64_t)b * kSyncStride] = 0;
-            if (app_ok) a.seq_lens[b] = (int32_t)(pos + 1);
-        }
-    }
     if (normal && warp == 0) cluster_threshold(sup, hist, nctas, kk, misc + kMT1);
     if (warp == 1) {
         const int f = lane < nctas ? (int)ld_cluster_u32(cluster_addr(misc + kMOvf, lane)) : 0;
@@ -501,20 +575,29 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     const int s_end = (int)(a.S < n ? a.S : n);
     const int w_beg = (int)(n - a.W > s_end ? n - a.W : s_end);
     int32_t *out = a.sel_idx + (int64_t)bh * a.cap_sel;
-    bool slow = !normal || misc[kMAnyOvf] != 0 || cnt_T1 > kInbinMax;
+    // the kept tokens of this CTA are placed through a bitmap of its range
+    // (after the in-bin lists in the idle ring); a range too long for it takes
+    // the slow path
+    uint4 *s_loc = reinterpret_cast<uint4 *>(ring);              // this CTA's in-bin tokens
+    uint4 *s_inb = reinterpret_cast<uint4 *>(ring) + kInbinMax;  // the cluster's
+    uint32_t *bmap = reinterpret_cast<uint32_t *>(ring + 2 * kInbinMax * 16);
+    constexpr int kBmapWords = (SS::RING_B - 2 * kInbinMax * 16) / 4;
+    const int nwords = (nloc + 31) / 32;
+    // (the same decision in every CTA of the cluster: the bitmap bound uses the
+    // longest range cta_range gives any CTA)
+    const int64_t max_range = ceil_div(ceil_div(n, nctas), 64) * 64;
+    const bool slow = !normal || misc[kMAnyOvf] != 0 || cnt_T1 > kInbinMax || ceil_div(max_range, 32) > kBmapWords;
 
-    int total_mid = 0;
     if (!slow) {
         // ---- fast path: classify this warp's candidates (definite: bin > T1,
         // in the threshold bin: listed for the cluster)
-        uint4 *s_loc = reinterpret_cast<uint4 *>(ring);              // this CTA's in-bin tokens
-        uint4 *s_inb = reinterpret_cast<uint4 *>(ring) + kInbinMax;  // the cluster's
+        for (int x = tid; x < nwords; x += NT) bmap[x] = 0u;
         int ndef = 0;
         for (int jb = 0; jb < ncand; jb += 32) {
             const int jj = jb + lane;
             uint2 e = make_uint2(0u, 0u);
             if (jj < ncand) e = cand_ref(jj);
-            const int t = (int)(t0 + wb + (int)e.x);
+            const int t = (int)(t0 + (int)e.x);
             const int bin = score_bin(key_to_float(e.y), inv2A);
             const bool inb = jj < ncand && bin == T1;
             const bool def = jj < ncand && bin > T1 && t >= s_end && t < w_beg;
@@ -525,15 +608,15 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
                 if (lane == 0) base = atomicAdd(misc + kMNinb, __popc(ib));
                 base = __shfl_sync(0xffffffffu, base, 0);
                 const int slot = base + __popc(ib & lt);
-                if (inb && slot < kInbinMax) s_loc[slot] = make_uint4(e.y, (uint32_t)t, (uint32_t)cta, (uint32_t)warp);
+                if (inb && slot < kInbinMax) s_loc[slot] = make_uint4(e.y, (uint32_t)t, (uint32_t)cta, 0u);
             }
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
-        if (lane == 0) s_wkeep[warp] = ndef;
+        if (lane == 0) s_wdef[warp] = ndef;
         __syncthreads();
         if (warp == 0) {  // publish (in-bin entries, definite middle tokens) into every CTA's s_cnt[cta]
-            int dsum = s_wkeep[lane];
+            int dsum = lane < NWARP ? s_wdef[lane] : 0;
 #pragma unroll
             for (int o = 16; o; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
             const int ni = min(misc[kMNinb], kInbinMax);
@@ -544,7 +627,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         }
         cluster_sync();  // (2)
         const int c1 = cnt_T1;
-        if (warp * 32 < c1) {  // thread e copies in-bin entry e from the CTA whose list holds it
+        {   // entry e of the cluster's in-bin list comes from the CTA whose list holds it
             const int ni = lane < nctas ? s_cnt[lane][0] : 0;
             int incl = ni;
 #pragma unroll
@@ -553,14 +636,18 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
                 if (lane >= o) incl += y;
             }
             const int excl = incl - ni;
-            int r = 0;
-            for (int qq = 1; qq < nctas; ++qq) r = __shfl_sync(0xffffffffu, excl, qq) <= tid ? qq : r;
-            const int off = tid - __shfl_sync(0xffffffffu, excl, r);
-            if (tid < c1) s_inb[tid] = ld_cluster_v4(cluster_addr(s_loc + off, r));
+            for (int e0 = warp * 32; e0 < c1; e0 += NT) {
+                const int e = e0 + lane;
+                int r = 0;
+                for (int qq = 1; qq < nctas; ++qq) r = __shfl_sync(0xffffffffu, excl, qq) <= e ? qq : r;
+                const int off = e - __shfl_sync(0xffffffffu, excl, r);
+                if (e < c1) s_inb[e] = ld_cluster_v4(cluster_addr(s_loc + off, r));
+            }
         }
         __syncthreads();
         cluster_arrive();  // (3): done with the other CTAs' shared memory
-        // rank the in-bin list: the need1-th (score desc, token asc) is the last selected
+        // rank the in-bin list: the need1-th (score desc, token asc) is the last
+        // selected; count the selected middle ones per CTA (output offsets)
         const int need1 = (int)kk - above1;
         if (c1 <= 32) {
             if (warp == 0) {
@@ -585,7 +672,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
                     const int cr = __popc(__ballot_sync(0xffffffffu, sel && (int)en.z == r));
                     if (lane == r) mid = s_cnt[r][1] + cr;
                 }
-                if (sel && (int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
                 int before = lane < cta ? mid : 0, tot = mid;
 #pragma unroll
                 for (int o = 16; o; o >>= 1) {
@@ -615,10 +701,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             for (int e = tid; e < c1; e += NT) {
                 const uint4 en = s_inb[e];
                 const int t = (int)en.y;
-                if (t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT))) {
-                    atomicAdd(&s_mid[en.z], 1);
-                    if ((int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
-                }
+                if (t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT))) atomicAdd(&s_mid[en.z], 1);
             }
             __syncthreads();
             if (tid == 0) {
@@ -634,25 +717,36 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         __syncthreads();
         const uint32_t Tkey = (uint32_t)misc[kMTkey];
         const int IT = misc[kMIT];
-        total_mid = misc[kMTotal];
-        // ordered emission: warp w writes its kept candidates after those of CTAs
-        // < cta and warps < w
-        int wpos = s_end + misc[kMBefore];
-        for (int w2 = 0; w2 < warp; ++w2) wpos += s_wkeep[w2];
+        const int total_mid = misc[kMTotal];
+        // kept middle tokens of this CTA into the bitmap, then written in
+        // token order after those of CTAs < cta
         for (int jb = 0; jb < ncand; jb += 32) {
             const int jj = jb + lane;
-            uint2 e = make_uint2(0u, 0u);
-            if (jj < ncand) e = cand_ref(jj);
-            const int t = (int)(t0 + wb + (int)e.x);
-            const int bin = score_bin(key_to_float(e.y), inv2A);
-            const bool keep = jj < ncand && t >= s_end && t < w_beg &&
-                              (bin > T1 || (bin == T1 && (e.y > Tkey || (e.y == Tkey && t <= IT))));
-            const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-            if (keep) {
-                const int p = wpos + __popc(kb & lt);
-                if (p < a.cap_sel) out[p] = t;
+            if (jj < ncand) {
+                const uint2 e = cand_ref(jj);
+                const int t = (int)(t0 + (int)e.x);
+                const int bin = score_bin(key_to_float(e.y), inv2A);
+                if (t >= s_end && t < w_beg && (bin > T1 || (bin == T1 && (e.y > Tkey || (e.y == Tkey && t <= IT)))))
+                    atomicOr(bmap + (e.x >> 5), 1u << (e.x & 31));
             }
-            wpos += __popc(kb);
+        }
+        __syncthreads();
+        {
+            const int per = (nwords + NT - 1) / NT;
+            const int w0 = tid * per, w1 = min(nwords, w0 + per);
+            int cnt = 0;
+            for (int x = w0; x < w1; ++x) cnt += __popc(bmap[x]);
+            int tot;
+            int p = s_end + misc[kMBefore] + block_excl_scan<NT>(cnt, s_warp, &tot);
+            for (int x = w0; x < w1; ++x) {
+                uint32_t m = bmap[x];
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (p < a.cap_sel) out[p] = (int32_t)(t0 + 32 * x + bit);
+                    ++p;
+                }
+            }
         }
         {   // the sinks, the window and the padding, spread over the cluster's CTAs
             const int wpos0 = s_end + total_mid;
@@ -678,7 +772,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         // tokens of bins >= T1 per CTA, and let CTA 0 resolve and emit.
         float *srow = a.ws.scores + (int64_t)bh * a.ws.ld;
         int32_t *cand = a.ws.cand + (int64_t)bh * a.ws.ld;
-        int *s_warp = s_wkeep;  // scratch for the block scan
         int seg = 0;
         if (normal) {
             for (int64_t base = t0; base < t1; base += NT) {
@@ -721,14 +814,13 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
 
     if constexpr (G > 0) {
         // ---- attention over the emitted list: CTA c takes an equal slice of it
-        __threadfence();
-        cluster_sync();  // (4): the whole list and its count are written
+        cluster_sync();  // (4): the whole list and its count are written (cluster-scope release / acquire)
         constexpr int HG = G < 4 ? G : 4;   // query heads per warp
         constexpr int NTEAM = G / HG;       // warp teams, each over every row for its HG heads
         constexpr int WPT = NWARP / NTEAM;  // warps per team
         constexpr int SL = 32 / HG;         // lanes per head: dim slices
         constexpr int DPL = D / SL;         // dims per lane
-        constexpr int TROWS = D == 128 ? 4 : 8;
+        constexpr int TROWS = 8;
         constexpr int ROW_B = D * 2;
         constexpr int TILE_B = TROWS * 2 * ROW_B;
         static_assert(DPL % 8 == 0 || DPL == 4 || DPL == 2, "dims per lane");
@@ -920,6 +1012,16 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             if (i == 0 && a.lse) a.lse[oq] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
         }
         cluster_sync();  // (6): no CTA leaves while another may still read its partial
+    }
+    if (appending && cta == 0 && tid == 0) {
+        // every CTA of this cluster read seq_lens[b] before barrier (1); the last
+        // cluster of the sequence to get here moves its length on
+        __threadfence();
+        const uint32_t old = atomicAdd(a.seq_arrive + (int64_t)b * kSyncStride, 1u);
+        if (old == (uint32_t)(kv.Hkv - 1)) {
+            a.seq_arrive[(int64_t)b * kSyncStride] = 0;
+            if (app_ok) a.seq_lens[b] = (int32_t)(pos + 1);
+        }
     }
 }
 

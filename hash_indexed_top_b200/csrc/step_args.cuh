@@ -6,15 +6,21 @@
 
 namespace dkv {
 
-constexpr int kStepThreads = 1024;
+constexpr int kStepThreads = 512;
 constexpr int kStepWarps = kStepThreads / 32;
 constexpr int kRingStages = 5;
 
+// The code stream runs in CTA-wide stages of STG_TOK consecutive tokens
+// (16 KB of codes): warp w takes the 32 TPL tokens [32 TPL w, 32 TPL (w + 1))
+// of every stage, lane l those congruent to l mod 32 (TPL of them, so the
+// per-stage bookkeeping of a warp is shared by several tokens per lane).
 template <int BITS>
 struct StepShape {
     static constexpr int CODE_B = BITS >= 64 ? BITS / 8 : 8;  // bytes of one token's code in memory
-    static constexpr int CHUNK_B = 32 * CODE_B;               // one warp step: 32 tokens
-    static constexpr int RING_B = kStepWarps * kRingStages * CHUNK_B;
+    static constexpr int TPL = BITS == 128 ? 2 : 4;            // tokens per lane per stage
+    static constexpr int STG_TOK = kStepThreads * TPL;         // tokens per stage
+    static constexpr int STG_B = STG_TOK * CODE_B;             // bytes per stage (16 KB)
+    static constexpr int RING_B = kRingStages * STG_B;
 };
 
 // Fixed part of the low shared region (byte offsets from the dynamic base).
@@ -27,20 +33,21 @@ struct StepLow {
     static constexpr int MISC = KNEW + kMaxDim * 4;                // int[64]
     static constexpr int NEWC = MISC + 64 * 4;                     // u32[4] appended key's code
     static constexpr int NEWR = NEWC + 16;                         // u32[4] the same in stored (rotated) order
-    static constexpr int MBAR = NEWR + 16;                         // u64[kStepWarps][kRingStages]
-    static constexpr int MBAR_ATT = MBAR + kStepWarps * kRingStages * 8;  // u64[kStepWarps][2]
-    static constexpr int WKEEP = MBAR_ATT + kStepWarps * 2 * 8;    // int[kStepWarps]
-    static constexpr int CNT = WKEEP + kStepWarps * 4;             // int[kMaxCluster][2]
+    static constexpr int MBAR = NEWR + 16;                         // u64[kRingStages] full barriers of the ring
+    static constexpr int STG_CNT = MBAR + kRingStages * 8;         // u32[kRingStages] warps done with a slot
+    static constexpr int MBAR_ATT = (STG_CNT + kRingStages * 4 + 7) / 8 * 8;  // u64[kStepWarps][2]
+    static constexpr int WDEF = MBAR_ATT + kStepWarps * 2 * 8;     // int[kStepWarps] definite tokens per warp
+    static constexpr int CNT = WDEF + kStepWarps * 4;              // int[kMaxCluster][2]
     static constexpr int MID = CNT + kMaxCluster * 8;              // int[kMaxCluster]
-    static constexpr int WKEY = MID + kMaxCluster * 4;             // unused pad
-    static constexpr int END = (WKEY + 255) / 256 * 256;           // candidate lists start here
+    static constexpr int WARPSCAN = MID + kMaxCluster * 4;         // int[32] block-scan scratch
+    static constexpr int END = (WARPSCAN + 128 + 255) / 256 * 256; // candidate lists start here
 };
-static_assert(StepLow::MBAR % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(StepLow::MBAR % 8 == 0 && StepLow::MBAR_ATT % 8 == 0, "mbarriers are 8-byte aligned");
 
 // misc[] slots
 enum : int {
     kMTloc = 0, kMIns = 1, kMNinb = 2, kMOvf = 3, kMT1 = 4, kMAbove = 5, kMCntT1 = 6,
-    kMTkey = 8, kMIT = 9, kMBefore = 10, kMTotal = 11, kMAnyOvf = 12, kMIbOvf = 13, kMAnyIbOvf = 14
+    kMTkey = 8, kMIT = 9, kMBefore = 10, kMTotal = 11, kMAnyOvf = 12, kMKept = 13
 };
 
 struct StepArgs {
