@@ -294,7 +294,8 @@ int setup_step_kernels(const dashkv_ctx *c) {
     }
     // the layout needs the low region below the LUT's 64 KB boundary, the LUT, the
     // code ring and some candidate room above it
-    const int ring = kStepWarps * kRingStages * 32 * (c->cfg.bits >= 64 ? c->cfg.bits / 8 : 8);
+    const int code_b = c->cfg.bits >= 64 ? c->cfg.bits / 8 : 8;
+    const int ring = kRingStages * kStreamWarps * 32 * (c->cfg.bits == 128 ? 2 : 4) * code_b;
     if (smem < 2 * 65536 + ring + 4096) return 0;
     for (int i = 0; i < nk; ++i) {
         cudaFuncSetAttribute(ks[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

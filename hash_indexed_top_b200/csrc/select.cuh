@@ -792,18 +792,27 @@ constexpr int kInbinMax = 1024;
 constexpr int kMaxCluster = 16;
 
 // Threshold of the cluster's summed histogram, computed by one full warp from
-// the CTAs' super-bin counts (coarse[64], super-bin s = bins [64 s, 64 s + 64))
-// and histograms (hist[kBins]), both read in place in every CTA's shared
-// memory.  Returns T1 to every lane; out (when not null) = {T1, tokens above
-// T1, tokens in T1} as threshold_bin.
+// the CTAs' super-bin counts (coarse[64], super-bin s = bins [PER s, PER s +
+// PER)) and histograms (hist[64 PER]), both read in place in every CTA's
+// shared memory (LOCAL: this CTA's alone, nranks ignored).  Returns the bin
+// holding the kk-th largest counted score to every lane, or -1 when fewer than
+// kk are counted; out (when not null and the bin exists) = {bin, tokens above
+// it, tokens in it} as threshold_bin.
+template <int PER = kBins / 64, bool LOCAL = false>
 __device__ __forceinline__ int cluster_threshold(const uint32_t *coarse, const uint32_t *hist, int nranks,
                                                  int64_t kk, int *out) {
+    static_assert(PER % 2 == 0 && PER <= 64, "fine bins per super-bin");
     const int lane = threadIdx.x & 31;
+    if (LOCAL) nranks = 1;
+    auto ld = [&](const uint32_t *p, int r) -> uint32_t {
+        if constexpr (LOCAL) return *reinterpret_cast<const volatile uint32_t *>(p);
+        else return ld_cluster_u32(cluster_addr(p, r));
+    };
     // lane l holds super-bins 63 - 2l (upper) and 62 - 2l (lower): lane 0 the top
     uint32_t cu = 0, cl = 0;
     for (int r = 0; r < nranks; ++r) {
-        cu += ld_cluster_u32(cluster_addr(coarse + (63 - 2 * lane), r));
-        cl += ld_cluster_u32(cluster_addr(coarse + (62 - 2 * lane), r));
+        cu += ld(coarse + (63 - 2 * lane), r);
+        cl += ld(coarse + (62 - 2 * lane), r);
     }
     int64_t incl = (int64_t)cu + cl;
 #pragma unroll
@@ -813,22 +822,25 @@ __device__ __forceinline__ int cluster_threshold(const uint32_t *coarse, const u
     }
     const int64_t excl = incl - cu - cl;
     const bool here = excl < kk && kk <= incl;
+    const uint32_t hb = __ballot_sync(0xffffffffu, here);
+    if (!hb) return -1;  // fewer than kk counted
     int sb = 0;
     int64_t above = 0;
     if (here) {
         if (excl + cu >= kk) { sb = 63 - 2 * lane; above = excl; }
         else { sb = 62 - 2 * lane; above = excl + cu; }
     }
-    const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
-    sb = __shfl_sync(0xffffffffu, sb, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    // the 64 bins of super-bin sb, the same way
-    const int bu = 64 * sb + 63 - 2 * lane, bl = bu - 1;
+    sb = __shfl_sync(0xffffffffu, sb, __ffs(hb) - 1);
+    above = __shfl_sync(0xffffffffu, above, __ffs(hb) - 1);
+    // the PER bins of super-bin sb, the same way (lanes >= PER / 2 hold none)
+    const bool has = lane < PER / 2;
+    const int bu = PER * sb + PER - 1 - 2 * lane, bl = bu - 1;
     uint32_t fu = 0, fl = 0;
-    for (int r = 0; r < nranks; ++r) {
-        fu += ld_cluster_u32(cluster_addr(hist + bu, r));
-        fl += ld_cluster_u32(cluster_addr(hist + bl, r));
-    }
+    if (has)
+        for (int r = 0; r < nranks; ++r) {
+            fu += ld(hist + bu, r);
+            fl += ld(hist + bl, r);
+        }
     int64_t fincl = (int64_t)fu + fl;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -837,13 +849,15 @@ __device__ __forceinline__ int cluster_threshold(const uint32_t *coarse, const u
     }
     const int64_t fexcl = above + fincl - fu - fl;
     fincl += above;
-    const bool hit = fexcl < kk && kk <= fincl;
+    const bool hit = has && fexcl < kk && kk <= fincl;
+    const uint32_t hm = __ballot_sync(0xffffffffu, hit);
+    if (!hm) return -1;  // (counts that did not add up: not reached with settled counts)
     const int t1 = hit ? (fexcl + fu >= kk ? bu : bl) : 0;
     if (hit && out) {
         if (fexcl + fu >= kk) { out[0] = bu; out[1] = (int)fexcl; out[2] = (int)fu; }
         else { out[0] = bl; out[1] = (int)(fexcl + fu); out[2] = (int)fl; }
     }
-    return __shfl_sync(0xffffffffu, t1, __ffs(__ballot_sync(0xffffffffu, hit)) - 1);
+    return __shfl_sync(0xffffffffu, t1, __ffs(hm) - 1);
 }
 
 }  // namespace dkv

@@ -10,31 +10,45 @@
 // paragraph of its CSA section (a recent window stays exact); DySCO page, Q3
 // (attention sinks).
 //
-// Grid: one thread-block cluster of C CTAs (1024 threads, one per SM) per
-// (sequence, kv head); CTA c owns a contiguous, 64-aligned token range.
+// Grid: one thread-block cluster of C CTAs (16 consumer warps and one producer
+// warp, one CTA per SM) per (sequence, kv head); CTA c owns a contiguous,
+// 64-aligned token range.
 //
 //  stream   the CTA streams its codes in stages of 16 KB through a ring in
 //           shared memory: dense caches by one bulk copy per stage
-//           (cp.async.bulk, completion counted in bytes on the stage's
-//           mbarrier, issued by the last warp to finish with the slot), paged
-//           caches by per-thread cp.async of each thread's own tokens.  Warp w
+//           (cp.async.bulk, completion counted in bytes on the stage's full
+//           mbarrier), issued by the producer warp as soon as every consumer
+//           warp has released the slot on its empty mbarrier; paged caches by
+//           per-thread cp.async of each thread's own tokens (warp 15 idles).
+//           A consumer warp (0..14)
+//           reads the next stage's codes into registers before it scores the
+//           current one, and releases a slot as soon as its codes are in
+//           registers.  Consumer warp w
 //           takes a 32- or 64-token slice of every stage and lane l scores the
 //           tokens t = l (mod 32) with the byte-LUT of the query (the codes are
 //           stored byte-rotated by t mod T, see store_code_rotated).  A token
-//           whose histogram bin reaches the CTA's running threshold is kept
-//           with its exact order key in the warp's candidate list in shared
-//           memory and counted in the CTA histogram; the running threshold is
-//           the bin of the CTA's k-th largest score so far (never above the
-//           final one), so every token that can be selected is kept and the
-//           histogram is exact for every bin at or above the final threshold.
+//           whose score reaches the CTA's threshold is kept with its exact
+//           order key in the warp's candidate list in shared memory; after the
+//           stream every warp counts its list into the CTA histogram.
+//  estimate the threshold comes from a stratified sample of the whole
+//           sequence scored before the stream (the same 32-token blocks in
+//           every CTA of the cluster): the bin of a sample rank set a few
+//           standard deviations above the one the k-th largest score is
+//           expected at.  It is an estimate and nothing rests on it: when the
+//           cluster's k-th largest counted score lies below the threshold (or
+//           fewer than k are counted) the estimate was too high, and a full
+//           candidate list means it was far too low; either way the exact slow
+//           path runs.
 //  select   the cluster sums its histograms through distributed shared
-//           memory and finds the bin T1 holding the k-th largest score; the
-//           warps classify their candidates, rank the few of bin T1 exactly
-//           (score desc, index asc), mark the kept tokens in a bitmap of the
-//           CTA's range and write them in order.  Heavy
-//           ties (more than kInbinMax tokens in T1) or a full candidate list
-//           take an exact slow path (re-score into the workspace, CTA 0 runs
-//           the two-kernel path's resolver).
+//           memory and finds the bin T1 holding the k-th largest score (exact:
+//           every CTA counted every token of every bin at or above its
+//           threshold, and no threshold is above T1); the warps classify their
+//           candidates, rank the few of bin T1 exactly (score desc, index
+//           asc), mark the kept tokens in a bitmap of the CTA's range and
+//           write them in order.  Heavy ties (more than kInbinMax tokens in
+//           T1), a full candidate list or a threshold estimate above T1 take
+//           an exact slow path (re-score and count every token into the
+//           workspace, CTA 0 runs the two-kernel path's resolver).
 //  attend   (G > 0) every CTA takes an equal slice of the emitted list, bulk
 //           copies the K and V rows into shared memory (two tiles in flight
 //           per warp) and runs an online softmax in fp32; the CTAs' partial
@@ -49,74 +63,6 @@
 #include "step_args.cuh"
 
 namespace dkv {
-
-// Bin of the CTA's kk-th largest counted score from its super-bin and bin
-// counts (one full warp; 0 when fewer than kk are counted).  Counts only grow
-// while this runs, so a stale read can only give a lower bin.
-__device__ __forceinline__ int local_threshold(const uint32_t *sup, const uint32_t *hist, int64_t kk) {
-    const int lane = threadIdx.x & 31;
-    const volatile uint32_t *vs = sup;
-    const volatile uint32_t *vh = hist;
-    const uint32_t cu = vs[63 - 2 * lane], cl = vs[62 - 2 * lane];
-    int64_t incl = (int64_t)cu + cl;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    const int64_t excl = incl - cu - cl;
-    const bool here = excl < kk && kk <= incl;
-    const uint32_t hb = __ballot_sync(0xffffffffu, here);
-    if (!hb) return 0;
-    int sb = 0;
-    int64_t above = 0;
-    if (here) {
-        if (excl + cu >= kk) { sb = 63 - 2 * lane; above = excl; }
-        else { sb = 62 - 2 * lane; above = excl + cu; }
-    }
-    const int src = __ffs(hb) - 1;
-    sb = __shfl_sync(0xffffffffu, sb, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    const int bu = 64 * sb + 63 - 2 * lane, bl = bu - 1;
-    const uint32_t fu = vh[bu], fl = vh[bl];
-    int64_t fincl = (int64_t)fu + fl;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int64_t y = __shfl_up_sync(0xffffffffu, fincl, o);
-        if (lane >= o) fincl += y;
-    }
-    const int64_t fexcl = above + fincl - fu - fl;
-    fincl += above;
-    const bool hit = fexcl < kk && kk <= fincl;
-    const uint32_t hm = __ballot_sync(0xffffffffu, hit);
-    if (!hm) return 64 * sb;  // counts moved under the read: the super-bin's floor is still a lower bound
-    const int t = hit ? (fexcl + fu >= kk ? bu : bl) : 0;
-    return __shfl_sync(0xffffffffu, t, __ffs(hm) - 1);
-}
-
-// Drop from a warp's candidate list (entries j < ncand, the first cap_lo in
-// lo[], the rest in hi[]) the ones whose bin is below tl, keeping their order;
-// returns the new count.  One full warp; out of line (rare).
-static __device__ __noinline__ int compact_candidates(uint2 *lo, uint2 *hi, int cap_lo, int ncand, int tl, float inv2A) {
-    const int lane = threadIdx.x & 31;
-    const uint32_t lt = (1u << lane) - 1u;
-    int kept = 0;
-    for (int jb = 0; jb < ncand; jb += 32) {
-        const int jj = jb + lane;
-        uint2 e = make_uint2(0u, 0u);
-        if (jj < ncand) e = jj < cap_lo ? lo[jj] : hi[jj - cap_lo];
-        const bool keep = jj < ncand && score_bin(key_to_float(e.y), inv2A) >= tl;
-        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-        __syncwarp();
-        if (keep) {
-            const int d = kept + __popc(kb & lt);
-            if (d < cap_lo) lo[d] = e; else hi[d - cap_lo] = e;
-        }
-        kept += __popc(kb);
-        __syncwarp();
-    }
-    return kept;
-}
 
 // fp32 LUT score of one token's (rotated) code words for a token t (any lane):
 // lane offset t mod 32 keeps the table order right (t mod T = lane mod T).
@@ -153,7 +99,7 @@ template <int BITS, int D, int G, bool PAGED, bool RADIUS>
 __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, const RBits R) {
     using SS = StepShape<BITS>;
     constexpr int NS = kRingStages;
-    constexpr int NWARP = kStepWarps, NT = kStepThreads;
+    constexpr int NWARP = kStepWarps, NT = kStepThreads, NCONS = kStreamWarps;
     constexpr int CODE_B = SS::CODE_B, TPL = SS::TPL, STG_TOK = SS::STG_TOK, STG_B = SS::STG_B;
     constexpr int T = BITS / 8;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -166,18 +112,21 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     const uint32_t smem_s = (uint32_t)__cvta_generic_to_shared(smem);
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + StepLow::HIST);
     uint32_t *sup = reinterpret_cast<uint32_t *>(smem + StepLow::SUP);
+    uint32_t *shist = reinterpret_cast<uint32_t *>(smem + StepLow::SHIST);
+    uint32_t *ssup = reinterpret_cast<uint32_t *>(smem + StepLow::SSUP);
     float *qsum = reinterpret_cast<float *>(smem + StepLow::QSUM);
     float *Qp = reinterpret_cast<float *>(smem + StepLow::QP);
     float *knew = reinterpret_cast<float *>(smem + StepLow::KNEW);
     int *misc = reinterpret_cast<int *>(smem + StepLow::MISC);
     uint32_t *newc = reinterpret_cast<uint32_t *>(smem + StepLow::NEWC);
     uint32_t *newr = reinterpret_cast<uint32_t *>(smem + StepLow::NEWR);
-    uint32_t *stg_cnt = reinterpret_cast<uint32_t *>(smem + StepLow::STG_CNT);
     int *s_wdef = reinterpret_cast<int *>(smem + StepLow::WDEF);
     int (*s_cnt)[2] = reinterpret_cast<int (*)[2]>(smem + StepLow::CNT);
     int *s_mid = reinterpret_cast<int *>(smem + StepLow::MID);
     int *s_warp = reinterpret_cast<int *>(smem + StepLow::WARPSCAN);
-    const uint32_t mbar_full = smem_s + StepLow::MBAR;  // [NS]
+    const uint32_t mbar_full = smem_s + StepLow::MBAR;         // [NS]
+    const uint32_t mbar_empty = smem_s + StepLow::MBAR_EMPTY;  // [NS]
+    const bool consumer = warp < NCONS;  // (during the stream; warp NCONS is its producer)
     const uint32_t mbar_att = smem_s + StepLow::MBAR_ATT + 8u * (uint32_t)(warp * 2);
     const uint32_t lut_s = (smem_s + StepLow::END + 65535u) & ~65535u;  // 64 KB aligned
     unsigned char *lut = smem + (lut_s - smem_s);
@@ -185,8 +134,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     unsigned char *ring = lut + 65536;
     const uint32_t end_s = smem_s + (uint32_t)a.smem_bytes;
     // candidate list of this warp: cap_lo entries below the LUT, cap_hi above the ring
-    const int cap_lo = (int)((lut_s - (smem_s + StepLow::END)) / (8u * NWARP));
-    const int cap_hi = end_s > ring_s + SS::RING_B ? (int)((end_s - ring_s - SS::RING_B) / (8u * NWARP)) : 0;
+    // (NCONS lists: warp NCONS has none and keeps ncand = 0)
+    const int cap_lo = (int)((lut_s - (smem_s + StepLow::END)) / (8u * NCONS));
+    const int cap_hi = end_s > ring_s + SS::RING_B ? (int)((end_s - ring_s - SS::RING_B) / (8u * NCONS)) : 0;
     uint2 *cand_lo = reinterpret_cast<uint2 *>(smem + StepLow::END) + warp * cap_lo;
     uint2 *cand_hi = reinterpret_cast<uint2 *>(ring + SS::RING_B) + warp * cap_hi;
     const int cap = cap_lo + cap_hi;
@@ -194,9 +144,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
 
     // ---- set-up: counters, barriers, this warp's hyperplane words
     for (int i = tid; i < kBins; i += NT) hist[i] = 0;
-    if (tid < 64) { sup[tid] = 0; misc[tid] = 0; }
+    for (int i = tid; i < kSampleBins; i += NT) shist[i] = 0;
+    if (tid < 64) { sup[tid] = 0; ssup[tid] = 0; misc[tid] = 0; }
     if (tid < 4) newc[tid] = 0;
-    if (tid < NS) { mbar_init(mbar_full + 8u * tid, 1); stg_cnt[tid] = 0; }
+    if (tid < NS) { mbar_init(mbar_full + 8u * tid, 1); mbar_init(mbar_empty + 8u * tid, NCONS); }
     if (tid >= 32 && tid < 32 + NWARP * 2) mbar_init(smem_s + StepLow::MBAR_ATT + 8u * (tid - 32), 1);
     if (tid < 32 + NWARP * 2) fence_mbar_init();
     static_assert(BITS % NWARP == 0, "hyperplanes per warp");
@@ -241,9 +192,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     // ---- the code ring.  Dense: stage s is one bulk copy of the stage's codes
     // (when they lie inside the capacity at a 16-byte aligned address; else its
     // tokens are read with plain loads), issued by whichever warp is the last
-    // to finish with the slot.  Paged: every thread copies its own tokens of the
+    // to release the slot.  Paged: every thread copies its own tokens of the
     // stage with cp.async (a stage's 32-token warp slices lie in single pages
-    // for pages of 64 or more tokens) and reads only what it copied.
+    // for pages of 64 or more tokens) and reads only what it copied.  Either
+    // way a warp reads stage s + 1 into registers before it scores stage s, and
+    // releases a slot once the codes it read from there have been scored.
     const unsigned char *codes_b = reinterpret_cast<const unsigned char *>(kv.codes);
     const unsigned char *dense_base = codes_b + ((int64_t)bh * kv.n_cap + t0) * CODE_B;
     auto stage_tokens = [&](int s) { return min(STG_TOK, nloc - s * STG_TOK); };
@@ -300,9 +253,19 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     int pgn[TPL];  // PAGED: pages of this lane's tokens of the next stage to issue
-    __syncthreads();  // barriers initialised
+
+    // the group's summed query and the appended key (their loads overlap the
+    // barrier set-up)
+    for (int i = tid; i < D; i += NT) {
+        const __nv_bfloat16 *qh = a.q + ((int64_t)b * a.Hq + (int64_t)h * a.G) * D + i;
+        float s = 0.0f;
+        for (int g = 0; g < a.G; ++g) s += __bfloat162float(qh[(int64_t)g * D]);
+        qsum[i] = s;
+    }
+    if (own_new && tid < D) knew[tid] = __bfloat162float(a.k_new[((int64_t)b * kv.Hkv + h) * D + tid]);
+    __syncthreads();  // barriers initialised; qsum, knew ready
     if constexpr (PAGED) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NS && consumer; ++s) {
             int pg[TPL];
 #pragma unroll
             for (int u = 0; u < TPL; ++u) pg[u] = lane_page(s, u);
@@ -311,19 +274,43 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
 #pragma unroll
         for (int u = 0; u < TPL; ++u) pgn[u] = lane_page(NS, u);
     } else {
-        if (tid == 0)
+        if (tid == NCONS * 32)  // the producer
             for (int s = 0; s < NS && s < nstg; ++s) issue_dense(s);
     }
 
-    // ---- LUT of the group's summed query (as the two-kernel scorer builds it)
-    for (int i = tid; i < D; i += NT) {
-        const __nv_bfloat16 *qh = a.q + ((int64_t)b * a.Hq + (int64_t)h * a.G) * D + i;
-        float s = 0.0f;
-        for (int g = 0; g < a.G; ++g) s += __bfloat162float(qh[(int64_t)g * D]);
-        qsum[i] = s;
+    // ---- the threshold estimate's sample: one 32-token block of each of
+    // `nstrata` strata of the whole sequence, at a pseudo-random offset in the
+    // stratum (the same blocks in every CTA of the cluster; the appended token
+    // is left out).  Its codes are loaded now; they are scored once the LUT is
+    // built.
+    const int64_t kk = a.topk < n ? a.topk : n;
+    const bool normal = n > 0 && kk < n;
+    const int nblk_all = (int)(n >> 5);
+    const int nstrata = normal ? min(kSampleStrata, nblk_all / 16) : 0;
+    constexpr int SPW = kSampleStrata / NWARP;  // blocks per warp
+    uint32_t smp[SPW][BITS / 32];
+    float smr[SPW];
+    bool sok[SPW];
+#pragma unroll
+    for (int q = 0; q < SPW; ++q) {
+        const int j = warp + NWARP * q;
+        sok[q] = false;
+        smr[q] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < BITS / 32; ++k) smp[q][k] = 0u;
+        if (j < nstrata) {
+            const int stride = nblk_all / nstrata;
+            uint32_t hsh = (uint32_t)j * 0x9E3779B1u ^ ((uint32_t)bh * 0x85EBCA77u);
+            hsh ^= hsh >> 15;
+            hsh *= 0x2C1B3C6Du;
+            hsh ^= hsh >> 12;
+            const int64_t t = 32 * ((int64_t)j * stride + (int64_t)(hsh % (uint32_t)stride)) + lane;
+            if (t != pos) sok[q] = load_code_plain<BITS>(kv, b, h, t, smp[q]);
+            if constexpr (RADIUS) smr[q] = sok[q] ? radius_of_token(kv, b, h, t) : 0.0f;
+        }
     }
-    if (own_new && tid < D) knew[tid] = __bfloat162float(a.k_new[((int64_t)b * kv.Hkv + h) * D + tid]);
-    __syncthreads();
+
+    // ---- LUT of the group's summed query (as the two-kernel scorer builds it)
     // Qp_j = sum_i R[j][i] qsum[i] (and, in the CTA that appends, the new key's
     // projections): warp w takes hyperplanes w, w + 32, ... and lane l the dims
     // l, l + 32, ...; a shuffle tree sums the lanes.  Exact on grid inputs.
@@ -404,19 +391,50 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             for (int k = 0; k < BITS / 32; ++k) newr[k] = w32[k];
         }
     }
-    const int64_t kk = a.topk < n ? a.topk : n;
-    const bool normal = n > 0 && kk < n;
     if (tid == 0) misc[kMTloc] = normal ? 0 : kBins;  // kBins: nothing is kept
     __syncthreads();  // LUT, newr, tloc ready
-
-    // ---- stream: score every token of the CTA's range, stage by stage
     const uint32_t lbase = lut_s | (4u * (uint32_t)lane);
 
-    const int wsl = warp * 32 * TPL;                      // this warp's slice of a stage
+    // ---- threshold estimate: the sample's histogram gives the bin of sample
+    // rank r_s = e + 3.5 sqrt(e) + 8, where e = k m / n is the number of sample
+    // tokens expected at or above the k-th largest score (m sample tokens).
+    if (nstrata > 0) {
+        int cnt = 0;
+#pragma unroll
+        for (int q = 0; q < SPW; ++q) {
+            if (sok[q]) {
+                float sc = lut_score<BITS>(smp[q], lbase);  // (t = lane mod 32)
+                if constexpr (RADIUS) sc = __fmul_rn(sc, smr[q]);
+                const int bin = score_bin(sc, inv2A);
+                atomicAdd(&shist[bin / kSampleDiv], 1u);
+                atomicAdd(&ssup[bin >> 6], 1u);
+            }
+            cnt += __popc(__ballot_sync(0xffffffffu, sok[q]));
+        }
+        if (lane == 0 && cnt) atomicAdd(misc + kMSamp, cnt);
+        __syncthreads();
+        if (warp == 0) {
+            const int m = misc[kMSamp];
+            const float e = (float)kk * (float)m / (float)n;
+            const int64_t rs = (int64_t)ceilf(e + 3.5f * sqrtf(e) + 8.0f);
+            const int cb = rs <= m ? cluster_threshold<kSampleBins / 64, true>(ssup, shist, 1, rs, nullptr) : -1;
+            if (lane == 0 && cb > 0) misc[kMTloc] = cb * kSampleDiv;
+        }
+        __syncthreads();
+    }
+
+    // ---- stream: score every token of the CTA's range, stage by stage
+    const int wsl = warp * 32 * TPL;  // this warp's slice of a stage
     int ncand = 0;
     bool ovf = false, tmo = false;
     float *srow_out = a.scores_out ? a.scores_out + (int64_t)bh * a.ld_out + t0 : nullptr;
-    volatile int *vtloc = misc + kMTloc;
+    // the candidate test: a score at or above thr_f, a little below the lowest
+    // score of bin tl (so every token of bins >= tl is kept: its bin is exact
+    // and checked when the lists are counted)
+    const int tl = misc[kMTloc];
+    const float thr_f = tl <= 0 || inv2A == 0.0f ? -INFINITY
+                        : (tl >= kBins ? INFINITY
+                                       : (((float)tl / (float)(kBins - 1) - 0.5f) - 1e-5f) / inv2A);
     float rad[TPL];
 #pragma unroll
     for (int u = 0; u < TPL; ++u) rad[u] = 0.0f;
@@ -433,30 +451,18 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     // the capacity)
     const bool bulk_mid = nstg > 1 && stage_bulk_bytes(nstg - 2) != 0u;
     const bool bulk_last = nstg > 0 && stage_bulk_bytes(nstg - 1) != 0u;
-    int s = 0, slot = 0;
-    uint32_t phase = 0;
-#pragma unroll 1
-    for (; s < nstg; ++s) {
-        bool bulk_bytes = false;
-        if constexpr (PAGED) {
-            asm volatile("cp.async.wait_group %0;" ::"n"(NS - 1) : "memory");
-        } else {
-            if (!mbar_wait(mbar_full + 8u * slot, phase)) { tmo = true; break; }
-            bulk_bytes = s + 1 < nstg ? bulk_mid : bulk_last;
+    // stage s's codes for this lane into w (dense: once the slot's copy landed);
+    // false when the wait gave up
+    auto read_stage = [&](int s, uint32_t (&w)[TPL][BITS / 32]) -> bool {
+        const int slot = s % NS;
+        if constexpr (!PAGED) {
+            if (!mbar_wait(mbar_full + 8u * (uint32_t)slot, (uint32_t)((s / NS) & 1))) return false;
         }
-        float rnow[TPL];
-#pragma unroll
-        for (int u = 0; u < TPL; ++u) rnow[u] = rad[u];
-        if constexpr (RADIUS) load_radius(s + 1);
-        // the stage's codes of this lane, then their scores (independent chains)
-        uint32_t w[TPL][BITS / 32];
-        bool valid[TPL];
+        const bool from_ring = PAGED || (s + 1 < nstg ? bulk_mid : bulk_last);
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
             const int li = wsl + 32 * u + lane;  // token within the stage
-            const int i = s * STG_TOK + li;      // CTA-local token
-            valid[u] = i < nloc;
-            if (PAGED || bulk_bytes) {
+            if (from_ring) {
                 const unsigned char *src = ring + slot * STG_B + li * CODE_B;
                 if constexpr (BITS == 128) {
                     const uint4 x = *reinterpret_cast<const uint4 *>(src);
@@ -467,108 +473,140 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
                 } else {
                     w[u][0] = *reinterpret_cast<const uint32_t *>(src);
                 }
-                if constexpr (PAGED) valid[u] = valid[u] && !((pbad >> (slot * TPL + u)) & 1u);
             } else {
 #pragma unroll
-                for (int k = 0; k < BITS / 32; ++k) w[u][k] = 0;
-                if (valid[u]) valid[u] = load_code_plain<BITS>(kv, b, h, t0 + i, w[u]);
-            }
-            if (i == pos_loc) {
-#pragma unroll
-                for (int k = 0; k < BITS / 32; ++k) w[u][k] = newr[k];
+                for (int k = 0; k < BITS / 32; ++k) w[u][k] = 0u;
+                const int i = s * STG_TOK + li;
+                if (i < nloc) load_code_plain<BITS>(kv, b, h, t0 + i, w[u]);
             }
         }
-        float sc[TPL];
-#pragma unroll
-        for (int u = 0; u < TPL; ++u) {
-            sc[u] = lut_score<BITS>(w[u], lbase);
-            if constexpr (RADIUS) sc[u] = __fmul_rn(sc[u], rnow[u]);
+        return true;
+    };
+    uint32_t cur[TPL][BITS / 32];
+    int s = 0;
+    if (!consumer) {
+        // ---- the producer: refills a slot with stage r as soon as every
+        // consumer warp has released it from stage r - NS
+        if constexpr (!PAGED) {
+            if (lane == 0)
+                for (int r = NS; r < nstg; ++r) {
+                    if (!mbar_wait(mbar_empty + 8u * (uint32_t)(r % NS), (uint32_t)((r / NS - 1) & 1))) break;
+                    issue_dense(r);
+                }
+            __syncwarp();
         }
-        const int tl = *vtloc;
-        int bins[TPL];
-        bool isc[TPL];
-        bool mine = false;
-#pragma unroll
-        for (int u = 0; u < TPL; ++u) {
-            const int i = s * STG_TOK + wsl + 32 * u + lane;
-            if (srow_out && valid[u]) srow_out[i] = sc[u];
-            bins[u] = score_bin(sc[u], inv2A);
-            isc[u] = valid[u] && bins[u] >= tl;
-            mine |= isc[u];
+    } else {
+        if (nstg > 0) {
+            if constexpr (PAGED) asm volatile("cp.async.wait_group %0;" ::"n"(NS - 1) : "memory");
+            tmo = !read_stage(0, cur);
+            __syncwarp();
+            if (!PAGED && lane == 0) mbar_arrive(mbar_empty);  // stage 0's codes are in registers
         }
-        if (__any_sync(0xffffffffu, mine)) {
+#pragma unroll 1
+        for (; s < nstg && !tmo; ++s) {
+            uint32_t nxt[TPL][BITS / 32];
+            if (s + 1 < nstg) {
+                if constexpr (PAGED) asm volatile("cp.async.wait_group %0;" ::"n"(NS - 2) : "memory");
+                tmo = !read_stage(s + 1, nxt);  // (stage s is still scored)
+            }
+            float rnow[TPL];
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) rnow[u] = rad[u];
+            if constexpr (RADIUS) load_radius(s + 1);
+            const int sbase = s * STG_TOK;
+            if (pos_loc >= sbase && pos_loc < sbase + STG_TOK) {
+                // the appended token is scored from the code computed above
+#pragma unroll
+                for (int u = 0; u < TPL; ++u)
+                    if (sbase + wsl + 32 * u + lane == pos_loc) {
+#pragma unroll
+                        for (int k = 0; k < BITS / 32; ++k) cur[u][k] = newr[k];
+                    }
+            }
+            float sc[TPL];
 #pragma unroll
             for (int u = 0; u < TPL; ++u) {
-                const uint32_t ball = __ballot_sync(0xffffffffu, isc[u]);
-                if (!ball) continue;
-                const int i = s * STG_TOK + wsl + 32 * u + lane;
-                if (isc[u]) {  // results unused: reductions, no round trip
-                    atomicAdd(&hist[bins[u]], 1u);
-                    atomicAdd(&sup[bins[u] >> 6], 1u);
-                }
-                const int nb = __popc(ball);
-                if (!ovf && ncand + nb > cap) {
-                    // full: raise the threshold to the CTA's current k-th bin and drop what is below
-                    const int tnew = local_threshold(sup, hist, kk);
-                    if (lane == 0) atomicMax(misc + kMTloc, tnew);
-                    __syncwarp();
-                    ncand = compact_candidates(cand_lo, cand_hi, cap_lo, ncand, *vtloc, inv2A);
-                    if (ncand + nb > cap) {
+                sc[u] = lut_score<BITS>(cur[u], lbase);
+                if constexpr (RADIUS) sc[u] = __fmul_rn(sc[u], rnow[u]);
+            }
+            const bool full_stage = sbase + STG_TOK <= nloc;
+            bool isc[TPL];
+            bool mine = false;
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                const int i = sbase + wsl + 32 * u + lane;
+                bool valid = full_stage || i < nloc;
+                if constexpr (PAGED) valid = valid && !((pbad >> ((s % NS) * TPL + u)) & 1u);
+                if (srow_out && valid) srow_out[i] = sc[u];
+                isc[u] = valid && sc[u] >= thr_f;
+                mine |= isc[u];
+            }
+            if (__any_sync(0xffffffffu, mine) && !ovf) {
+#pragma unroll
+                for (int u = 0; u < TPL; ++u) {
+                    const uint32_t ball = __ballot_sync(0xffffffffu, isc[u]);
+                    const int nb = __popc(ball);
+                    if (ncand + nb > cap) {  // full: the exact slow path takes over
                         ovf = true;
                         if (lane == 0) misc[kMOvf] = 1;
+                        break;
                     }
-                }
-                if (!ovf) {
-                    if (isc[u]) cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)i, float_key(sc[u]));
+                    if (isc[u]) cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)(sbase + wsl + 32 * u + lane), float_key(sc[u]));
                     ncand += nb;
                 }
             }
-        }
-        // once per stage one warp (in turn) moves the CTA's threshold up to the
-        // bin of its current k-th largest counted score
-        if (warp == (s % NWARP) && tl < kBins) {
-            const int tnew = local_threshold(sup, hist, kk);
-            if (lane == 0 && tnew > tl) atomicMax(misc + kMTloc, tnew);
-        }
-        // release the slot and refill it with stage s + NS
-        __syncwarp();
-        if constexpr (PAGED) {
-            int pg[TPL];
+            __syncwarp();
+            if constexpr (PAGED) {
+                // refill slot s % NS (its codes were read a stage ago) with stage s + NS
+                int pg[TPL];
 #pragma unroll
-            for (int u = 0; u < TPL; ++u) pg[u] = pgn[u];
+                for (int u = 0; u < TPL; ++u) pg[u] = pgn[u];
 #pragma unroll
-            for (int u = 0; u < TPL; ++u) pgn[u] = lane_page(s + NS + 1, u);
-            issue_paged(s + NS, pg);
-        } else {
-            if (lane == 0) {
-                // the last of the warps to finish with the slot refills it (the
-                // count only grows: every NWARP arrivals are one use of the slot)
-                const uint32_t old = atomicAdd(stg_cnt + slot, 1u);
-                if ((old + 1u) % NWARP == 0u && s + NS < nstg) issue_dense(s + NS);
+                for (int u = 0; u < TPL; ++u) pgn[u] = lane_page(s + NS + 1, u);
+                issue_paged(s + NS, pg);
+            } else {
+                // release stage s + 1's slot: its codes are in registers (the
+                // arrive orders the loads before it)
+                if (lane == 0 && s + 1 < nstg && !tmo) mbar_arrive(mbar_empty + 8u * (uint32_t)((s + 1) % NS));
             }
+#pragma unroll
+            for (int u = 0; u < TPL; ++u)
+#pragma unroll
+                for (int k = 0; k < BITS / 32; ++k) cur[u][k] = nxt[u][k];
         }
-        if (++slot == NS) {
-            slot = 0;
-            phase ^= 1u;
+        if constexpr (PAGED) asm volatile("cp.async.wait_group 0;" ::: "memory");
+        if (tmo) {  // give the copies still in flight a bounded chance to land before the buffers are reused
+            for (int c = s; c < nstg && c < s + NS; ++c) mbar_wait(mbar_full + 8u * (c % NS), (uint32_t)((c / NS) & 1));
+            if (lane == 0) misc[kMOvf] = 1;
+            ovf = true;
         }
-    }
-    if constexpr (PAGED) asm volatile("cp.async.wait_group 0;" ::: "memory");
-    if (tmo) {  // give the copies still in flight a bounded chance to land before the buffers are reused
-        for (int c = s; c < nstg && c < s + NS; ++c) mbar_wait(mbar_full + 8u * (c % NS), (uint32_t)((c / NS) & 1));
-        if (lane == 0) misc[kMOvf] = 1;
-        ovf = true;
+        // the CTA histogram of the kept tokens of bins >= tl, from this warp's list
+        if (!ovf)
+            for (int j = lane; j < ncand; j += 32) {
+                const int bin = score_bin(key_to_float(cand_ref(j).y), inv2A);
+                if (bin >= tl) {
+                    atomicAdd(&hist[bin], 1u);
+                    atomicAdd(&sup[bin >> 6], 1u);
+                }
+            }
     }
     __syncthreads();  // every warp's list and the histogram are complete
 
-    // ---- the cluster's threshold bin T1 (exact: every CTA counted every token
-    // of every bin at or above it)
+    // ---- the cluster's threshold bin T1 (exact when found: every CTA counted
+    // every token of every bin at or above its threshold, and no CTA's
+    // threshold is above T1; not found: the estimate was too high)
     if (tid == 0) { misc[kMT1] = kBins; misc[kMAbove] = 0; misc[kMCntT1] = 0; misc[kMNinb] = 0; misc[kMKept] = 0; }
     cluster_sync();  // (1)
     if (normal && warp == 0) cluster_threshold(sup, hist, nctas, kk, misc + kMT1);
     if (warp == 1) {
+        // any CTA's list overflowed, and the highest CTA threshold (T1 below it
+        // means that CTA did not count every token of bin T1 and above)
         const int f = lane < nctas ? (int)ld_cluster_u32(cluster_addr(misc + kMOvf, lane)) : 0;
+        int tmax = lane < nctas ? (int)ld_cluster_u32(cluster_addr(misc + kMTloc, lane)) : 0;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
         const uint32_t any = __ballot_sync(0xffffffffu, f != 0);
-        if (lane == 0) misc[kMAnyOvf] = any != 0;
+        if (lane == 0) { misc[kMAnyOvf] = any != 0; misc[kMTmax] = tmax; }
     }
     __syncthreads();
     const int T1 = misc[kMT1], above1 = misc[kMAbove], cnt_T1 = misc[kMCntT1];
@@ -586,7 +624,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     // (the same decision in every CTA of the cluster: the bitmap bound uses the
     // longest range cta_range gives any CTA)
     const int64_t max_range = ceil_div(ceil_div(n, nctas), 64) * 64;
-    const bool slow = !normal || misc[kMAnyOvf] != 0 || cnt_T1 > kInbinMax || ceil_div(max_range, 32) > kBmapWords;
+    const bool slow = !normal || T1 == kBins || T1 < misc[kMTmax] || misc[kMAnyOvf] != 0 || cnt_T1 > kInbinMax ||
+                      ceil_div(max_range, 32) > kBmapWords;
 
     if (!slow) {
         // ---- fast path: classify this warp's candidates (definite: bin > T1,
@@ -767,30 +806,46 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         }
         cluster_wait();  // (3)
     } else {
-        // ---- exact slow path (heavy ties, a full candidate list, or all / none
-        // selected): re-score the CTA's range into the workspace rows, list the
-        // tokens of bins >= T1 per CTA, and let CTA 0 resolve and emit.
+        // ---- exact slow path (heavy ties, a full candidate list, a threshold
+        // estimate above T1, or all / none selected): re-score the CTA's range
+        // into the workspace rows counting every token (the stream counted
+        // only those at or above its threshold; a token whose page is out of
+        // range scores as the all-zero code, as in the two-kernel scorer), find
+        // T1 from the full histograms, list the tokens of bins >= T1 per CTA,
+        // and let CTA 0 resolve and emit.
         float *srow = a.ws.scores + (int64_t)bh * a.ws.ld;
         int32_t *cand = a.ws.cand + (int64_t)bh * a.ws.ld;
         int seg = 0;
         if (normal) {
-            for (int64_t base = t0; base < t1; base += NT) {
-                const int64_t t = base + warp * 32 + lane;
-                bool flag = false;
-                if (t < t1) {
-                    uint32_t w[BITS / 32];
-                    bool ok = true;
-                    if (t == pos) {
+            cluster_sync();  // (s1): no CTA reads the stream's counts any more
+            for (int i = tid; i < kBins; i += NT) hist[i] = 0;
+            if (tid < 64) sup[tid] = 0;
+            if (tid == 0) { misc[kMT1] = kBins; misc[kMAbove] = 0; misc[kMCntT1] = 0; }
+            __syncthreads();
+            for (int64_t t = t0 + tid; t < t1; t += NT) {
+                uint32_t w[BITS / 32];
+                if (t == pos) {
 #pragma unroll
-                        for (int k = 0; k < BITS / 32; ++k) w[k] = newr[k];
-                    } else {
-                        ok = load_code_plain<BITS>(kv, b, h, t, w);
-                    }
-                    float sc = ok ? lut_score_any<BITS>(w, lut_s, t) : 0.0f;
-                    if constexpr (RADIUS) sc = __fmul_rn(sc, radius_of_token(kv, b, h, t));
-                    srow[t] = sc;
-                    flag = ok && score_bin(sc, inv2A) >= T1;
+                    for (int k = 0; k < BITS / 32; ++k) w[k] = newr[k];
+                } else if (!load_code_plain<BITS>(kv, b, h, t, w)) {
+#pragma unroll
+                    for (int k = 0; k < BITS / 32; ++k) w[k] = 0u;
                 }
+                float sc = lut_score_any<BITS>(w, lut_s, t);
+                if constexpr (RADIUS) sc = __fmul_rn(sc, radius_of_token(kv, b, h, t));
+                srow[t] = sc;
+                const int bin = score_bin(sc, inv2A);
+                atomicAdd(&hist[bin], 1u);
+                atomicAdd(&sup[bin >> 6], 1u);
+            }
+            cluster_sync();  // (s2): every CTA's full histogram
+            if (warp == 0) cluster_threshold(sup, hist, nctas, kk, misc + kMT1);
+            __syncthreads();
+            const int T1s = misc[kMT1];
+            // (each thread reads back the scores it wrote)
+            for (int64_t base = t0; base < t1; base += NT) {
+                const int64_t t = base + tid;
+                const bool flag = t < t1 && score_bin(srow[t], inv2A) >= T1s;
                 const uint32_t fb = __ballot_sync(0xffffffffu, flag);
                 int tot;
                 const int wex = block_excl_scan<NT>(lane == 0 ? __popc(fb) : 0, s_warp, &tot);
@@ -804,7 +859,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         cluster_sync();  // (2s): segments complete
         if (cta == 0) {
             SelState st;
-            st.T1 = T1; st.above1 = above1; st.cnt_T1 = cnt_T1;
+            st.T1 = misc[kMT1]; st.above1 = misc[kMAbove]; st.cnt_T1 = misc[kMCntT1];
             st.flags = n == 0 ? kStateEmpty : (normal ? kStateNormal : kStateAll);
             st.inv2A = inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
             resolve_emit<NT, 4096>(a.ws, bh, nctas, st, a.S, a.W, a.cap_sel, a.sel_idx, a.sel_cnt,
