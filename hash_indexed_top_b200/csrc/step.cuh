@@ -49,10 +49,15 @@
 //           T1), a full candidate list or a threshold estimate above T1 take
 //           an exact slow path (re-score and count every token into the
 //           workspace, CTA 0 runs the two-kernel path's resolver).
-//  attend   (G > 0) every CTA takes an equal slice of the emitted list, bulk
-//           copies the K and V rows into shared memory (two tiles in flight
-//           per warp) and runs an online softmax in fp32; the CTAs' partial
-//           states are merged through distributed shared memory.
+//  attend   (G > 0) every CTA attends over its own kept tokens (listed in
+//           shared memory as it emits them), its share of the window and, in
+//           CTA 0, the sinks (the slow path: an equal slice of the emitted
+//           list).  Warps copy the K / V rows into shared memory with 16-byte
+//           cp.async (a row per warp instruction; two tiles in flight per warp)
+//           and run an online softmax in fp32.  Each CTA
+//           pushes its partial state, element by element, into the shared
+//           memory of the CTA that merges that element, and after one cluster
+//           barrier every CTA merges and writes the elements it owns.
 //  append   (k_new given) the CTA that owns position seq_lens[b] encodes the
 //           new key, writes its code and K/V rows there and scores it from
 //           the code it computed; the last cluster of a sequence to finish
@@ -127,7 +132,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     const uint32_t mbar_full = smem_s + StepLow::MBAR;         // [NS]
     const uint32_t mbar_empty = smem_s + StepLow::MBAR_EMPTY;  // [NS]
     const bool consumer = warp < NCONS;  // (during the stream; warp NCONS is its producer)
-    const uint32_t mbar_att = smem_s + StepLow::MBAR_ATT + 8u * (uint32_t)(warp * 2);
     const uint32_t lut_s = (smem_s + StepLow::END + 65535u) & ~65535u;  // 64 KB aligned
     unsigned char *lut = smem + (lut_s - smem_s);
     const uint32_t ring_s = lut_s + 65536u;
@@ -135,7 +139,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     const uint32_t end_s = smem_s + (uint32_t)a.smem_bytes;
     // candidate list of this warp: cap_lo entries below the LUT, cap_hi above the ring
     // (NCONS lists: warp NCONS has none and keeps ncand = 0)
-    const int cap_lo = (int)((lut_s - (smem_s + StepLow::END)) / (8u * NCONS));
+    const uint32_t recv_s = lut_s - (uint32_t)kRecvBytes;  // the attention merge's inbox (G > 0)
+    const int cap_lo = (int)((recv_s - (smem_s + StepLow::END)) / (8u * NCONS));
     const int cap_hi = end_s > ring_s + SS::RING_B ? (int)((end_s - ring_s - SS::RING_B) / (8u * NCONS)) : 0;
     uint2 *cand_lo = reinterpret_cast<uint2 *>(smem + StepLow::END) + warp * cap_lo;
     uint2 *cand_hi = reinterpret_cast<uint2 *>(ring + SS::RING_B) + warp * cap_hi;
@@ -148,8 +153,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     if (tid < 64) { sup[tid] = 0; ssup[tid] = 0; misc[tid] = 0; }
     if (tid < 4) newc[tid] = 0;
     if (tid < NS) { mbar_init(mbar_full + 8u * tid, 1); mbar_init(mbar_empty + 8u * tid, NCONS); }
-    if (tid >= 32 && tid < 32 + NWARP * 2) mbar_init(smem_s + StepLow::MBAR_ATT + 8u * (tid - 32), 1);
-    if (tid < 32 + NWARP * 2) fence_mbar_init();
+    if (tid < NS) fence_mbar_init();
     static_assert(BITS % NWARP == 0, "hyperplanes per warp");
     uint32_t rw[BITS / NWARP][D / 32];
 #pragma unroll
@@ -184,6 +188,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     }
     int64_t t0, t1;
     cta_range(n, cta, nctas, t0, t1);
+    const int s_end = (int)(a.S < n ? a.S : n);  // sinks [0, s_end), window [w_beg, n)
+    const int w_beg = (int)(n - a.W > s_end ? n - a.W : s_end);
+    // this CTA's share of the window rows for the attention: [wt0, wt0 + nw)
+    const int per_w = (int)ceil_div(n - w_beg, (int64_t)nctas);
+    const int64_t wt0 = w_beg + (int64_t)cta * per_w;
+    const int nw = (int)max((int64_t)0, min((int64_t)per_w, n - wt0));
     const int nloc = (int)(t1 - t0);
     const int nstg = (nloc + STG_TOK - 1) / STG_TOK;  // stages of this CTA
     const bool own_new = pos >= t0 && pos < t1;
@@ -214,7 +224,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         const uint32_t bytes = stage_bulk_bytes(s);
         if (bytes) {
             mbar_arrive_expect_tx(mb, bytes);
-            bulk_g2s(ring_s + (uint32_t)((s % NS) * STG_B), dense_base + (int64_t)s * STG_B, bytes, mb);
+            // codes are read once: first out of L2, ahead of the K / V rows kept there
+            bulk_g2s_hint(ring_s + (uint32_t)((s % NS) * STG_B), dense_base + (int64_t)s * STG_B, bytes, mb,
+                          l2_policy_evict_first());
         } else {
             mbar_arrive(mb);  // completes the phase with no data
         }
@@ -551,7 +563,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
                         if (lane == 0) misc[kMOvf] = 1;
                         break;
                     }
-                    if (isc[u]) cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)(sbase + wsl + 32 * u + lane), float_key(sc[u]));
+                    if (isc[u]) {
+                        const int i = sbase + wsl + 32 * u + lane;
+                        cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)i, float_key(sc[u]));
+                    }
                     ncand += nb;
                 }
             }
@@ -610,8 +625,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     }
     __syncthreads();
     const int T1 = misc[kMT1], above1 = misc[kMAbove], cnt_T1 = misc[kMCntT1];
-    const int s_end = (int)(a.S < n ? a.S : n);
-    const int w_beg = (int)(n - a.W > s_end ? n - a.W : s_end);
     int32_t *out = a.sel_idx + (int64_t)bh * a.cap_sel;
     // the kept tokens of this CTA are placed through a bitmap of its range
     // (after the in-bin lists in the idle ring); a range too long for it takes
@@ -624,8 +637,13 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     // (the same decision in every CTA of the cluster: the bitmap bound uses the
     // longest range cta_range gives any CTA)
     const int64_t max_range = ceil_div(ceil_div(n, nctas), 64) * 64;
+    // the attention list of this CTA (G > 0), in the candidate area once the
+    // candidates are emitted: its kept middle tokens (after the sinks in CTA 0)
+    int32_t *att_list = reinterpret_cast<int32_t *>(smem + StepLow::END);
+    const int att_cap = (int)((recv_s - (smem_s + StepLow::END)) / 4u);
+    int att_n = 0;
     const bool slow = !normal || T1 == kBins || T1 < misc[kMTmax] || misc[kMAnyOvf] != 0 || cnt_T1 > kInbinMax ||
-                      ceil_div(max_range, 32) > kBmapWords;
+                      ceil_div(max_range, 32) > kBmapWords || (G > 0 && kk + a.S > att_cap);
 
     if (!slow) {
         // ---- fast path: classify this warp's candidates (definite: bin > T1,
@@ -776,16 +794,25 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             int cnt = 0;
             for (int x = w0; x < w1; ++x) cnt += __popc(bmap[x]);
             int tot;
-            int p = s_end + misc[kMBefore] + block_excl_scan<NT>(cnt, s_warp, &tot);
+            const int lp = block_excl_scan<NT>(cnt, s_warp, &tot);
+            int p = s_end + misc[kMBefore] + lp;
+            int q = (cta == 0 ? s_end : 0) + lp;  // (the candidate lists are dead: the bitmap holds them)
             for (int x = w0; x < w1; ++x) {
                 uint32_t m = bmap[x];
                 while (m) {
                     const int bit = __ffs(m) - 1;
                     m &= m - 1;
-                    if (p < a.cap_sel) out[p] = (int32_t)(t0 + 32 * x + bit);
+                    const int32_t tok = (int32_t)(t0 + 32 * x + bit);
+                    if (p < a.cap_sel) out[p] = tok;
+                    if constexpr (G > 0) att_list[q] = tok;
                     ++p;
+                    ++q;
                 }
             }
+            att_n = (cta == 0 ? s_end : 0) + tot;
+            if constexpr (G > 0)
+                if (cta == 0)
+                    for (int x = tid; x < s_end; x += NT) att_list[x] = x;
         }
         {   // the sinks, the window and the padding, spread over the cluster's CTAs
             const int wpos0 = s_end + total_mid;
@@ -804,7 +831,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             }
             if (cta == 0 && tid == 0) a.sel_cnt[bh] = total;
         }
-        cluster_wait();  // (3)
+        __syncthreads();  // the attention list is complete
+        cluster_wait();  // (3): no CTA reads this one's ring any more
     } else {
         // ---- exact slow path (heavy ties, a full candidate list, a threshold
         // estimate above T1, or all / none selected): re-score the CTA's range
@@ -868,205 +896,290 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     }
 
     if constexpr (G > 0) {
-        // ---- attention over the emitted list: CTA c takes an equal slice of it
-        cluster_sync();  // (4): the whole list and its count are written (cluster-scope release / acquire)
-        constexpr int HG = G < 4 ? G : 4;   // query heads per warp
-        constexpr int NTEAM = G / HG;       // warp teams, each over every row for its HG heads
-        constexpr int WPT = NWARP / NTEAM;  // warps per team
-        constexpr int SL = 32 / HG;         // lanes per head: dim slices
-        constexpr int DPL = D / SL;         // dims per lane
-        constexpr int TROWS = 8;
+        // ---- exact attention over this CTA's share of the selection: n_sl
+        // tokens listed in att_list, then the nw window tokens wt0 + j, then
+        // n_gl tokens of the global list gl (the slow path's share)
+        int n_sl = 0, n_win = 0, n_gl = 0;
+        const int32_t *gl = nullptr;
+        if (!slow) {
+            n_sl = att_n;
+            n_win = nw;
+        } else {
+            cluster_sync();  // (4s): CTA 0's list and count are written (cluster-scope release / acquire)
+            const int cnt = __ldcg(a.sel_cnt + bh);
+            const int per = (cnt + nctas - 1) / nctas;
+            const int r0 = min(cnt, cta * per), r1 = min(cnt, r0 + per);
+            gl = a.sel_idx + (int64_t)bh * a.cap_sel + r0;
+            n_gl = r1 - r0;
+        }
+        const int natt = n_sl + n_win + n_gl;
+        auto token_of = [&](int r) -> int {
+            if (r < n_sl) return att_list[r];
+            if (r < n_sl + n_win) return (int)(wt0 + (r - n_sl));
+            return __ldcg(gl + (r - n_sl - n_win));
+        };
+        // Lane l owns dims [DL l, DL l + DL) of every one of the G query heads,
+        // and a tile is TR rows.  The G TR partial dot products of a tile are
+        // summed over the warp by a transpose butterfly that leaves the one of
+        // head lv / TR and row lv % TR (lv: the low log2(G TR) bits of l) in
+        // lane l.  At the level that pairs lanes across bit k every lane sends
+        // the upper half of its values and keeps the lower half; that is the
+        // right half for both lanes because a lane keeps its heads and rows in
+        // the order XOR-ed with lv (slot hh holds head hh ^ hperm, slot r row
+        // r ^ rperm).
+        constexpr int DL = D / 32;               // dims per lane
+        constexpr int TR = G >= 4 ? 32 / G : 8;  // rows per tile
+        constexpr int V = G * TR;                // partial products per lane
         constexpr int ROW_B = D * 2;
-        constexpr int TILE_B = TROWS * 2 * ROW_B;
-        static_assert(DPL % 8 == 0 || DPL == 4 || DPL == 2, "dims per lane");
-        const int team = warp / WPT, wt = warp % WPT;
-        const int gl = lane / SL, sl = lane % SL;
-        const int g = team * HG + gl;
-        float qf[DPL];
-        {
-            const __nv_bfloat16 *qr = a.q + ((int64_t)b * a.Hq + (int64_t)h * G + g) * D + sl * DPL;
+        constexpr int TILE_B = TR * 2 * ROW_B;
+        constexpr int WSTAGE_B = 2 * TILE_B + 128;  // two tiles and 32 softmax weights per warp
+        static_assert(G <= kMaxG && V <= 32 && (V & (V - 1)) == 0 && (DL == 2 || DL == 4), "tile shape");
+        const int lv = lane & (V - 1);
+        const int hperm = lv / TR, rperm = lv % TR;
+        float qf[G][DL];
 #pragma unroll
-            for (int e = 0; e < DPL; e += 2) {
-                const uint32_t x = *reinterpret_cast<const uint32_t *>(qr + e);
-                qf[e] = bf16_lo(x) * a.scale_log2;
-                qf[e + 1] = bf16_hi(x) * a.scale_log2;
+        for (int hh = 0; hh < G; ++hh) {
+            const __nv_bfloat16 *qr = a.q + ((int64_t)b * a.Hq + (int64_t)h * G + (hh ^ hperm)) * D + DL * lane;
+            if constexpr (DL == 4) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(qr);
+                qf[hh][0] = bf16_lo(w.x) * a.scale_log2; qf[hh][1] = bf16_hi(w.x) * a.scale_log2;
+                qf[hh][2] = bf16_lo(w.y) * a.scale_log2; qf[hh][3] = bf16_hi(w.y) * a.scale_log2;
+            } else {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(qr);
+                qf[hh][0] = bf16_lo(w) * a.scale_log2; qf[hh][1] = bf16_hi(w) * a.scale_log2;
             }
         }
-        float m = -INFINITY, l = 0.0f, acc[DPL];
+        float acc[G][DL];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = 0.0f;
-        const int cnt = __ldcg(a.sel_cnt + bh);
-        const int32_t *list = a.sel_idx + (int64_t)bh * a.cap_sel;
-        const int per = (cnt + nctas - 1) / nctas;
-        const int r0 = cta * per, r1 = min(cnt, r0 + per);
-        const int ntiles = r1 > r0 ? (r1 - r0 + TROWS - 1) / TROWS : 0;
-        const uint32_t stage_s = lut_s + (uint32_t)(warp * 2 * TILE_B);
-        const unsigned char *stage = lut + warp * 2 * TILE_B;
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+            for (int d = 0; d < DL; ++d) acc[hh][d] = 0.0f;
+        float m = -INFINITY, lsum = 0.0f;  // of head hperm (the same in its TR lanes)
+        const int ntiles = (natt + TR - 1) / TR;
+        // two staging tiles per warp over the LUT and the code ring (both idle now)
+        const uint32_t stage_s = lut_s + (uint32_t)(warp * WSTAGE_B);
+        const unsigned char *stage = lut + warp * WSTAGE_B;
+        float *s_p = reinterpret_cast<float *>(lut + warp * WSTAGE_B + 2 * TILE_B);  // [TR][G]
         const __nv_bfloat16 *kn_row = appending ? a.k_new + ((int64_t)b * kv.Hkv + h) * D : nullptr;
         const __nv_bfloat16 *vn_row = appending ? a.v_new + ((int64_t)b * kv.Hkv + h) * D : nullptr;
-        // the rows of tile `tile` into buffer `buf`; returns the valid-row mask
+        // the rows of tile `tile` into buffer `buf` with 16-byte cp.async (one
+        // commit group per call; rows that are not valid are zero-filled);
+        // returns the valid-row mask
+        constexpr int CPR = 2 * ROW_B / 16;  // 16-byte chunks per row (K then V)
+        constexpr int RPI = 32 / CPR;        // rows per warp-wide copy
+        static_assert(CPR * RPI == 32 && TR % RPI == 0, "copy shape");
+        // dense rows of (b, h): token t's K / V row starts at element rbase + t D
+        const int64_t rbase = ((int64_t)b * kv.Hkv + h) * kv.n_cap * D;
         auto fetch = [&](int tile, int buf) -> uint32_t {
-            const int r = r0 + tile * TROWS + lane;
-            int64_t off = -1;
-            int tok = -1;
-            if (lane < TROWS && r < r1) {
-                tok = __ldcg(list + r);
-                if (tok < 0 || tok >= capn) {
-                    raise_error(kErrCapacity);
-                    tok = -1;
-                } else if (tok != pos) {
-                    off = kv.row(b, h, tok);
-                    if (off < 0) tok = -1;
+            // lanes < TR resolve row tile TR + lane: PAGED the element offset of
+            // the row, dense the token; -2: the appended token, -1: none
+            int64_t key = -1;
+            if (lane < TR) {
+                const int r = tile * TR + lane;
+                if (r < natt) {
+                    const int tok = token_of(r);
+                    if (tok < 0 || tok >= capn) {
+                        raise_error(kErrCapacity);
+                    } else if (tok == pos) {
+                        key = -2;
+                    } else if constexpr (PAGED) {
+                        key = kv.row(b, h, tok);  // (-1: page out of range)
+                    } else {
+                        key = tok;
+                    }
                 }
             }
-            const uint32_t vm = __ballot_sync(0xffffffffu, tok >= 0);
-            const uint32_t mb = mbar_att + 8u * (uint32_t)buf;
-            if (lane == 0) {
-                if (vm) mbar_arrive_expect_tx(mb, (uint32_t)__popc(vm) * 2u * ROW_B);
-                else mbar_arrive(mb);
+            const uint32_t vm = __ballot_sync(0xffffffffu, key != -1);
+            const int c = lane % CPR;  // this lane's chunk of its row
+            const bool isv = c >= CPR / 2;
+            const int ce = (isv ? c - CPR / 2 : c) * 8;  // first element of the chunk
+            const __nv_bfloat16 *cache = isv ? kv.v : kv.k;
+            const __nv_bfloat16 *fresh = (isv ? vn_row : kn_row) + ce;
+#pragma unroll
+            for (int i = 0; i < TR / RPI; ++i) {
+                const int r = i * RPI + lane / CPR;
+                int64_t o;
+                if constexpr (PAGED) {
+                    o = __shfl_sync(0xffffffffu, key, r);
+                } else {
+                    const int tk = __shfl_sync(0xffffffffu, (int)key, r);
+                    o = tk >= 0 ? rbase + (int64_t)tk * D : tk;
+                }
+                const __nv_bfloat16 *src = o >= 0 ? cache + o + ce : (o == -2 ? fresh : kv.k);
+                const uint32_t sz = o != -1 ? 16u : 0u;  // (zero-filled when not valid)
+                const uint32_t dst = stage_s + (uint32_t)(buf * TILE_B + r * 2 * ROW_B + c * 16);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
             }
-            __syncwarp();
-            if (tok >= 0) {
-                const uint32_t dst = stage_s + (uint32_t)(buf * TILE_B + lane * 2 * ROW_B);
-                const void *ks = tok == pos ? (const void *)kn_row : (const void *)(kv.k + off);
-                const void *vs = tok == pos ? (const void *)vn_row : (const void *)(kv.v + off);
-                bulk_g2s(dst, ks, ROW_B, mb);
-                bulk_g2s(dst + ROW_B, vs, ROW_B, mb);
-            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
             return vm;
         };
-        uint32_t vmask[2] = {0u, 0u};
+        // this lane's DL dims of a staged bf16 row
+        auto load_row = [&](const unsigned char *row, float (&f)[DL]) {
+            if constexpr (DL == 4) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(row + lane * 8);
+                f[0] = bf16_lo(w.x); f[1] = bf16_hi(w.x); f[2] = bf16_lo(w.y); f[3] = bf16_hi(w.y);
+            } else {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(row + lane * 4);
+                f[0] = bf16_lo(w); f[1] = bf16_hi(w);
+            }
+        };
         int k = 0;
-        if (wt < ntiles) vmask[0] = fetch(wt, 0);
-        if (wt + WPT < ntiles) vmask[1] = fetch(wt + WPT, 1);
-        for (int tile = wt; tile < ntiles; tile += WPT, ++k) {
+        // two commit groups in flight per lane (empty ones past the last tile);
+        // vm0 / vm1: the valid-row masks of the tiles in buffers k & 1 = 0 / 1
+        uint32_t vm0 = warp < ntiles ? fetch(warp, 0) : 0u;
+        uint32_t vm1 = warp + NWARP < ntiles ? fetch(warp + NWARP, 1) : 0u;
+        if (warp >= ntiles) asm volatile("cp.async.commit_group;" ::: "memory");
+        if (warp + NWARP >= ntiles) asm volatile("cp.async.commit_group;" ::: "memory");
+        for (int tile = warp; tile < ntiles; tile += NWARP, ++k) {
             const int buf = k & 1;
-            if (!mbar_wait(mbar_att + 8u * buf, (uint32_t)((k >> 1) & 1))) break;
+            asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's group has landed
+            __syncwarp();  // (and every lane's copies are visible to the warp)
             const unsigned char *tb = stage + buf * TILE_B;
-            const uint32_t vm = vmask[buf];
-            float x[TROWS];
+            const uint32_t vm = buf ? vm1 : vm0;
+            // partial q . k of (slot head hh, slot row r); rows that are not
+            // valid are zeros and masked below
+            float x[V];
 #pragma unroll
-            for (int r = 0; r < TROWS; ++r) {
-                const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(tb + r * 2 * ROW_B) + sl * DPL;
-                float2 d2 = make_float2(0.0f, 0.0f);
+            for (int r = 0; r < TR; ++r) {
+                float kf[DL];
+                load_row(tb + (r ^ rperm) * 2 * ROW_B, kf);
 #pragma unroll
-                for (int e = 0; e < DPL; e += 8) {
-                    if constexpr (DPL >= 8) {
-                        const uint4 w4 = *reinterpret_cast<const uint4 *>(kr + e);
-                        d2 = ffma2(make_float2(qf[e], qf[e + 1]), bf16x2_to_float2(w4.x), d2);
-                        d2 = ffma2(make_float2(qf[e + 2], qf[e + 3]), bf16x2_to_float2(w4.y), d2);
-                        d2 = ffma2(make_float2(qf[e + 4], qf[e + 5]), bf16x2_to_float2(w4.z), d2);
-                        d2 = ffma2(make_float2(qf[e + 6], qf[e + 7]), bf16x2_to_float2(w4.w), d2);
-                    }
-                }
-                if constexpr (DPL == 4) {
-                    const uint2 w2 = *reinterpret_cast<const uint2 *>(kr);
-                    d2 = ffma2(make_float2(qf[0], qf[1]), bf16x2_to_float2(w2.x), d2);
-                    d2 = ffma2(make_float2(qf[2], qf[3]), bf16x2_to_float2(w2.y), d2);
-                } else if constexpr (DPL == 2) {
-                    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(kr);
-                    d2 = ffma2(make_float2(qf[0], qf[1]), bf16x2_to_float2(w1), d2);
-                }
-                x[r] = d2.x + d2.y;
-            }
+                for (int hh = 0; hh < G; hh += 2) {
+                    if constexpr (G == 1) {
+                        float s = 0.0f;
 #pragma unroll
-            for (int o = SL / 2; o; o >>= 1)
-#pragma unroll
-                for (int r = 0; r < TROWS; ++r) x[r] += __shfl_xor_sync(0xffffffffu, x[r], o);
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < TROWS; ++r) {
-                x[r] = ((vm >> r) & 1u) ? x[r] : -INFINITY;
-                tmax = fmaxf(tmax, x[r]);
-            }
-            if (tmax != -INFINITY) {
-                const float mn = fmaxf(m, tmax);
-                const float c = fast_exp2(m - mn);
-                m = mn;
-                l *= c;
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) acc[e] *= c;
-#pragma unroll
-                for (int r = 0; r < TROWS; ++r) {
-                    // invalid rows were not copied: their staging bytes are stale
-                    if (!((vm >> r) & 1u)) continue;
-                    const float p = fast_exp2(x[r] - mn);
-                    l += p;
-                    const __nv_bfloat16 *vr =
-                        reinterpret_cast<const __nv_bfloat16 *>(tb + r * 2 * ROW_B + ROW_B) + sl * DPL;
-                    const float2 p2 = make_float2(p, p);
-                    if constexpr (DPL >= 8) {
-#pragma unroll
-                        for (int e = 0; e < DPL; e += 8) {
-                            const uint4 w4 = *reinterpret_cast<const uint4 *>(vr + e);
-                            float2 a0 = ffma2(p2, bf16x2_to_float2(w4.x), make_float2(acc[e], acc[e + 1]));
-                            float2 a1 = ffma2(p2, bf16x2_to_float2(w4.y), make_float2(acc[e + 2], acc[e + 3]));
-                            float2 a2 = ffma2(p2, bf16x2_to_float2(w4.z), make_float2(acc[e + 4], acc[e + 5]));
-                            float2 a3 = ffma2(p2, bf16x2_to_float2(w4.w), make_float2(acc[e + 6], acc[e + 7]));
-                            acc[e] = a0.x; acc[e + 1] = a0.y; acc[e + 2] = a1.x; acc[e + 3] = a1.y;
-                            acc[e + 4] = a2.x; acc[e + 5] = a2.y; acc[e + 6] = a3.x; acc[e + 7] = a3.y;
-                        }
-                    } else if constexpr (DPL == 4) {
-                        const uint2 w2 = *reinterpret_cast<const uint2 *>(vr);
-                        float2 a0 = ffma2(p2, bf16x2_to_float2(w2.x), make_float2(acc[0], acc[1]));
-                        float2 a1 = ffma2(p2, bf16x2_to_float2(w2.y), make_float2(acc[2], acc[3]));
-                        acc[0] = a0.x; acc[1] = a0.y; acc[2] = a1.x; acc[3] = a1.y;
+                        for (int d = 0; d < DL; ++d) s = fmaf(qf[0][d], kf[d], s);
+                        x[r] = s;
                     } else {
-                        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(vr);
-                        float2 a0 = ffma2(p2, bf16x2_to_float2(w1), make_float2(acc[0], acc[1]));
-                        acc[0] = a0.x; acc[1] = a0.y;
+                        float2 s2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                        for (int d = 0; d < DL; ++d)
+                            s2 = ffma2(make_float2(qf[hh][d], qf[hh + 1][d]), make_float2(kf[d], kf[d]), s2);
+                        x[hh * TR + r] = s2.x;
+                        x[(hh + 1) * TR + r] = s2.y;
                     }
                 }
             }
-            __syncwarp();  // the buffer is refilled next
-            if (tile + 2 * WPT < ntiles) vmask[buf] = fetch(tile + 2 * WPT, buf);
-        }
-        __syncthreads();  // every warp is done with its staging buffers
-        // CTA merge of the warps' states: [warp][HG] (m, l) and [warp][HG][D] acc at the LUT base
-        float *s_acc = reinterpret_cast<float *>(lut);
-        float *s_ml = s_acc + NWARP * HG * D;
-        if (sl == 0) { s_ml[(warp * HG + gl) * 2] = m; s_ml[(warp * HG + gl) * 2 + 1] = l; }
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) s_acc[(warp * HG + gl) * D + sl * DPL + e] = acc[e];
+            for (int half = V / 2; half >= 1; half >>= 1)
+#pragma unroll
+                for (int i = 0; i < half; ++i) x[i] += __shfl_xor_sync(0xffffffffu, x[i + half], half);
+#pragma unroll
+            for (int o = 16; o >= V; o >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], o);
+            // online softmax of head hperm over the tile's rows (its TR lanes)
+            const bool ok = (vm >> rperm) & 1u;
+            const float sc = ok ? x[0] : -INFINITY;
+            float tmax = sc;
+#pragma unroll
+            for (int o = TR / 2; o; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+            const float mn = fmaxf(m, tmax);
+            const float c = m == -INFINITY ? 0.0f : fast_exp2(m - mn);
+            const float pv = ok ? fast_exp2(sc - mn) : 0.0f;
+            float ps = pv;
+#pragma unroll
+            for (int o = TR / 2; o; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+            lsum = fmaf(lsum, c, ps);
+            m = mn;
+            if (lane < V) s_p[rperm * G + hperm] = pv;
+            float ch[G];
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) ch[hh] = __shfl_sync(0xffffffffu, c, hh * TR);
+            __syncwarp();
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+                for (int d = 0; d < DL; ++d) acc[hh][d] *= ch[hh];
+#pragma unroll
+            for (int r = 0; r < TR; ++r) {
+                // (rows that are not valid are zeros with weight 0)
+                float vf[DL];
+                load_row(tb + r * 2 * ROW_B + ROW_B, vf);
+                float p[G];
+#pragma unroll
+                for (int hh = 0; hh < G; hh += 4) {
+                    if constexpr (G >= 4) {
+                        const float4 p4 = *reinterpret_cast<const float4 *>(s_p + r * G + hh);
+                        p[hh] = p4.x; p[hh + 1] = p4.y; p[hh + 2] = p4.z; p[hh + 3] = p4.w;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < G; ++u) p[u] = s_p[r * G + u];
+                    }
+                }
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+                    for (int d = 0; d < DL; d += 2) {
+                        const float2 a2 = ffma2(make_float2(p[hh], p[hh]), make_float2(vf[d], vf[d + 1]),
+                                                make_float2(acc[hh][d], acc[hh][d + 1]));
+                        acc[hh][d] = a2.x;
+                        acc[hh][d + 1] = a2.y;
+                    }
+            }
+            __syncwarp();  // the weights and the buffer are refilled next
+            if (tile + 2 * NWARP < ntiles) {
+                const uint32_t v = fetch(tile + 2 * NWARP, buf);
+                if (buf) vm1 = v; else vm0 = v;
+            } else {
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            }
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();  // every warp is done with its staging buffers
+        // CTA merge of the warps' states: [warp][G] (m, l) and [warp][G][D] acc at the LUT base
+        float *s_acc = reinterpret_cast<float *>(lut);
+        float *s_ml = s_acc + NWARP * G * D;
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+            const float mh = __shfl_sync(0xffffffffu, m, hh * TR);
+            const float lh = __shfl_sync(0xffffffffu, lsum, hh * TR);
+            if (lane == 0) { s_ml[(warp * G + hh) * 2] = mh; s_ml[(warp * G + hh) * 2 + 1] = lh; }
+#pragma unroll
+            for (int d = 0; d < DL; ++d) s_acc[(warp * G + hh) * D + DL * lane + d] = acc[hh][d];
+        }
         __syncthreads();
-        // this CTA's partial (m, l, acc) per query head, in the low region (read by the cluster)
-        float *cpart = reinterpret_cast<float *>(smem + StepLow::END);  // [G][D + 2]
+        // this CTA's partial (M, L, A) per query head g and dim i, element
+        // x = g D + i: A goes to the CTA that merges x (x mod C, slot
+        // [cta][x / C] of its inbox), every CTA gets each head's (M, L)
+        float *recv_acc = reinterpret_cast<float *>(smem + (recv_s - smem_s));  // [C][slots]
+        float *recv_ml = recv_acc + kRecvAccFloats;                              // [C][G][2]
+        const int slots = (G * D + nctas - 1) / nctas;
         for (int x2 = tid; x2 < G * D; x2 += NT) {
             const int gg = x2 / D, i = x2 % D;
-            const int tm = gg / HG, gq = gg % HG;
             float M = -INFINITY;
-            for (int w2 = tm * WPT; w2 < (tm + 1) * WPT; ++w2) M = fmaxf(M, s_ml[(w2 * HG + gq) * 2]);
+            for (int w2 = 0; w2 < NWARP; ++w2) M = fmaxf(M, s_ml[(w2 * G + gg) * 2]);
             float L = 0.0f, A = 0.0f;
             if (M != -INFINITY) {
-                for (int w2 = tm * WPT; w2 < (tm + 1) * WPT; ++w2) {
-                    const float c = fast_exp2(s_ml[(w2 * HG + gq) * 2] - M);
-                    L = fmaf(s_ml[(w2 * HG + gq) * 2 + 1], c, L);
-                    A = fmaf(s_acc[(w2 * HG + gq) * D + i], c, A);
+                for (int w2 = 0; w2 < NWARP; ++w2) {
+                    const float c = fast_exp2(s_ml[(w2 * G + gg) * 2] - M);
+                    L = fmaf(s_ml[(w2 * G + gg) * 2 + 1], c, L);
+                    A = fmaf(s_acc[(w2 * G + gg) * D + i], c, A);
                 }
             }
-            cpart[gg * (D + 2) + i] = A;
-            if (i == 0) { cpart[gg * (D + 2) + D] = M; cpart[gg * (D + 2) + D + 1] = L; }
+            st_cluster_f32(cluster_addr(recv_acc + cta * slots + x2 / nctas, x2 % nctas), A);
+            if (i == 0)
+                for (int r = 0; r < nctas; ++r) {
+                    st_cluster_f32(cluster_addr(recv_ml + (cta * G + gg) * 2, r), M);
+                    st_cluster_f32(cluster_addr(recv_ml + (cta * G + gg) * 2 + 1, r), L);
+                }
         }
-        cluster_sync();  // (5): every CTA's partial is complete
-        // the cluster merge, element x handled by CTA x mod C
+        cluster_sync();  // (5): every partial is in its merging CTA's inbox
+        // the cluster merge of the elements this CTA owns (from its inbox only)
         for (int x2 = cta + nctas * tid; x2 < G * D; x2 += nctas * NT) {
             const int gg = x2 / D, i = x2 % D;
             float M = -INFINITY;
-            for (int r = 0; r < nctas; ++r) M = fmaxf(M, ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + D, r)));
+            for (int r = 0; r < nctas; ++r) M = fmaxf(M, recv_ml[(r * G + gg) * 2]);
             float L = 0.0f, A = 0.0f;
             if (M != -INFINITY) {
                 for (int r = 0; r < nctas; ++r) {
-                    const float pm = ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + D, r));
-                    const float c = fast_exp2(pm - M);
-                    L = fmaf(ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + D + 1, r)), c, L);
-                    A = fmaf(ld_cluster_f32(cluster_addr(cpart + gg * (D + 2) + i, r)), c, A);
+                    const float c = fast_exp2(recv_ml[(r * G + gg) * 2] - M);
+                    L = fmaf(recv_ml[(r * G + gg) * 2 + 1], c, L);
+                    A = fmaf(recv_acc[r * slots + x2 / nctas], c, A);
                 }
             }
             const int64_t oq = (int64_t)b * a.Hq + (int64_t)h * G + gg;
             a.out[oq * D + i] = L > 0.0f ? A / L : 0.0f;
             if (i == 0 && a.lse) a.lse[oq] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
         }
-        cluster_sync();  // (6): no CTA leaves while another may still read its partial
     }
     if (appending && cta == 0 && tid == 0) {
         // every CTA of this cluster read seq_lens[b] before barrier (1); the last

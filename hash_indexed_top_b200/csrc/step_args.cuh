@@ -33,6 +33,14 @@ constexpr int kSampleDiv = 4;
 constexpr int kSampleBins = kBins / kSampleDiv;
 constexpr int kSampleStrata = 64;  // sampled 32-token blocks (at most)
 
+// The attention's cluster merge: CTA c receives, for the elements x = g D + i
+// with x mod C = c, every CTA's partial sum (slot [cta][x / C]) and every
+// CTA's per-head (max, sum) pair, in a region just below the LUT that nothing
+// else uses.
+constexpr int kMaxG = 8;
+constexpr int kRecvAccFloats = kMaxG * kMaxDim + kMaxCluster;
+constexpr int kRecvBytes = (kRecvAccFloats + kMaxCluster * kMaxG * 2) * 4;
+
 // Fixed part of the low shared region (byte offsets from the dynamic base).
 struct StepLow {
     static constexpr int HIST = 0;                                 // u32[kBins]
@@ -47,15 +55,13 @@ struct StepLow {
     static constexpr int NEWR = NEWC + 16;                         // u32[4] the same in stored (rotated) order
     static constexpr int MBAR = NEWR + 16;                         // u64[kRingStages] full barriers of the ring
     static constexpr int MBAR_EMPTY = MBAR + kRingStages * 8;      // u64[kRingStages] slots released by every consumer
-    static constexpr int MBAR_ATT = MBAR_EMPTY + kRingStages * 8;  // u64[kStepWarps][2]
-    static constexpr int WDEF = MBAR_ATT + kStepWarps * 2 * 8;     // int[kStepWarps] definite tokens per warp
+    static constexpr int WDEF = MBAR_EMPTY + kRingStages * 8;      // int[kStepWarps] definite tokens per warp
     static constexpr int CNT = WDEF + kStepWarps * 4;              // int[kMaxCluster][2]
     static constexpr int MID = CNT + kMaxCluster * 8;              // int[kMaxCluster]
     static constexpr int WARPSCAN = MID + kMaxCluster * 4;         // int[32] block-scan scratch
     static constexpr int END = (WARPSCAN + 128 + 255) / 256 * 256; // candidate lists start here
 };
-static_assert(StepLow::MBAR % 8 == 0 && StepLow::MBAR_EMPTY % 8 == 0 && StepLow::MBAR_ATT % 8 == 0,
-              "mbarriers are 8-byte aligned");
+static_assert(StepLow::MBAR % 8 == 0 && StepLow::MBAR_EMPTY % 8 == 0, "mbarriers are 8-byte aligned");
 
 // misc[] slots
 enum : int {
