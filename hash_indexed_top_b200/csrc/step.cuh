@@ -995,7 +995,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             const int ce = (isv ? c - CPR / 2 : c) * 8;  // first element of the chunk
             const __nv_bfloat16 *cache = isv ? kv.v : kv.k;
             const __nv_bfloat16 *fresh = (isv ? vn_row : kn_row) + ce;
-#pragma unroll
+#pragma unroll 1
             for (int i = 0; i < TR / RPI; ++i) {
                 const int r = i * RPI + lane / CPR;
                 int64_t o;
@@ -1089,7 +1089,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
             for (int hh = 0; hh < G; ++hh)
 #pragma unroll
                 for (int d = 0; d < DL; ++d) acc[hh][d] *= ch[hh];
-#pragma unroll
+#pragma unroll 2
             for (int r = 0; r < TR; ++r) {
                 // (rows that are not valid are zeros with weight 0)
                 float vf[DL];
