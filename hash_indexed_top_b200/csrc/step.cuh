@@ -136,16 +136,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     unsigned char *lut = smem + (lut_s - smem_s);
     const uint32_t ring_s = lut_s + 65536u;
     unsigned char *ring = lut + 65536;
-    const uint32_t end_s = smem_s + (uint32_t)a.smem_bytes;
-    // candidate list of this warp: cap_lo entries below the LUT, cap_hi above the ring
-    // (NCONS lists: warp NCONS has none and keeps ncand = 0)
+    // candidate list of this warp: cap entries (token in the CTA's range, order
+    // key) between the low region and the attention merge's inbox below the LUT
     const uint32_t recv_s = lut_s - (uint32_t)kRecvBytes;  // the attention merge's inbox (G > 0)
-    const int cap_lo = (int)((recv_s - (smem_s + StepLow::END)) / (8u * NCONS));
-    const int cap_hi = end_s > ring_s + SS::RING_B ? (int)((end_s - ring_s - SS::RING_B) / (8u * NCONS)) : 0;
-    uint2 *cand_lo = reinterpret_cast<uint2 *>(smem + StepLow::END) + warp * cap_lo;
-    uint2 *cand_hi = reinterpret_cast<uint2 *>(ring + SS::RING_B) + warp * cap_hi;
-    const int cap = cap_lo + cap_hi;
-    auto cand_ref = [&](int j) -> uint2 & { return j < cap_lo ? cand_lo[j] : cand_hi[j - cap_lo]; };
+    // (NCONS lists: warp NCONS has none and keeps ncand = 0)
+    const int cap = (int)((recv_s - (smem_s + StepLow::END)) / (8u * NCONS));
+    uint2 *cand = reinterpret_cast<uint2 *>(smem + StepLow::END) + warp * cap;
 
     // ---- set-up: counters, barriers, this warp's hyperplane words
     for (int i = tid; i < kBins; i += NT) hist[i] = 0;
@@ -565,7 +561,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
                     }
                     if (isc[u]) {
                         const int i = sbase + wsl + 32 * u + lane;
-                        cand_ref(ncand + __popc(ball & lt)) = make_uint2((uint32_t)i, float_key(sc[u]));
+                        cand[ncand + __popc(ball & lt)] = make_uint2((uint32_t)i, float_key(sc[u]));
                     }
                     ncand += nb;
                 }
@@ -598,7 +594,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         // the CTA histogram of the kept tokens of bins >= tl, from this warp's list
         if (!ovf)
             for (int j = lane; j < ncand; j += 32) {
-                const int bin = score_bin(key_to_float(cand_ref(j).y), inv2A);
+                const int bin = score_bin(key_to_float(cand[j].y), inv2A);
                 if (bin >= tl) {
                     atomicAdd(&hist[bin], 1u);
                     atomicAdd(&sup[bin >> 6], 1u);
@@ -653,7 +649,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         for (int jb = 0; jb < ncand; jb += 32) {
             const int jj = jb + lane;
             uint2 e = make_uint2(0u, 0u);
-            if (jj < ncand) e = cand_ref(jj);
+            if (jj < ncand) e = cand[jj];
             const int t = (int)(t0 + (int)e.x);
             const int bin = score_bin(key_to_float(e.y), inv2A);
             const bool inb = jj < ncand && bin == T1;
@@ -780,7 +776,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
         for (int jb = 0; jb < ncand; jb += 32) {
             const int jj = jb + lane;
             if (jj < ncand) {
-                const uint2 e = cand_ref(jj);
+                const uint2 e = cand[jj];
                 const int t = (int)(t0 + (int)e.x);
                 const int bin = score_bin(key_to_float(e.y), inv2A);
                 if (t >= s_end && t < w_beg && (bin > T1 || (bin == T1 && (e.y > Tkey || (e.y == Tkey && t <= IT)))))
