@@ -345,11 +345,14 @@ def run_dashkv(args, cfg, world, rank, local):
     assert eng.get_error() == 0
     enc_ms = e_enc[0].elapsed_time(e_enc[1])
     enc_keys = int(seq.sum()) * cfg.Hkv
-    fma_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * 1.965e9  # fp32 FLOP/s
+    # the encode is b d signed adds per key-head (R is +-1): its roof is one fp32
+    # add per lane per clock
+    add_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 1.965e9  # fp32 adds/s
+    adds_per_s = cfg.bits * cfg.d * enc_keys / (enc_ms * 1e-3)
     encode = {"ms": enc_ms, "key_heads": enc_keys, "key_heads_per_s": enc_keys / (enc_ms * 1e-3),
-              "alu_tflops": 2.0 * cfg.bits * cfg.d * enc_keys / (enc_ms * 1e-3) / 1e12,
-              "alu_frac": 2.0 * cfg.bits * cfg.d * enc_keys / (enc_ms * 1e-3) / fma_peak,
-              "peak": "fp32 FMA lanes: SMs x 128 x 2 x 1.965 GHz",
+              "alu_tadds_per_s": adds_per_s / 1e12,
+              "alu_frac": adds_per_s / add_peak,
+              "peak": "fp32 add lanes: SMs x 128 x 1.965 GHz (one signed add per key element and hyperplane)",
               "bytes": enc_keys * (cfg.d * 2 + cfg.bits // 8), "timing": "one call, L2 flushed before it"}
 
     # One CUDA graph per step (append -> select -> decode on that step's inputs);

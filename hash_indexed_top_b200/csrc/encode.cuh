@@ -85,11 +85,15 @@ encode_keys_kernel(KV kv, const int32_t *__restrict__ seq_lens, const RBits R, i
             const float4 *r4 = reinterpret_cast<const float4 *>(rrow + i * BITS);
 #pragma unroll
             for (int q = 0; q < S::JPT / 4; ++q) {
+                // R is +-1: each product is exact, so a packed fma per two
+                // hyperplanes rounds exactly like the add (or subtract) it is
                 float4 r = r4[q];
-                acc[4 * q + 0] = fmaf(r.x, kx, acc[4 * q + 0]);
-                acc[4 * q + 1] = fmaf(r.y, kx, acc[4 * q + 1]);
-                acc[4 * q + 2] = fmaf(r.z, kx, acc[4 * q + 2]);
-                acc[4 * q + 3] = fmaf(r.w, kx, acc[4 * q + 3]);
+                const float2 a01 = ffma2(make_float2(r.x, r.y), make_float2(kx, kx),
+                                         make_float2(acc[4 * q + 0], acc[4 * q + 1]));
+                const float2 a23 = ffma2(make_float2(r.z, r.w), make_float2(kx, kx),
+                                         make_float2(acc[4 * q + 2], acc[4 * q + 3]));
+                acc[4 * q + 0] = a01.x; acc[4 * q + 1] = a01.y;
+                acc[4 * q + 2] = a23.x; acc[4 * q + 3] = a23.y;
             }
         }
         uint64_t word = 0;
