@@ -363,10 +363,12 @@ def run_dashkv(args, cfg, world, rank, local):
     K = args.steps
     T = min(K, args.trace_steps)
     n_sel_kernels = eng.select_kernels(cache.capacity)
-    sel_names = ["select_step"] if n_sel_kernels == 1 else ["score_hist", "collect_select"]
-    # the whole step as one clustered launch (dashkv_decode_step) for token
-    # selection on the clustered path; the separate calls otherwise
-    fused = not (cfg.block or cfg.radius or args.split_step or n_sel_kernels != 1)
+    sel_names = ["select_fused"] if n_sel_kernels == 1 else ["score_hist", "collect_select"]
+    # --path step: the whole step as one clustered launch (dashkv_decode_step),
+    # for token selection on the clustered path; otherwise the separate calls
+    # (append, select, sparse decode), captured into one graph with
+    # programmatic dependent launches between them
+    fused = args.path == "step" and not (cfg.block or cfg.radius or n_sel_kernels != 1)
     # the kernels of one step, in launch order, and the calls that launch them
     if fused:
         calls = [("decode_step", ["decode_step"])]
@@ -595,8 +597,9 @@ def main():
     ap.add_argument("--cpu-steps", type=int, default=2)
     ap.add_argument("--two-kernel-select", action="store_true",
                     help="use the two-kernel selection path (and the separate calls)")
-    ap.add_argument("--split-step", action="store_true",
-                    help="time append_keys + select + sparse_decode instead of the one-launch decode step")
+    ap.add_argument("--path", choices=["calls", "step"], default="calls",
+                    help="calls: append_keys + select + sparse_decode, one graph per step (the faster path "
+                         "at every configured workload); step: the one-launch dashkv_decode_step")
     ap.add_argument("--trace-steps", type=int, default=10,
                     help="extra traced steps for the per-kernel durations")
     ap.add_argument("--clock-reps", type=int, default=20,

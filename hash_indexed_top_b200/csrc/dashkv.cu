@@ -315,6 +315,18 @@ void set_attrs_bd() {
                          (int)ScoreShape<BITS>::SMEM);
     cudaFuncSetAttribute(score_hist_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)ScoreShape<BITS>::SMEM);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, false, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(select_fused_kernel<BITS, D, true, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
 }
 
 template <int D, int G>
@@ -571,9 +583,47 @@ SelWS carve_selws(const WsLayout &L, char *w, int64_t cap, float *scores) {
     return ws;
 }
 
-// One selection over `k` (the token cache, or the block codes): the clustered
-// step kernel (selection only), or score + collect followed by the optional
-// copy of the scores (rows of length cap).  The workspace is carved as L lays it out.
+// Fused selection: a grid of (C, B * Hkv) CTAs in clusters of C (one cluster
+// per (b, h)) that may also start early behind the preceding kernel.
+template <int BITS, int D>
+void launch_fused_bd(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                     int nctas, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    const int G = ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads;
+    auto kern = kv.radius ? (kv.page_size ? select_fused_kernel<BITS, D, true, true>
+                                          : select_fused_kernel<BITS, D, false, true>)
+                          : (kv.page_size ? select_fused_kernel<BITS, D, true> : select_fused_kernel<BITS, D, false>);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nctas, BH);
+    cfg.blockDim = dim3(kScoreThreads);
+    cfg.dynamicSmemBytes = ScoreShape<BITS>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nctas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, kern, kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, G, seq, ctx->R,
+                       ws, a.topk, a.sink, a.window, a.cap_sel, sel_idx, sel_cnt);
+}
+
+template <int D>
+void launch_fused_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *seq, const SelWS &ws,
+                    int nctas, const SelArgs &a, int32_t *si, int32_t *sc, cudaStream_t st) {
+    switch (ctx->cfg.bits) {
+        case 32: launch_fused_bd<32, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
+        case 64: launch_fused_bd<64, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
+        default: launch_fused_bd<128, D>(ctx, kv, q, seq, ws, nctas, a, si, sc, st); break;
+    }
+}
+
+// One selection over `k` (the token cache, or the block codes): the fused
+// clustered selection, or score + collect, followed by the optional copy of the
+// scores (rows of length cap).  The workspace is carved as L lays it out.
 void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout &L, char *w, const void *q,
                 const int32_t *seq_lens, const SelArgs &a, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
                 Tracer &tr, cudaStream_t st) {
@@ -590,11 +640,11 @@ void run_select(const dashkv_ctx *ctx, const KV &k, int64_t cap, const WsLayout 
     };
     if (use_fused(ctx)) {
         const int nc = fused_cluster(ctx, cap);
-        const StepArgs s = select_args(ctx, k, q, seq_lens, ws, a, sel_idx, sel_cnt, scores, cap);
         tr.before();
-        launch_step(ctx, step_kern(ctx->cfg.bits, ctx->cfg.head_dim, 0, k.page_size != 0, k.radius != nullptr), nc, s,
-                    st);
+        if (ctx->cfg.head_dim == 64) launch_fused_d<64>(ctx, k, q, seq_lens, ws, nc, a, sel_idx, sel_cnt, st);
+        else launch_fused_d<128>(ctx, k, q, seq_lens, ws, nc, a, sel_idx, sel_cnt, st);
         tr.after();
+        copy_scores();
         return;
     }
     tr.before();

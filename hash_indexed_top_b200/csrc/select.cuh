@@ -43,6 +43,9 @@ constexpr int kMaxSelCtas = 512;
 constexpr int kCandSmem = 2048;   // in-bin candidates ranked in shared memory
 constexpr int kListSmem = 8192;   // candidate list held in shared memory by the resolver
 constexpr int kCollectTile = kSelThreads * 16;
+// The fused selection records, per 32-token chunk of a CTA's range, the largest
+// bin in the chunk (uint16 in shared memory, for the first kCmaxCap chunks).
+constexpr int kCmaxCap = 16384;
 
 enum : int { kStateNormal = 0, kStateAll = 1, kStateEmpty = 2 };
 
@@ -135,7 +138,7 @@ struct ScoreShape {
     static constexpr int NW = BITS / 32;       // 32-bit code words per token
     static constexpr uint32_t LUT_BYTES = 256 * 256;
     static constexpr uint32_t SCRATCH_BYTES = kBins * 4 + (kMaxDim + kMaxBits + 64) * 4;  // hist + scratch
-    static constexpr uint32_t LOW_BYTES = SCRATCH_BYTES;
+    static constexpr uint32_t LOW_BYTES = SCRATCH_BYTES + kCmaxCap * 2;               // + chunk maxima
     using Vec = typename std::conditional<BITS == 128, uint4, uint2>::type;  // one token's code
     // per-thread cp.async ring of upcoming codes (one token per thread per stage)
     static constexpr int STAGES = 5;
@@ -217,13 +220,17 @@ struct ScoreOut {
     int R;               // tokens per warp range (multiple of 32)
     float inv2A;
     unsigned char *lut;  // 64 KB LUT region, free for reuse once scoring is done
+    uint16_t *cmax;      // [kCmaxCap] largest bin per 32-token chunk (FUSED only)
 };
 
+// FUSED: the fused selection -- record the chunk maxima, and let the dependent
+// launch (the sparse decode, whose window CTAs need nothing from the selection)
+// start right after the wait on the preceding kernel.
 // RADIUS: radius-scaled scores s' = r~ s (Spherical KV page, section 2.1 ADA: a
 // quantized key radius beside the angle code scales the logit), r~ = (c + 1/2)/4
 // from the token's 8-bit code c in kv.radius; the bins span r~_max times the
 // unscaled range.
-template <int BITS, int D, bool PAGED, bool RADIUS = false>
+template <int BITS, int D, bool PAGED, bool FUSED = false, bool RADIUS = false>
 __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
                                                 const int32_t *__restrict__ seq_lens, const RBits &R,
                                                 const SelWS &ws, int nctas, unsigned char *smem) {
@@ -311,8 +318,10 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
     ScoreOut o;
     o.inv2A = red[0];
     o.lut = lut;
+    o.cmax = reinterpret_cast<uint16_t *>(smem + S::SCRATCH_BYTES);
     // everything above depends on q only; codes and lengths come from the append
     griddep_wait();
+    if constexpr (FUSED) griddep_trigger();
     o.n = clamp_len(kv, seq_lens, b);
     cta_range(o.n, blockIdx.x, nctas, o.t0, o.t1);
     const int64_t t0 = o.t0, t1 = o.t1;
@@ -415,6 +424,11 @@ __device__ __forceinline__ ScoreOut score_phase(const KV &kv, const __nv_bfloat1
                 srow[i] = sc;
                 bin = score_bin(sc, inv2A);
                 atomicAdd(&hist[bin], 1u);
+            }
+            if constexpr (FUSED) {
+                const unsigned m = __reduce_max_sync(0xffffffffu, (unsigned)bin);
+                const int c = (wb >> 5) + k;  // chunk of local tokens [32 c, 32 c + 32)
+                if (lane == 0 && c < kCmaxCap) o.cmax[c] = (uint16_t)m;
             }
         }
     }
@@ -860,6 +874,382 @@ __device__ __forceinline__ int cluster_threshold(const uint32_t *coarse, const u
         else { out[0] = bl; out[1] = (int)(fexcl + fu); out[2] = (int)fl; }
     }
     return __shfl_sync(0xffffffffu, t1, __ffs(hm) - 1);
+}
+
+// Smallest finite float s with score_bin(s, inv2A) >= T, or +inf if there is
+// none, so that for every finite s:  s >= result  <=>  score_bin(s) >= T.
+// score_bin is monotone in s (a correctly rounded fma with a non-negative
+// factor, a clamp, a scale and a truncation), hence monotone along the
+// order-preserving keys.  A full warp first tests the 32 keys around the
+// algebraic estimate; if the boundary is not among them it narrows the whole
+// key range 32-fold per round.  Every lane returns the result.
+__device__ __forceinline__ float bin_floor_value(int T, float inv2A) {
+    const int lane = threadIdx.x & 31;
+    if (T <= 0) return -INFINITY;
+    if (T >= kBins) return INFINITY;
+    auto P = [&](uint32_t key) { return score_bin(key_to_float(key), inv2A) >= T; };
+    if (inv2A > 0.0f) {
+        const float est = ((float)T / (float)(kBins - 1) - 0.5f) / inv2A;
+        const uint32_t k0 = float_key(est) - 16u;
+        const uint32_t b = __ballot_sync(0xffffffffu, P(k0 + (uint32_t)lane));
+        const int f = __ffs(b) - 1;  // a boundary inside the window: false below lane f, true from it
+        if (f > 0 && b == (0xffffffffu << f)) return key_to_float(k0 + (uint32_t)f);
+    }
+    const uint32_t none = 0xff800000u;     // key of +inf: one past the key of FLT_MAX
+    uint64_t lo = 0x00800000u, hi = none;  // key of -FLT_MAX; answer in [lo, hi]
+    while (lo < hi) {
+        const uint64_t n = hi - lo;
+        const uint64_t step = (n + 31) / 32;
+        const uint64_t x = lo + (uint64_t)lane * step;
+        const uint32_t b = __ballot_sync(0xffffffffu, x < hi && P((uint32_t)x));
+        if (b) {
+            const int f = __ffs(b) - 1;    // false at lo + (f - 1) step, true at lo + f step
+            hi = lo + (uint64_t)f * step;
+            if (f) lo += (uint64_t)(f - 1) * step + 1;
+        } else {                           // every tested point is false
+            const uint64_t last = (n - 1) / step < 31 ? (n - 1) / step : 31;
+            lo += last * step + 1;
+        }
+    }
+    return key_to_float((uint32_t)lo);     // `none` maps to +inf
+}
+
+template <int BITS, int D, bool PAGED, bool RADIUS = false>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+select_fused_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq, int G,
+                    const int32_t *__restrict__ seq_lens, const RBits R, SelWS ws, int topk, int S, int W,
+                    int cap_sel, int32_t *sel_idx, int32_t *sel_cnt) {
+    constexpr int NT = kScoreThreads;
+    constexpr int NWARP = NT / 32;
+    constexpr int CW = 64;  // candidates per warp kept in shared memory (more go to the global segment)
+    // hit chunks whose scores one warp stages per round trip: [FB][32] floats per
+    // warp in the code ring, which is idle once the scores are written
+    constexpr int FB = (int)(ScoreShape<BITS>::RING_BYTES / (NWARP * 32 * 4)) < 16
+                           ? (int)(ScoreShape<BITS>::RING_BYTES / (NWARP * 32 * 4)) : 16;
+    static_assert(FB >= 1 && (size_t)FB * NWARP * 32 * 4 <= ScoreShape<BITS>::RING_BYTES, "staging exceeds the ring");
+    // the LUT region (64 KB) after scoring: in-bin list | warp candidates | gathered list, or the resolver
+    static_assert(kInbinMax * 16 <= 16384 && NWARP * CW * 8 <= 16384, "fast-path lists exceed their slots");
+    static_assert(sizeof(ResolveSmem<4096>) <= ScoreShape<BITS>::LUT_BYTES, "resolver exceeds the LUT region");
+    extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ int s_warp[32];
+    __shared__ int s_thr[4];
+    __shared__ int s_misc[4];
+    __shared__ float s_theta[2];
+    __shared__ uint32_t s_coarse[64];      // this CTA's histogram per super-bin (read by the cluster)
+    __shared__ int s_cnt[kMaxCluster][2];  // per CTA of the cluster: in-bin entries, definite middle tokens
+    __shared__ int s_mid[kMaxCluster];
+    __shared__ int s_wkeep[NWARP];
+    __shared__ int s_hlist[NWARP][32];     // per warp: its hit chunks of the current group
+    __shared__ int s_ninb;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.y, cta = blockIdx.x;  // cta = rank in the cluster (cluster = the row of CTAs)
+    const int nctas = gridDim.x;
+    const ScoreOut so = score_phase<BITS, D, PAGED, true, RADIUS>(kv, q, Hq, G, seq_lens, R, ws, nctas, smem);
+    const uint32_t *hist = reinterpret_cast<const uint32_t *>(smem);
+    {   // super-bin counts: 16 threads per super-bin, 4 bins each
+        uint32_t c = hist[4 * tid] + hist[4 * tid + 1] + hist[4 * tid + 2] + hist[4 * tid + 3];
+#pragma unroll
+        for (int o = 8; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if ((lane & 15) == 0) s_coarse[tid >> 4] = c;
+    }
+    const int64_t n = so.n, t0 = so.t0, t1 = so.t1;
+    const int64_t kk = topk < n ? topk : n;
+    const bool normal = n > 0 && kk < n;
+    if (tid == 0) { s_thr[0] = kBins; s_thr[1] = 0; s_thr[2] = 0; s_ninb = 0; }
+    cluster_sync();  // (1): every histogram of the cluster is complete
+    const float inv2A = so.inv2A;
+    if (normal && warp < 2) {  // both find T1; warp 0 then theta(T1), warp 1 theta(T1 + 1)
+        const int T1w = cluster_threshold(s_coarse, hist, nctas, kk, warp == 0 ? s_thr : nullptr);
+        const float th = bin_floor_value(T1w + warp, inv2A);
+        if (lane == 0) s_theta[warp] = th;
+    }
+    __syncthreads();
+    const int T1 = s_thr[0], above1 = s_thr[1], cnt_T1 = s_thr[2];
+    const bool fallback = normal && cnt_T1 > kInbinMax;
+    const int s_end = (int)(S < n ? S : n);
+    const int w_beg = (int)(n - W > s_end ? n - W : s_end);
+    int32_t *cand = ws.cand + (int64_t)bh * ws.ld;
+    uint32_t *ckey = ws.ckey + (int64_t)bh * ws.ld;
+    const float *srow = ws.scores + (int64_t)bh * ws.ld;
+    int32_t *out = sel_idx + (int64_t)bh * cap_sel;
+
+    if (!normal || fallback) {
+        // ---- exact resolver of the two-kernel path (heavy ties, everything or nothing selected):
+        // CTA segments [t0, t0 + seg) of the tokens with bin >= T1, ascending
+        int seg = 0;
+        if (normal) {
+            for (int64_t base = t0; base < t1; base += (int64_t)NT * 32) {
+                const int64_t tb = base + (int64_t)tid * 32;
+                uint32_t flags = 0;
+                for (int e = 0; e < 32; ++e)
+                    if (tb + e < t1 && score_bin(__ldcg(srow + tb + e), inv2A) >= T1) flags |= 1u << e;
+                int tot;
+                int r = block_excl_scan<NT>(__popc(flags), s_warp, &tot);
+                while (flags) {
+                    const int j = __ffs(flags) - 1;
+                    flags &= flags - 1;
+                    cand[t0 + seg + r++] = (int32_t)(tb + j);
+                }
+                seg += tot;
+            }
+        }
+        if (tid == 0) ws.seg_cnt[(int64_t)bh * kMaxSelCtas + cta] = seg;
+        __threadfence();
+        cluster_sync();  // (2): segments complete (nothing reads another CTA's shared memory after this)
+        if (cta != 0) return;
+        SelState st;
+        st.T1 = T1; st.above1 = above1; st.cnt_T1 = cnt_T1;
+        st.flags = n == 0 ? kStateEmpty : (normal ? kStateNormal : kStateAll);
+        st.inv2A = inv2A; st.pad = 0.0f; st.kk = (int32_t)kk; st.n = (int32_t)n;
+        resolve_emit<NT, 4096>(ws, bh, nctas, st, S, W, cap_sel, sel_idx, sel_cnt,
+                               *reinterpret_cast<ResolveSmem<4096> *>(so.lut));
+        return;
+    }
+
+    // ---- fast path.  Warp w owns the 32-token chunks of its range; only the
+    // chunks whose maximum bin reaches T1 are re-read (lane = token, up to FB
+    // chunks per memory round trip, staged in shared memory so that the code
+    // that runs once per step stays a pair of short loops).  A token is a candidate iff its score >=
+    // theta (exactly bin >= T1) and in the threshold bin iff also score <
+    // theta2.  The warp keeps its candidates in token order with their order
+    // keys -- the first CW in shared memory, the rest in its slice of the global
+    // segment -- lists the in-bin ones for the cluster and counts the definite
+    // middle ones.
+    uint4 *s_loc = reinterpret_cast<uint4 *>(so.lut);                      // this CTA's in-bin tokens
+    uint2 *wcand = reinterpret_cast<uint2 *>(so.lut + 16384) + warp * CW;  // per-warp candidates
+    uint4 *s_inb = reinterpret_cast<uint4 *>(so.lut + 32768);              // the cluster's in-bin tokens
+    const float theta = s_theta[0], theta2 = s_theta[1];
+    const int wb = warp * so.R;
+    const int we = (int)min((int64_t)(wb + so.R), t1 - t0);
+    const int nch = we > wb ? (we - wb + 31) >> 5 : 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    int ncand = 0, ndef = 0;
+    auto chunk_hit = [&](int c) {
+        const int gc = (wb >> 5) + c;
+        return c < nch && (gc >= kCmaxCap || (int)so.cmax[gc] >= T1);
+    };
+    // per-warp staging buffer [FB][32] of scores, in the (now idle) code ring,
+    // and the warp's list of hit chunks of the current group of 32
+    float *fbuf = reinterpret_cast<float *>(so.lut + 65536) + warp * (FB * 32);
+    const uint32_t fbuf_s = (uint32_t)__cvta_generic_to_shared(fbuf);
+    int *hlist = s_hlist[warp];
+    const int wlen = we - wb;  // tokens of this warp
+    for (int g0 = 0; g0 < nch; g0 += 32) {
+        const bool hc = chunk_hit(g0 + lane);
+        const uint32_t hb = __ballot_sync(0xffffffffu, hc);
+        if (hc) hlist[__popc(hb & lt)] = g0 + lane;
+        __syncwarp();
+        const int nh = __popc(hb);
+        for (int h0 = 0; h0 < nh; h0 += FB) {
+            const int nf = min(FB, nh - h0);
+            // stage the scores of chunks h0 .. h0 + nf - 1: 16 bytes per lane, 4 chunks
+            // per instruction, all in flight at once (whole chunks: rows are padded
+            // to 64 tokens, so a chunk never runs past its row)
+#pragma unroll 1
+            for (int q = lane; q < 8 * nf; q += 32) {
+                const int c = hlist[h0 + (q >> 3)];
+                const float *src = srow + t0 + wb + 32 * c + 4 * (q & 7);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(fbuf_s + 16u * (uint32_t)q), "l"(src)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+            __syncwarp();
+#pragma unroll 2
+            for (int f = 0; f < nf; ++f) {
+                const int li = 32 * hlist[h0 + f] + lane;  // warp-local token
+                const float sv = fbuf[32 * f + lane];
+                const bool hit = li < wlen && sv >= theta;
+                const uint32_t ball = __ballot_sync(0xffffffffu, hit);
+                if (hit) {
+                    const int j = ncand + __popc(ball & lt);
+                    const int t = (int)(t0 + wb + li);
+                    const uint32_t key = float_key(sv);
+                    if (j < CW) wcand[j] = make_uint2((uint32_t)t, key);
+                    else { cand[t0 + wb + j] = t; ckey[t0 + wb + j] = key; }
+                }
+                ncand += __popc(ball);
+            }
+            __syncwarp();  // the buffer is refilled by the next batch
+        }
+    }
+    auto cand_at = [&](int j, int &t, uint32_t &key) {
+        if (j < CW) { const uint2 c = wcand[j]; t = (int)c.x; key = c.y; }
+        else { t = __ldcg(cand + t0 + wb + j); key = __ldcg(ckey + t0 + wb + j); }
+    };
+    __syncwarp();
+    // classify the warp's candidates, 32 at a time: in the threshold bin (score <
+    // theta2: listed for the cluster, one reservation per group) or definite
+    // (counted when in the middle range)
+    const uint32_t key2 = float_key(theta2);  // order keys follow scores
+    for (int jb = 0; jb < ncand; jb += 32) {
+        const int j = jb + lane;
+        int t = 0;
+        uint32_t key = 0;
+        if (j < ncand) cand_at(j, t, key);
+        const bool inb = j < ncand && key < key2;
+        const bool def = j < ncand && !inb && t >= s_end && t < w_beg;
+        ndef += __popc(__ballot_sync(0xffffffffu, def)) * (lane == 0);
+        const uint32_t ib = __ballot_sync(0xffffffffu, inb);
+        if (ib) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&s_ninb, __popc(ib));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int slot = base + __popc(ib & lt);
+            if (inb && slot < kInbinMax) s_loc[slot] = make_uint4(key, (uint32_t)t, (uint32_t)cta, (uint32_t)warp);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
+    if (lane == 0) s_wkeep[warp] = ndef;  // kept candidates of the warp: + its selected in-bin ones
+    __syncthreads();
+    if (warp == 0) {
+        // publish (in-bin entries, definite middle tokens) into every CTA's s_cnt[cta]
+        int d = s_wkeep[lane];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        const int ni = min(s_ninb, kInbinMax);
+        if (lane < nctas) {
+            st_cluster_u32(cluster_addr(&s_cnt[cta][0], lane), (uint32_t)ni);
+            st_cluster_u32(cluster_addr(&s_cnt[cta][1], lane), (uint32_t)d);
+        }
+    }
+    cluster_sync();  // (2): every CTA's in-bin list is complete and its counts delivered
+
+    // ---- gather the cluster's in-bin lists (their sizes sum to cnt_T1 <= NT):
+    // thread e copies entry e from the CTA whose list holds it
+    const int c1 = cnt_T1;
+    if (warp * 32 < c1) {
+        const int ni = lane < nctas ? s_cnt[lane][0] : 0;
+        int incl = ni;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int excl = incl - ni;
+        int r = 0;
+        for (int q = 1; q < nctas; ++q) r = __shfl_sync(0xffffffffu, excl, q) <= tid ? q : r;
+        const int off = tid - __shfl_sync(0xffffffffu, excl, r);
+        if (tid < c1) s_inb[tid] = ld_cluster_v4(cluster_addr(s_loc + off, r));
+    }
+    __syncthreads();
+    cluster_arrive();  // (3): done with the other CTAs' shared memory
+
+    // ---- rank the in-bin list (score desc, token asc): the need1-th entry
+    // (Tkey, IT) is the last one selected.  Credit the selected middle ones to
+    // their CTA (output offsets) and, for this CTA's, to their warp.
+    const int need1 = (int)kk - above1;  // 1 <= need1 <= c1
+    if (c1 <= 32) {
+        if (warp == 0) {  // one warp, entry e in lane e
+            const uint4 en = lane < c1 ? s_inb[lane] : make_uint4(0u, 0u, 0u, 0u);
+            uint32_t Tkey = 0u;
+            int IT = 0x7fffffff;
+            if (need1 < c1) {
+                int rank = 0;
+                for (int f = 0; f < c1; ++f) {
+                    const uint32_t kf = __shfl_sync(0xffffffffu, en.x, f);
+                    const uint32_t tf = __shfl_sync(0xffffffffu, en.y, f);
+                    rank += (kf > en.x) || (kf == en.x && tf < en.y);
+                }
+                const int src = __ffs(__ballot_sync(0xffffffffu, lane < c1 && rank == need1 - 1)) - 1;
+                Tkey = __shfl_sync(0xffffffffu, en.x, src);
+                IT = (int)__shfl_sync(0xffffffffu, en.y, src);
+            }
+            const int t = (int)en.y;
+            const bool sel = lane < c1 && t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT));
+            int mid = 0;  // lane r < nctas: selected middle tokens of CTA r
+            for (int r = 0; r < nctas; ++r) {
+                const int cr = __popc(__ballot_sync(0xffffffffu, sel && (int)en.z == r));
+                if (lane == r) mid = s_cnt[r][1] + cr;
+            }
+            if (sel && (int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
+            int before = lane < cta ? mid : 0, total = mid;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                before += __shfl_xor_sync(0xffffffffu, before, o);
+                total += __shfl_xor_sync(0xffffffffu, total, o);
+            }
+            if (lane == 0) { s_misc[0] = (int)Tkey; s_misc[1] = IT; s_misc[2] = before; s_misc[3] = total; }
+        }
+    } else {  // a long list: every thread ranks its entries
+        if (tid == 0) { s_misc[0] = 0; s_misc[1] = 0x7fffffff; }
+        if (tid < nctas) s_mid[tid] = s_cnt[tid][1];
+        __syncthreads();
+        if (need1 < c1) {
+            for (int e = tid; e < c1; e += NT) {
+                const uint32_t ke = s_inb[e].x, ie = s_inb[e].y;
+                int rank = 0;
+                for (int f = 0; f < c1; ++f) {
+                    const uint32_t kf = s_inb[f].x;
+                    rank += (kf > ke) || (kf == ke && s_inb[f].y < ie);
+                }
+                if (rank == need1 - 1) { s_misc[0] = (int)ke; s_misc[1] = (int)ie; }
+            }
+        }
+        __syncthreads();
+        const uint32_t Tkey = (uint32_t)s_misc[0];
+        const int IT = s_misc[1];
+        for (int e = tid; e < c1; e += NT) {
+            const uint4 en = s_inb[e];
+            const int t = (int)en.y;
+            if (t >= s_end && t < w_beg && (en.x > Tkey || (en.x == Tkey && t <= IT))) {
+                atomicAdd(&s_mid[en.z], 1);
+                if ((int)en.z == cta) atomicAdd(&s_wkeep[en.w], 1);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int before = 0, total = 0;
+            for (int r = 0; r < nctas; ++r) {
+                before += r < cta ? s_mid[r] : 0;
+                total += s_mid[r];
+            }
+            s_misc[2] = before;
+            s_misc[3] = total;
+        }
+    }
+    __syncthreads();
+    const uint32_t Tkey = (uint32_t)s_misc[0];
+    const int IT = s_misc[1];
+    const int total_mid = s_misc[3];
+    auto keep = [&](int t, uint32_t key) {
+        if (t < s_end || t >= w_beg) return false;
+        return key_to_float(key) >= theta2 || key > Tkey || (key == Tkey && t <= IT);
+    };
+    // ---- ordered emission: warp w writes its kept candidates from offset
+    // s_end + (this CTA's offset) + (kept candidates of warps < w)
+    int wpos = s_end + s_misc[2];
+    for (int w2 = 0; w2 < warp; ++w2) wpos += s_wkeep[w2];
+    for (int jb = 0; jb < ncand; jb += 32) {
+        const int j = jb + lane;
+        int t = 0; uint32_t key = 0;
+        if (j < ncand) cand_at(j, t, key);
+        const bool k2 = j < ncand && keep(t, key);
+        const uint32_t ball = __ballot_sync(0xffffffffu, k2);
+        if (k2) {
+            const int p = wpos + __popc(ball & lt);
+            if (p < cap_sel) out[p] = t;
+        }
+        wpos += __popc(ball);
+    }
+    {   // the sinks, the window and the padding, spread over the cluster's CTAs
+        const int wpos0 = s_end + total_mid;
+        const int nwin = (int)(n - w_beg);
+        const int total = min(wpos0 + nwin, cap_sel);
+        const int nall = s_end + nwin + (cap_sel - total);
+        for (int x = cta * NT + tid; x < nall; x += nctas * NT) {
+            if (x < s_end) {
+                out[x] = x;
+            } else if (x < s_end + nwin) {
+                const int tw = x - s_end;
+                if (wpos0 + tw < cap_sel) out[wpos0 + tw] = w_beg + tw;
+            } else {
+                out[total + (x - s_end - nwin)] = -1;
+            }
+        }
+        if (cta == 0 && tid == 0) sel_cnt[bh] = total;
+    }
+    cluster_wait();  // (3): no CTA leaves while another may still read its shared memory
 }
 
 }  // namespace dkv
