@@ -83,14 +83,16 @@ typedef enum dashkv_status {
                                     up (a bulk copy did not land); results invalid    */
 } dashkv_status;
 
-/* Selection path.  By default dashkv_select (and dashkv_decode_step) runs one
- * kernel with one thread-block cluster per (sequence, kv head): its CTAs (one
- * per SM, up to 16 per cluster) stream the codes through bulk-copy rings, keep
- * the candidates in shared memory and exchange histograms and boundary tokens
- * through distributed shared memory and hardware cluster barriers.  Without
- * cluster launch support, or with this flag, the selection runs two ordinary
- * kernels instead (and dashkv_decode_step the three separate calls).  All
- * give identical selections. */
+/* Selection path.  By default dashkv_select runs one kernel with one
+ * thread-block cluster per (sequence, kv head): its CTAs (one per SM, up to 16
+ * per cluster) stream the codes, build a histogram of the scores and exchange
+ * histograms and boundary tokens through distributed shared memory and
+ * hardware cluster barriers; dashkv_decode_step runs its own clustered kernel
+ * (append, selection and attention in one launch: its CTAs keep candidates
+ * at or above a sampled threshold in shared memory and attend over what they
+ * kept).  Without cluster launch support, or with this flag, the selection runs
+ * two ordinary kernels instead (and dashkv_decode_step the three separate
+ * calls).  All give identical selections. */
 #define DASHKV_FLAG_TWO_KERNEL_SELECT 1
 
 /* Problem description.  Supported: head_dim in {64, 128}; bits in
