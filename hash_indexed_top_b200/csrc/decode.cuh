@@ -8,9 +8,12 @@
 // selected ids; the optional first wy rows hold window CTAs (see the kernel).  A lane group of LPR
 // lanes owns one row at a time (DPL = d / LPR dims per lane), gathers its K and
 // V slices with 16-byte loads once, and serves all G query heads of the group
-// from them.  Rows are processed in tiles of RT per lane group: the logits of
-// the tile are formed first, then one running-max update and one rescale of
-// the accumulators per tile (fp32, base-2 exponentials).  Each CTA merges its
+// from them.  Rows are processed in tiles of RT per lane group: the RT G
+// partial logits of the tile are formed first and summed over the group by a
+// transpose butterfly that leaves one (row, head) logit per lane; each lane
+// updates its head's running max and sum, the weights go back to the group
+// through shared memory, and the accumulators are rescaled once per tile
+// (fp32, base-2 exponentials).  Each CTA merges its
 // lane groups' states in shared memory and writes one partial; the last CTA of
 // the (b, h) to arrive (atomic counter, no waiting) merges the partials with a
 // log-sum-exp reduction and writes out / lse.
@@ -35,13 +38,16 @@ struct DecodeShape {
     static constexpr int NWARP = kAttnThreads / 32;
     static constexpr int NST = NWARP * RPW;            // lane groups (running states) per CTA
     static constexpr int RT0 = RPW >= 8 ? 1 : 8 / RPW;
-    static constexpr int RT = RT0 * G > 32 ? 32 / G : RT0;  // rows per lane group per tile (<= 32 logits)
+    static constexpr int RT1 = RT0 * G > 32 ? 32 / G : RT0;
+    static constexpr int RT = RT1 * G > LPR ? (LPR / G > 0 ? LPR / G : 1) : RT1;  // rows per lane group per tile:
+                                                                                  // its logits fit the group's lanes
     static constexpr int TROWS = RPW * RT;             // rows per warp tile
     static constexpr int STAGES = TROWS <= 4 ? 3 : 2;  // cp.async pipeline depth per warp
     static constexpr int CPR = D / 8;                  // 16-byte chunks per K (or V) row
     // per warp: STAGES buffers x TROWS rows x (K, V) x D bf16
     static constexpr size_t STAGE_BYTES = (size_t)NWARP * STAGES * TROWS * 2 * D * 2;
-    static constexpr size_t SMEM = STAGE_BYTES + (size_t)NST * G * (D + 2) * 4 + 16;
+    static constexpr int V = RT * G;                   // logits of a lane group's tile (<= LPR)
+    static constexpr size_t SMEM = STAGE_BYTES + (size_t)NST * G * (D + 2) * 4 + (size_t)NST * V * 4 + 16;
 };
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
@@ -71,16 +77,26 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                      const int32_t *__restrict__ seq_lens, int n_sink, int n_window, int topk, int wy, int nw) {
     using S = DecodeShape<D, G>;
     constexpr int DPL = S::DPL, LPR = S::LPR, RPW = S::RPW, NST = S::NST, RT = S::RT;
-    constexpr int TROWS = S::TROWS, CPR = S::CPR, NWARP = S::NWARP, STAGES = S::STAGES;
+    constexpr int TROWS = S::TROWS, CPR = S::CPR, NWARP = S::NWARP, STAGES = S::STAGES, V = S::V;
+    static_assert((V & (V - 1)) == 0 && V <= LPR, "a lane group's logits fit its lanes");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(smem_raw);               // [NWARP][STAGES][TROWS][2][D]
     float *s_acc = reinterpret_cast<float *>(smem_raw + S::STAGE_BYTES);              // [NST][G][D]
     float *s_m = s_acc + NST * G * D;                                                  // [NST][G]
     float *s_l = s_m + NST * G;                                                        // [NST][G]
+    float *s_p = s_l + NST * G;                                                        // [NST][V] weights
     __shared__ int s_last;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = lane / LPR, li = lane % LPR;
+    // The V = RT G logits of a lane group's tile are summed over its LPR lanes
+    // by a transpose butterfly: at the level that pairs lanes across bit k every
+    // lane sends the upper half of its values and keeps the lower half, and
+    // after it lane li holds the logit of (row lv / G, head lv % G), lv = li &
+    // (V - 1).  The halves line up because a lane keeps its slots in an order
+    // XOR-ed with lv: slot (j, g) holds row j ^ jperm and head g ^ gperm.
+    const int lv = li & (V - 1);
+    const int gperm = lv % G, jperm = lv / G;
     // Roles.  With wy > 0 the first wy rows of the grid hold nw window CTAs per
     // (b, h): between them they attend over the sinks and the window, which
     // every selection contains, straight from the token range, so they do not
@@ -98,11 +114,11 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     const int b = bh / kv.Hkv, h = bh % kv.Hkv;
     const int64_t cap_tokens = kv.capacity();
 
-    // this lane's slice of every query head of the group
+    // this lane's slice of every query head of the group (slot g: head g ^ gperm)
     float qf[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        const __nv_bfloat16 *qr = q + ((int64_t)b * Hq + h * G + g) * D + li * DPL;
+        const __nv_bfloat16 *qr = q + ((int64_t)b * Hq + h * G + (g ^ gperm)) * D + li * DPL;
 #pragma unroll
         for (int e = 0; e < DPL; e += 2) {
             const uint32_t w = *reinterpret_cast<const uint32_t *>(qr + e);
@@ -110,14 +126,12 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             qf[g][e + 1] = bf16_hi(w);
         }
     }
-    float m[G], l[G], acc[G][DPL];
+    float m = -INFINITY, lsum = 0.0f;  // of head lv % G (the same in all its lanes)
+    float acc[G][DPL];                 // every head (in order) at this lane's dims
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-        l[g] = 0.0f;
+    for (int g = 0; g < G; ++g)
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[g][e] = 0.0f;
-    }
 
     // q is an input of the step; the selection comes from the preceding kernel
     // (the window CTAs need none of it: the lengths and rows they read were
@@ -221,12 +235,11 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
         __syncwarp();
         const __nv_bfloat16 *tile = wstage + (size_t)buf * TROWS * 2 * D;
 
-        float x[RT][G];  // logits, then softmax weights
-        bool ok[RT];
+        // partial q . k of slot (j, g): row j ^ jperm, head g ^ gperm
+        float x[V];
 #pragma unroll
         for (int j = 0; j < RT; ++j) {
-            const int jr = j * RPW + sub;  // row within the tile
-            ok[j] = __shfl_sync(0xffffffffu, tok[buf], jr) >= 0;
+            const int jr = (j ^ jperm) * RPW + sub;  // row within the tile
             const __nv_bfloat16 *kr = tile + (size_t)jr * 2 * D + li * DPL;
             float kf[DPL];
             if constexpr (DPL >= 8) {
@@ -246,39 +259,42 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
 #pragma unroll
                 for (int e = 0; e < DPL; e += 2)
                     d2 = ffma2(make_float2(qf[g][e], qf[g][e + 1]), make_float2(kf[e], kf[e + 1]), d2);
-                x[j][g] = d2.x + d2.y;
+                x[j * G + g] = d2.x + d2.y;
             }
         }
 #pragma unroll
-        for (int o = LPR / 2; o; o >>= 1)
+        for (int half = V / 2; half >= 1; half >>= 1)
 #pragma unroll
-            for (int j = 0; j < RT; ++j)
+            for (int i = 0; i < half; ++i) x[i] += __shfl_xor_sync(0xffffffffu, x[i + half], half);
 #pragma unroll
-                for (int g = 0; g < G; ++g) x[j][g] += __shfl_xor_sync(0xffffffffu, x[j][g], o);
+        for (int o = LPR / 2; o >= V; o >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], o);
+        // online softmax of head lv % G over its RT rows (lanes lv, lv + G, ...)
+        const bool okl = __shfl_sync(0xffffffffu, tok[buf], (lv / G) * RPW + sub) >= 0;
+        const float sc = okl ? x[0] * scale_log2 : -INFINITY;
+        float tmax = sc;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float tmax = -INFINITY;
+        for (int o = G; o < V; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+        const float mn = fmaxf(m, tmax);
+        const float c = mn == -INFINITY ? 1.0f : fast_exp2(m - mn);  // 0 while m = -inf
+        const float pw = okl ? fast_exp2(sc - mn) : 0.0f;
+        float ps = pw;
 #pragma unroll
-            for (int j = 0; j < RT; ++j) {
-                x[j][g] = ok[j] ? x[j][g] * scale_log2 : -INFINITY;
-                tmax = fmaxf(tmax, x[j][g]);
-            }
-            if (tmax == -INFINITY) {  // no valid row in this lane group's tile
+        for (int o = G; o < V; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        lsum = fmaf(lsum, c, ps);
+        m = mn;
+        // the weights to the whole lane group through shared memory, each head's
+        // rescale factor by shuffle
+        float *sp = s_p + (warp * RPW + sub) * V;  // [RT][G]
+        if (li < V) sp[li] = pw;
+        float ch[G];
 #pragma unroll
-                for (int j = 0; j < RT; ++j) x[j][g] = 0.0f;
-                continue;
-            }
-            const float mn = fmaxf(m[g], tmax);
-            const float c = fast_exp2(m[g] - mn);
-            m[g] = mn;
-            float psum = 0.0f;
+        for (int g = 0; g < G; ++g) ch[g] = __shfl_sync(0xffffffffu, c, sub * LPR + g);
+        __syncwarp();
 #pragma unroll
-            for (int j = 0; j < RT; ++j) { x[j][g] = fast_exp2(x[j][g] - mn); psum += x[j][g]; }
-            l[g] = fmaf(l[g], c, psum);
+        for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[g][e] *= c;
-        }
-        // P.V for the tile
+            for (int e = 0; e < DPL; ++e) acc[g][e] *= ch[g];
+        // P.V for the tile (rows that are not valid are zero-filled, weight 0)
 #pragma unroll
         for (int j = 0; j < RT; ++j) {
             const int jr = j * RPW + sub;
@@ -295,9 +311,20 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                 const uint2 w = *reinterpret_cast<const uint2 *>(vrow);
                 vf[0] = bf16_lo(w.x); vf[1] = bf16_hi(w.x); vf[2] = bf16_lo(w.y); vf[3] = bf16_hi(w.y);
             }
+            float pj[G];
+            if constexpr (G >= 4) {
+#pragma unroll
+                for (int g = 0; g < G; g += 4) {
+                    const float4 p4 = *reinterpret_cast<const float4 *>(sp + j * G + g);
+                    pj[g] = p4.x; pj[g + 1] = p4.y; pj[g + 2] = p4.z; pj[g + 3] = p4.w;
+                }
+            } else {
+#pragma unroll
+                for (int g = 0; g < G; ++g) pj[g] = sp[j * G + g];
+            }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float2 p2 = make_float2(x[j][g], x[j][g]);
+                const float2 p2 = make_float2(pj[g], pj[g]);
 #pragma unroll
                 for (int e = 0; e < DPL; e += 2) {
                     const float2 a2 = ffma2(p2, make_float2(vf[e], vf[e + 1]), make_float2(acc[g][e], acc[g][e + 1]));
@@ -314,7 +341,9 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     const int st = warp * RPW + sub;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        if (li == 0) { s_m[st * G + g] = m[g]; s_l[st * G + g] = l[g]; }
+        const float mg = __shfl_sync(0xffffffffu, m, sub * LPR + g);
+        const float lg = __shfl_sync(0xffffffffu, lsum, sub * LPR + g);
+        if (li == 0) { s_m[st * G + g] = mg; s_l[st * G + g] = lg; }
 #pragma unroll
         for (int e = 0; e < DPL; ++e) s_acc[(st * G + g) * D + li * DPL + e] = acc[g][e];
     }
