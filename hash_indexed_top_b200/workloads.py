@@ -85,6 +85,9 @@ CONFIGS["c128k_blocks4"] = CONFIGS["c128k"].scaled(name="c128k_blocks4", block=4
 CONFIGS["c1m_blocks4"] = CONFIGS["c1m"].scaled(name="c1m_blocks4", block=4)
 # the 128K workload selected on radius-scaled scores
 CONFIGS["c128k_radius"] = CONFIGS["c128k"].scaled(name="c128k_radius", radius=True)
+# the 1M-token workload's shape at half the length: a case small enough for
+# multi-pass profiler captures of the same kernels
+CONFIGS["c512k"] = CONFIGS["c1m"].scaled(name="c512k", N=524288)
 
 
 def grid(x: torch.Tensor) -> torch.Tensor:
