@@ -460,3 +460,114 @@ void dko_radius_scale(int B, int Hkv, int64_t n_cap, const int32_t *page_table, 
                 out[i] = (double)prod + 0.0;
             }
 }
+
+/* ------------------------------------------------------ precision tiers */
+/*
+ * Tier-homogeneous pages (Spherical KV page, section 2.2 RDR: every retained
+ * state gets a precision tier, protected states keep the highest one, and
+ * states are grouped into pages of one tier so that the decode reads a page
+ * in one pass guided by its header; DASH-KV page, section
+ * "技术架构：动态混合精度机制", paras 2-3: the tokens that matter keep full
+ * floating-point precision, the others a cheaper form; DeepSeek DSA->CSA/HCA
+ * page: the KV store itself is mixed-precision).
+ *
+ * Two tiers.  Tier 0: the bf16 rows as stored.  Tier 1: FP8 E4M3 rows (OCP
+ * 8-bit floating point, "FN" variant: 1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits, no infinities, S.1111.111 is NaN, largest finite 448)
+ * with one power-of-two scale per (token, kv head) row and per tensor (K, V):
+ *   s   = the largest integer with amax * 2^s <= 448, capped at 127
+ *         (amax = max_i |x_i| over the row; s = 0 for an all-zero row);
+ *   c_i = e4m3 code of x_i * 2^s, rounded to nearest, ties to even;
+ *   x~_i = value(c_i) * 2^-s.
+ * A page's tier is a byte per physical page (its header).  The controller:
+ * a page is demoted to tier 1 when every one of its tokens lies in the
+ * middle [S, N - W) of its sequence (no sink, no window token), it is still
+ * tier 0 and the caller did not protect it.  Attention over a selection reads
+ * x~ for rows of tier-1 pages and the bf16 rows otherwise, exactly as before.
+ *
+ * FP8 arrays: k8 / v8 [P][page][Hkv][d] uint8 (the K / V page layout),
+ * exps [P][page][Hkv][2] int8 (s of the K row, then of the V row).
+ */
+double dko_e4m3_value(uint8_t c) {
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest e4m3 code of v, ties to the even code; |v| above 448 saturates to
+ * +-448 (never reached for scaled rows). */
+uint8_t dko_e4m3_encode(double v) {
+    uint8_t sign = (v < 0.0 || (v == 0.0 && signbit(v))) ? 0x80 : 0;
+    double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    /* quantum of the binade of a: 2^(E-3) for a in [2^E, 2^(E+1)), E >= -6;
+     * 2^-9 below 2^-6 (subnormals) */
+    int E;
+    if (a < ldexp(1.0, -6)) E = -6;
+    else {
+        frexp(a, &E);  /* a = f * 2^E, f in [0.5, 1) */
+        E -= 1;
+    }
+    double quantum = ldexp(1.0, E - 3);
+    double n = a / quantum;            /* exact: power-of-two divisor */
+    double r = floor(n);
+    double frac = n - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double q = r * quantum;            /* the rounded magnitude */
+    if (q > 448.0) q = 448.0;
+    /* the code of q */
+    if (q < ldexp(1.0, -6)) return sign | (uint8_t)(q / ldexp(1.0, -9));
+    int Eq;
+    double f = frexp(q, &Eq);          /* q = f * 2^Eq = (2f) * 2^(Eq-1) */
+    int e = Eq - 1 + 7;
+    int m = (int)((2.0 * f - 1.0) * 8.0);
+    return sign | (uint8_t)((e << 3) | m);
+}
+
+int dko_tier_exponent(const double *x, int d) {
+    double amax = 0.0;
+    for (int i = 0; i < d; ++i)
+        if (fabs(x[i]) > amax) amax = fabs(x[i]);
+    if (amax == 0.0) return 0;
+    /* amax = f * 2^E, f in [0.5, 1); 448 = 0.875 * 2^9 */
+    int E;
+    double f = frexp(amax, &E);
+    int s = (f <= 0.875) ? 9 - E : 8 - E;
+    return s > 127 ? 127 : s;
+}
+
+/* Scale exponent and codes of one row. */
+void dko_tier_quantize_row(const double *x, int d, uint8_t *codes, int8_t *s_out) {
+    int s = dko_tier_exponent(x, d);
+    for (int i = 0; i < d; ++i) codes[i] = dko_e4m3_encode(ldexp(x[i], s));
+    *s_out = (int8_t)s;
+}
+
+/* The controller over every (sequence, logical page) of a paged cache:
+ * demote the eligible pages (see above), writing their codes and exponents
+ * and setting tier[p] = 1.  protect may be NULL.  Returns the number of pages
+ * demoted. */
+int dko_demote_pages(int B, int Hkv, int d, int page, const int32_t *page_table, int max_pages,
+                     const double *K, const double *V, const int32_t *seq_lens, int S, int W,
+                     const uint8_t *protect, uint8_t *tier, uint8_t *k8, uint8_t *v8, int8_t *exps) {
+    int demoted = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t n = seq_lens[b];
+        for (int p = 0; p < max_pages; ++p) {
+            int64_t lo = (int64_t)p * page, hi = lo + page;  /* tokens [lo, hi) */
+            if (lo < S || hi > n - W) continue;
+            int32_t phys = page_table[(int64_t)b * max_pages + p];
+            if (phys < 0 || tier[phys] != 0 || (protect && protect[phys])) continue;
+            for (int slot = 0; slot < page; ++slot)
+                for (int h = 0; h < Hkv; ++h) {
+                    int64_t row = ((int64_t)phys * page + slot) * Hkv + h;
+                    dko_tier_quantize_row(K + row * d, d, k8 + row * d, exps + row * 2);
+                    dko_tier_quantize_row(V + row * d, d, v8 + row * d, exps + row * 2 + 1);
+                }
+            tier[phys] = 1;
+            ++demoted;
+        }
+    }
+    return demoted;
+}

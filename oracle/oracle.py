@@ -63,6 +63,15 @@ def lib():
         L.dko_radius_value.restype = ctypes.c_double
         L.dko_radius_codes.argtypes = [I, I, I, I64, P, I, I, P, P, P]
         L.dko_radius_scale.argtypes = [I, I, I64, P, I, I, P, P, P, P]
+        L.dko_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.dko_e4m3_value.restype = ctypes.c_double
+        L.dko_e4m3_encode.argtypes = [ctypes.c_double]
+        L.dko_e4m3_encode.restype = ctypes.c_uint8
+        L.dko_tier_exponent.argtypes = [P, I]
+        L.dko_tier_exponent.restype = I
+        L.dko_tier_quantize_row.argtypes = [P, I, P, P]
+        L.dko_demote_pages.argtypes = [I, I, I, I, P, I, P, P, P, I, I, P, P, P, P, P]
+        L.dko_demote_pages.restype = I
         L.dko_set_threads.argtypes = [I]
         L.dko_get_threads.restype = I
         _lib = L
@@ -282,3 +291,76 @@ def decode_step_radius(layout: Layout, Hq, q, K, V, codes, rc, seq_lens, R, topk
     idx, cnt = select(ss, seq_lens, topk, sink, window)
     out, lse = attend(layout, Hq, q, K, V, idx, cnt)
     return dict(scores=ss, unscaled=sc, bound=bound, sel_idx=idx, sel_cnt=cnt, out=out, lse=lse)
+
+
+# ---------------------------------------------------------------- precision tiers
+# Tier-homogeneous pages (Spherical KV page, section 2.2 RDR; DASH-KV page,
+# section "技术架构：动态混合精度机制"): pages whose tokens all lie between the
+# sinks and the window are demoted to FP8 E4M3 rows with a power-of-two scale
+# per (token, kv head) row; attention reads those rows dequantized.  The C
+# file's section on precision tiers has the exact definitions.
+
+def e4m3_value(c: int) -> float:
+    """Value of an FP8 E4M3 (FN) code (NaN for the two NaN codes)."""
+    return float(lib().dko_e4m3_value(int(c) & 0xFF))
+
+
+def e4m3_encode(v: float) -> int:
+    """Nearest E4M3 code of v, ties to even (|v| <= 448)."""
+    return int(lib().dko_e4m3_encode(float(v)))
+
+
+def tier_exponent(x) -> int:
+    """s = the largest integer with max|x| * 2^s <= 448, capped at 127 (0 for a zero row)."""
+    x = _f64(x)
+    return int(lib().dko_tier_exponent(_p(x), int(x.shape[-1])))
+
+
+def tier_quantize_row(x):
+    """(codes uint8 [d], s) of one row."""
+    x = _f64(x)
+    codes = np.empty(x.shape[-1], dtype=np.uint8)
+    s = np.zeros(1, dtype=np.int8)
+    lib().dko_tier_quantize_row(_p(x), int(x.shape[-1]), _p(codes), _p(s))
+    return codes, int(s[0])
+
+
+def tier_arrays(num_pages: int, page: int, Hkv: int, d: int):
+    """Zeroed (tier [P], k8 [P,page,Hkv,d], v8, exps [P,page,Hkv,2]) arrays."""
+    return (np.zeros(num_pages, dtype=np.uint8), np.zeros((num_pages, page, Hkv, d), dtype=np.uint8),
+            np.zeros((num_pages, page, Hkv, d), dtype=np.uint8), np.zeros((num_pages, page, Hkv, 2), dtype=np.int8))
+
+
+def demote_pages(layout: Layout, K, V, seq_lens, sink: int, window: int, tier, k8, v8, exps, protect=None) -> int:
+    """The page controller on a paged layout; updates tier / k8 / v8 / exps in
+    place and returns the number of pages demoted."""
+    assert layout.page > 0, "tiers are defined on paged layouts"
+    for a, dt in ((tier, np.uint8), (k8, np.uint8), (v8, np.uint8), (exps, np.int8)):
+        assert a.dtype == dt and a.flags.c_contiguous
+    pr = None if protect is None else np.ascontiguousarray(protect, dtype=np.uint8)
+    return int(lib().dko_demote_pages(layout.B, layout.Hkv, layout.d, layout.page, _p(layout.page_table),
+                                      layout.max_pages, _p(_f64(K)), _p(_f64(V)), _p(_i32(seq_lens)), int(sink),
+                                      int(window), _p(pr), _p(tier), _p(k8), _p(v8), _p(exps)))
+
+
+def e4m3_table() -> np.ndarray:
+    """Values of all 256 codes (float64)."""
+    return np.array([e4m3_value(c) for c in range(256)])
+
+
+def dequantized(K, V, tier, k8, v8, exps):
+    """K / V as attention reads them: rows of tier-1 pages replaced by
+    value(c) * 2^-s, the others unchanged (paged layout, float64)."""
+    K = _f64(K).copy()
+    V = _f64(V).copy()
+    tab = e4m3_table()
+    for p in np.nonzero(np.asarray(tier) == 1)[0]:
+        K[p] = tab[k8[p]] * np.ldexp(1.0, -exps[p][..., 0:1].astype(np.int64))
+        V[p] = tab[v8[p]] * np.ldexp(1.0, -exps[p][..., 1:2].astype(np.int64))
+    return K, V
+
+
+def attend_tiered(layout: Layout, Hq, q, K, V, tier, k8, v8, exps, sel_idx, sel_cnt):
+    """Exact attention over the selection with tier-1 rows dequantized."""
+    Kd, Vd = dequantized(K, V, tier, k8, v8, exps)
+    return attend(layout, Hq, q, Kd, Vd, sel_idx, sel_cnt)
