@@ -227,7 +227,9 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
     sequence's cache.  Appends (and the summary of a block an append completes)
     are untimed too."""
     from oracle import oracle as O
-    one = cfg.scaled(B=1, steps=n_steps + 1)
+    # one sequence of the workload's longest length, dense (a paged workload's
+    # page permutation changes nothing in the oracle's arithmetic)
+    one = cfg.scaled(B=1, steps=n_steps + 1, page_size=0, n_min=0)
     w = W.make_workload(one, device="cpu", steps=n_steps + 1)
     R = O.hyperplanes(W.HYPERPLANE_SEED, cfg.bits, cfg.d)
     L = O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=w.n_cap)
@@ -244,16 +246,36 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
         O.append(L, K, V, codes, seq, w.k_new[s].double().numpy(), w.v_new[s].double().numpy(), R)
         if m:
             oracle_block_update(L, K, bcodes, int(seq[0]), m, R)
+        if cfg.tiers:  # the appended row into the paged copy too (its page is in the window: bf16)
+            t = int(seq[0]) - 1
+            Kp[t // cfg.page_size, t % cfg.page_size] = K[0, :, t]
+            Vp[t // cfg.page_size, t % cfg.page_size] = V[0, :, t]
         if cfg.radius:  # the appended token's radius code
             n = int(seq[0])
             rc[:, :, n - 1] = O.radius_codes(O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, n_cap=1),
                                              np.ascontiguousarray(K[:, :, n - 1:n]), np.array([1], np.int32))[:, :, 0]
 
     rc = O.radius_codes(L, K, seq) if cfg.radius else None
+    if cfg.tiers:  # the same sequence as a paged cache, its middle pages demoted (untimed)
+        ps = cfg.page_size
+        npg = (w.n_cap + ps - 1) // ps
+        Lp = O.Layout(1, cfg.Hkv, cfg.d, cfg.bits, page_table=np.arange(npg, dtype=np.int32).reshape(1, npg), page=ps)
+        Kp = np.zeros((npg * ps, cfg.Hkv, cfg.d))
+        Vp = np.zeros((npg * ps, cfg.Hkv, cfg.d))
+        Kp[:w.n_cap] = K[0].transpose(1, 0, 2)
+        Vp[:w.n_cap] = V[0].transpose(1, 0, 2)
+        Kp = Kp.reshape(npg, ps, cfg.Hkv, cfg.d)
+        Vp = Vp.reshape(npg, ps, cfg.Hkv, cfg.d)
+        tarr = O.tier_arrays(npg, ps, cfg.Hkv, cfg.d)
+        O.demote_pages(Lp, Kp, Vp, seq, cfg.sink, cfg.window, *tarr)
 
     def decode(s):
         q = w.q[s].double().numpy()
-        if cfg.radius:
+        if cfg.tiers:
+            sc, _ = O.scores(L, cfg.Hq, q, codes, seq, R)
+            idx, cnt = O.select(sc, seq, cfg.topk, cfg.sink, cfg.window)
+            O.attend_tiered(Lp, cfg.Hq, q, Kp, Vp, *tarr, idx, cnt)
+        elif cfg.radius:
             O.decode_step_radius(L, cfg.Hq, q, K, V, codes, rc, seq, R, cfg.topk, cfg.sink, cfg.window)
         elif m:
             O.decode_step_blocks(L, cfg.Hq, q, K, V, bcodes, seq, R, m, cfg.topk // m, cfg.sink, cfg.window,
@@ -276,6 +298,8 @@ def oracle_sample(cfg: W.Config, n_steps: int, seq_index: int = 0) -> dict:
     one_thread_s = time.perf_counter() - t0
     O.set_threads(cores)
     how = f", blocks of {m}" if m else (", radius-scaled scores" if cfg.radius else "")
+    if cfg.tiers:
+        how = ", middle pages as FP8 rows (attention reads them dequantized; appended rows stay bf16)"
     return dict(times=times, cores=cores, one_thread_s=one_thread_s,
                 sample=f"sequence {seq_index} of {cfg.B} (N={cfg.N}, all {cfg.Hkv} KV / {cfg.Hq} query heads{how}), "
                        f"{n_steps} decode steps, oracle encode untimed")
@@ -333,6 +357,26 @@ def run_dashkv(args, cfg, world, rank, local):
     if cfg.radius:  # radius codes of the prefilled cache (untimed)
         radius = dk.KVCache.empty_radius_like(w.K, w.paged)
         eng.encode_radius(cache, radius, seq)
+    tiers = demote = None
+    if cfg.tiers:  # the controller over the prefilled cache: middle pages to FP8 rows
+        tiers = dk.PageTiers.empty_for(cache)
+        eng.demote_pages(cache, tiers, seq)  # (loads the kernel; repeated below, timed)
+        torch.cuda.synchronize(dev)
+        tiers.tier.zero_()
+        flush(0)
+        e_dem = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e_dem[0].record(stream)
+        eng.demote_pages(cache, tiers, seq)
+        e_dem[1].record(stream)
+        torch.cuda.synchronize(dev)
+        n_pages = int(tiers.tier.sum())
+        rows = n_pages * cfg.page_size * cfg.Hkv
+        dem_ms = e_dem[0].elapsed_time(e_dem[1])
+        demote = {"ms": dem_ms, "pages": n_pages, "of_pages": int(tiers.tier.numel()),
+                  "bytes": rows * (2 * cfg.d * 2 + 2 * cfg.d + 2),
+                  "gbs": rows * (2 * cfg.d * 2 + 2 * cfg.d + 2) / (dem_ms * 1e-3) / 1e9,
+                  "timing": "one full controller pass over the prefilled cache, L2 flushed before it; a decode loop "
+                            "runs it again when a page leaves the window (once per page of steps)"}
     torch.cuda.synchronize(dev)
     assert eng.get_error() == 0
     # the prefill encode, timed on its own (a second, identical call: cold L2, kernel already loaded)
@@ -368,7 +412,7 @@ def run_dashkv(args, cfg, world, rank, local):
     # for token selection on the clustered path; otherwise the separate calls
     # (append, select, sparse decode), captured into one graph with
     # programmatic dependent launches between them
-    fused = args.path == "step" and not (cfg.block or cfg.radius or n_sel_kernels != 1)
+    fused = args.path == "step" and not (cfg.block or cfg.radius or cfg.tiers or n_sel_kernels != 1)
     # the kernels of one step, in launch order, and the calls that launch them
     if fused:
         calls = [("decode_step", ["decode_step"])]
@@ -382,7 +426,7 @@ def run_dashkv(args, cfg, world, rank, local):
             calls += [("append_radius", ["append_radius"]), ("select_radius", sel_names)]
         else:
             calls += [("select", sel_names)]
-        calls += [("sparse_decode", ["sparse_decode"])]
+        calls += [("sparse_decode_tiered" if cfg.tiers else "sparse_decode", ["sparse_decode"])]
     kernels = [k for _, ks in calls for k in ks]
     n_graph = args.warmup + K + T
 
@@ -406,6 +450,8 @@ def run_dashkv(args, cfg, world, rank, local):
                 eng.select_radius(cache, radius, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
             elif name == "select":
                 eng.select(cache, q, seq, buf["sel_idx"], buf["sel_cnt"], None, ws)
+            elif name == "sparse_decode_tiered":
+                eng.sparse_decode_tiered(cache, tiers, q, buf["sel_idx"], buf["sel_cnt"], out, lse, ws, seq_lens=seq)
             else:
                 eng.sparse_decode(cache, q, buf["sel_idx"], buf["sel_cnt"], out, lse, ws, seq_lens=seq)
             j += len(ks)
@@ -481,6 +527,13 @@ def run_dashkv(args, cfg, world, rank, local):
     code_bytes = float(scanned.sum()) * cfg.Hkv * cfg.bits / 8
     sel_rows = float(buf["sel_cnt"].sum())
     kv_bytes = sel_rows * 2 * cfg.d * 2
+    fp8_rows = None
+    if tiers is not None:  # rows of FP8 pages: 2 d code bytes + 2 exponents; every row: its page's tier byte
+        idx = buf["sel_idx"].long()
+        valid = torch.arange(idx.shape[-1], device=dev)[None, None, :] < buf["sel_cnt"][..., None]
+        phys = w.page_table.long()[torch.arange(cfg.B, device=dev)[:, None, None], idx.clamp(min=0) // cfg.page_size]
+        fp8_rows = float(((tiers.tier.long()[phys] == 1) & valid).sum())
+        kv_bytes = (sel_rows - fp8_rows) * 2 * cfg.d * 2 + fp8_rows * (2 * cfg.d + 2) + sel_rows
     qo_bytes = cfg.B * cfg.Hq * cfg.d * (2 + 4)
     step_bytes = code_bytes + kv_bytes + qo_bytes
     peaks = measured_peaks()
@@ -561,6 +614,7 @@ def run_dashkv(args, cfg, world, rank, local):
             "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
                        "bits": cfg.bits, "topk": cfg.topk, "sink": cfg.sink, "window": cfg.window,
                        "block": cfg.block or None, "radius": cfg.radius or None,
+                       "tiers": "pages between the sinks and the window as FP8 E4M3 rows" if cfg.tiers else None,
                        "layout": "paged" if w.paged else "dense", "l2": "flushed before every step: 2 x L2 write, then 2 x L2 clean read (no pending write-backs)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs,
@@ -576,6 +630,8 @@ def run_dashkv(args, cfg, world, rank, local):
             "per_head_queries_per_s": value * cfg.Hq,
             "warm_ms_per_step": warm_ms,
             "encode": encode,
+            "demote": demote,
+            "fp8_selected_rows": fp8_rows,
             "codes_scanned_per_s": float(scanned.sum()) * cfg.Hkv / (ms_per_step * 1e-3),
             "selected_kv_bytes_per_s": kv_bytes / (ms_per_step * 1e-3),
             "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": len(kernels) * K, "clocks": clk,

@@ -19,6 +19,7 @@
 #include "radius.cuh"
 #include "select.cuh"
 #include "step_args.cuh"
+#include "tiers.cuh"
 
 namespace dkv {
 __device__ unsigned g_error_word;  // the device error word (declared in common.cuh)
@@ -331,7 +332,9 @@ void set_attrs_bd() {
 
 template <int D, int G>
 void set_attr_decode() {
-    cudaFuncSetAttribute(sparse_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(sparse_decode_kernel<D, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)DecodeShape<D, G>::SMEM);
+    cudaFuncSetAttribute(sparse_decode_kernel<D, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)DecodeShape<D, G>::SMEM);
 }
 
@@ -543,26 +546,29 @@ int window_ctas(const dashkv_ctx *ctx, int64_t cap, const int32_t *seq_lens, int
 template <int D, int G>
 void launch_decode_dg(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *si, const int32_t *sc,
                       float *out, float *lse, const AttnWS &ws, const int32_t *seq_lens, int64_t cap,
-                      cudaStream_t st) {
+                      const Tiers *tiers, cudaStream_t st) {
     const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
     const int splits = attn_splits(ctx);
     const int nw = window_ctas(ctx, cap, seq_lens, splits);
     const int wy = (BH * nw + splits - 1) / splits;  // grid rows of window CTAs
     const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    launch_pdl(sparse_decode_kernel<D, G>, dim3(splits, BH + wy), dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st,
-               kv, static_cast<const __nv_bfloat16 *>(q), ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws,
-               splits, scale_log2, seq_lens, ctx->cfg.sink, ctx->cfg.window, ctx->cfg.topk, wy, nw > 0 ? nw : 1);
+    const Tiers tr = tiers ? *tiers : Tiers{};
+    launch_pdl(tiers ? sparse_decode_kernel<D, G, true> : sparse_decode_kernel<D, G, false>, dim3(splits, BH + wy),
+               dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st, kv, static_cast<const __nv_bfloat16 *>(q),
+               ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws, splits, scale_log2, seq_lens, ctx->cfg.sink,
+               ctx->cfg.window, ctx->cfg.topk, wy, nw > 0 ? nw : 1, tr);
 }
 
 template <int D>
 void launch_decode_d(const dashkv_ctx *ctx, const KV &kv, const void *q, const int32_t *si, const int32_t *sc,
-                     float *out, float *lse, const AttnWS &ws, const int32_t *seq, int64_t cap, cudaStream_t st) {
+                     float *out, float *lse, const AttnWS &ws, const int32_t *seq, int64_t cap, const Tiers *tiers,
+                     cudaStream_t st) {
     switch (ctx->cfg.num_q_heads / ctx->cfg.num_kv_heads) {
-        case 1: launch_decode_dg<D, 1>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
-        case 2: launch_decode_dg<D, 2>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
-        case 4: launch_decode_dg<D, 4>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
-        default: launch_decode_dg<D, 8>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, st); break;
+        case 1: launch_decode_dg<D, 1>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, tiers, st); break;
+        case 2: launch_decode_dg<D, 2>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, tiers, st); break;
+        case 4: launch_decode_dg<D, 4>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, tiers, st); break;
+        default: launch_decode_dg<D, 8>(ctx, kv, q, si, sc, out, lse, ws, seq, cap, tiers, st); break;
     }
 }
 
@@ -775,6 +781,51 @@ void static_scratch_forget(int dev) {
     StaticScratch &s = g_static[dev];
     s.hist_off = s.hist_bytes = s.arrive_off = s.arrive_bytes = 0;
 }
+
+// Tier view of a paged cache (tiers.cuh): all four arrays, FP8 rows 16-byte aligned.
+dashkv_status check_tiers(const dashkv_ctx *ctx, const dashkv_tier_view *tv) {
+    if (!tv || !tv->tier || !tv->k8 || !tv->v8 || !tv->exps) return DASHKV_ERR_INVALID_ARG;
+    if (!ctx->cfg.page_size) return DASHKV_ERR_UNSUPPORTED;  // tiers are per page
+    if (!aligned(tv->k8, 16) || !aligned(tv->v8, 16) || !aligned(tv->exps, 2)) return DASHKV_ERR_INVALID_ARG;
+    return DASHKV_OK;
+}
+
+Tiers make_tiers(const dashkv_tier_view *tv) {
+    Tiers t;
+    t.tier = tv->tier;
+    t.k8 = tv->k8;
+    t.v8 = tv->v8;
+    t.exps = tv->exps;
+    return t;
+}
+
+// dashkv_sparse_decode, with FP8 rows for the tier-1 pages when `tiers` is set.
+dashkv_status run_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, const Tiers *tiers, const void *q,
+                         const int32_t *seq_lens, const int32_t *sel_idx, const int32_t *sel_cnt, float *out,
+                         float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!ctx || !q || !sel_idx || !sel_cnt || !out || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
+    dashkv_status s = check_view(ctx, kv, true, false);
+    if (s != DASHKV_OK) return s;
+    const WsLayout L = ws_layout(ctx->cfg, view_capacity(ctx, kv));
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
+    char *w = static_cast<char *>(workspace);
+    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
+    AttnWS ws;
+    ws.part = reinterpret_cast<float *>(w + L.part);
+    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive) + 2 * BH * kSyncStride;
+    const KV k = make_kv(ctx, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Tracer tr(ctx, st);
+    tr.before();
+    const int64_t cap = view_capacity(ctx, kv);
+    if (ctx->cfg.head_dim == 64)
+        launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, tiers, st);
+    else
+        launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, tiers, st);
+    tr.after();
+    return launch_status();
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -928,25 +979,41 @@ dashkv_status dashkv_sparse_decode(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    const int32_t *seq_lens, const int32_t *sel_idx, const int32_t *sel_cnt,
                                    float *out, float *lse, void *workspace, size_t workspace_bytes,
                                    void *stream) {
-    if (!ctx || !q || !sel_idx || !sel_cnt || !out || !aligned(q, 16)) return DASHKV_ERR_INVALID_ARG;
+    return run_decode(ctx, kv, nullptr, q, seq_lens, sel_idx, sel_cnt, out, lse, workspace, workspace_bytes,
+                      stream);
+}
+
+dashkv_status dashkv_demote_pages(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_tier_view *tv,
+                                  const int32_t *seq_lens, const uint8_t *protect, void *stream) {
+    if (!ctx || !seq_lens) return DASHKV_ERR_INVALID_ARG;
     dashkv_status s = check_view(ctx, kv, true, false);
+    if (s == DASHKV_OK) s = check_tiers(ctx, tv);
     if (s != DASHKV_OK) return s;
-    const WsLayout L = ws_layout(ctx->cfg, view_capacity(ctx, kv));
-    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return DASHKV_ERR_WORKSPACE;
-    char *w = static_cast<char *>(workspace);
-    const int BH = ctx->cfg.batch * ctx->cfg.num_kv_heads;
-    AttnWS ws;
-    ws.part = reinterpret_cast<float *>(w + L.part);
-    ws.arrive = reinterpret_cast<uint32_t *>(w + L.arrive) + 2 * BH * kSyncStride;
     const KV k = make_kv(ctx, kv);
+    const Tiers tr = make_tiers(tv);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    Tracer tr(ctx, st);
-    tr.before();
-    const int64_t cap = view_capacity(ctx, kv);
-    if (ctx->cfg.head_dim == 64) launch_decode_d<64>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
-    else launch_decode_d<128>(ctx, k, q, sel_idx, sel_cnt, out, lse, ws, seq_lens, cap, st);
-    tr.after();
+    Tracer trc(ctx, st);
+    trc.before();
+    const dim3 grid((unsigned)kv->max_pages, (unsigned)ctx->cfg.batch);
+    if (ctx->cfg.head_dim == 64)
+        demote_pages_kernel<64><<<grid, kDemoteThreads, 0, st>>>(k, tr, protect, seq_lens, ctx->cfg.sink,
+                                                                 ctx->cfg.window);
+    else
+        demote_pages_kernel<128><<<grid, kDemoteThreads, 0, st>>>(k, tr, protect, seq_lens, ctx->cfg.sink,
+                                                                  ctx->cfg.window);
+    trc.after();
     return launch_status();
+}
+
+dashkv_status dashkv_sparse_decode_tiered(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_tier_view *tv,
+                                          const void *q, const int32_t *seq_lens, const int32_t *sel_idx,
+                                          const int32_t *sel_cnt, float *out, float *lse, void *workspace,
+                                          size_t workspace_bytes, void *stream) {
+    if (!ctx) return DASHKV_ERR_INVALID_ARG;
+    const dashkv_status s = check_tiers(ctx, tv);
+    if (s != DASHKV_OK) return s;
+    const Tiers tr = make_tiers(tv);
+    return run_decode(ctx, kv, &tr, q, seq_lens, sel_idx, sel_cnt, out, lse, workspace, workspace_bytes, stream);
 }
 
 dashkv_status dashkv_decode_step(dashkv_ctx *ctx, const dashkv_kv_view *kv, const void *q, const void *k_new,

@@ -17,8 +17,15 @@
 // lane groups' states in shared memory and writes one partial; the last CTA of
 // the (b, h) to arrive (atomic counter, no waiting) merges the partials with a
 // log-sum-exp reduction and writes out / lse.
+//
+// TIERED: rows of tier-1 pages (see tiers.cuh) are gathered as their FP8 K and
+// V rows (128 + 128 bytes at d = 128 instead of 256 + 256) into the first half
+// of the same staging slots, and read back as value(code) * 2^-s; the owner
+// lane of a tile row loads its page's tier byte and the row's two exponents
+// with the token id, one tile ahead.
 #pragma once
 #include "common.cuh"
+#include "tiers.cuh"
 
 namespace dkv {
 
@@ -69,12 +76,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-template <int D, int G>
+template <int D, int G, bool TIERED = false>
 __global__ void __launch_bounds__(kAttnThreads, 2)
 sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
                      const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt, int cap_sel,
                      float *__restrict__ out, float *__restrict__ lse, AttnWS ws, int splits, float scale_log2,
-                     const int32_t *__restrict__ seq_lens, int n_sink, int n_window, int topk, int wy, int nw) {
+                     const int32_t *__restrict__ seq_lens, int n_sink, int n_window, int topk, int wy, int nw,
+                     Tiers tiers) {
     using S = DecodeShape<D, G>;
     constexpr int DPL = S::DPL, LPR = S::LPR, RPW = S::RPW, NST = S::NST, RT = S::RT;
     constexpr int TROWS = S::TROWS, CPR = S::CPR, NWARP = S::NWARP, STAGES = S::STAGES, V = S::V;
@@ -184,16 +192,31 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
         if (kv.page_size && kv.page_of(b, t) < 0) return -1;
         return t;
     };
+    // Tier of the row of token t (from tile_token: -1 or a valid token) --
+    // 1 | s_K << 8 | s_V << 16 for an FP8 row, 0 otherwise.
+    auto tile_meta = [&](int t) -> uint32_t {
+        if constexpr (!TIERED) {
+            return 0u;
+        } else {
+            if (t < 0) return 0u;
+            const int64_t p = kv.page_of(b, t);
+            const int64_t row = (p * kv.page_size + t % kv.page_size) * kv.Hkv + h;
+            const uint32_t tr = __ldg(tiers.tier + p);
+            const uint32_t e2 = __ldg(reinterpret_cast<const unsigned short *>(tiers.exps) + row);
+            return tr ? 1u | (e2 << 8) : 0u;
+        }
+    };
     // Gather a tile's K and V rows into buffer `buf` (zero-filled when invalid);
     // tok: this lane's tile_token() of the tile.
     // Lane l copies row l / LPT of the tile: chunks l % LPT, l % LPT + LPT, ...
     // of its K and V rows (so each lane computes one row address per tile).
     constexpr int LPT = 32 / TROWS;               // lanes per tile row
     constexpr int CPL = 2 * CPR / LPT;            // 16-byte chunks per lane (K then V)
-    auto prefetch = [&](int tok, int buf) {
+    auto prefetch = [&](int tok, uint32_t meta, int buf) {
         __nv_bfloat16 *dst0 = wstage + (size_t)buf * TROWS * 2 * D;
         const int j = lane / LPT, c0 = lane % LPT;
         const int t = __shfl_sync(0xffffffffu, tok, j);
+        const bool f8 = TIERED && (__shfl_sync(0xffffffffu, meta, j) & 1u);
         const int64_t off = t >= 0 ? kv.row(b, h, t) : 0;
         const int nbytes = t >= 0 ? 16 : 0;
         __nv_bfloat16 *dst = dst0 + (size_t)j * 2 * D;
@@ -202,8 +225,14 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             const int c = c0 + m * LPT;       // chunk of the (K, V) pair of rows
             const bool isv = c >= CPR;        // compile-time per m when LPT divides CPR
             const int cc = isv ? c - CPR : c;
-            const __nv_bfloat16 *src = (isv ? kv.v : kv.k) + off + cc * 8;
-            cp_async16(dst + (isv ? D : 0) + cc * 8, src, nbytes);
+            if (TIERED && f8) {  // the FP8 row: its CPR / 2 chunks into the slot's first half
+                const bool in = cc < CPR / 2 && t >= 0;
+                const uint8_t *src = in ? (isv ? tiers.v8 : tiers.k8) + off + cc * 16 : tiers.k8;
+                cp_async16(dst + (isv ? D : 0) + cc * 8, src, in ? 16 : 0);
+            } else {
+                const __nv_bfloat16 *src = (isv ? kv.v : kv.k) + off + cc * 8;
+                cp_async16(dst + (isv ? D : 0) + cc * 8, src, nbytes);
+            }
         }
         cp_async_commit();
     };
@@ -211,12 +240,16 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
     constexpr int WSTEP = NWARP * TROWS;  // rows per CTA tile round
     int base = r0 + warp * TROWS;
     int tok[STAGES];
+    uint32_t meta[STAGES];
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) meta[s] = 0u;
 #pragma unroll
     for (int s = 0; s < STAGES - 1; ++s) {
         tok[s] = -1;
         if (base + s * WSTEP < r1) {
             tok[s] = tile_token(base + s * WSTEP);
-            prefetch(tok[s], s);
+            meta[s] = tile_meta(tok[s]);
+            prefetch(tok[s], meta[s], s);
         } else {
             cp_async_commit();
         }
@@ -227,7 +260,8 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
         const int abuf = (k + STAGES - 1) % STAGES;
         if (ahead < r1) {
             tok[abuf] = tile_token(ahead);
-            prefetch(tok[abuf], abuf);
+            meta[abuf] = tile_meta(tok[abuf]);
+            prefetch(tok[abuf], meta[abuf], abuf);
         } else {
             cp_async_commit();
         }
@@ -242,7 +276,11 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             const int jr = (j ^ jperm) * RPW + sub;  // row within the tile
             const __nv_bfloat16 *kr = tile + (size_t)jr * 2 * D + li * DPL;
             float kf[DPL];
-            if constexpr (DPL >= 8) {
+            const uint32_t mk = TIERED ? __shfl_sync(0xffffffffu, meta[buf], jr) : 0u;
+            if (TIERED && (mk & 1u)) {
+                e4m3_row<DPL>(reinterpret_cast<const uint8_t *>(tile + (size_t)jr * 2 * D) + li * DPL,
+                              pow2_neg((int)(int8_t)(mk >> 8)), kf);
+            } else if constexpr (DPL >= 8) {
 #pragma unroll
                 for (int e = 0; e < DPL; e += 8) {
                     const uint4 w = *reinterpret_cast<const uint4 *>(kr + e);
@@ -300,7 +338,11 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             const int jr = j * RPW + sub;
             const __nv_bfloat16 *vrow = tile + ((size_t)jr * 2 + 1) * D + li * DPL;
             float vf[DPL];
-            if constexpr (DPL >= 8) {
+            const uint32_t mv = TIERED ? __shfl_sync(0xffffffffu, meta[buf], jr) : 0u;
+            if (TIERED && (mv & 1u)) {
+                e4m3_row<DPL>(reinterpret_cast<const uint8_t *>(tile + ((size_t)jr * 2 + 1) * D) + li * DPL,
+                              pow2_neg((int)(int8_t)(mv >> 16)), vf);
+            } else if constexpr (DPL >= 8) {
 #pragma unroll
                 for (int e = 0; e < DPL; e += 8) {
                     const uint4 w = *reinterpret_cast<const uint4 *>(vrow + e);

@@ -29,7 +29,8 @@ SYMBOLS = ("dashkv_create", "dashkv_destroy", "dashkv_workspace_size", "dashkv_e
            "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_get_error",
            "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_kernels", "dashkv_status_str",
            "dashkv_select_static", "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks",
-           "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius", "dashkv_decode_step")
+           "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius", "dashkv_decode_step",
+           "dashkv_demote_pages", "dashkv_sparse_decode_tiered")
 
 
 class DashKVError(RuntimeError):
@@ -49,6 +50,11 @@ class KVView(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("n_cap", ctypes.c_int64), ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32)]
+
+
+class TierView(ctypes.Structure):
+    _fields_ = [("tier", ctypes.c_void_p), ("k8", ctypes.c_void_p), ("v8", ctypes.c_void_p),
+                ("exps", ctypes.c_void_p)]
 
 
 class BlockView(ctypes.Structure):
@@ -86,6 +92,9 @@ def lib() -> ctypes.CDLL:
         L.dashkv_encode_radius.argtypes = [P, ctypes.POINTER(KVView), P, P, P]
         L.dashkv_append_radius.argtypes = [P, ctypes.POINTER(KVView), P, P, P]
         L.dashkv_select_radius.argtypes = [P, ctypes.POINTER(KVView), P, P, P, P, P, P, P, SZ, P]
+        L.dashkv_demote_pages.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(TierView), P, P, P]
+        L.dashkv_sparse_decode_tiered.argtypes = [P, ctypes.POINTER(KVView), ctypes.POINTER(TierView), P, P, P, P,
+                                                  P, P, P, SZ, P]
         L.dashkv_get_error.argtypes = [P]
         L.dashkv_hyperplanes.argtypes = [U64, I32, I32, P]
         L.dashkv_set_trace.argtypes = [P, P, I32]
@@ -96,7 +105,8 @@ def lib() -> ctypes.CDLL:
         for f in ("dashkv_encode_keys", "dashkv_append_keys", "dashkv_select", "dashkv_sparse_decode", "dashkv_decode_step",
                   "dashkv_get_error", "dashkv_hyperplanes", "dashkv_set_trace", "dashkv_select_static",
                   "dashkv_encode_blocks", "dashkv_append_blocks", "dashkv_select_blocks",
-                  "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius", "dashkv_decode_step"):
+                  "dashkv_encode_radius", "dashkv_append_radius", "dashkv_select_radius", "dashkv_decode_step",
+           "dashkv_demote_pages", "dashkv_sparse_decode_tiered"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -216,6 +226,32 @@ class BlockIndex:
         return BlockIndex(torch.zeros((batch, Hkv, nb_cap, W), dtype=torch.int64, device=cache.k.device), int(block))
 
 
+@dataclasses.dataclass
+class PageTiers:
+    """Precision tiers of a paged cache's pages: tier [P] uint8 (0 = bf16
+    rows, 1 = FP8 rows), k8 / v8 [P, page, Hkv, d] uint8 (FP8 E4M3 codes) and
+    exps [P, page, Hkv, 2] int8 (the rows' power-of-two scale exponents)."""
+    tier: torch.Tensor
+    k8: torch.Tensor
+    v8: torch.Tensor
+    exps: torch.Tensor
+
+    def view(self) -> TierView:
+        return TierView(self.tier.data_ptr(), self.k8.data_ptr(), self.v8.data_ptr(), self.exps.data_ptr())
+
+    @staticmethod
+    def empty_for(cache: "KVCache") -> "PageTiers":
+        """Every page tier 0 (zeroed arrays shaped like the cache's pages)."""
+        if not cache.paged:
+            raise ValueError("precision tiers are defined on paged caches")
+        P, page, Hkv, d = cache.k.shape
+        dev = cache.k.device
+        return PageTiers(torch.zeros(P, dtype=torch.uint8, device=dev),
+                         torch.zeros((P, page, Hkv, d), dtype=torch.uint8, device=dev),
+                         torch.zeros((P, page, Hkv, d), dtype=torch.uint8, device=dev),
+                         torch.zeros((P, page, Hkv, 2), dtype=torch.int8, device=dev))
+
+
 class DashKV:
     """One problem configuration (shapes, bits, k, S, W, layout, seed)."""
 
@@ -299,6 +335,26 @@ class DashKV:
                                                                   _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt),
                                                                   _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                                                   _stream(stream)))
+
+    def demote_pages(self, cache: KVCache, tiers: PageTiers, seq_lens: torch.Tensor,
+                     protect: Optional[torch.Tensor] = None, stream=None) -> None:
+        """Move every page that holds no sink and no window token (and is not
+        protected) to the FP8 tier."""
+        v, t = cache.view(), tiers.view()
+        _check("dashkv_demote_pages", lib().dashkv_demote_pages(self._ctx, ctypes.byref(v), ctypes.byref(t),
+                                                                _ptr(seq_lens), _ptr(protect), _stream(stream)))
+
+    def sparse_decode_tiered(self, cache: KVCache, tiers: PageTiers, q: torch.Tensor, sel_idx: torch.Tensor,
+                             sel_cnt: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None,
+                             seq_lens: Optional[torch.Tensor] = None) -> None:
+        """sparse_decode with the rows of FP8-tier pages read from `tiers`."""
+        ws = workspace if workspace is not None else self.workspace(cache.capacity, q.device)
+        v, t = cache.view(), tiers.view()
+        _check("dashkv_sparse_decode_tiered",
+               lib().dashkv_sparse_decode_tiered(self._ctx, ctypes.byref(v), ctypes.byref(t), _ptr(q),
+                                                 _ptr(seq_lens), _ptr(sel_idx), _ptr(sel_cnt), _ptr(out), _ptr(lse),
+                                                 _ptr(ws), ws.numel(), _stream(stream)))
 
     def decode_step(self, cache: KVCache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                     seq_lens: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor, out: torch.Tensor,

@@ -53,6 +53,7 @@ class Config:
     seed: int = 1234
     block: int = 0         # > 0: select through summaries of blocks of this many tokens
     radius: bool = False   # select on radius-scaled scores (8-bit key-norm codes)
+    tiers: bool = False    # paged: pages between the sinks and the window held as FP8 rows
 
     @property
     def G(self) -> int:
@@ -85,6 +86,9 @@ CONFIGS["c128k_blocks4"] = CONFIGS["c128k"].scaled(name="c128k_blocks4", block=4
 CONFIGS["c1m_blocks4"] = CONFIGS["c1m"].scaled(name="c1m_blocks4", block=4)
 # the 128K workload selected on radius-scaled scores
 CONFIGS["c128k_radius"] = CONFIGS["c128k"].scaled(name="c128k_radius", radius=True)
+# the ragged paged workload with every page between the sinks and the window
+# demoted to FP8 rows (the pages' mixed-precision KV store)
+CONFIGS["ragged_paged_fp8"] = CONFIGS["ragged_paged"].scaled(name="ragged_paged_fp8", tiers=True)
 # the 1M-token workload's shape at half the length: a case small enough for
 # multi-pass profiler captures of the same kernels
 CONFIGS["c512k"] = CONFIGS["c1m"].scaled(name="c512k", N=524288)

@@ -310,6 +310,51 @@ dashkv_status dashkv_select_radius(dashkv_ctx *ctx, const dashkv_kv_view *kv, co
                                    const int32_t *seq_lens, int32_t *sel_idx, int32_t *sel_cnt, float *scores,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Precision tiers of pages (paged caches only).
+ *
+ * Spherical KV page, section 2.2 RDR: every retained state gets a precision
+ * tier, protected states keep the highest one, and states are grouped into
+ * pages of a single tier so that the decode reads each page in one pass
+ * guided by its header.  DASH-KV page, section "技术架构：动态混合精度机制",
+ * paras 2-3: the tokens that matter keep full floating-point precision, the
+ * others a cheaper form.
+ *
+ * Tier 0: the bf16 rows of kv->k / kv->v.  Tier 1: FP8 E4M3 (OCP "FN"
+ * encoding) rows with one power-of-two scale per (token, kv head) row and
+ * tensor: s = the largest integer with max_i |x_i| * 2^s <= 448, capped at
+ * 127 (0 for a zero row); code_i = E4M3(x_i * 2^s), nearest, ties to even;
+ * the row reads back as value(code_i) * 2^-s (exact in fp32).  The page
+ * header is one tier byte per physical page.
+ * ------------------------------------------------------------------------ */
+typedef struct dashkv_tier_view {
+    uint8_t *tier;  /* device u8 [num_pages]: 0 = bf16 rows, 1 = FP8 rows.  The caller
+                       zero-fills it once and zeroes the byte of a page it reassigns */
+    uint8_t *k8;    /* device u8 [num_pages][page][Hkv][d] FP8 keys (16-byte aligned) */
+    uint8_t *v8;    /* device u8 [num_pages][page][Hkv][d] FP8 values (16-byte aligned) */
+    int8_t *exps;   /* device i8 [num_pages][page][Hkv][2]: s of the K row, then of the V row */
+} dashkv_tier_view;
+
+/* The tier controller.  For every sequence b and logical page p whose tokens
+ * [p page, (p + 1) page) all lie in [S, seq_lens[b] - W) -- no sink, no window
+ * token -- and whose physical page is still tier 0 and not protected
+ * (protect: optional device u8 [num_pages], nonzero = keep bf16), the page's K
+ * and V rows of every kv head are quantized into tv->k8 / tv->v8 / tv->exps
+ * and its tier byte is set to 1.  Pages already tier 1 are left alone (their
+ * rows must not change afterwards).  A page-table entry outside
+ * [0, num_pages) sets the device error word and is skipped.  A physical page
+ * must belong to one sequence.  DASHKV_ERR_UNSUPPORTED for dense caches. */
+dashkv_status dashkv_demote_pages(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_tier_view *tv,
+                                  const int32_t *seq_lens, const uint8_t *protect, void *stream);
+
+/* dashkv_sparse_decode over a tiered paged cache: the same selection, the
+ * same exact fp32 attention, with the rows of tier-1 pages read from tv (their
+ * dequantized FP8 values) and the others from kv->k / kv->v. */
+dashkv_status dashkv_sparse_decode_tiered(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_tier_view *tv,
+                                          const void *q, const int32_t *seq_lens, const int32_t *sel_idx,
+                                          const int32_t *sel_cnt, float *out, float *lse, void *workspace,
+                                          size_t workspace_bytes, void *stream);
+
 /* Synchronise `stream`, then read and clear the current device's error
  * word: DASHKV_OK, DASHKV_ERR_TIMEOUT, DASHKV_ERR_DEVICE, DASHKV_ERR_CAPACITY
  * (in that order of precedence), or DASHKV_ERR_CUDA when the stream reports an

@@ -121,3 +121,21 @@ def test_block_view_layout_and_index_shapes():
     paged = dk.KVCache(Kp, Kp, dk.KVCache.empty_codes_like(Kp, 64, True), pt)
     idx = dk.BlockIndex.empty_for(paged, 2, 64, 16)
     assert tuple(idx.codes.shape) == (2, 4, 7 * 64 // 16, 1)
+
+
+def test_tier_view_layout_and_page_tier_shapes():
+    # dashkv_tier_view: { uint8_t *tier; uint8_t *k8; uint8_t *v8; int8_t *exps; }
+    assert ctypes.sizeof(dk.TierView) == 32
+    assert [dk.TierView.tier.offset, dk.TierView.k8.offset, dk.TierView.v8.offset,
+            dk.TierView.exps.offset] == [0, 8, 16, 24]
+    Kp = torch.zeros((10, 64, 4, 128), dtype=torch.bfloat16)
+    pt = torch.zeros((2, 7), dtype=torch.int32)
+    paged = dk.KVCache(Kp, Kp, dk.KVCache.empty_codes_like(Kp, 64, True), pt)
+    t = dk.PageTiers.empty_for(paged)
+    assert tuple(t.tier.shape) == (10,) and t.tier.dtype == torch.uint8
+    assert tuple(t.k8.shape) == (10, 64, 4, 128) and tuple(t.v8.shape) == (10, 64, 4, 128)
+    assert tuple(t.exps.shape) == (10, 64, 4, 2) and t.exps.dtype == torch.int8
+    assert not t.tier.any() and t.view().tier == t.tier.data_ptr()
+    K = torch.zeros((3, 2, 100, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dk.PageTiers.empty_for(dk.KVCache(K, K, dk.KVCache.empty_codes_like(K, 64, False)))
