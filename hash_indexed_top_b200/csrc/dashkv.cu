@@ -335,7 +335,7 @@ void set_attr_decode() {
     cudaFuncSetAttribute(sparse_decode_kernel<D, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)DecodeShape<D, G>::SMEM);
     cudaFuncSetAttribute(sparse_decode_kernel<D, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)DecodeShape<D, G>::SMEM);
+                         (int)(DecodeShape<D, G>::SMEM + DecodeShape<D, G>::EX_BYTES));
 }
 
 void set_attrs() {
@@ -554,8 +554,9 @@ void launch_decode_dg(const dashkv_ctx *ctx, const KV &kv, const void *q, const 
     const int cap_sel = ctx->cfg.topk + ctx->cfg.sink + ctx->cfg.window;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     const Tiers tr = tiers ? *tiers : Tiers{};
+    const size_t smem = DecodeShape<D, G>::SMEM + (tiers ? DecodeShape<D, G>::EX_BYTES : 0);
     launch_pdl(tiers ? sparse_decode_kernel<D, G, true> : sparse_decode_kernel<D, G, false>, dim3(splits, BH + wy),
-               dim3(kAttnThreads), DecodeShape<D, G>::SMEM, st, kv, static_cast<const __nv_bfloat16 *>(q),
+               dim3(kAttnThreads), smem, st, kv, static_cast<const __nv_bfloat16 *>(q),
                ctx->cfg.num_q_heads, si, sc, cap_sel, out, lse, ws, splits, scale_log2, seq_lens, ctx->cfg.sink,
                ctx->cfg.window, ctx->cfg.topk, wy, nw > 0 ? nw : 1, tr);
 }
@@ -782,11 +783,12 @@ void static_scratch_forget(int dev) {
     s.hist_off = s.hist_bytes = s.arrive_off = s.arrive_bytes = 0;
 }
 
-// Tier view of a paged cache (tiers.cuh): all four arrays, FP8 rows 16-byte aligned.
+// Tier view of a paged cache (tiers.cuh): all four arrays, FP8 rows 16-byte
+// aligned, exponents 4-byte aligned (the decode copies them in 4-byte words).
 dashkv_status check_tiers(const dashkv_ctx *ctx, const dashkv_tier_view *tv) {
     if (!tv || !tv->tier || !tv->k8 || !tv->v8 || !tv->exps) return DASHKV_ERR_INVALID_ARG;
     if (!ctx->cfg.page_size) return DASHKV_ERR_UNSUPPORTED;  // tiers are per page
-    if (!aligned(tv->k8, 16) || !aligned(tv->v8, 16) || !aligned(tv->exps, 2)) return DASHKV_ERR_INVALID_ARG;
+    if (!aligned(tv->k8, 16) || !aligned(tv->v8, 16) || !aligned(tv->exps, 4)) return DASHKV_ERR_INVALID_ARG;
     return DASHKV_OK;
 }
 

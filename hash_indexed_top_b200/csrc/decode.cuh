@@ -21,8 +21,9 @@
 // TIERED: rows of tier-1 pages (see tiers.cuh) are gathered as their FP8 K and
 // V rows (128 + 128 bytes at d = 128 instead of 256 + 256) into the first half
 // of the same staging slots, and read back as value(code) * 2^-s; the owner
-// lane of a tile row loads its page's tier byte and the row's two exponents
-// with the token id, one tile ahead.
+// lane of a tile row loads its page's tier byte with the token id, one tile
+// ahead, and copies the 4-byte word holding the row's two exponents into
+// shared memory with the row's copies (no register waits on it).
 #pragma once
 #include "common.cuh"
 #include "tiers.cuh"
@@ -55,6 +56,8 @@ struct DecodeShape {
     static constexpr size_t STAGE_BYTES = (size_t)NWARP * STAGES * TROWS * 2 * D * 2;
     static constexpr int V = RT * G;                   // logits of a lane group's tile (<= LPR)
     static constexpr size_t SMEM = STAGE_BYTES + (size_t)NST * G * (D + 2) * 4 + (size_t)NST * V * 4 + 16;
+    // TIERED: per warp and stage, the exponent word of each tile row (after SMEM)
+    static constexpr size_t EX_BYTES = (size_t)NWARP * STAGES * TROWS * 4;
 };
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
@@ -192,18 +195,24 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
         if (kv.page_size && kv.page_of(b, t) < 0) return -1;
         return t;
     };
-    // Tier of the row of token t (from tile_token: -1 or a valid token) --
-    // 1 | s_K << 8 | s_V << 16 for an FP8 row, 0 otherwise.
-    auto tile_meta = [&](int t) -> uint32_t {
+    // Tier of the row of token t (from tile_token: -1 or a valid token) of
+    // a tile staged in buffer buf: 1 | (row & 1) << 1 for an FP8 row, 0
+    // otherwise.  For an FP8 row the aligned exponent word holding the row's
+    // pair is copied to word (warp * STAGES + buf) * TROWS + lane after SMEM,
+    // committed with the row's copies.
+    auto tile_meta = [&](int t, int buf) -> uint32_t {
         if constexpr (!TIERED) {
             return 0u;
         } else {
             if (t < 0) return 0u;
             const int64_t p = kv.page_of(b, t);
             const int64_t row = (p * kv.page_size + t % kv.page_size) * kv.Hkv + h;
-            const uint32_t tr = __ldg(tiers.tier + p);
-            const uint32_t e2 = __ldg(reinterpret_cast<const unsigned short *>(tiers.exps) + row);
-            return tr ? 1u | (e2 << 8) : 0u;
+            if (!__ldg(tiers.tier + p)) return 0u;
+            const unsigned dst = (unsigned)__cvta_generic_to_shared(smem_raw + S::SMEM) +
+                                 4u * (unsigned)((warp * STAGES + buf) * TROWS + lane);
+            const int8_t *src = tiers.exps + (row & ~(int64_t)1) * 2;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+            return 1u | (uint32_t)(row & 1) << 1;
         }
     };
     // Gather a tile's K and V rows into buffer `buf` (zero-filled when invalid);
@@ -248,7 +257,7 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
         tok[s] = -1;
         if (base + s * WSTEP < r1) {
             tok[s] = tile_token(base + s * WSTEP);
-            meta[s] = tile_meta(tok[s]);
+            meta[s] = tile_meta(tok[s], s);
             prefetch(tok[s], meta[s], s);
         } else {
             cp_async_commit();
@@ -260,7 +269,7 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
         const int abuf = (k + STAGES - 1) % STAGES;
         if (ahead < r1) {
             tok[abuf] = tile_token(ahead);
-            meta[abuf] = tile_meta(tok[abuf]);
+            meta[abuf] = tile_meta(tok[abuf], abuf);
             prefetch(tok[abuf], meta[abuf], abuf);
         } else {
             cp_async_commit();
@@ -276,10 +285,18 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             const int jr = (j ^ jperm) * RPW + sub;  // row within the tile
             const __nv_bfloat16 *kr = tile + (size_t)jr * 2 * D + li * DPL;
             float kf[DPL];
-            const uint32_t mk = TIERED ? __shfl_sync(0xffffffffu, meta[buf], jr) : 0u;
-            if (TIERED && (mk & 1u)) {
-                e4m3_row<DPL>(reinterpret_cast<const uint8_t *>(tile + (size_t)jr * 2 * D) + li * DPL,
-                              pow2_neg((int)(int8_t)(mk >> 8)), kf);
+            bool f8 = false;
+            if constexpr (TIERED) {
+                const uint32_t mk = __shfl_sync(0xffffffffu, meta[buf], jr);
+                if (mk & 1u) {
+                    const uint32_t ew = reinterpret_cast<const uint32_t *>(smem_raw + S::SMEM)
+                                            [(warp * STAGES + buf) * TROWS + jr] >> ((mk & 2u) ? 16 : 0);
+                    e4m3_row<DPL>(reinterpret_cast<const uint8_t *>(tile + (size_t)jr * 2 * D) + li * DPL,
+                                  pow2_neg((int)(int8_t)ew), kf);
+                    f8 = true;
+                }
+            }
+            if (f8) {
             } else if constexpr (DPL >= 8) {
 #pragma unroll
                 for (int e = 0; e < DPL; e += 8) {
@@ -338,10 +355,18 @@ sparse_decode_kernel(KV kv, const __nv_bfloat16 *__restrict__ q, int Hq,
             const int jr = j * RPW + sub;
             const __nv_bfloat16 *vrow = tile + ((size_t)jr * 2 + 1) * D + li * DPL;
             float vf[DPL];
-            const uint32_t mv = TIERED ? __shfl_sync(0xffffffffu, meta[buf], jr) : 0u;
-            if (TIERED && (mv & 1u)) {
-                e4m3_row<DPL>(reinterpret_cast<const uint8_t *>(tile + ((size_t)jr * 2 + 1) * D) + li * DPL,
-                              pow2_neg((int)(int8_t)(mv >> 16)), vf);
+            bool f8v = false;
+            if constexpr (TIERED) {
+                const uint32_t mv = __shfl_sync(0xffffffffu, meta[buf], jr);
+                if (mv & 1u) {
+                    const uint32_t ew = reinterpret_cast<const uint32_t *>(smem_raw + S::SMEM)
+                                            [(warp * STAGES + buf) * TROWS + jr] >> ((mv & 2u) ? 16 : 0);
+                    e4m3_row<DPL>(reinterpret_cast<const uint8_t *>(tile + ((size_t)jr * 2 + 1) * D) + li * DPL,
+                                  pow2_neg((int)(int8_t)(ew >> 8)), vf);
+                    f8v = true;
+                }
+            }
+            if (f8v) {
             } else if constexpr (DPL >= 8) {
 #pragma unroll
                 for (int e = 0; e < DPL; e += 8) {

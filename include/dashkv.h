@@ -332,7 +332,8 @@ typedef struct dashkv_tier_view {
                        zero-fills it once and zeroes the byte of a page it reassigns */
     uint8_t *k8;    /* device u8 [num_pages][page][Hkv][d] FP8 keys (16-byte aligned) */
     uint8_t *v8;    /* device u8 [num_pages][page][Hkv][d] FP8 values (16-byte aligned) */
-    int8_t *exps;   /* device i8 [num_pages][page][Hkv][2]: s of the K row, then of the V row */
+    int8_t *exps;   /* device i8 [num_pages][page][Hkv][2]: s of the K row, then of the V row
+                       (4-byte aligned) */
 } dashkv_tier_view;
 
 /* The tier controller.  For every sequence b and logical page p whose tokens
