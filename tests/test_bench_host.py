@@ -59,3 +59,15 @@ def test_oracle_block_update_matches_a_whole_cache_encode():
         completed += int(seq[0]) % cfg.block == 0
         assert np.array_equal(bcodes, O.encode_blocks(L, K, seq, cfg.block, R, nb_cap)), s
     assert completed >= 2
+
+
+def test_oracle_sample_runs_paged_and_tiered_workloads_as_one_dense_sequence():
+    # the CPU baseline times one sequence of the workload at its longest
+    # length, dense; the tiered workload demotes its middle pages first
+    from hash_indexed_top_b200 import workloads as W
+    for name in ("ragged_paged", "ragged_paged_fp8"):
+        cfg = W.CONFIGS[name].scaled(N=3000, n_min=500, topk=128, window=64)
+        r = bench.oracle_sample(cfg, 2)
+        assert len(r["times"]) == 2 and all(t > 0 for t in r["times"])
+        assert "N=3000" in r["sample"]
+        assert ("FP8" in r["sample"]) == (name == "ragged_paged_fp8")
