@@ -350,7 +350,10 @@ dashkv_status dashkv_demote_pages(dashkv_ctx *ctx, const dashkv_kv_view *kv, con
 
 /* dashkv_sparse_decode over a tiered paged cache: the same selection, the
  * same exact fp32 attention, with the rows of tier-1 pages read from tv (their
- * dequantized FP8 values) and the others from kv->k / kv->v. */
+ * dequantized FP8 values) and the others from kv->k / kv->v.  Same arguments,
+ * workspace and error behaviour as dashkv_sparse_decode; in addition
+ * DASHKV_ERR_INVALID_ARG for a missing or misaligned tier view and
+ * DASHKV_ERR_UNSUPPORTED for dense caches. */
 dashkv_status dashkv_sparse_decode_tiered(dashkv_ctx *ctx, const dashkv_kv_view *kv, const dashkv_tier_view *tv,
                                           const void *q, const int32_t *seq_lens, const int32_t *sel_idx,
                                           const int32_t *sel_cnt, float *out, float *lse, void *workspace,
