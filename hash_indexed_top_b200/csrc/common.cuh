@@ -92,7 +92,7 @@ __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
 }
 
 // ---- shared-memory barriers and bulk copies (global -> this CTA's shared
-// memory, completion counted in bytes on an mbarrier; never multicast).
+// memory only, completion counted in bytes on an mbarrier).
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
 }
